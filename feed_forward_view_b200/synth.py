@@ -1,0 +1,139 @@
+"""Seeded synthetic inputs for the VGGT attention path.
+
+This module only *draws* inputs; it holds none of the attention arithmetic.
+Both the CUDA path and the CPU oracle consume the same tensors built here.
+
+Token layout (VGGT aggregator, one scene, B = 1):
+
+* ``S`` frames, each with ``T = 5 + g*g`` tokens: one camera token and four
+  register tokens (the five "special" tokens), then the ``g x g`` patch grid in
+  row-major order (vggt-jax README, attention benchmark table: ``[2,930,16,64]``
+  is 2 frames of 25*37 patches + 5 specials).
+* ``q``, ``k``, ``v`` are ``[S*T, H, D]`` bf16, token-major with heads
+  interleaved, as in the ``[B, N, H, D]`` shapes of that table.
+* ``pos`` is ``[S*T, 2]`` fp32 ``(row, col)``: special tokens at ``(0, 0)``,
+  patch ``(r, c)`` at ``(r + 1, c + 1)``.
+
+Values are i.i.d. N(0, 1) drawn in fp32 from a CPU ``torch.Generator`` and
+rounded to bf16 (round-to-nearest-even, torch's own conversion).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+N_SPECIAL = 5
+HEADS = 16
+HEAD_DIM = 64
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention workload: kind, frame count, grid side and pooling factor."""
+
+    name: str
+    kind: str  # "global" | "frame" | "descriptor"
+    S: int
+    g: int
+    kv_down: int = 1
+    H: int = HEADS
+    D: int = HEAD_DIM
+
+    @property
+    def T(self) -> int:
+        return N_SPECIAL + self.g * self.g
+
+    @property
+    def n_q(self) -> int:
+        return self.S * self.T
+
+    @property
+    def T_k(self) -> int:
+        if self.kind != "descriptor":
+            return self.T
+        nc = -(-self.g // self.kv_down) if self.g > 0 else 0
+        return N_SPECIAL + nc * nc
+
+    @property
+    def n_k(self) -> int:
+        return self.S * self.T_k
+
+    def flops(self) -> float:
+        """Algorithmic attention FLOPs: 4 * H * D per (query, key) pair."""
+        if self.kind == "frame":
+            pairs = self.S * self.T * self.T
+        else:
+            pairs = self.n_q * self.n_k
+        return 4.0 * self.H * self.D * pairs
+
+
+# The five workloads of the pages' shapes (two 224^2 frames; eight 518^2 frames
+# at patch 14; nine 1024^2 frames at patch 16; 200 518^2 frames pooled 4x4).
+WORKLOADS = {
+    w.name: w
+    for w in (
+        Workload("global_s2_g16", "global", S=2, g=16),
+        Workload("frame_s8_g37", "frame", S=8, g=37),
+        Workload("global_s8_g37", "global", S=8, g=37),
+        Workload("global_s9_g64", "global", S=9, g=64),
+        Workload("descriptor_s200_g37_kd4", "descriptor", S=200, g=37, kv_down=4),
+    )
+}
+
+
+def grid_side(T: int) -> int:
+    """Side of the square patch grid for ``T`` tokens per frame, or -1."""
+    p = T - N_SPECIAL
+    if p < 0:
+        return -1
+    g = math.isqrt(p)
+    return g if g * g == p else -1
+
+
+def grid_positions(S: int, g: int) -> torch.Tensor:
+    """``[S*T, 2]`` fp32 (row, col): specials at (0,0), patch (r,c) at (r+1,c+1)."""
+    T = N_SPECIAL + g * g
+    one = torch.zeros(T, 2, dtype=torch.float32)
+    if g > 0:
+        r = torch.arange(g, dtype=torch.float32).repeat_interleave(g)
+        c = torch.arange(g, dtype=torch.float32).repeat(g)
+        one[N_SPECIAL:, 0] = r + 1.0
+        one[N_SPECIAL:, 1] = c + 1.0
+    return one.repeat(S, 1).contiguous()
+
+
+def normal_bf16(shape, seed: int) -> torch.Tensor:
+    """N(0,1) fp32 from a seeded CPU generator, rounded to bf16."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_qkv(S: int, g: int, seed: int, H: int = HEADS, D: int = HEAD_DIM):
+    """Return ``(q, k, v, pos)`` CPU tensors for one scene.
+
+    q, k, v are drawn from three generators seeded ``3*seed``, ``3*seed+1``,
+    ``3*seed+2`` so each tensor is reproducible on its own.
+    """
+    T = N_SPECIAL + g * g
+    n = S * T
+    q = normal_bf16((n, H, D), 3 * seed)
+    k = normal_bf16((n, H, D), 3 * seed + 1)
+    v = normal_bf16((n, H, D), 3 * seed + 2)
+    return q, k, v, grid_positions(S, g)
+
+
+def make_workload(w: Workload, seed: int):
+    return make_qkv(w.S, w.g, seed, w.H, w.D)
+
+
+def sample_rows(n: int, count: int, seed: int) -> torch.Tensor:
+    """Sorted, distinct query-row indices spread over ``[0, n)``, always
+    including the first and the last row (the ragged tail)."""
+    count = min(count, n)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(10_000 + int(seed))
+    idx = torch.randperm(n, generator=gen)[:count]
+    return torch.unique(torch.cat([idx, torch.tensor([0, n - 1])]))

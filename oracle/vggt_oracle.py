@@ -1,0 +1,336 @@
+"""CPU oracle for the VGGT alternating-attention path, in float64.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. The product path (the
+CUDA library and its Python binding) never calls it and shares no code with it.
+
+What it computes, per head, for bf16 inputs widened exactly to float64:
+
+1. QK prologue: ``x_hat = RoPE2D(LayerNorm(x), pos)`` for every query and key
+   head vector (64 dims).
+   * LayerNorm over the head's 64 dims, centered, biased variance, eps 1e-5,
+     no affine ("Norm: Layer Normalization" slide, ``(x - mu) / sigma``, in the
+     VGGT paper-report slides; ``layer_norm_eps 1e-05`` in the VGGT-Omega
+     config.json field table; vggt-jax README keeps "centered FP32 LayerNorm"
+     and tunes the Q/K LayerNorm shapes).
+   * 2D rotary embedding with base 100 (``rope_base: 100.0`` in the VGGT-Omega
+     config.json field table). Dims 0-31 rotate by the row position, dims 32-63
+     by the column position; within each 32-dim half, dim ``j`` pairs with dim
+     ``j + 16`` and turns by ``pos * base**(-2j/32)`` -- the frequency schedule
+     of the sinusoidal positional-encoding formula on the "Positional
+     Encoding (4/6)" slide, ``pos / 10000^(2i/d)``.
+2. Scores ``s_ij = q_hat_i . k_hat_j / sqrt(64)``, softmax over ``j``, and
+   ``o_i = sum_j p_ij v_j`` ("Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V"
+   and "softmax(x)_i = e^{x_i} / sum_j e^{x_j}" slides, Section V).
+3. Which keys a query sees:
+   * frame attention: the keys of its own frame ("Frame Attention" panel of the
+     "Global + Frame Attention" architecture slide);
+   * global attention: all ``S*T`` keys of the scene ("Global Attention" panel);
+   * descriptor attention: all frames' compressed descriptors -- each frame's
+     five special tokens unchanged plus one average per ``kd x kd`` cell of the
+     patch grid (ceil mode), at the cell's mean position (FlashVGGT README,
+     Overview: cross-attention between all image tokens and the per-frame
+     descriptor set; Key Arguments: ``--kv_downfactor`` 4).
+
+Evaluating a subset of query rows is the same definition restricted to those
+rows: every output row depends only on its own query and the key set, so
+``rows=`` changes nothing about any row that is computed.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+N_SPECIAL = 5
+LN_EPS = 1e-5
+ROPE_BASE = 100.0
+HEAD_DIM = 64
+
+# --------------------------------------------------------------------------
+# bf16 <-> float helpers (exact widening; correctly rounded narrowing)
+# --------------------------------------------------------------------------
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of raw bf16 bit patterns (uint16) as float64."""
+    b = np.ascontiguousarray(bits).view(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact value of raw bf16 bit patterns (uint16) as float32."""
+    b = np.ascontiguousarray(bits).view(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16, round-to-nearest-even, as uint16 bits.
+
+    bf16 keeps the top 16 bits of the float32 pattern. Rounding to nearest
+    with ties to even adds ``0x7FFF`` plus the lowest kept bit before
+    truncating. NaN stays a quiet NaN with its sign.
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    rounded = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = np.isnan(np.asarray(x, dtype=np.float32))
+    if nan.any():
+        sign = ((u >> 16) & 0x8000).astype(np.uint16)
+        rounded = np.where(nan, sign | np.uint16(0x7FC0), rounded)
+    return rounded
+
+
+# --------------------------------------------------------------------------
+# Softmax, LayerNorm, RoPE
+# --------------------------------------------------------------------------
+
+
+def softmax(x: np.ndarray, axis: int = -1) -> np.ndarray:
+    """``e^{x_i} / sum_j e^{x_j}`` along ``axis`` (Section V, softmax slide).
+
+    The row maximum is subtracted first; that leaves every quotient unchanged
+    and keeps ``exp`` finite.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(x - np.max(x, axis=axis, keepdims=True))
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+def layer_norm(x: np.ndarray, eps: float = LN_EPS) -> np.ndarray:
+    """``(x - mu) / sqrt(var + eps)`` over the last axis; biased variance,
+    computed from the centered values; no scale or shift."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    c = x - mu
+    var = (c * c).mean(axis=-1, keepdims=True)
+    return c / np.sqrt(var + eps)
+
+
+def rope_frequencies(base: float, d: int) -> np.ndarray:
+    """``base ** (-2i / d)`` for ``i = 0 .. d/2 - 1``: the angular frequency of
+    pair ``i`` in the sinusoidal formula ``PE(pos, 2i) = sin(pos / base^(2i/d))``
+    (Positional Encoding (4/6) slide)."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return base ** (-2.0 * i / d)
+
+
+def sinusoidal_pe(pos: float, d: int, base: float) -> np.ndarray:
+    """The slide's sinusoidal encoding: sin on even dims, cos on odd dims."""
+    f = rope_frequencies(base, d)
+    out = np.empty(d, dtype=np.float64)
+    out[0::2] = np.sin(pos * f)
+    out[1::2] = np.cos(pos * f)
+    return out
+
+
+def rope_2d(x: np.ndarray, pos: np.ndarray, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotate head vectors ``x[..., 64]`` by their 2D positions ``pos[..., 2]``.
+
+    Half ``a`` (a=0: dims 0-31, row position; a=1: dims 32-63, column
+    position) is split into ``x1 = dims 0-15`` and ``x2 = dims 16-31`` of the
+    half; pair ``(x1_j, x2_j)`` turns by ``theta_j = p_a * base**(-2j/32)``:
+    ``x1' = x1 cos - x2 sin``, ``x2' = x2 cos + x1 sin``.
+    ``pos`` broadcasts against ``x[..., 0]``.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    pos = np.asarray(pos, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    quarter = half // 2
+    freq = rope_frequencies(base, half)  # quarter entries
+    out = np.empty_like(x)
+    for a in range(2):
+        theta = pos[..., a][..., None] * freq  # [..., quarter]
+        c, s = np.cos(theta), np.sin(theta)
+        x1 = x[..., a * half: a * half + quarter]
+        x2 = x[..., a * half + quarter: (a + 1) * half]
+        out[..., a * half: a * half + quarter] = x1 * c - x2 * s
+        out[..., a * half + quarter: (a + 1) * half] = x2 * c + x1 * s
+    return out
+
+
+def qk_prologue(x: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """LayerNorm then 2D RoPE for ``x[N, H, D]`` at ``pos[N, 2]``."""
+    return rope_2d(layer_norm(x), np.asarray(pos)[:, None, :])
+
+
+# --------------------------------------------------------------------------
+# Grid geometry and K/V descriptor pooling
+# --------------------------------------------------------------------------
+
+
+def grid_side(T: int) -> int:
+    """Side ``g`` of the square patch grid when ``T = 5 + g*g``, else -1."""
+    p = T - N_SPECIAL
+    if p < 0:
+        return -1
+    g = math.isqrt(p)
+    return g if g * g == p else -1
+
+
+def pool_cells(g: int, kd: int):
+    """Ceil-mode ``kd x kd`` cells of a ``g x g`` grid, row-major.
+
+    Each cell is a list of member patch indices ``r*g + c`` in row-major
+    order; edge cells keep only the members that lie inside the grid.
+    """
+    nc = -(-g // kd) if g > 0 else 0
+    cells = []
+    for cr in range(nc):
+        for cc in range(nc):
+            rows = range(cr * kd, min(cr * kd + kd, g))
+            cols = range(cc * kd, min(cc * kd + kd, g))
+            cells.append([r * g + c for r in rows for c in cols])
+    return cells
+
+
+def pooled_tokens_per_frame(T: int, kd: int) -> int:
+    g = grid_side(T)
+    nc = -(-g // kd) if g > 0 else 0
+    return N_SPECIAL + nc * nc
+
+
+def kv_pool(k: np.ndarray, v: np.ndarray, pos: np.ndarray, S: int, T: int, kd: int):
+    """Per-frame descriptors in float64: the 5 special tokens unchanged, then
+    the mean of each ceil-mode ``kd x kd`` cell of the patch grid (K, V and
+    position alike). Inputs are ``[S*T, H, D]`` and ``[S*T, 2]``."""
+    g = grid_side(T)
+    cells = pool_cells(g, kd)
+    Tk = N_SPECIAL + len(cells)
+    k = np.asarray(k, dtype=np.float64).reshape(S, T, *k.shape[1:])
+    v = np.asarray(v, dtype=np.float64).reshape(S, T, *v.shape[1:])
+    pos = np.asarray(pos, dtype=np.float64).reshape(S, T, 2)
+    kp = np.empty((S, Tk) + k.shape[2:])
+    vp = np.empty((S, Tk) + v.shape[2:])
+    pp = np.empty((S, Tk, 2))
+    kp[:, :N_SPECIAL] = k[:, :N_SPECIAL]
+    vp[:, :N_SPECIAL] = v[:, :N_SPECIAL]
+    pp[:, :N_SPECIAL] = pos[:, :N_SPECIAL]
+    for ci, members in enumerate(cells):
+        idx = N_SPECIAL + np.asarray(members)
+        kp[:, N_SPECIAL + ci] = k[:, idx].mean(axis=1)
+        vp[:, N_SPECIAL + ci] = v[:, idx].mean(axis=1)
+        pp[:, N_SPECIAL + ci] = pos[:, idx].mean(axis=1)
+    return (kp.reshape(S * Tk, *k.shape[2:]), vp.reshape(S * Tk, *v.shape[2:]),
+            pp.reshape(S * Tk, 2))
+
+
+def kv_pool_bf16_reference(k_bits, v_bits, pos, S: int, T: int, kd: int):
+    """The stored form of the pooled descriptors, bit for bit.
+
+    For every cell and channel: float32 sum of the members in row-major order
+    (each addition rounded to float32), divided in float32 by the member
+    count, rounded to bf16 (nearest, ties to even). Positions: the same float32
+    sum and division, kept in float32. Special tokens are copied unchanged.
+    Returns ``(k_bits, v_bits, pos_f32)``.
+    """
+    g = grid_side(T)
+    cells = pool_cells(g, kd)
+    Tk = N_SPECIAL + len(cells)
+    k32 = bf16_bits_to_f32(k_bits).reshape(S, T, -1)
+    v32 = bf16_bits_to_f32(v_bits).reshape(S, T, -1)
+    p32 = np.asarray(pos, dtype=np.float32).reshape(S, T, 2)
+    kb = np.asarray(k_bits).view(np.uint16).reshape(S, T, -1)
+    vb = np.asarray(v_bits).view(np.uint16).reshape(S, T, -1)
+    ko = np.empty((S, Tk, kb.shape[2]), dtype=np.uint16)
+    vo = np.empty((S, Tk, vb.shape[2]), dtype=np.uint16)
+    po = np.empty((S, Tk, 2), dtype=np.float32)
+    ko[:, :N_SPECIAL] = kb[:, :N_SPECIAL]
+    vo[:, :N_SPECIAL] = vb[:, :N_SPECIAL]
+    po[:, :N_SPECIAL] = p32[:, :N_SPECIAL]
+    for ci, members in enumerate(cells):
+        ak = np.zeros((S, k32.shape[2]), dtype=np.float32)
+        av = np.zeros((S, v32.shape[2]), dtype=np.float32)
+        ap = np.zeros((S, 2), dtype=np.float32)
+        for m in members:  # row-major member order
+            t = N_SPECIAL + m
+            ak = ak + k32[:, t]
+            av = av + v32[:, t]
+            ap = ap + p32[:, t]
+        n = np.float32(len(members))
+        ko[:, N_SPECIAL + ci] = f32_to_bf16_bits(ak / n)
+        vo[:, N_SPECIAL + ci] = f32_to_bf16_bits(av / n)
+        po[:, N_SPECIAL + ci] = ap / n
+    return ko.reshape(S * Tk, -1), vo.reshape(S * Tk, -1), po.reshape(S * Tk, 2)
+
+
+# --------------------------------------------------------------------------
+# Attention
+# --------------------------------------------------------------------------
+
+ROW_GROUP = 1024  # rows evaluated together; rows are independent
+
+
+def _attend(qh: np.ndarray, kh: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """``softmax(qh kh^T / sqrt(D)) v`` for one head: qh [n,D], kh [m,D], v [m,Dv]."""
+    scores = (qh @ kh.T) / math.sqrt(qh.shape[-1])
+    return softmax(scores, axis=-1) @ v
+
+
+def cross_attention(q_hat, k_hat, v, rows=None) -> np.ndarray:
+    """Every selected query row attends to every key, each head on its own.
+
+    ``q_hat [Nq,H,D]``, ``k_hat [Nk,H,D]`` already through the prologue;
+    ``v [Nk,H,D]``. Returns ``[len(rows), H, D]``.
+    """
+    rows = np.arange(q_hat.shape[0]) if rows is None else np.asarray(rows)
+    H = q_hat.shape[1]
+    out = np.empty((rows.size, H, v.shape[2]))
+    for h in range(H):
+        kh, vh = k_hat[:, h], v[:, h]
+        for s0 in range(0, rows.size, ROW_GROUP):
+            r = rows[s0:s0 + ROW_GROUP]
+            out[s0:s0 + ROW_GROUP, h] = _attend(q_hat[r, h], kh, vh)
+    return out
+
+
+def _rows(n: int, rows):
+    return np.arange(n) if rows is None else np.asarray(rows)
+
+
+def attn_global(q, k, v, pos, S: int, T: int, rows=None) -> np.ndarray:
+    """Global attention: all ``S*T`` tokens attend to all ``S*T`` tokens."""
+    rows = _rows(S * T, rows)
+    q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows])
+    k_hat = qk_prologue(k, pos)
+    return cross_attention(q_hat, k_hat, np.asarray(v, dtype=np.float64))
+
+
+def attn_frame(q, k, v, pos, S: int, T: int, rows=None) -> np.ndarray:
+    """Frame attention: each token attends to the ``T`` tokens of its frame."""
+    rows = _rows(S * T, rows)
+    q, k, pos = np.asarray(q), np.asarray(k), np.asarray(pos)
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty((rows.size, q.shape[1], v.shape[2]))
+    frames = rows // T
+    for s in np.unique(frames):
+        sel = np.nonzero(frames == s)[0]
+        lo, hi = s * T, (s + 1) * T
+        q_hat = qk_prologue(q[rows[sel]], pos[rows[sel]])
+        k_hat = qk_prologue(k[lo:hi], pos[lo:hi])
+        out[sel] = cross_attention(q_hat, k_hat, v[lo:hi])
+    return out
+
+
+def attn_descriptor(q, k, v, pos, S: int, T: int, kd: int, rows=None) -> np.ndarray:
+    """Descriptor attention: every query attends to all frames' pooled
+    descriptors; the pooled keys go through the prologue at their cell-mean
+    positions, pooled values are used as they are."""
+    kp, vp, pp = kv_pool(k, v, pos, S, T, kd)
+    rows = _rows(S * T, rows)
+    q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows])
+    k_hat = qk_prologue(kp, pp)
+    return cross_attention(q_hat, k_hat, vp)
+
+
+def flops(kind: str, S: int, T: int, Tk: int, H: int, D: int, n_rows=None) -> float:
+    """Algorithmic attention FLOPs, ``4*H*D`` per (query, key) pair."""
+    if kind == "frame":
+        keys = T
+    elif kind == "descriptor":
+        keys = S * Tk
+    else:
+        keys = S * T
+    n = S * T if n_rows is None else n_rows
+    return 4.0 * H * D * n * keys

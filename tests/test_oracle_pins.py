@@ -1,0 +1,416 @@
+"""Pins for the fp64 CPU oracle: worked examples printed on the pages, closed
+forms, invariants and special cases that reduce to a library routine.
+
+Each test is built so that a plausible slip in the oracle (a dropped scale, a
+wrong sign or pair index, the wrong half for rows/columns, an unbiased
+variance, the wrong key set for a frame, column-major pooling order) fails.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import vggt_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _f64(t: torch.Tensor) -> np.ndarray:
+    return O.bf16_bits_to_f64(_bits(t))
+
+
+# ----------------------------------------------------------------- fixtures
+
+
+def _read_kv(path):
+    rows = {}
+    for line in open(path, encoding="utf-8"):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, _, rest = line.partition(" ")
+        rows[key] = rest
+    return rows
+
+
+def test_softmax_worked_example():
+    g = _read_kv(os.path.join(GOLDEN, "softmax_worked_example.txt"))
+    x = np.array([float(t) for t in g["input"].split()])
+    want = np.array([float(t) for t in g["expected"].split()])
+    half_unit = 0.5 * 10.0 ** -int(g["decimals"])
+    got = O.softmax(x)
+    assert np.all(np.abs(got - want) <= half_unit + 1e-12), got
+    assert abs(got.sum() - 1.0) < 1e-15
+
+
+def test_sinusoid_worked_example_pins_frequency_schedule():
+    path = os.path.join(GOLDEN, "sinusoid_worked_example.txt")
+    meta, rows = {}, []
+    for line in open(path, encoding="utf-8"):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("pos "):
+            p, vals = line[4:].split(":")
+            rows.append((float(p), np.array([float(t) for t in vals.split()])))
+        else:
+            k, v = line.split()
+            meta[k] = float(v)
+    half_unit = 0.5 * 10.0 ** -int(meta["decimals"])
+    for p, want in rows:
+        got = O.sinusoidal_pe(p, int(meta["d"]), meta["base"])
+        assert np.all(np.abs(got - want) <= half_unit + 1e-12), (p, got, want)
+
+
+def test_softmax_rows_sum_to_one_and_shift_invariance():
+    rng = np.random.default_rng(0)
+    x = rng.normal(scale=30.0, size=(7, 50))
+    p = O.softmax(x)
+    assert np.allclose(p.sum(-1), 1.0, atol=1e-14, rtol=0)
+    assert np.all(p >= 0)
+    assert np.allclose(O.softmax(x + 123.0), p, atol=1e-15)
+    # the largest score always gets the largest weight
+    assert np.all(p.argmax(-1) == x.argmax(-1))
+
+
+# ----------------------------------------------------------------- LayerNorm
+
+
+def test_layernorm_alternating_closed_form():
+    for a in (1e-3, 0.5, 3.0):
+        x = np.tile([a, -a], 32)
+        want = np.tile([1.0, -1.0], 32) * a / math.sqrt(a * a + O.LN_EPS)
+        assert np.allclose(O.layer_norm(x), want, atol=1e-15, rtol=1e-13)
+
+
+def test_layernorm_moments_use_biased_variance_and_eps():
+    rng = np.random.default_rng(1)
+    for scale in (1e-3, 1.0, 40.0):
+        x = rng.normal(loc=3.0, scale=scale, size=(5, 64))
+        y = O.layer_norm(x)
+        sigma2 = np.var(x, axis=-1)  # population variance (ddof=0)
+        assert np.allclose(y.mean(-1), 0.0, atol=1e-12)
+        assert np.allclose(np.var(y, axis=-1), sigma2 / (sigma2 + O.LN_EPS), rtol=1e-10)
+    # shift invariance
+    assert np.allclose(O.layer_norm(x + 17.25), O.layer_norm(x), atol=1e-10)
+    # a constant vector normalises to exactly zero
+    assert np.all(O.layer_norm(np.full(64, 2.5)) == 0.0)
+
+
+# ----------------------------------------------------------------- RoPE
+
+
+def _unit(i, d=64):
+    e = np.zeros(d)
+    e[i] = 1.0
+    return e
+
+
+def test_rope_identity_at_origin():
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=(9, 64))
+    assert np.array_equal(O.rope_2d(x, np.zeros((9, 2))), x)
+
+
+@pytest.mark.parametrize(
+    "dim,partner,pos,freq",
+    [
+        (8, 24, (5.0, 0.0), 0.1),      # row half, j=8: 100^(-8/16) = 0.1
+        (0, 16, (2.0, 0.0), 1.0),      # row half, j=0: frequency 1
+        (40, 56, (0.0, 5.0), 0.1),     # column half, j=8
+        (36, 52, (0.0, 3.0), 100 ** (-4 / 16)),  # column half, j=4
+    ],
+)
+def test_rope_pair_layout_and_sign(dim, partner, pos, freq):
+    theta = (pos[0] if dim < 32 else pos[1]) * freq
+    out = O.rope_2d(_unit(dim), np.array(pos))
+    want = np.zeros(64)
+    want[dim] = math.cos(theta)
+    want[partner] = math.sin(theta)
+    assert np.allclose(out, want, atol=1e-15)
+    # the second member of the pair turns the other way
+    out2 = O.rope_2d(_unit(partner), np.array(pos))
+    want2 = np.zeros(64)
+    want2[partner] = math.cos(theta)
+    want2[dim] = -math.sin(theta)
+    assert np.allclose(out2, want2, atol=1e-15)
+
+
+def test_rope_row_position_leaves_column_half_alone():
+    rng = np.random.default_rng(3)
+    x = rng.normal(size=64)
+    out = O.rope_2d(x, np.array([7.0, 0.0]))
+    assert np.array_equal(out[32:], x[32:])
+    out = O.rope_2d(x, np.array([0.0, 7.0]))
+    assert np.array_equal(out[:32], x[:32])
+
+
+def test_rope_norm_and_relative_position():
+    rng = np.random.default_rng(4)
+    q, k = rng.normal(size=64), rng.normal(size=64)
+    p, pp = np.array([3.0, 11.0]), np.array([17.0, 2.0])
+    rq, rk = O.rope_2d(q, p), O.rope_2d(k, pp)
+    # norm of every rotated pair is kept
+    for a in (0, 32):
+        for j in range(16):
+            n0 = q[a + j] ** 2 + q[a + j + 16] ** 2
+            n1 = rq[a + j] ** 2 + rq[a + j + 16] ** 2
+            assert abs(n0 - n1) < 1e-12
+    # the score depends only on the position difference
+    lhs = rq @ rk
+    rhs = q @ O.rope_2d(k, pp - p)
+    assert abs(lhs - rhs) < 1e-12
+
+
+# ----------------------------------------------------------------- attention
+
+
+def test_cross_attention_two_keys_closed_form_pins_scale():
+    # q_hat = 8 e0, k1 = e0, k2 = 0 -> s1 = 8*1/sqrt(64) = 1, s2 = 0
+    qh = np.zeros((1, 1, 64))
+    qh[0, 0, 0] = 8.0
+    kh = np.zeros((2, 1, 64))
+    kh[0, 0, 0] = 1.0
+    v = np.zeros((2, 1, 64))
+    v[0, 0, :] = 1.0
+    v[1, 0, :] = -3.0
+    p1 = math.e / (1.0 + math.e)
+    want = p1 * 1.0 + (1 - p1) * -3.0
+    out = O.cross_attention(qh, kh, v)
+    assert np.allclose(out, want, atol=1e-14)
+
+
+def test_cross_attention_single_key_returns_its_value():
+    rng = np.random.default_rng(5)
+    qh, kh, v = rng.normal(size=(4, 2, 64)), rng.normal(size=(1, 2, 64)), rng.normal(size=(1, 2, 64))
+    out = O.cross_attention(qh, kh, v)
+    assert np.allclose(out, np.broadcast_to(v, out.shape), atol=1e-14)
+
+
+def test_cross_attention_brute_force_tiny():
+    rng = np.random.default_rng(6)
+    nq, nk, d = 3, 4, 64
+    qh, kh, v = rng.normal(size=(nq, 1, d)), rng.normal(size=(nk, 1, d)), rng.normal(size=(nk, 1, d))
+    out = O.cross_attention(qh, kh, v)
+    for i in range(nq):
+        w = []
+        for j in range(nk):
+            dot = 0.0
+            for c in range(d):
+                dot += qh[i, 0, c] * kh[j, 0, c]
+            w.append(math.exp(dot / 8.0))
+        tot = sum(w)
+        for c in range(d):
+            acc = 0.0
+            for j in range(nk):
+                acc += w[j] / tot * v[j, 0, c]
+            assert abs(acc - out[i, 0, c]) < 1e-12
+
+
+def _scene(S, g, H=2, seed=0):
+    T = 5 + g * g
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(S * T, H, 64))
+    k = rng.normal(size=(S * T, H, 64))
+    v = rng.normal(size=(S * T, H, 64))
+    pos = np.zeros((S * T, 2))
+    for s in range(S):
+        for r in range(g):
+            for c in range(g):
+                pos[s * T + 5 + r * g + c] = (r + 1, c + 1)
+    return q, k, v, pos, T
+
+
+def test_constant_values_return_the_constant():
+    q, k, v, pos, T = _scene(2, 3)
+    v[:] = 0.75
+    for out in (O.attn_global(q, k, v, pos, 2, T), O.attn_frame(q, k, v, pos, 2, T),
+                O.attn_descriptor(q, k, v, pos, 2, T, 2)):
+        assert np.allclose(out, 0.75, atol=1e-14)
+
+
+def test_zero_queries_average_exactly_the_visible_keys():
+    # q = 0 -> LayerNorm gives 0 -> every score is 0 -> output = mean of V over
+    # the keys the query can see. This pins each variant's key set.
+    S, g = 3, 3
+    q, k, v, pos, T = _scene(S, g)
+    q[:] = 0.0
+    og = O.attn_global(q, k, v, pos, S, T)
+    assert np.allclose(og, v.mean(axis=0, keepdims=True), atol=1e-13)
+    of = O.attn_frame(q, k, v, pos, S, T)
+    for s in range(S):
+        want = v[s * T:(s + 1) * T].mean(axis=0)
+        assert np.allclose(of[s * T:(s + 1) * T], want, atol=1e-13)
+    # descriptor with kd >= g: per frame 5 specials + the mean of the grid
+    od = O.attn_descriptor(q, k, v, pos, S, T, kd=g)
+    desc = []
+    for s in range(S):
+        fr = v[s * T:(s + 1) * T]
+        desc.extend(list(fr[:5]))
+        desc.append(fr[5:].mean(axis=0))
+    assert np.allclose(od, np.mean(desc, axis=0), atol=1e-13)
+
+
+def test_global_attention_is_equivariant_to_frame_permutation():
+    S, g = 3, 2
+    q, k, v, pos, T = _scene(S, g, seed=7)
+    perm = [2, 0, 1]
+    idx = np.concatenate([np.arange(s * T, (s + 1) * T) for s in perm])
+    out = O.attn_global(q, k, v, pos, S, T)
+    outp = O.attn_global(q[idx], k[idx], v[idx], pos[idx], S, T)
+    assert np.allclose(outp, out[idx], atol=1e-13)
+
+
+def test_frame_attention_single_frame_equals_global():
+    q, k, v, pos, T = _scene(1, 3, seed=8)
+    assert np.allclose(O.attn_frame(q, k, v, pos, 1, T), O.attn_global(q, k, v, pos, 1, T), atol=1e-14)
+
+
+def test_frame_attention_ignores_other_frames():
+    S, g = 3, 2
+    q, k, v, pos, T = _scene(S, g, seed=9)
+    base = O.attn_frame(q, k, v, pos, S, T)
+    k2, v2 = k.copy(), v.copy()
+    k2[T:2 * T] += 5.0 * np.random.default_rng(1).normal(size=k2[T:2 * T].shape)
+    v2[T:2 * T] -= 2.0
+    alt = O.attn_frame(q, k2, v2, pos, S, T)
+    assert np.allclose(alt[:T], base[:T], atol=1e-15)
+    assert np.allclose(alt[2 * T:], base[2 * T:], atol=1e-15)
+    assert not np.allclose(alt[T:2 * T], base[T:2 * T])
+
+
+def test_descriptor_kd1_equals_global():
+    S, g = 2, 3
+    q, k, v, pos, T = _scene(S, g, seed=10)
+    assert np.allclose(O.attn_descriptor(q, k, v, pos, S, T, 1), O.attn_global(q, k, v, pos, S, T),
+                       atol=1e-13)
+
+
+def test_row_subsets_match_full_evaluation():
+    S, g = 2, 3
+    q, k, v, pos, T = _scene(S, g, seed=11)
+    rows = np.array([0, 4, 5, T, 2 * T - 1])
+    for full, part in (
+        (O.attn_global(q, k, v, pos, S, T), O.attn_global(q, k, v, pos, S, T, rows=rows)),
+        (O.attn_frame(q, k, v, pos, S, T), O.attn_frame(q, k, v, pos, S, T, rows=rows)),
+        (O.attn_descriptor(q, k, v, pos, S, T, 2), O.attn_descriptor(q, k, v, pos, S, T, 2, rows=rows)),
+    ):
+        assert np.allclose(full[rows], part, atol=1e-15)
+
+
+# ----------------------------------------------------------------- pooling
+
+
+def test_grid_helpers():
+    assert O.grid_side(1374) == 37 and O.grid_side(261) == 16 and O.grid_side(4101) == 64
+    assert O.grid_side(5) == 0 and O.grid_side(930) == -1 and O.grid_side(4) == -1
+    assert O.pooled_tokens_per_frame(1374, 4) == 105
+    assert O.pooled_tokens_per_frame(1374, 1) == 1374
+    assert O.pooled_tokens_per_frame(1374, 40) == 6
+    cells = O.pool_cells(5, 2)
+    assert len(cells) == 9
+    assert cells[0] == [0, 1, 5, 6]          # row-major members
+    assert cells[2] == [4, 9]                # right edge: one column
+    assert cells[8] == [24]                  # corner: one member
+
+
+def test_pool_kd1_is_identity_and_large_kd_is_grid_mean():
+    S, g = 2, 4
+    q, k, v, pos, T = _scene(S, g, seed=12)
+    kp, vp, pp = O.kv_pool(k, v, pos, S, T, 1)
+    assert np.array_equal(kp, k) and np.array_equal(vp, v) and np.array_equal(pp, pos)
+    kp, vp, pp = O.kv_pool(k, v, pos, S, T, 9)
+    assert kp.shape[0] == S * 6
+    for s in range(S):
+        fr = slice(s * T, (s + 1) * T)
+        assert np.array_equal(kp[s * 6:s * 6 + 5], k[fr][:5])
+        assert np.allclose(kp[s * 6 + 5], k[fr][5:].mean(axis=0), atol=1e-15)
+        assert np.allclose(vp[s * 6 + 5], v[fr][5:].mean(axis=0), atol=1e-15)
+        assert np.allclose(pp[s * 6 + 5], [(g + 1) / 2, (g + 1) / 2])
+
+
+def test_pool_ceil_mode_edge_cells_and_centres():
+    S, g, kd = 1, 5, 2
+    q, k, v, pos, T = _scene(S, g, seed=13)
+    kp, vp, pp = O.kv_pool(k, v, pos, S, T, kd)
+    assert kp.shape[0] == 5 + 9
+    assert np.array_equal(kp[5 + 8], k[5 + 24])            # corner = the member itself
+    assert np.allclose(kp[5 + 2], (k[5 + 4] + k[5 + 9]) / 2)  # right edge, 2 members
+    assert np.allclose(pp[5 + 0], [1.5, 1.5])
+    assert np.allclose(pp[5 + 2], [1.5, 5.0])
+    assert np.allclose(pp[5 + 8], [5.0, 5.0])
+    # 37x37 with kd=4: cell 0 centre 2.5, last cell a single row at 37
+    _, _, pp = O.kv_pool(np.zeros((1374, 1, 1)), np.zeros((1374, 1, 1)),
+                         np.asarray(_scene(1, 37, H=1)[3]), 1, 1374, 4)
+    assert np.allclose(pp[5], [2.5, 2.5]) and np.allclose(pp[5 + 99], [37.0, 37.0])
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(14)
+    x = rng.normal(scale=10.0, size=20000).astype(np.float32)
+    # exact ties: bf16 value + half an ulp
+    ties = (torch.randn(200).to(torch.bfloat16).to(torch.float32).numpy().view(np.uint32) | 0x8000)
+    x = np.concatenate([x, ties.view(np.float32), np.array([np.inf, -np.inf, 0.0, -0.0], np.float32)])
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.f32_to_bf16_bits(x), want)
+    assert np.isnan(O.bf16_bits_to_f32(O.f32_to_bf16_bits(np.array([np.nan], np.float32))))[0]
+
+
+def test_bf16_widening_is_exact():
+    t = torch.randn(5000).to(torch.bfloat16)
+    assert np.array_equal(_f64(t), t.to(torch.float64).numpy())
+
+
+def _bf16_scene(S, g, H, seed):
+    T = 5 + g * g
+    gen = torch.Generator().manual_seed(seed)
+    k = torch.randn(S * T, H, 64, generator=gen).to(torch.bfloat16)
+    v = torch.randn(S * T, H, 64, generator=gen).to(torch.bfloat16)
+    return k, v, T
+
+
+def test_pool_reference_bits_equal_correctly_rounded_mean_when_sums_are_exact():
+    # multiples of 1/16 in [-8, 8]: every fp32 partial sum is exact, so the
+    # stored value must be the correctly rounded mean.
+    S, g, H, kd = 2, 7, 2, 3
+    T = 5 + g * g
+    gen = torch.Generator().manual_seed(15)
+    k = (torch.randint(-128, 129, (S * T, H, 64), generator=gen).float() / 16).to(torch.bfloat16)
+    v = (torch.randint(-128, 129, (S * T, H, 64), generator=gen).float() / 16).to(torch.bfloat16)
+    pos = np.asarray(_scene(S, g, H=1)[3], dtype=np.float32)
+    kb, vb, pb = O.kv_pool_bf16_reference(_bits(k), _bits(v), pos, S, T, kd)
+    kp, vp, pp = O.kv_pool(_f64(k), _f64(v), pos, S, T, kd)
+    want_k = torch.from_numpy(kp.reshape(kb.shape)).to(torch.float32).to(torch.bfloat16)
+    want_v = torch.from_numpy(vp.reshape(vb.shape)).to(torch.float32).to(torch.bfloat16)
+    assert np.array_equal(kb, _bits(want_k))
+    assert np.array_equal(vb, _bits(want_v))
+    assert np.array_equal(pb, pp.astype(np.float32))
+
+
+def test_pool_reference_sums_members_in_row_major_order():
+    # one 2x2 cell: row-major [2^24, 1, -2^24, 1] sums to 1 in fp32 (2^24 + 1
+    # rounds back to 2^24); column-major order would give 2.
+    S, g, kd, H = 1, 2, 2, 1
+    T = 5 + g * g
+    k = torch.zeros(T, H, 64)
+    k[5, 0, :], k[6, 0, :], k[7, 0, :], k[8, 0, :] = 2.0 ** 24, 1.0, -(2.0 ** 24), 1.0
+    k = k.to(torch.bfloat16)
+    pos = np.asarray(_scene(S, g, H=1)[3], dtype=np.float32)
+    kb, vb, _ = O.kv_pool_bf16_reference(_bits(k), _bits(k), pos, S, T, kd)
+    assert np.all(O.bf16_bits_to_f32(kb[5]) == 0.25)
+    assert np.array_equal(kb[:5], _bits(k)[:5].reshape(5, -1))
+
+
+def test_pool_reference_kd1_is_bit_identity():
+    k, v, T = _bf16_scene(2, 5, 2, 16)
+    pos = np.asarray(_scene(2, 5, H=1)[3], dtype=np.float32)
+    kb, vb, pb = O.kv_pool_bf16_reference(_bits(k), _bits(v), pos, 2, T, 1)
+    assert np.array_equal(kb, _bits(k).reshape(kb.shape))
+    assert np.array_equal(vb, _bits(v).reshape(vb.shape))
+    assert np.array_equal(pb, pos)
