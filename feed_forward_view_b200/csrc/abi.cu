@@ -1,0 +1,244 @@
+// abi.cu -- the extern "C" entry points declared in include/vggt_attn.h.
+//
+// Each call validates every argument on the host (nothing is launched for an
+// invalid call), takes its scratch with cudaMallocAsync on the caller's
+// stream, launches the kernels in stream order and frees the scratch with
+// cudaFreeAsync on the same stream. No call synchronises the stream.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+
+#include <cuda_runtime.h>
+
+#include "vggt_attn.h"
+#include "vggt_internal.h"
+
+namespace {
+
+using vggt::AttnProblem;
+using vggt::PrologueJob;
+
+constexpr long long kDefaultWaitLimit = 1LL << 32;  // SM cycles (~2 s at 2 GHz)
+constexpr int kMaxDevices = 64;
+
+__device__ int g_device_status;  // non-zero once a bounded device wait ran out
+
+struct DeviceState {
+    int* status = nullptr;  // device address of g_device_status
+    long long wait_limit = kDefaultWaitLimit;
+};
+DeviceState g_dev[kMaxDevices];
+
+// State of the current device, with the status word's device address looked
+// up once per device (with that device current).
+DeviceState* device_state() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    DeviceState& st = g_dev[dev];
+    if (!st.status) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        st.status = static_cast<int*>(p);
+    }
+    return &st;
+}
+
+int grid_side(int T) {
+    const int p = T - VGGT_N_SPECIAL;
+    if (p < 0) return -1;
+    int g = static_cast<int>(std::lround(std::sqrt(static_cast<double>(p))));
+    while (g * g > p) --g;
+    while ((g + 1) * (g + 1) <= p) ++g;
+    return g * g == p ? g : -1;
+}
+
+// Every tensor is read or written with 16-byte vector accesses or by TMA,
+// which needs 16-byte aligned global addresses.
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared checks. Returns VGGT_OK to proceed, 1 for an empty problem, or an
+// error status.
+int check_common(const void* q, const void* k, const void* v, const void* pos, const void* out,
+                 int S, int T, int H, int D) {
+    if (S < 0 || T < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    if (grid_side(T) < 0) return VGGT_ERR_SHAPE;
+    if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS) return VGGT_ERR_SHAPE;
+    if (H > 65535) return VGGT_ERR_SHAPE;
+    if (S == 0 || H == 0) return 1;
+    if (!q || !k || !v || !pos || !out) return VGGT_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(pos) || !aligned16(out))
+        return VGGT_ERR_UNSUPPORTED;
+    return VGGT_OK;
+}
+
+size_t head_plane_bytes(long long n_tokens, int H) {
+    return static_cast<size_t>(n_tokens) * H * VGGT_HEAD_DIM * sizeof(uint16_t);
+}
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA; }
+
+// Prologue on (q, pos) and (k, pos_k), then attention; frees the scratch.
+int run_attention(const uint16_t* q, const float* pos, const uint16_t* k, const float* pos_k,
+                  const uint16_t* v, uint16_t* out, int n_seg, int q_len, int k_len, int H,
+                  void* extra_scratch, cudaStream_t stream) {
+    DeviceState* st = device_state();
+    if (!st) {
+        if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
+        return VGGT_ERR_CUDA;
+    }
+    const long long nq = static_cast<long long>(n_seg) * q_len;
+    const long long nk = static_cast<long long>(n_seg) * k_len;
+    void* scratch = nullptr;
+    if (cudaMallocAsync(&scratch, head_plane_bytes(nq, H) + head_plane_bytes(nk, H), stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
+        return VGGT_ERR_ALLOC;
+    }
+    uint16_t* q_hat = static_cast<uint16_t*>(scratch);
+    uint16_t* k_hat = q_hat + head_plane_bytes(nq, H) / sizeof(uint16_t);
+    PrologueJob jq{q, pos, q_hat, static_cast<int>(nq)};
+    PrologueJob jk{k, pos_k, k_hat, static_cast<int>(nk)};
+    int rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
+    if (rc == VGGT_OK) {
+        AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H};
+        rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
+    }
+    cudaFreeAsync(scratch, stream);
+    if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
+    return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vggt_attn_frame(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                    vggt_bf16* out, int S, int T, int H, int D, int kv_down, cudaStream_t stream) {
+    int rc = check_common(q, k, v, pos, out, S, T, H, D);
+    if (rc == VGGT_OK && kv_down != 0 && kv_down != 1) rc = VGGT_ERR_SHAPE;
+    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
+    return run_attention(q, pos, k, pos, v, out, S, T, T, H, nullptr, stream);
+}
+
+int vggt_attn_global(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                     vggt_bf16* out, int S, int T, int H, int D, int kv_down, cudaStream_t stream) {
+    int rc = check_common(q, k, v, pos, out, S, T, H, D);
+    if (rc == VGGT_OK && kv_down != 0 && kv_down != 1) rc = VGGT_ERR_SHAPE;
+    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
+    const int n = S * T;
+    return run_attention(q, pos, k, pos, v, out, 1, n, n, H, nullptr, stream);
+}
+
+int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int N, int H, int D,
+                     cudaStream_t stream) {
+    if (N < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    if (N > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
+    if (N == 0 || H == 0) return VGGT_OK;
+    if (!x || !pos || !x_hat) return VGGT_ERR_NULL;
+    if (!aligned16(x) || !aligned16(pos) || !aligned16(x_hat)) return VGGT_ERR_UNSUPPORTED;
+    PrologueJob j{x, pos, x_hat, N};
+    PrologueJob none{nullptr, nullptr, nullptr, 0};
+    return to_status(vggt::launch_qk_prologue(j, none, H, stream));
+}
+
+int vggt_kv_pool_tokens(int T, int kv_down) {
+    const int g = grid_side(T);
+    if (g < 0 || kv_down < 1) return VGGT_ERR_SHAPE;
+    const int nc = g > 0 ? (g + kv_down - 1) / kv_down : 0;
+    return VGGT_N_SPECIAL + nc * nc;
+}
+
+int vggt_kv_pool(const vggt_bf16* k, const vggt_bf16* v, const float* pos, vggt_bf16* k_out,
+                 vggt_bf16* v_out, float* pos_out, int S, int T, int H, int D, int kv_down,
+                 cudaStream_t stream) {
+    if (S < 0 || T < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    const int g = grid_side(T);
+    if (g < 0 || kv_down < 1) return VGGT_ERR_SHAPE;
+    if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
+    if (S == 0 || H == 0) return VGGT_OK;
+    if (!k || !v || !pos || !k_out || !v_out || !pos_out) return VGGT_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(pos) || !aligned16(k_out) ||
+        !aligned16(v_out) || !aligned16(pos_out))
+        return VGGT_ERR_UNSUPPORTED;
+    return to_status(vggt::launch_kv_pool(k, v, pos, k_out, v_out, pos_out, S, T, g, kv_down, H,
+                                          stream));
+}
+
+int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                         const float* pos, vggt_bf16* out, int S, int T, int H, int D, int kv_down,
+                         cudaStream_t stream) {
+    int rc = check_common(q, k, v, pos, out, S, T, H, D);
+    if (rc == VGGT_OK && kv_down < 1) rc = VGGT_ERR_SHAPE;
+    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
+    const int g = grid_side(T);
+    const int Tk = vggt_kv_pool_tokens(T, kv_down);
+    const long long nk = static_cast<long long>(S) * Tk;
+    // pooled k, pooled v, pooled positions
+    const size_t kv_bytes = head_plane_bytes(nk, H);
+    const size_t pos_bytes = static_cast<size_t>(nk) * 2 * sizeof(float);
+    void* pooled = nullptr;
+    if (cudaMallocAsync(&pooled, 2 * kv_bytes + pos_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_ALLOC;
+    }
+    uint16_t* kp = static_cast<uint16_t*>(pooled);
+    uint16_t* vp = kp + kv_bytes / sizeof(uint16_t);
+    float* pp = reinterpret_cast<float*>(vp + kv_bytes / sizeof(uint16_t));
+    rc = to_status(vggt::launch_kv_pool(k, v, pos, kp, vp, pp, S, T, g, kv_down, H, stream));
+    if (rc != VGGT_OK) {
+        cudaFreeAsync(pooled, stream);
+        return rc;
+    }
+    // Every query row attends to all S*Tk descriptors: one segment.
+    return run_attention(q, pos, kp, pp, vp, out, 1, S * T, static_cast<int>(nk), H, pooled,
+                         stream);
+}
+
+int vggt_get_device_status(cudaStream_t stream) {
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return VGGT_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return VGGT_ERR_CUDA;
+        return VGGT_ERR_TIMEOUT;
+    }
+    return VGGT_OK;
+}
+
+const char* vggt_status_string(int status) {
+    switch (status) {
+        case VGGT_OK: return "VGGT_OK";
+        case VGGT_ERR_NULL: return "VGGT_ERR_NULL: a required pointer is NULL";
+        case VGGT_ERR_UNSUPPORTED: return "VGGT_ERR_UNSUPPORTED: head dimension must be 64";
+        case VGGT_ERR_SHAPE: return "VGGT_ERR_SHAPE: invalid sizes";
+        case VGGT_ERR_ALLOC: return "VGGT_ERR_ALLOC: scratch allocation failed";
+        case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA: CUDA call or launch failed";
+        case VGGT_ERR_TIMEOUT: return "VGGT_ERR_TIMEOUT: a bounded device wait ran out";
+        default: return "unknown vggt_status";
+    }
+}
+
+long long vggt_set_wait_limit(long long cycles) {
+    DeviceState* st = device_state();
+    if (!st) return -1;
+    const long long prev = st->wait_limit;
+    st->wait_limit = cycles < 1 ? kDefaultWaitLimit : cycles;
+    return prev;
+}
+
+int vggt_debug_wait_timeout(cudaStream_t stream) {
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    return to_status(vggt::launch_wait_probe(st->status, st->wait_limit, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// vggt_internal.h -- host-side launchers shared by the C ABI (abi.cu) and the
+// kernel translation units. Not part of the public interface.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime_api.h>
+
+namespace vggt {
+
+constexpr int kNSpecial = 5;
+constexpr int kHeadDim = 64;
+
+// One tensor to normalise and rotate: x [n, H, 64] token-major in, x_hat
+// [H, n, 64] head-major out, positions pos [n, 2] (row, col).
+struct PrologueJob {
+    const uint16_t* x;
+    const float* pos;
+    uint16_t* x_hat;
+    int n;
+};
+
+// LayerNorm (eps 1e-5, no affine) + 2D RoPE (base 100) over one or two jobs in
+// a single launch. Returns the launch's cudaError_t.
+cudaError_t launch_qk_prologue(const PrologueJob& a, const PrologueJob& b, int H,
+                               cudaStream_t stream);
+
+// Ceil-mode kd x kd average pooling of the patch grid of every frame, special
+// tokens copied. k,v [S*T, H, 64] -> [S*Tk, H, 64]; pos [S*T,2] -> [S*Tk,2].
+cudaError_t launch_kv_pool(const uint16_t* k, const uint16_t* v, const float* pos,
+                           uint16_t* k_out, uint16_t* v_out, float* pos_out,
+                           int S, int T, int g, int kd, int H, cudaStream_t stream);
+
+// Attention over segments: segment s has queries rows [s*q_len, (s+1)*q_len)
+// of q_hat and keys rows [s*k_len, (s+1)*k_len) of k_hat / v.
+//   q_hat [H, n_seg*q_len, 64] and k_hat [H, n_seg*k_len, 64] head-major,
+//   v [n_seg*k_len, H, 64] and out [n_seg*q_len, H, 64] token-major.
+struct AttnProblem {
+    const uint16_t* q_hat;
+    const uint16_t* k_hat;
+    const uint16_t* v;
+    uint16_t* out;
+    int n_seg;
+    int q_len;
+    int k_len;
+    int H;
+};
+
+// Returns cudaSuccess, or an error from tensor-map encoding or the launch.
+cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_limit,
+                             cudaStream_t stream);
+
+// A one-thread kernel that waits on a barrier nothing completes.
+cudaError_t launch_wait_probe(int* status, long long wait_limit, cudaStream_t stream);
+
+}  // namespace vggt

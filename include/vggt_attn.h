@@ -1,0 +1,168 @@
+/*
+ * vggt_attn.h -- C ABI of libvggt_attn.so: the attention core of the VGGT
+ * aggregator (frame, global and compressed-descriptor attention, each with a
+ * fused per-head QK LayerNorm + 2D RoPE prologue) for NVIDIA B200 (sm_100a).
+ *
+ * Operation (all variants, per head h):
+ *   q_hat = RoPE2D(LayerNorm(q), pos),  k_hat = RoPE2D(LayerNorm(k), pos_k)
+ *   out_i = sum_j softmax_j(q_hat_i . k_hat_j / sqrt(D)) v_j
+ * - LayerNorm over the D = 64 dims of one head, centered, biased variance,
+ *   eps = 1e-5, no scale/shift ("Norm: Layer Normalization" slide of the VGGT
+ *   paper-report deck; layer_norm_eps 1e-05 in the VGGT-Omega config.json
+ *   field table).
+ * - 2D RoPE, base 100 (rope_base 100.0, VGGT-Omega config.json field table):
+ *   dims 0-31 turn by the row position, dims 32-63 by the column position;
+ *   inside each half, dim j pairs with dim j+16 and turns by
+ *   pos * 100^(-2j/32) (frequency schedule of the sinusoidal formula on the
+ *   deck's "Positional Encoding (4/6)" slide).
+ * - softmax(Q K^T / sqrt(d_k)) V: deck, Section V "Attention" slides.
+ *
+ * Data layout (every pointer is DEVICE memory owned by the caller):
+ *   q, k, v, out : [S, T, H, D] bf16 (raw uint16 bits), contiguous, token-major
+ *                  with heads interleaved -- the [B, N, H, D] layout of the
+ *                  vggt-jax README attention table.
+ *   pos          : [S, T, 2] fp32 (row, col). VGGT places the five special
+ *                  tokens (camera + 4 registers) at (0, 0) and patch (r, c) at
+ *                  (r + 1, c + 1); the library uses whatever pos holds.
+ *   Each frame holds T = 5 + g*g tokens: the 5 special tokens first, then the
+ *   g x g patch grid row-major. Only the descriptor pooling depends on this
+ *   order; frame and global attention use pos alone.
+ *
+ * Common rules:
+ *   - D must be 64 (VGGT: 16 heads x 64 dims). H >= 1 is free.
+ *   - Every pointer must be 16-byte aligned (TMA and 16-byte vector access).
+ *   - S == 0 or H == 0 is an empty problem: VGGT_OK, nothing is launched.
+ *   - Everything is asynchronous on `stream`; no call synchronises it.
+ *   - Scratch (normalised q/k, pooled k/v) is taken with cudaMallocAsync and
+ *     released with cudaFreeAsync on `stream`.
+ *   - Outputs must not overlap inputs.
+ *   - Every argument is checked on the host before any launch; an invalid call
+ *     returns a negative vggt_status and launches nothing.
+ *   - No call traps on the device. Device-side waits are bounded; a wait that
+ *     runs out sets a device status word that vggt_get_device_status() reads.
+ */
+#ifndef VGGT_ATTN_H
+#define VGGT_ATTN_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define VGGT_API __attribute__((visibility("default")))
+#else
+#define VGGT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t vggt_bf16; /* raw bf16 bits */
+
+typedef enum vggt_status {
+    VGGT_OK = 0,
+    VGGT_ERR_NULL = -1,        /* a required pointer is NULL                      */
+    VGGT_ERR_UNSUPPORTED = -2, /* D != 64, or a pointer not 16-byte aligned        */
+    VGGT_ERR_SHAPE = -3,       /* negative sizes, T != 5 + g*g, bad kv_down, or a
+                                  size beyond the library's limits                */
+    VGGT_ERR_ALLOC = -4,       /* scratch allocation failed                        */
+    VGGT_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed             */
+    VGGT_ERR_TIMEOUT = -6      /* a bounded device-side wait ran out (reported by
+                                  vggt_get_device_status)                          */
+} vggt_status;
+
+/* Number of special (camera + register) tokens at the head of every frame. */
+#define VGGT_N_SPECIAL 5
+/* Head dimension the kernels are built for. */
+#define VGGT_HEAD_DIM 64
+/* Largest S*T (or S*T_k) accepted: keeps every row index inside int32 and
+   every tensor below 2^31 elements of one head-major scratch plane. */
+#define VGGT_MAX_TOKENS (1 << 21)
+
+/*
+ * Frame attention: every token attends only to the T tokens of its own frame
+ * ("Frame Attention" panel, "Global + Frame Attention" architecture slide).
+ * kv_down must be 0 or 1. Writes out[S, T, H, D].
+ */
+VGGT_API int vggt_attn_frame(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                    const float* pos, vggt_bf16* out,
+                    int S, int T, int H, int D, int kv_down, cudaStream_t stream);
+
+/*
+ * Global attention: all S*T tokens attend to all S*T tokens ("Global
+ * Attention" panel of the same slide; vggt-jax README global shape
+ * [1, 1860, 16, 64]). kv_down must be 0 or 1. Writes out[S, T, H, D].
+ */
+VGGT_API int vggt_attn_global(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                     const float* pos, vggt_bf16* out,
+                     int S, int T, int H, int D, int kv_down, cudaStream_t stream);
+
+/*
+ * Compressed-descriptor attention (FlashVGGT README, Overview; --kv_downfactor,
+ * default 4): K/V are first pooled per frame as vggt_kv_pool does, then every
+ * query of every frame attends to all S frames' descriptors (S * T_k keys).
+ * The pooled keys get the prologue at their pooled positions; pooled values
+ * are used as stored. kv_down >= 1 (kv_down == 1 is dense global attention).
+ * Writes out[S, T, H, D].
+ */
+VGGT_API int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                         const float* pos, vggt_bf16* out,
+                         int S, int T, int H, int D, int kv_down, cudaStream_t stream);
+
+/*
+ * The QK prologue on its own: for every token t < N and head h < H,
+ *   x_hat[h, t, :] = RoPE2D(LayerNorm(x[t, h, :]), pos[t])
+ * with the LayerNorm and rotary embedding defined at the top of this header.
+ * x [N, H, D] bf16 token-major in; x_hat [H, N, D] bf16 head-major out (the
+ * layout the attention kernel reads); pos [N, 2] fp32. The attention entry
+ * points run this step internally; it is exported for users who need the
+ * normalised, rotated vectors themselves. N == 0 or H == 0 is a no-op.
+ */
+VGGT_API int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat,
+                              int N, int H, int D, cudaStream_t stream);
+
+/*
+ * Per-frame K/V descriptors (FlashVGGT README: "spatially resampling keys and
+ * values"; the grid is g x g with g = sqrt(T - 5)):
+ *   - the 5 special tokens of each frame are copied unchanged;
+ *   - the grid is cut into ceil(g/kv_down)^2 cells of up to kv_down x kv_down
+ *     patches (edge cells keep only the patches inside the grid); each cell
+ *     becomes one token whose K and V are, per channel, the float32 sum of its
+ *     members in row-major order divided in float32 by the member count and
+ *     rounded to bf16 (nearest, ties to even); its position is the same
+ *     float32 mean of the members' positions.
+ * Outputs: k_out, v_out [S, T_k, H, D] bf16, pos_out [S, T_k, 2] fp32 with
+ * T_k = vggt_kv_pool_tokens(T, kv_down). kv_down >= 1.
+ */
+VGGT_API int vggt_kv_pool(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                 vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out,
+                 int S, int T, int H, int D, int kv_down, cudaStream_t stream);
+
+/* Tokens per frame after pooling (5 + ceil(g/kv_down)^2), or a negative
+   vggt_status when T is not 5 + g*g or kv_down < 1. Host only. */
+VGGT_API int vggt_kv_pool_tokens(int T, int kv_down);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+   the current device: VGGT_OK, or VGGT_ERR_TIMEOUT when a bounded device wait
+   ran out since the last call; VGGT_ERR_CUDA if the synchronisation failed. */
+VGGT_API int vggt_get_device_status(cudaStream_t stream);
+
+/* Human-readable name of a vggt_status value (static storage). */
+VGGT_API const char* vggt_status_string(int status);
+
+/* Upper bound, in SM clock cycles, of every device-side wait in the library's
+   kernels (default about 2^32 cycles, roughly two seconds). Values < 1 restore
+   the default. Returns the previous limit. Applies to launches made after the
+   call on the current device. */
+VGGT_API long long vggt_set_wait_limit(long long cycles);
+
+/* Launches one block that waits, with the current limit, on a barrier that
+   nothing ever completes, then records VGGT_ERR_TIMEOUT in the status word.
+   It exercises the timeout path without any risk to the device. */
+VGGT_API int vggt_debug_wait_timeout(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VGGT_ATTN_H */

@@ -1,0 +1,109 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+exactly what include/vggt_attn.h declares, and rejects invalid arguments
+before touching the device."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import feed_forward_view_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vggt_attn.h")
+
+OK, E_NULL, E_UNSUP, E_SHAPE = 0, -1, -2, -3
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"VGGT_API\s+[\w\s\*]+?\b(vggt_\w+)\s*\(", src))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == set(F.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol_and_nothing_else():
+    out = subprocess.run(["nm", "-D", "--defined-only", F.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    text_syms = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert declared_functions() <= text_syms
+    assert all(s.startswith("vggt_") for s in text_syms), text_syms
+    for name in declared_functions():
+        assert hasattr(F.lib, name)
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert F.vggt_status_string(code).startswith("VGGT_")
+    assert "unknown" in F.vggt_status_string(7)
+
+
+def test_pool_token_counts():
+    assert F.vggt_kv_pool_tokens(1374, 4) == 105
+    assert F.vggt_kv_pool_tokens(1374, 1) == 1374
+    assert F.vggt_kv_pool_tokens(4101, 4) == 5 + 16 * 16
+    assert F.vggt_kv_pool_tokens(261, 3) == 5 + 36
+    assert F.vggt_kv_pool_tokens(5, 4) == 5
+    assert F.vggt_kv_pool_tokens(930, 4) == E_SHAPE  # 25x37 is not square
+    assert F.vggt_kv_pool_tokens(1374, 0) == E_SHAPE
+    assert F.vggt_kv_pool_tokens(4, 1) == E_SHAPE
+
+
+ATTN = ("vggt_attn_frame", "vggt_attn_global", "vggt_attn_descriptor")
+FAKE = 0x1000  # never dereferenced: every case below fails validation first
+
+
+@pytest.mark.parametrize("name", ATTN)
+def test_attention_argument_checks(name):
+    fn = getattr(F.lib, name)
+    kd = 4 if name == "vggt_attn_descriptor" else 1
+    p = [FAKE] * 5
+    assert fn(*p, 2, 261, 16, 32, kd, None) == E_UNSUP
+    assert fn(*p, 2, 262, 16, 64, kd, None) == E_SHAPE      # T - 5 not a square
+    assert fn(*p, 2, 4, 16, 64, kd, None) == E_SHAPE        # fewer than 5 tokens
+    assert fn(*p, -1, 261, 16, 64, kd, None) == E_SHAPE
+    assert fn(*p, 2, 261, -1, 64, kd, None) == E_SHAPE
+    assert fn(*p, 1 << 20, 261, 16, 64, kd, None) == E_SHAPE  # beyond VGGT_MAX_TOKENS
+    for i in range(5):
+        q = list(p)
+        q[i] = None
+        assert fn(*q, 2, 261, 16, 64, kd, None) == E_NULL
+    for i in range(5):
+        q = list(p)
+        q[i] = FAKE + 8  # not 16-byte aligned
+        assert fn(*q, 2, 261, 16, 64, kd, None) == E_UNSUP
+    # empty problems succeed without touching any pointer
+    assert fn(None, None, None, None, None, 0, 261, 16, 64, kd, None) == OK
+    assert fn(None, None, None, None, None, 3, 261, 0, 64, kd, None) == OK
+
+
+def test_kv_down_rules():
+    p = [FAKE] * 5
+    assert F.lib.vggt_attn_frame(*p, 2, 261, 16, 64, 2, None) == E_SHAPE
+    assert F.lib.vggt_attn_global(*p, 2, 261, 16, 64, 4, None) == E_SHAPE
+    assert F.lib.vggt_attn_descriptor(*p, 2, 261, 16, 64, 0, None) == E_SHAPE
+
+
+def test_pool_and_prologue_argument_checks():
+    p6 = [FAKE] * 6
+    assert F.lib.vggt_kv_pool(*p6, 2, 261, 16, 32, 4, None) == E_UNSUP
+    assert F.lib.vggt_kv_pool(*p6, 2, 262, 16, 64, 4, None) == E_SHAPE
+    assert F.lib.vggt_kv_pool(*p6, 2, 261, 16, 64, 0, None) == E_SHAPE
+    assert F.lib.vggt_kv_pool(None, *p6[1:], 2, 261, 16, 64, 4, None) == E_NULL
+    assert F.lib.vggt_kv_pool(None, None, None, None, None, None, 0, 261, 16, 64, 4, None) == OK
+    assert F.lib.vggt_qk_prologue(FAKE, FAKE, FAKE, 10, 16, 48, None) == E_UNSUP
+    assert F.lib.vggt_qk_prologue(FAKE, FAKE, FAKE, -1, 16, 64, None) == E_SHAPE
+    assert F.lib.vggt_qk_prologue(FAKE, None, FAKE, 10, 16, 64, None) == E_NULL
+    assert F.lib.vggt_qk_prologue(None, None, None, 0, 16, 64, None) == OK
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+
+    q = torch.zeros(261 * 2, 16, 64, dtype=torch.bfloat16)
+    pos = torch.zeros(261 * 2, 2)
+    with pytest.raises(ValueError):
+        F.vggt_attn_global(q, q, q, pos, q.clone(), S=2, T=261)

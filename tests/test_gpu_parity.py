@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle on
+the same seeded inputs.
+
+Bars (fixed by the method's statement of the target):
+* attention outputs: max-abs error <= 2e-2 and relative Frobenius error
+  <= 5e-3 against the oracle, over every compared row;
+* pooled K/V: bit-exact against the oracle's bf16 form of the float32 mean;
+  pooled positions: exact;
+* prologue: within one bf16 rounding of the exact value (2^-8 relative) plus a
+  small absolute allowance for float32 arithmetic.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vggt_oracle as O
+from feed_forward_view_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_FRO = 5e-3
+
+
+@pytest.fixture(scope="module")
+def F():
+    import feed_forward_view_b200 as F
+
+    return F
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return O.bf16_bits_to_f64(bits(t)).reshape(t.shape)
+
+
+def errors(got: np.ndarray, ref: np.ndarray):
+    d = got - ref
+    return float(np.abs(d).max()), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30))
+
+
+def oracle_rows(kind, q, k, v, pos, S, T, kd, rows):
+    qn, kn, vn, pn = f64(q), f64(k), f64(v), pos.numpy().astype(np.float64)
+    if kind == "global":
+        return O.attn_global(qn, kn, vn, pn, S, T, rows=rows)
+    if kind == "frame":
+        return O.attn_frame(qn, kn, vn, pn, S, T, rows=rows)
+    return O.attn_descriptor(qn, kn, vn, pn, S, T, kd, rows=rows)
+
+
+def run_gpu(F, kind, q, k, v, pos, S, T, kd, stream=None):
+    dev = torch.device("cuda:0")
+    qd, kd_, vd, pd = (t.to(dev) for t in (q, k, v, pos))
+    out = torch.empty_like(qd)
+    fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
+          "descriptor": F.vggt_attn_descriptor}[kind]
+    fn(qd, kd_, vd, pd, out, S=S, T=T, kv_down=kd, stream=stream)
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    return out.cpu()
+
+
+def check_attention(F, kind, S, g, kd, seed, rows=None):
+    q, k, v, pos = synth.make_qkv(S, g, seed)
+    T = 5 + g * g
+    out = run_gpu(F, kind, q, k, v, pos, S, T, kd)
+    rows = np.arange(S * T) if rows is None else np.asarray(rows)
+    ref = oracle_rows(kind, q, k, v, pos, S, T, kd, rows)
+    got = f64(out)[rows]
+    mx, rf = errors(got, ref)
+    assert np.isfinite(got).all()
+    assert mx <= MAX_ABS and rf <= REL_FRO, (kind, S, g, kd, mx, rf)
+    return mx, rf
+
+
+# ------------------------------------------------------------------ prologue
+
+
+@pytest.mark.parametrize("S,g,H", [(2, 22, 16), (1, 0, 3), (3, 7, 5)])
+def test_prologue_matches_oracle(F, S, g, H):
+    x, _, _, pos = synth.make_qkv(S, g, seed=5, H=H)
+    xh = F.vggt_qk_prologue(x.cuda(), pos.cuda(), H=H)
+    torch.cuda.synchronize()
+    ref = O.qk_prologue(f64(x), pos.numpy().astype(np.float64)).transpose(1, 0, 2)
+    got = f64(xh.cpu())
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4)
+
+
+def test_prologue_large_positions(F):
+    # 64x64 grid: angles up to 64 rad
+    x, _, _, pos = synth.make_qkv(1, 64, seed=6)
+    xh = F.vggt_qk_prologue(x.cuda(), pos.cuda())
+    torch.cuda.synchronize()
+    ref = O.qk_prologue(f64(x), pos.numpy().astype(np.float64)).transpose(1, 0, 2)
+    got = f64(xh.cpu())
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4)
+
+
+# ------------------------------------------------------------------ pooling
+
+
+@pytest.mark.parametrize("S,g,kd", [(2, 37, 4), (3, 5, 2), (2, 6, 1), (2, 7, 9), (1, 0, 4), (4, 16, 3)])
+def test_kv_pool_bit_exact(F, S, g, kd):
+    _, k, v, pos = synth.make_qkv(S, g, seed=7)
+    T = 5 + g * g
+    ko, vo, po = F.vggt_kv_pool(k.cuda(), v.cuda(), pos.cuda(), S=S, T=T, kv_down=kd)
+    torch.cuda.synchronize()
+    kb, vb, pb = O.kv_pool_bf16_reference(bits(k), bits(v), pos.numpy(), S, T, kd)
+    assert np.array_equal(bits(ko).reshape(kb.shape), kb)
+    assert np.array_equal(bits(vo).reshape(vb.shape), vb)
+    assert np.array_equal(po.cpu().numpy(), pb)
+
+
+def test_kv_pool_sums_in_row_major_order(F):
+    S, g, kd, H = 1, 2, 2, 16
+    T = 5 + g * g
+    k = torch.zeros(T, H, 64)
+    k[5], k[6], k[7], k[8] = 2.0 ** 24, 1.0, -(2.0 ** 24), 1.0
+    k = k.to(torch.bfloat16)
+    pos = synth.grid_positions(S, g)
+    ko, _, _ = F.vggt_kv_pool(k.cuda(), k.cuda(), pos.cuda(), S=S, T=T, kv_down=kd)
+    torch.cuda.synchronize()
+    assert torch.all(ko[5].float().cpu() == 0.25)
+
+
+# ------------------------------------------------------------------ attention
+
+SMALL = [
+    ("global", 2, 16, 1),      # 522 tokens: 4 full tiles + 10-row tail
+    ("frame", 3, 20, 1),       # 405 tokens per frame: 3 tiles + 21-row tail
+    ("frame", 2, 11, 1),       # 126 tokens per frame: one partial tile
+    ("global", 1, 15, 1),      # 230 tokens: an odd pair with a partial second tile
+    ("global", 1, 0, 1),       # 5 special tokens only
+    ("global", 2, 1, 1),       # 6 tokens per frame
+    ("descriptor", 4, 37, 4),  # 420 pooled keys
+    ("descriptor", 3, 9, 3),   # 3x3 cells
+    ("descriptor", 2, 10, 1),  # kv_down 1 == dense global
+    ("descriptor", 2, 7, 9),   # one cell per frame
+]
+
+
+@pytest.mark.parametrize("kind,S,g,kd", SMALL)
+def test_attention_small_full(F, kind, S, g, kd):
+    check_attention(F, kind, S, g, kd, seed=11)
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_attention_full_workloads(F, name):
+    w = synth.WORKLOADS[name]
+    n = w.n_q
+    rows = None if n <= 12000 and w.kind == "frame" or n <= 600 else synth.sample_rows(n, 384, seed=3).numpy()
+    check_attention(F, w.kind, w.S, w.g, w.kv_down, seed=1, rows=rows)
+
+
+def test_descriptor_kd1_equals_global_on_gpu(F):
+    q, k, v, pos = synth.make_qkv(2, 12, seed=13)
+    T = 5 + 144
+    a = run_gpu(F, "descriptor", q, k, v, pos, 2, T, 1)
+    b = run_gpu(F, "global", q, k, v, pos, 2, T, 1)
+    mx, rf = errors(a.double().numpy(), b.double().numpy())
+    assert mx <= 1e-2 and rf <= 2e-3
+
+
+def test_zero_queries_average_values(F):
+    # q = 0 -> every score is 0 -> out = mean of the visible V rows.
+    S, g = 2, 12
+    q, k, v, pos = synth.make_qkv(S, g, seed=14)
+    T = 5 + g * g
+    q.zero_()
+    out = f64(run_gpu(F, "frame", q, k, v, pos, S, T, 1))
+    vv = f64(v)
+    for s in range(S):
+        want = vv[s * T:(s + 1) * T].mean(axis=0)
+        assert np.abs(out[s * T:(s + 1) * T] - want).max() < 4e-3
+
+
+def test_output_guard_regions_untouched(F):
+    S, g = 2, 16
+    q, k, v, pos = synth.make_qkv(S, g, seed=15)
+    T = 5 + g * g
+    n = S * T * 16 * 64
+    G = 4096
+    buf = torch.full((n + 2 * G,), -7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[G:G + n].view(S * T, 16, 64)
+    F.vggt_attn_global(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), out, S=S, T=T)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:G] == -7.0) and torch.all(buf[G + n:] == -7.0)
+    assert torch.isfinite(out).all()
+
+
+def test_repeatable_and_stream_ordered(F):
+    S, g = 3, 20
+    q, k, v, pos = synth.make_qkv(S, g, seed=16)
+    T = 5 + g * g
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = run_gpu(F, "frame", q, k, v, pos, S, T, 1, stream=s)
+        b = run_gpu(F, "frame", q, k, v, pos, S, T, 1, stream=s)
+    assert torch.equal(a, b)
+
+
+def test_empty_problem_is_a_no_op(F):
+    q = torch.zeros(0, 16, 64, dtype=torch.bfloat16, device="cuda")
+    pos = torch.zeros(0, 2, device="cuda")
+    out = torch.zeros(0, 16, 64, dtype=torch.bfloat16, device="cuda")
+    F.vggt_attn_global(q, q, q, pos, out, S=0, T=261)
+    assert F.vggt_get_device_status() == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(F):
+    prev = F.vggt_set_wait_limit(200_000)
+    try:
+        F.vggt_debug_wait_timeout()
+        assert F.vggt_get_device_status() == -6
+        assert F.vggt_get_device_status() == 0  # cleared by the read
+    finally:
+        F.vggt_set_wait_limit(prev)
+    check_attention(F, "global", 1, 15, 1, seed=17)
