@@ -1,0 +1,455 @@
+"""Benchmark of the VGGT attention path on B200.
+
+Default workload: dense global attention over 9 frames of 1024x1024 at patch
+16 (64x64 patches + 5 special tokens = 4101 tokens/frame, 36 909 tokens,
+16 heads x 64 dims). One step = one ``vggt_attn_global`` call through the C
+ABI (QK LayerNorm + 2D RoPE prologue, then the tcgen05 attention kernel) on
+inputs already resident in HBM. ``value`` = algorithmic attention FLOPs
+(4*H*D per query-key pair) / device time, summed over all ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+
+Multi-GPU (``torchrun``): every rank runs an independent replica of the
+workload (the path has no data exchange); the job's time is the max over
+ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "global-attention fwd TFLOP/s and tokens/s on 1 B200; % of dense bf16 peak"
+DEFAULT_WORKLOAD = "global_s9_g64"
+L2_BYTES = 126 * 1024 * 1024
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_kernel_global_s6_g64.txt")
+KERNEL_SOURCES = ("feed_forward_view_b200/csrc/attn_fwd.cu", "feed_forward_view_b200/csrc/sm100.cuh")
+
+
+# ----------------------------------------------------------------------------- helpers
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(w):
+    """DRAM bytes per attention launch for workload ``w``, from the committed
+    ncu summary of a smaller dense-global case scaled by the token count
+    (every byte the kernel moves -- q_hat, k_hat, v in, out -- grows linearly
+    with the tokens while one head's keys fit in L2), or None when the summary
+    is missing, covers another kind, or was taken on different kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY) or w.kind != "global":
+        return None
+    fields = {}
+    for line in open(PROFILE_SUMMARY):
+        if ":" in line and not line.startswith("#"):
+            k, _, v = line.partition(":")
+            fields[k.strip()] = v.strip().split()[0] if v.strip() else ""
+    if fields.get("source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"]) * w.n_q / float(fields["tokens"])
+    except (KeyError, ValueError, ZeroDivisionError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, cmax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            sm.append(clk)
+            mx = cmax
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [c for c in sm if c > 0.5 * max(sm)]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if n_gpus > 0 else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, local, world
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar across ranks (identity at world size 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+
+class OracleLeg:
+    """The fp64 oracle, as it stands, on a sample of query rows of workload
+    ``w``. Setup (widening the inputs, the keys' prologue and pooling: a fixed
+    O(N_k) cost that a full run amortises) happens once, untimed; ``run``
+    times ``n_rows`` query rows against all keys, all heads."""
+
+    def __init__(self, w, seed: int = 0):
+        import numpy as np
+        import torch
+
+        from feed_forward_view_b200 import synth
+        from oracle import vggt_oracle as O
+
+        self.w, self.O, self.synth = w, O, synth
+        q, k, v, pos = synth.make_workload(w, seed)
+
+        def f64(t):
+            return O.bf16_bits_to_f64(t.contiguous().view(torch.int16).numpy().view(np.uint16)).reshape(t.shape)
+
+        self.q, self.k, self.v, self.pos = f64(q), f64(k), f64(v), pos.numpy().astype(np.float64)
+        if w.kind == "descriptor":
+            kp, vp, pp = O.kv_pool(self.k, self.v, self.pos, w.S, w.T, w.kv_down)
+            self.k_hat, self.vv = O.qk_prologue(kp, pp), vp
+        elif w.kind == "global":
+            self.k_hat, self.vv = O.qk_prologue(self.k, self.pos), self.v
+
+    def run(self, n_rows: int, seed: int = 0):
+        """Returns (TFLOP/s, seconds, rows)."""
+        w, O = self.w, self.O
+        rows = self.synth.sample_rows(w.n_q, n_rows, seed).numpy()
+        t0 = time.perf_counter()
+        if w.kind == "frame":
+            O.attn_frame(self.q, self.k, self.v, self.pos, w.S, w.T, rows=rows)
+            keys = w.T
+        else:
+            O.cross_attention(O.qk_prologue(self.q[rows], self.pos[rows]), self.k_hat, self.vv)
+            keys = w.n_k
+        dt = time.perf_counter() - t0
+        return 4.0 * w.H * w.D * rows.size * keys / dt / 1e12, dt, int(rows.size)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, bounded sample per step."""
+    from feed_forward_view_b200 import synth
+
+    rank, _, world = int(os.environ.get("RANK", "0")), 0, int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    w = synth.ALL_WORKLOADS[args.workload]
+    leg = OracleLeg(w)
+    # size each step from a short calibration so the whole run stays bounded
+    _, dt, rows = leg.run(32)
+    per_row = dt / rows
+    budget = args.reference_budget_s / max(1, args.steps + args.warmup)
+    n_rows = int(min(4096, max(8, budget / per_row)))
+    for i in range(args.warmup):
+        leg.run(n_rows, seed=i)
+    vals, times = [], []
+    for i in range(args.steps):
+        tf, dt, rows = leg.run(n_rows, seed=100 + i)
+        vals.append(tf)
+        times.append(dt)
+    threads = blas_threads()
+    value = statistics.median(vals)
+    sample = (f"{rows} query rows x all {w.n_k if w.kind != 'frame' else w.T} keys x {w.H} heads per step "
+              f"(of {w.n_q} rows), key prologue precomputed")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
+                   "keys": w.n_k if w.kind != "frame" else w.T, "H": w.H, "D": w.D,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+
+def run_gpu(args):
+    import torch
+
+    import feed_forward_view_b200 as F
+    from feed_forward_view_b200 import synth
+
+    rank, local, world = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.ALL_WORKLOADS[args.workload]
+    fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
+          "descriptor": F.vggt_attn_descriptor}[w.kind]
+
+    q_h, k_h, v_h, pos_h = synth.make_workload(w, seed=rank)
+    q, k, v, pos = (t.to(dev) for t in (q_h, k_h, v_h, pos_h))
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, pos))
+
+    def step():
+        fn(q, k, v, pos, out, S=w.S, T=w.T, kv_down=w.kv_down)
+
+    # ---- warm-up, then the timed region: K steps between two barriers
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if F.vggt_get_device_status() != 0:
+        raise RuntimeError("device wait timeout during warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    clocks.stop()
+    ms_local = e0.elapsed_time(e1)
+    status = F.vggt_get_device_status()
+    ms_total = max_over_ranks(ms_local, world, dev)
+    launches = 2 + (1 if w.kind == "descriptor" else 0)  # prologue + attention (+ pool)
+    ms_step = ms_total / args.steps
+    flops = w.flops()
+    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+    tokens_s = world * w.n_q * args.steps / (ms_total * 1e-3)
+
+    # ---- kernel-only timings (same kernels, launched one by one with events)
+    H = w.H
+    q_hat = torch.empty((H, w.n_q, 64), dtype=torch.bfloat16, device=dev)
+    k_hat = torch.empty((H, w.n_k, 64), dtype=torch.bfloat16, device=dev)
+    if w.kind == "descriptor":
+        kp, vp, pp = F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down)
+        F.vggt_qk_prologue(kp, pp, k_hat)
+        v_use = vp
+    else:
+        F.vggt_qk_prologue(k, pos, k_hat)
+        v_use = v
+    F.vggt_qk_prologue(q, pos, q_hat)
+    n_seg, q_len, k_len = (w.S, w.T, w.T) if w.kind == "frame" else (1, w.n_q, w.n_k)
+    reps = max(5, min(args.steps, 50))
+    for _ in range(3):
+        F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
+    torch.cuda.synchronize(dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(reps):
+        F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    attn_ms = a0.elapsed_time(a1) / reps
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(reps):
+        F.vggt_qk_prologue(q, pos, q_hat)
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    pro_ms = p0.elapsed_time(p1) / reps
+    pro_bytes = 2 * w.n_q * H * 64 * 2 + w.n_q * 8  # read x + pos, write x_hat
+
+    # ---- end to end through the public call with host buffers
+    e2e = None
+    if not args.skip_e2e:
+        hq, hk, hv, hp = (t.pin_memory() for t in (q_h, k_h, v_h, pos_h))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dk, dv, dp = (torch.empty_like(t) for t in (q, k, v, pos))
+        dout = torch.empty_like(out)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dp.copy_(hp, non_blocking=True)
+            fn(dq, dk, dv, dp, dout, S=w.S, T=w.T, kv_down=w.kv_down)
+            hout.copy_(dout, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 30))
+        barrier(world, dev)
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        x1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, dev) / n_e2e
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size(),
+               "ms_per_step": e2e_ms}
+
+    status2 = F.vggt_get_device_status()
+
+    # ---- CPU oracle baseline (rank 0 at N = 1 only)
+    cpu = None
+    if world == 1 and not args.skip_cpu:
+        tf, dt, rows = OracleLeg(w).run(args.cpu_rows)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{rows} of {w.n_q} query rows x all keys x {w.H} heads, fp64 numpy, "
+                         f"{dt:.1f} s; key prologue precomputed"}
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        attn_tf = flops / (attn_ms * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        traffic = profiled_traffic(w)
+        clk = clocks.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
+                       "keys": w.n_k if w.kind != "frame" else w.T, "H": w.H, "D": w.D,
+                       "kv_down": w.kv_down, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs {in_bytes / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
+            "tokens_per_s": tokens_s,
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tf,
+                         "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
+                         "peak_source": f"{peak_src} bf16 burst",
+                         "frac_of_sustained": attn_tf / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "traffic": traffic, "kernel_ms": attn_ms,
+                         "share_of_step": attn_ms / ms_step},
+            "kernels": {"qk_prologue": {"ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
+                                        "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"])}},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches * args.steps,
+            "clocks": clk,
+            "device_status": status or status2,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-rows", type=int, default=768)
+    ap.add_argument("--reference-budget-s", type=float, default=150.0)
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle leg")
+    ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
+    args = ap.parse_args(argv)
+    if args.impl == "native":
+        args.warmup = max(args.warmup, 3)  # at least three untimed steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

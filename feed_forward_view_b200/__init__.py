@@ -26,6 +26,7 @@ __all__ = [
     "vggt_kv_pool",
     "vggt_kv_pool_tokens",
     "vggt_qk_prologue",
+    "vggt_attn_core",
     "vggt_get_device_status",
     "vggt_status_string",
     "vggt_set_wait_limit",
@@ -36,6 +37,7 @@ __all__ = [
 # every symbol include/vggt_attn.h declares
 EXPORTED_SYMBOLS = (
     "vggt_qk_prologue",
+    "vggt_attn_core",
     "vggt_attn_frame",
     "vggt_attn_global",
     "vggt_attn_descriptor",
@@ -64,6 +66,8 @@ lib.vggt_kv_pool.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.vggt_kv_pool.restype = _i
 lib.vggt_qk_prologue.argtypes = [_p, _p, _p, _i, _i, _i, _p]
 lib.vggt_qk_prologue.restype = _i
+lib.vggt_attn_core.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+lib.vggt_attn_core.restype = _i
 lib.vggt_kv_pool_tokens.argtypes = [_i, _i]
 lib.vggt_kv_pool_tokens.restype = _i
 lib.vggt_get_device_status.argtypes = [_p]
@@ -150,6 +154,15 @@ def vggt_qk_prologue(x, pos, x_hat=None, N=None, H=16, D=64, stream=None):
                               _stream(stream))
     _check(rc, "vggt_qk_prologue")
     return x_hat
+
+
+def vggt_attn_core(q_hat, k_hat, v, out, n_seg, q_len, k_len, H=16, D=64, stream=None):
+    """Attention on prologue outputs (head-major q_hat / k_hat). Returns ``out``."""
+    rc = lib.vggt_attn_core(_ptr(q_hat, torch.bfloat16, "q_hat"), _ptr(k_hat, torch.bfloat16, "k_hat"),
+                            _ptr(v, torch.bfloat16, "v"), _ptr(out, torch.bfloat16, "out"),
+                            int(n_seg), int(q_len), int(k_len), int(H), int(D), _stream(stream))
+    _check(rc, "vggt_attn_core")
+    return out
 
 
 def vggt_kv_pool_tokens(T: int, kv_down: int) -> int:

@@ -144,6 +144,24 @@ int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int
     return to_status(vggt::launch_qk_prologue(j, none, H, stream));
 }
 
+int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
+                   vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
+                   cudaStream_t stream) {
+    if (n_seg < 0 || q_len < 0 || k_len < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    if (static_cast<long long>(n_seg) * q_len > VGGT_MAX_TOKENS ||
+        static_cast<long long>(n_seg) * k_len > VGGT_MAX_TOKENS || H > 65535)
+        return VGGT_ERR_SHAPE;
+    if (n_seg == 0 || q_len == 0 || k_len == 0 || H == 0) return VGGT_OK;
+    if (!q_hat || !k_hat || !v || !out) return VGGT_ERR_NULL;
+    if (!aligned16(q_hat) || !aligned16(k_hat) || !aligned16(v) || !aligned16(out))
+        return VGGT_ERR_UNSUPPORTED;
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H};
+    return to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
+}
+
 int vggt_kv_pool_tokens(int T, int kv_down) {
     const int g = grid_side(T);
     if (g < 0 || kv_down < 1) return VGGT_ERR_SHAPE;

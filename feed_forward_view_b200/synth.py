@@ -82,6 +82,11 @@ WORKLOADS = {
     )
 }
 
+# A smaller dense-global case whose inputs (151 MB) still exceed the 126 MB L2,
+# used for hardware-counter captures of the attention kernel.
+PROFILE_WORKLOADS = {w.name: w for w in (Workload("global_s6_g64", "global", S=6, g=64),)}
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS}
+
 
 def grid_side(T: int) -> int:
     """Side of the square patch grid for ``T`` tokens per frame, or -1."""

@@ -122,6 +122,22 @@ VGGT_API int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x
                               int N, int H, int D, cudaStream_t stream);
 
 /*
+ * Attention on vectors that already went through the prologue (for callers
+ * that reuse normalised keys across calls, or attend between arbitrary token
+ * sets). Segment s (0 <= s < n_seg): queries [s*q_len, (s+1)*q_len) attend to
+ * keys [s*k_len, (s+1)*k_len); softmax(q_hat k_hat^T / sqrt(D)) v.
+ *   q_hat [H, n_seg*q_len, D], k_hat [H, n_seg*k_len, D] bf16 head-major (the
+ *   layout vggt_qk_prologue writes); v [n_seg*k_len, H, D] and
+ *   out [n_seg*q_len, H, D] bf16 token-major.
+ * Frame attention is n_seg = S, q_len = k_len = T; global attention is
+ * n_seg = 1, q_len = k_len = S*T. Takes no scratch. n_seg, q_len or k_len
+ * == 0, or H == 0, is a no-op.
+ */
+VGGT_API int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
+                            vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
+                            cudaStream_t stream);
+
+/*
  * Per-frame K/V descriptors (FlashVGGT README: "spatially resampling keys and
  * values"; the grid is g x g with g = sqrt(T - 5)):
  *   - the 5 special tokens of each frame are copied unchanged;

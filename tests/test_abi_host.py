@@ -100,6 +100,16 @@ def test_pool_and_prologue_argument_checks():
     assert F.lib.vggt_qk_prologue(None, None, None, 0, 16, 64, None) == OK
 
 
+def test_core_argument_checks():
+    p = [FAKE] * 4
+    assert F.lib.vggt_attn_core(*p, 1, 100, 100, 16, 32, None) == E_UNSUP
+    assert F.lib.vggt_attn_core(*p, -1, 100, 100, 16, 64, None) == E_SHAPE
+    assert F.lib.vggt_attn_core(*p, 1, 1 << 22, 100, 16, 64, None) == E_SHAPE
+    assert F.lib.vggt_attn_core(None, *p[1:], 1, 100, 100, 16, 64, None) == E_NULL
+    assert F.lib.vggt_attn_core(FAKE + 4, *p[1:], 1, 100, 100, 16, 64, None) == E_UNSUP
+    assert F.lib.vggt_attn_core(None, None, None, None, 1, 0, 100, 16, 64, None) == OK
+
+
 def test_binding_rejects_host_tensors():
     import torch
 

@@ -1,0 +1,89 @@
+"""Host logic of bench.py without a GPU: max-over-ranks timing across two gloo
+ranks (the path of a multi-GPU run, where every rank is an independent
+replica), clock-sample parsing and the profile/traffic bookkeeping."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, local, w = bench.dist_setup(n_gpus=0)  # gloo
+    assert (r, local, w) == (rank, rank, world)
+    bench.barrier(w)
+    mx = bench.max_over_ranks(10.0 + 5.0 * rank, w)
+    bench.barrier(w)
+    results[rank] = mx
+    import torch.distributed as dist
+
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert dict(results) == {0: 15.0, 1: 15.0}
+
+
+def test_max_over_ranks_single_process_is_identity():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_clock_summary_parsing():
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 1965, 1965, 300.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1335, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1350, 1965, 995.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 120, 1965, 90.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage",
+    ]
+    s = cs.summary()
+    assert s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    assert s["sm_mhz"] == 1350  # idle sample (120 MHz) excluded, median of the rest
+    assert s["samples"] == 4
+
+
+def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
+    from feed_forward_view_b200 import synth
+
+    w = synth.WORKLOADS["global_s9_g64"]
+    f = tmp_path / "summary.txt"
+    f.write_text(f"tokens: {w.n_q // 3}\nsource_sha256_16: {bench.kernel_source_hash()}\n"
+                 "dram_bytes_per_launch: 1000\n")
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(f))
+    assert bench.profiled_traffic(w) == 3000.0
+    assert bench.profiled_traffic(synth.WORKLOADS["frame_s8_g37"]) is None
+    f.write_text("tokens: 10\nsource_sha256_16: 0000\ndram_bytes_per_launch: 1234\n")
+    assert bench.profiled_traffic(w) is None
+
+
+@pytest.mark.parametrize("name", ["global_s2_g16", "frame_s8_g37", "descriptor_s200_g37_kd4"])
+def test_oracle_leg_runs_on_a_small_sample(name):
+    from feed_forward_view_b200 import synth
+
+    w = synth.WORKLOADS[name]
+    if w.n_q > 50000:
+        pytest.skip("large setup; covered by the reference arm")
+    tf, dt, rows = bench.OracleLeg(w).run(8)
+    assert tf > 0 and dt > 0 and rows >= 8

@@ -155,6 +155,22 @@ def test_attention_full_workloads(F, name):
     check_attention(F, w.kind, w.S, w.g, w.kv_down, seed=1, rows=rows)
 
 
+def test_core_on_prologue_outputs_equals_the_fused_call(F):
+    # vggt_attn_core on vggt_qk_prologue outputs runs the same kernels as
+    # vggt_attn_global / vggt_attn_frame: the results are identical.
+    S, g = 3, 13
+    q, k, v, pos = synth.make_qkv(S, g, seed=12)
+    T = 5 + g * g
+    qd, kd_, vd, pd = (t.cuda() for t in (q, k, v, pos))
+    qh = F.vggt_qk_prologue(qd, pd)
+    kh = F.vggt_qk_prologue(kd_, pd)
+    for kind, n_seg, ql in (("global", 1, S * T), ("frame", S, T)):
+        out = torch.empty_like(qd)
+        F.vggt_attn_core(qh, kh, vd, out, n_seg, ql, ql)
+        torch.cuda.synchronize()
+        assert torch.equal(out.cpu(), run_gpu(F, kind, q, k, v, pos, S, T, 1))
+
+
 def test_descriptor_kd1_equals_global_on_gpu(F):
     q, k, v, pos = synth.make_qkv(2, 12, seed=13)
     T = 5 + 144
