@@ -27,6 +27,7 @@ __all__ = [
     "vggt_kv_pool_tokens",
     "vggt_qk_prologue",
     "vggt_attn_core",
+    "vggt_attn_global_noalloc",
     "vggt_get_device_status",
     "vggt_status_string",
     "vggt_set_wait_limit",
@@ -38,6 +39,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "vggt_qk_prologue",
     "vggt_attn_core",
+    "vggt_attn_global_noalloc",
     "vggt_attn_frame",
     "vggt_attn_global",
     "vggt_attn_descriptor",
@@ -59,7 +61,8 @@ lib = ctypes.CDLL(LIB_PATH)
 _p = ctypes.c_void_p
 _i = ctypes.c_int
 _ATTN_ARGS = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
-for _name in ("vggt_attn_frame", "vggt_attn_global", "vggt_attn_descriptor"):
+for _name in ("vggt_attn_frame", "vggt_attn_global", "vggt_attn_descriptor",
+              "vggt_attn_global_noalloc"):
     getattr(lib, _name).argtypes = _ATTN_ARGS
     getattr(lib, _name).restype = _i
 lib.vggt_kv_pool.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
@@ -142,6 +145,13 @@ def vggt_attn_descriptor(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, kv_
                          stream=None):
     """Compressed-descriptor attention (pooled K/V). Returns ``out``."""
     return _attn(lib.vggt_attn_descriptor, q, k, v, pos, out, S, T, H, D, kv_down, stream)
+
+
+def vggt_attn_global_noalloc(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, kv_down=0,
+                             stream=None):
+    """Global attention drawing its scratch from the library's fixed array
+    instead of allocating (see include/vggt_attn.h). Returns ``out``."""
+    return _attn(lib.vggt_attn_global_noalloc, q, k, v, pos, out, S, T, H, D, kv_down, stream)
 
 
 def vggt_qk_prologue(x, pos, x_hat=None, N=None, H=16, D=64, stream=None):

@@ -112,6 +112,18 @@ int run_attention(const uint16_t* q, const float* pos, const uint16_t* k, const 
 
 }  // namespace
 
+namespace vggt {
+
+bool device_status_word(int** status, long long* wait_limit) {
+    DeviceState* st = device_state();
+    if (!st) return false;
+    *status = st->status;
+    *wait_limit = st->wait_limit;
+    return true;
+}
+
+}  // namespace vggt
+
 extern "C" {
 
 int vggt_attn_frame(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,

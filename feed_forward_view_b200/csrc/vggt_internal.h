@@ -50,6 +50,10 @@ struct AttnProblem {
 cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_limit,
                              cudaStream_t stream);
 
+// Device address of the library's device status word and the current
+// bounded-wait limit, for the current device; false if the lookup failed.
+bool device_status_word(int** status, long long* wait_limit);
+
 // A one-thread kernel that waits on a barrier nothing completes.
 cudaError_t launch_wait_probe(int* status, long long wait_limit, cudaStream_t stream);
 

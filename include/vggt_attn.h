@@ -154,6 +154,32 @@ VGGT_API int vggt_kv_pool(const vggt_bf16* k, const vggt_bf16* v, const float* p
                  vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out,
                  int S, int T, int H, int D, int kv_down, cudaStream_t stream);
 
+/* Size of the fixed scratch array vggt_attn_global_noalloc draws on. */
+#define VGGT_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * Global attention that allocates nothing, for callers that must not allocate
+ * device memory while they run -- e.g. inference loops that reserve their
+ * whole memory budget at start-up, or processes without the stream-ordered
+ * allocator. (No counterpart on the pages: it exists only for such callers.)
+ * Same arguments, layouts and result as vggt_attn_global; the caller still
+ * provides q, k, v, pos and out. The normalised q and k live in a fixed
+ * VGGT_NOALLOC_SCRATCH_BYTES array inside the library, so the call needs
+ * 2 * S*T * H * D * 2 bytes <= VGGT_NOALLOC_SCRATCH_BYTES (S*T <= 4096 at
+ * H = 16) and returns VGGT_ERR_SHAPE beyond that, launching nothing.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Every GPU that loads the library keeps the array until the process exits.
+ * - All calls share the array: calls that overlap on the GPU (e.g. on two
+ *   unordered streams) race and corrupt each other's results. Order them.
+ * - It never calls cudaMalloc, cudaMallocAsync, cudaFree or any allocator.
+ */
+VGGT_API int vggt_attn_global_noalloc(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                                      const float* pos, vggt_bf16* out,
+                                      int S, int T, int H, int D, int kv_down,
+                                      cudaStream_t stream);
+
 /* Tokens per frame after pooling (5 + ceil(g/kv_down)^2), or a negative
    vggt_status when T is not 5 + g*g or kv_down < 1. Host only. */
 VGGT_API int vggt_kv_pool_tokens(int T, int kv_down);
