@@ -6,36 +6,55 @@
 //  Attention" slide; shapes [B, N, 16, 64] from the vggt-jax README table.)
 //
 // One CTA owns two 128-row query tiles of one head (256 queries) and streams
-// that head's keys/values in 128-row blocks:
+// that head's keys/values in 96-row blocks:
 //
-//   warp 0      TMA producer: Q tiles once, then K_j / V_j into a 3-stage ring.
-//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T (SS, M=128 N=128 K=64)
-//               into TMEM, and O_t += P_t V_j (TS: P read from TMEM, M=128
-//               N=64 K=128). Allocates / frees the 512 TMEM columns.
-//   warps 2-3   idle (they complete the first warpgroup).
+//   warp 0      TMA producer: Q tiles once, then K_j and V_j together into a
+//               5-slot ring (one full / one empty barrier per slot).
+//   warps 1, 2  MMA issuers, one per query tile t (one thread each):
+//               S_{t,j} = Q_t K_j^T (SS, M=128 N=96 K=64) into TMEM and
+//               O_t += P_{t,j} V_j (TS: P read from TMEM, M=128 N=64 K=96).
+//               A tcgen05.mma costs a single issuing thread about as long as a
+//               small MMA takes to execute, so each tile gets its own issuer.
+//   warp 3      idle (completes the first warpgroup).
 //   warps 4-7   softmax for tile 0, warps 8-11 softmax for tile 1: each thread
-//               owns one query row (its TMEM lane), reads the row's 128 scores
+//               owns one query row (its TMEM lane), reads the row's 96 scores
 //               from TMEM, runs the online softmax in fp32 with exp2, writes P
 //               as bf16 back to TMEM, and finally normalises O and stores it.
 //
-// TMEM columns (fp32 unless noted): S0 [0,128) S1 [128,256) O0 [256,320)
-// O1 [320,384) P0 [384,448) P1 [448,512) (P: 128 bf16 packed in 64 columns).
+// TMEM columns, tile t: S_{t,0} [256t, +96), S_{t,1} [256t + 96, +96) (fp32),
+// O_t [256t + 192, +64) (fp32); 512 in all. P_{t,b} (96 bf16 per row, packed
+// in 48 columns) is written over the first half of S_{t,b} once the scores
+// have been read. S is double-buffered: the issuer computes S_{t,j+1} while
+// the softmax warps work on block j.
+//
+// Issue order for tile t: S_{t,0}, S_{t,1}, then for every block j:
+// [P_{t,j} ready] PV_{t,j}, commit kv_empty[j's slot], [K_{j+2} loaded]
+// S_{t,j+2} into buffer j%2 (after PV_{t,j} has read P_{t,j} from it: the
+// tcgen05 MMAs of one thread run in issue order), commit bar_s[t][j%2]; at the
+// end, commit bar_o[t]. A commit tracks every earlier tcgen05 operation of the
+// thread, so S_{t,j} complete implies PV_{t,j-2} finished (P_{t,j} may be
+// written over buffer j%2) and S_{t,j+1} complete implies PV_{t,j-1} finished
+// (O_t may be rescaled).
+//
+// Barrier phases: a parity wait is unambiguous only while the barrier is at
+// most one phase away from the awaited one, in either direction. bar_s and
+// bar_p exist once per S buffer (blocks b, b+2, ...): the previous phase of
+// the same buffer (block j-2) has always been observed, and block j+2 cannot
+// start before block j is consumed. The K/V ring follows the same rule.
 //
 // Online softmax: m is the running row maximum in log2 units
 // (score * log2(e) / 8); p = 2^(score * log2(e)/8 - m). A block whose maximum
 // exceeds m by more than kLazy (8, i.e. p <= 256) triggers a rescale of O and
 // of the running sum l by 2^(m_old - m_new); smaller increases keep the stale
-// m, which is exact because the final O / l uses the same m for both.
+// m, which is exact because the final O / l uses the same m for both. After
+// the QK LayerNorm every |score| <= 8 (|q_hat|, |k_hat| <= 8): 2^x is only
+// ever needed for x in [-24, 24], so the last block, which has no later S to
+// wait on for the rescale, simply keeps the stale maximum (p <= 2^24 stays
+// far inside fp32 and bf16 range).
 //
-// Ordering: the MMA thread issues, per key block j and tile t, PV_{t,j-1} and
-// then S_{t,j}, and commits S_{t,j} to bar_s[t]. A tcgen05.commit tracks every
-// earlier tcgen05 operation of the thread, so when the softmax warps see
-// S_{t,j} complete, PV_{t,j-1} has also finished: P_t may be overwritten and
-// O_t may be rescaled in place.
-//
-// Every wait is bounded (vggt::mbar_wait); on timeout the CTA records the
-// timeout in the device status word, stops issuing work, drains what it has
-// in flight and frees its tensor memory before exiting.
+// Every wait is bounded; on timeout the CTA records the timeout in the device
+// status word, stops issuing work, drains what it has in flight and frees its
+// tensor memory before exiting.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -45,31 +64,79 @@
 namespace vggt {
 namespace {
 
-constexpr int kBM = 128;                       // query rows per tile
-constexpr int kBN = 128;                       // keys per block
-constexpr int kStages = 3;                     // K/V ring depth
-constexpr int kTileBytes = kBM * kHeadDim * 2; // 16 KB per bf16 tile
+constexpr int kBM = 128;                          // query rows per tile
+constexpr int kBN = 96;                           // keys per block
+constexpr int kStages = 5;                        // K/V ring depth
+constexpr int kQTileBytes = kBM * kHeadDim * 2;   // 16 KB
+constexpr int kKVTileBytes = kBN * kHeadDim * 2;  // 12 KB
 constexpr int kThreads = 384;
+// Register split: 168 per thread at launch (the cap for 12 warps); the
+// TMA/MMA warpgroup gives up to 80, the two softmax warpgroups take 208:
+// 128 * 80 + 256 * 208 = 63488 <= 384 * 168.
+constexpr uint32_t kRegsControl = 80;
+constexpr uint32_t kRegsSoftmax = 208;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * 168,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
-// TMEM column of S_t, O_t and P_t for query tile t in {0, 1}.
-__device__ __forceinline__ constexpr uint32_t col_s(int t) { return 128u * t; }
-__device__ __forceinline__ constexpr uint32_t col_o(int t) { return 256u + 64u * t; }
-__device__ __forceinline__ constexpr uint32_t col_p(int t) { return 384u + 64u * t; }
+
+// TMEM column of S_{t,b} (P_{t,b} aliases its first 48 columns) and of O_t.
+__device__ __forceinline__ constexpr uint32_t col_s(int t, int b) { return 256u * t + 96u * b; }
+__device__ __forceinline__ constexpr uint32_t col_o(int t) { return 256u * t + 192u; }
+
 constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64)
 constexpr float kLazy = 8.0f;
 
+// Exponentials per key block: of every 8 consecutive score pairs,
+// kExp2OnFma pairs are evaluated on the FMA pipe (polynomial below) and the
+// rest with the MUFU ex2 instruction, so that the two units share the work.
+#ifndef VGGT_EXP2_ON_FMA_PER8
+#define VGGT_EXP2_ON_FMA_PER8 2
+#endif
+constexpr int kExp2OnFma = VGGT_EXP2_ON_FMA_PER8;
+
+// 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [-1/2, 1/2]: minimax in relative error
+// (Remez exchange, fit by fit_exp2_poly.py in this directory); worst relative
+// error of the whole float32 evaluation over [-24, 8] is 7.5e-5.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+// 2^x for both lanes of a packed pair on the FMA pipe. x = j + f with
+// j = round(x) (taken by adding 1.5 * 2^23 in round-to-nearest, which leaves
+// j in the low mantissa bits of t) and f = x - j exactly, |f| <= 1/2; then
+// 2^x = p(f) * 2^j with 2^j applied by adding j << 23 to the bit pattern.
+// Valid for x in [-125, 127].
+__device__ __forceinline__ uint64_t exp2_fma_pair(uint64_t x) {
+    const uint64_t t = f2_add(x, f2_pack(kRoundMagic, kRoundMagic));
+    const uint64_t j = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
+    const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
+    uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+    p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+    p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+    uint32_t p0, p1, t0, t1;
+    u2_unpack(p, p0, p1);
+    u2_unpack(t, t0, t1);
+    return u2_pack(p0 + (t0 << 23), p1 + (t1 << 23));
+}
+
+// 2^x for both lanes with the MUFU ex2 instruction (exact 0 for -inf).
+__device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t x) {
+    float a, b;
+    f2_unpack(x, a, b);
+    return f2_pack(ex2_approx(a), ex2_approx(b));
+}
+
 struct SharedStorage {
-    uint8_t q[2][kTileBytes];
-    uint8_t k[kStages][kTileBytes];
-    uint8_t v[kStages][kTileBytes];
+    uint8_t q[2][kQTileBytes];
+    uint8_t kv[kStages][2][kKVTileBytes];  // [slot][K, V]
     uint64_t bar_q;
-    uint64_t bar_kfull[kStages];
-    uint64_t bar_kempty[kStages];
-    uint64_t bar_vfull[kStages];
-    uint64_t bar_vempty[kStages];
-    uint64_t bar_s[2];
-    uint64_t bar_p[2];
-    uint64_t bar_o;
+    uint64_t bar_kvfull[kStages];
+    uint64_t bar_kvempty[kStages];
+    uint64_t bar_s[2][2];  // [tile][buffer]: S_{t,j} computed (blocks j = b, b+2, ...)
+    uint64_t bar_p[2][2];  // [tile][buffer]: P_{t,j} written (blocks j = b, b+2, ...)
+    uint64_t bar_o[2];     // [tile]: every MMA of the tile finished (once)
     uint32_t tmem_base;
     int abort;
 };
@@ -85,7 +152,11 @@ struct Params {
 };
 
 // Bounded wait that also gives up once this CTA or any other CTA reported a
-// timeout; records a timeout of its own.
+// timeout; records a timeout of its own. The barrier is polled back to back
+// (try_wait itself suspends the thread for a while); the abort flag, the clock
+// and the global status word are only looked at every 256 polls, so that a
+// phase that completes is noticed within one poll and not one global-memory
+// round trip later.
 struct Waiter {
     long long limit;
     volatile int* abort;
@@ -94,17 +165,19 @@ struct Waiter {
     __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
         if (mbar_try_wait(bar, parity)) return true;
         const long long t0 = clock64();
-        while (true) {
+        for (uint32_t it = 1;; ++it) {
             if (mbar_try_wait(bar, parity)) return true;
-            if (*abort) return false;
-            if (*reinterpret_cast<volatile int*>(status)) {
-                *abort = 1;
-                return false;
-            }
-            if (clock64() - t0 > limit) {
-                *abort = 1;
-                atomicOr(status, kStatusTimeout);
-                return false;
+            if ((it & 255u) == 0) {
+                if (*abort) return false;
+                if (*reinterpret_cast<volatile int*>(status)) {
+                    *abort = 1;
+                    return false;
+                }
+                if (clock64() - t0 > limit) {
+                    *abort = 1;
+                    atomicOr(status, kStatusTimeout);
+                    return false;
+                }
             }
         }
     }
@@ -119,15 +192,38 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
     }
 }
 
-// Row maximum of 128 scores with 8 independent running maxima (little extra
-// register pressure next to the 128 live scores).
-__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+// Row maximum of 96 scores: 8 independent running maxima fed two scores at a
+// time with the three-input max of sm_100.
+__device__ __forceinline__ float row_max96(const float (&s)[96]) {
     float m[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = s[i];
 #pragma unroll
-    for (int c = 8; c < 128; ++c) m[c & 7] = fmaxf(m[c & 7], s[c]);
-    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+    for (int k = 0; k < 44; ++k) m[k & 7] = fmax3(m[k & 7], s[8 + 2 * k], s[9 + 2 * k]);
+    return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// p = 2^(s * log2(e)/8 - m) for 96 scores, packed to bf16 pairs in pk, with
+// the fp32 row sum of p returned. kMixed: share the exponentials between the
+// FMA pipe and MUFU; otherwise MUFU only (blocks with masked -inf scores).
+template <bool kMixed>
+__device__ __forceinline__ float exp_pack_row(const float (&s)[96], float m, uint32_t (&pk)[48]) {
+    const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
+    const uint64_t negm2 = f2_pack(-m, -m);
+    uint64_t acc[4] = {0, 0, 0, 0};  // packed partial sums (0 bits == 0.0f, 0.0f)
+#pragma unroll
+    for (int c = 0; c < 48; ++c) {
+        const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, negm2);
+        const uint64_t p = (kMixed && (c & 7) < kExp2OnFma) ? exp2_fma_pair(x) : exp2_mufu_pair(x);
+        acc[c & 3] = f2_add(acc[c & 3], p);
+        float p0, p1;
+        f2_unpack(p, p0, p1);
+        pk[c] = pack_bf16x2(p0, p1);
+    }
+    const uint64_t a = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+    float lo, hi;
+    f2_unpack(a, lo, hi);
+    return lo + hi;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -150,42 +246,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int nkb = (prm.k_len + kBN - 1) / kBN;
     const int last_valid = prm.k_len - (nkb - 1) * kBN;  // keys in the last block
 
-    // Shared-memory addresses of the barriers and tiles; stage / tile indices
+    // Shared-memory addresses of the barriers and tiles; slot / tile indices
     // are runtime values, so they are formed arithmetically (no local arrays).
     const uint32_t bar_q = smem_u32(&sm.bar_q);
-    const uint32_t bar_kfull0 = smem_u32(&sm.bar_kfull[0]);
-    const uint32_t bar_kempty0 = smem_u32(&sm.bar_kempty[0]);
-    const uint32_t bar_vfull0 = smem_u32(&sm.bar_vfull[0]);
-    const uint32_t bar_vempty0 = smem_u32(&sm.bar_vempty[0]);
-    const uint32_t bar_s0 = smem_u32(&sm.bar_s[0]);
-    const uint32_t bar_p0 = smem_u32(&sm.bar_p[0]);
-    const uint32_t bar_o = smem_u32(&sm.bar_o);
+    const uint32_t bar_kvfull0 = smem_u32(&sm.bar_kvfull[0]);
+    const uint32_t bar_kvempty0 = smem_u32(&sm.bar_kvempty[0]);
+    const uint32_t bar_s0 = smem_u32(&sm.bar_s[0][0]);
+    const uint32_t bar_p0 = smem_u32(&sm.bar_p[0][0]);
+    const uint32_t bar_o0 = smem_u32(&sm.bar_o[0]);
     const uint32_t q_smem0 = smem_u32(sm.q[0]);
-    const uint32_t k_smem0 = smem_u32(sm.k[0]);
-    const uint32_t v_smem0 = smem_u32(sm.v[0]);
-    auto bar_kfull = [&](int s) { return bar_kfull0 + 8u * s; };
-    auto bar_kempty = [&](int s) { return bar_kempty0 + 8u * s; };
-    auto bar_vfull = [&](int s) { return bar_vfull0 + 8u * s; };
-    auto bar_vempty = [&](int s) { return bar_vempty0 + 8u * s; };
-    auto bar_s = [&](int t) { return bar_s0 + 8u * t; };
-    auto bar_p = [&](int t) { return bar_p0 + 8u * t; };
-    auto q_smem = [&](int t) { return q_smem0 + static_cast<uint32_t>(kTileBytes) * t; };
-    auto k_smem = [&](int s) { return k_smem0 + static_cast<uint32_t>(kTileBytes) * s; };
-    auto v_smem = [&](int s) { return v_smem0 + static_cast<uint32_t>(kTileBytes) * s; };
+    const uint32_t kv_smem0 = smem_u32(sm.kv[0][0]);
+    auto bar_kvfull = [&](int s) { return bar_kvfull0 + 8u * s; };
+    auto bar_kvempty = [&](int s) { return bar_kvempty0 + 8u * s; };
+    auto bar_s = [&](int t, int b) { return bar_s0 + 16u * t + 8u * b; };
+    auto bar_p = [&](int t, int b) { return bar_p0 + 16u * t + 8u * b; };
+    auto bar_o = [&](int t) { return bar_o0 + 8u * t; };
+    auto q_smem = [&](int t) { return q_smem0 + static_cast<uint32_t>(kQTileBytes) * t; };
+    auto k_smem = [&](int s) { return kv_smem0 + static_cast<uint32_t>(2 * kKVTileBytes) * s; };
+    auto v_smem = [&](int s) { return k_smem(s) + static_cast<uint32_t>(kKVTileBytes); };
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_kfull(s), 1);
-            mbar_init(bar_kempty(s), 1);
-            mbar_init(bar_vfull(s), 1);
-            mbar_init(bar_vempty(s), 1);
+            mbar_init(bar_kvfull(s), 1);
+            mbar_init(bar_kvempty(s), ntile);  // one commit per tile issuer
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_s(t), 1);
-            mbar_init(bar_p(t), 4);  // one arrival per softmax warp
+            mbar_init(bar_s(t, 0), 1);
+            mbar_init(bar_s(t, 1), 1);
+            mbar_init(bar_p(t, 0), 4);  // one arrival per softmax warp
+            mbar_init(bar_p(t, 1), 4);
+            mbar_init(bar_o(t), 1);
         }
-        mbar_init(bar_o, 1);
         sm.abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -205,90 +297,84 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = sm.tmem_base;
     const Waiter wait{prm.wait_limit, &sm.abort, prm.status};
 
+    if (warp < 4) regs_dec<kRegsControl>();
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int n_issued = 0;  // K/V blocks whose loads were started
-            mbar_arrive_expect_tx(bar_q, ntile * kTileBytes);
+            int n_issued = 0;  // blocks whose loads were started
+            mbar_arrive_expect_tx(bar_q, ntile * kQTileBytes);
             tma_load_3d(q_smem(0), &tm_q, bar_q, 0, q_row0, h);
             if (ntile == 2) tma_load_3d(q_smem(1), &tm_q, bar_q, 0, q_row0 + kBM, h);
-            bool v_pending = false;  // K of the last block started, V not
             for (int j = 0; j < nkb; ++j) {
                 const int s = j % kStages;
                 const uint32_t use = j / kStages;
-                if (use > 0 && !wait(bar_kempty(s), (use - 1) & 1)) break;
-                mbar_arrive_expect_tx(bar_kfull(s), kTileBytes);
-                tma_load_3d(k_smem(s), &tm_k, bar_kfull(s), 0, k_row0 + j * kBN, h);
+                if (use > 0 && !wait(bar_kvempty(s), (use - 1) & 1)) break;
+                mbar_arrive_expect_tx(bar_kvfull(s), 2 * kKVTileBytes);
+                tma_load_3d(k_smem(s), &tm_k, bar_kvfull(s), 0, k_row0 + j * kBN, h);
+                tma_load_3d(v_smem(s), &tm_v, bar_kvfull(s), 0, h, k_row0 + j * kBN);
                 ++n_issued;
-                if (use > 0 && !wait(bar_vempty(s), (use - 1) & 1)) {
-                    v_pending = true;
-                    break;
-                }
-                mbar_arrive_expect_tx(bar_vfull(s), kTileBytes);
-                tma_load_3d(v_smem(s), &tm_v, bar_vfull(s), 0, h, k_row0 + j * kBN);
             }
             // Every copy this CTA started must land before the CTA exits: the
             // last kStages blocks started are the only ones that can still be
             // in flight.
             drain_wait(bar_q, 0, prm.wait_limit);
-            for (int j = max(0, n_issued - kStages); j < n_issued; ++j) {
-                const int s = j % kStages;
-                const uint32_t par = (j / kStages) & 1;
-                drain_wait(bar_kfull(s), par, prm.wait_limit);
-                if (!(v_pending && j == n_issued - 1)) drain_wait(bar_vfull(s), par, prm.wait_limit);
-            }
+            for (int j = max(0, n_issued - kStages); j < n_issued; ++j)
+                drain_wait(bar_kvfull(j % kStages), (j / kStages) & 1, prm.wait_limit);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------------ MMA issuers
+        const int t = warp - 1;
+        if (lane == 0 && t < ntile) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, kHeadDim, true);
+            const uint64_t qdesc = smem_desc_sw128(q_smem(t), 16, 1024);
+            // S_{t,j} = Q_t K_j^T into buffer j % 2: 4 steps of 16 head dims.
+            auto issue_s = [&](int j) {
+                const uint64_t kdesc = smem_desc_sw128(k_smem(j % kStages), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                    mma_ss(tmem + col_s(t, j & 1), qdesc + static_cast<uint64_t>((kk * 32) >> 4),
+                           kdesc + static_cast<uint64_t>((kk * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
+                mma_commit(bar_s(t, j & 1));
+            };
             bool ok = wait(bar_q, 0);
             tc_fence_after();
-            for (int j = 0; ok && j <= nkb; ++j) {
-                const int s = j % kStages;
-                const int sp = (j + kStages - 1) % kStages;  // stage of block j-1
-                if (j < nkb && !wait(bar_kfull(s), (j / kStages) & 1)) break;
-                if (j > 0 && !wait(bar_vfull(sp), ((j - 1) / kStages) & 1)) break;
-                tc_fence_after();
-                const uint64_t kdesc = smem_desc_sw128(k_smem(s), 16, 1024);
-                const uint64_t vdesc = smem_desc_sw128(v_smem(sp), 16, 1024);
-                for (int t = 0; t < ntile; ++t) {
-                    if (j > 0) {
-                        if (!wait(bar_p(t), (j - 1) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        // O_t (+)= P_t V_{j-1}: 8 steps of 16 keys.
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_ts(tmem + col_o(t), tmem + col_p(t) + kk * 8,
-                                   vdesc + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_o,
-                                   (j > 1 || kk > 0) ? 1u : 0u);
-                    }
-                    if (j < nkb) {
-                        // S_t = Q_t K_j^T: 4 steps of 16 head dims.
-                        const uint64_t qdesc = smem_desc_sw128(q_smem(t), 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                            mma_ss(tmem + col_s(t), qdesc + static_cast<uint64_t>((kk * 32) >> 4),
-                                   kdesc + static_cast<uint64_t>((kk * 32) >> 4), idesc_s,
-                                   kk > 0 ? 1u : 0u);
-                        mma_commit(bar_s(t));
-                    }
+            for (int j = 0; ok && j < min(2, nkb); ++j) {
+                if (!wait(bar_kvfull(j % kStages), (j / kStages) & 1)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) break;
-                if (j < nkb) mma_commit(bar_kempty(s));
-                if (j > 0) mma_commit(bar_vempty(sp));
+                tc_fence_after();
+                issue_s(j);
             }
-            // Completes once every MMA issued above has finished; the softmax
-            // warps wait on it before reading O, and it doubles as the drain.
-            mma_commit(bar_o);
-            drain_wait(bar_o, 0, prm.wait_limit);
+            for (int j = 0; ok && j < nkb; ++j) {
+                const int s = j % kStages;
+                if (!wait(bar_p(t, j & 1), (j >> 1) & 1)) break;
+                tc_fence_after();
+                // O_t (+)= P_{t,j} V_j: 6 steps of 16 keys; P sits in the first
+                // 48 columns of S_{t, j%2}.
+                const uint64_t vdesc = smem_desc_sw128(v_smem(s), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ts(tmem + col_o(t), tmem + col_s(t, j & 1) + kk * 8,
+                           vdesc + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_o,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar_kvempty(s));  // K_j and V_j no longer needed by this tile
+                const int jn = j + 2;
+                if (jn < nkb) {
+                    if (!wait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
+                    tc_fence_after();
+                    issue_s(jn);
+                }
+            }
+            // Completes once every MMA of this tile has finished: the softmax
+            // warps wait on it before the epilogue; it doubles as the drain.
+            mma_commit(bar_o(t));
+            drain_wait(bar_o(t), 0, prm.wait_limit);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------ softmax
+        regs_inc<kRegsSoftmax>();
         const int t = (warp >> 2) - 1;
         const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
         const int row = quarter * 32 + lane;
@@ -297,34 +383,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             float m = 0.f, l = 0.f;
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
-                if (!wait(bar_s(t), j & 1)) {
+                const int b = j & 1;
+                if (!wait(bar_s(t, b), (j >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                float s[128];
+                float s[96];
                 {
-                    uint32_t r[64];
+                    uint32_t r[96];
+                    tmem_ld96(lane_base + col_s(t, b), r);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        tmem_ld64(lane_base + col_s(t) + 64 * c, r);
-#pragma unroll
-                        for (int i = 0; i < 64; ++i) s[64 * c + i] = __uint_as_float(r[i]);
-                    }
+                    for (int i = 0; i < 96; ++i) s[i] = __uint_as_float(r[i]);
                 }
-                if (j == nkb - 1 && last_valid < kBN) {
+                const bool masked = (j == nkb - 1) && last_valid < kBN;
+                if (masked) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
+                    for (int c = 0; c < 96; ++c)
                         if (c >= last_valid) s[c] = -INFINITY;
                 }
-                const float mx = row_max128(s) * kScaleLog2;
+                const float mx = row_max96(s) * kScaleLog2;
                 // Lazy rescale: only when the block maximum exceeds the running
-                // maximum by more than kLazy (log2 units) anywhere in the warp.
+                // maximum by more than kLazy (log2 units) anywhere in the warp,
+                // and never on the last block (see the header comment).
                 float f = 1.0f;
                 bool rescale = false;
                 if (j == 0) {
                     m = mx;
-                } else {
+                } else if (j + 1 < nkb) {
                     const bool need = mx > m + kLazy;
                     rescale = __any_sync(0xFFFFFFFFu, need);
                     if (need) {
@@ -332,21 +418,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         m = mx;
                     }
                 }
-                float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[64];
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float p0 = ex2_approx(fmaf(s[2 * c], kScaleLog2, -m));
-                    const float p1 = ex2_approx(fmaf(s[2 * c + 1], kScaleLog2, -m));
-                    part[c & 7] += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
-                }
-                tmem_st64(lane_base + col_p(t), pk);
-                l = l * f + (((part[0] + part[1]) + (part[2] + part[3])) +
-                             ((part[4] + part[5]) + (part[6] + part[7])));
+                uint32_t pk[48];
+                const float row_sum = masked ? exp_pack_row<false>(s, m, pk) : exp_pack_row<true>(s, m, pk);
+                tmem_st48(lane_base + col_s(t, b), pk);
+                l = l * f + row_sum;
                 if (rescale) {
-                    // O_t holds sum_{i<j} P_i V_i at the old maximum (PV_{t,j-1}
-                    // finished before S_{t,j} was signalled).
+                    // O_t must hold sum_{i<j} P_i V_i: S_{t,j+1} complete
+                    // implies PV_{t,j-1} finished.
+                    if (!wait(bar_s(t, b ^ 1), ((j + 1) >> 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                     uint32_t o[64];
                     tmem_ld64(lane_base + col_o(t), o);
 #pragma unroll
@@ -355,9 +438,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_p(t));
+                if (lane == 0) mbar_arrive(bar_p(t, b));
             }
-            if (ok && wait(bar_o, 0)) {
+            if (ok && wait(bar_o(t), 0)) {
                 tc_fence_after();
                 const int row_in_seg = (tile0 + t) * kBM + row;
                 const float inv = 1.0f / l;
@@ -447,10 +530,10 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     const uint64_t nk = static_cast<uint64_t>(p.n_seg) * p.k_len;
     const uint64_t row_bytes = kHeadDim * 2;
     CUtensorMap tm_q, tm_k, tm_v;
-    // q_hat / k_hat: [H][n][64] -> dims {64, n, H}, box {64, 128, 1}
+    // q_hat / k_hat: [H][n][64] -> dims {64, n, H}, box {64, rows, 1}
     if (!make_map(&tm_q, p.q_hat, nq, p.H, row_bytes, nq * row_bytes, kBM, 1) ||
         !make_map(&tm_k, p.k_hat, nk, p.H, row_bytes, nk * row_bytes, kBN, 1) ||
-        // v: [n][H][64] -> dims {64, H, n}, box {64, 1, 128}
+        // v: [n][H][64] -> dims {64, H, n}, box {64, 1, rows}
         !make_map(&tm_v, p.v, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
         return cudaErrorInvalidValue;
 
@@ -458,7 +541,16 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        // The register split (setmaxnreg) needs the full 168 registers per
+        // thread at launch; with fewer, the softmax warpgroups' increase could
+        // never be granted. Refuse to launch such a build.
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
+        if (e != cudaSuccess) return e;
+        if (static_cast<uint32_t>(fa.numRegs) * kThreads < 128 * kRegsControl + 256 * kRegsSoftmax)
+            return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes));
         if (e != cudaSuccess) return e;
