@@ -6,26 +6,34 @@
 //  Attention" slide; shapes [B, N, 16, 64] from the vggt-jax README table.)
 //
 // One CTA owns two 128-row query tiles of one head (256 queries) and streams
-// that head's keys/values in 96-row blocks:
+// that head's keys/values in 80-row blocks:
 //
 //   warp 0      TMA producer: Q tiles once, then K_j and V_j together into a
 //               5-slot ring (one full / one empty barrier per slot).
-//   warps 1, 2  MMA issuers, one per query tile t (one thread each):
-//               S_{t,j} = Q_t K_j^T (SS, M=128 N=96 K=64) into TMEM and
-//               O_t += P_{t,j} V_j (TS: P read from TMEM, M=128 N=64 K=96).
-//               A tcgen05.mma costs a single issuing thread about as long as a
-//               small MMA takes to execute, so each tile gets its own issuer.
+//   warps 1, 2  MMA issuers, one per query tile t. The whole warp runs the
+//               loop; one elected lane issues the tcgen05 instructions:
+//               S_{t,j} = Q_t K_j^T (SS, M=128 N=80 K=64) into TMEM and
+//               [O_t | l_t] += P_{t,j} [V_j | 1] (TS: P read from TMEM, M=128
+//               N=80 K=80). A tcgen05.mma costs its issuing thread about as
+//               long as a small MMA takes to run, so each tile gets an issuer.
 //   warp 3      idle (completes the first warpgroup).
 //   warps 4-7   softmax for tile 0, warps 8-11 softmax for tile 1: each thread
-//               owns one query row (its TMEM lane), reads the row's 96 scores
+//               owns one query row (its TMEM lane), reads the row's 80 scores
 //               from TMEM, runs the online softmax in fp32 with exp2, writes P
 //               as bf16 back to TMEM, and finally normalises O and stores it.
 //
-// TMEM columns, tile t: S_{t,0} [256t, +96), S_{t,1} [256t + 96, +96) (fp32),
-// O_t [256t + 192, +64) (fp32); 512 in all. P_{t,b} (96 bf16 per row, packed
-// in 48 columns) is written over the first half of S_{t,b} once the scores
-// have been read. S is double-buffered: the issuer computes S_{t,j+1} while
-// the softmax warps work on block j.
+// Row sums on the tensor core: the PV MMA's B operand is 80 columns wide --
+// V_j (64 columns) followed by a constant shared-memory tile whose first
+// column is 1 and the rest 0 (the descriptor's leading byte offset points
+// from each V slot to it). Column 64 of the accumulator therefore collects
+// l = sum_j P_j from the same bf16 P that multiplies V, and the softmax warps
+// do no additions of their own.
+//
+// TMEM columns, tile t: S_{t,0} [256t, +80), S_{t,1} [256t + 80, +80) (fp32),
+// [O_t | l_t] [256t + 160, +80) (fp32); 496 of 512 used. P_{t,b} (80 bf16 per
+// row, packed in 40 columns) is written over the first half of S_{t,b} once
+// the scores have been read. S is double-buffered: the issuer computes
+// S_{t,j+1} while the softmax warps work on block j.
 //
 // Issue order for tile t: S_{t,0}, S_{t,1}, then for every block j:
 // [P_{t,j} ready] PV_{t,j}, commit kv_empty[j's slot], [K_{j+2} loaded]
@@ -44,13 +52,13 @@
 //
 // Online softmax: m is the running row maximum in log2 units
 // (score * log2(e) / 8); p = 2^(score * log2(e)/8 - m). A block whose maximum
-// exceeds m by more than kLazy (8, i.e. p <= 256) triggers a rescale of O and
-// of the running sum l by 2^(m_old - m_new); smaller increases keep the stale
-// m, which is exact because the final O / l uses the same m for both. After
-// the QK LayerNorm every |score| <= 8 (|q_hat|, |k_hat| <= 8): 2^x is only
-// ever needed for x in [-24, 24], so the last block, which has no later S to
-// wait on for the rescale, simply keeps the stale maximum (p <= 2^24 stays
-// far inside fp32 and bf16 range).
+// exceeds m by more than kLazy (8, i.e. p <= 256) triggers a rescale of
+// [O | l] by 2^(m_old - m_new); smaller increases keep the stale m, which is
+// exact because the final O / l uses the same m for both. After the QK
+// LayerNorm every |score| <= 8 (|q_hat|, |k_hat| <= 8): 2^x is only ever
+// needed for x in [-24, 24], so the last block, which has no later S to wait
+// on for the rescale, simply keeps the stale maximum (p <= 2^24 stays far
+// inside fp32 and bf16 range).
 //
 // Every wait is bounded; on timeout the CTA records the timeout in the device
 // status word, stops issuing work, drains what it has in flight and frees its
@@ -65,23 +73,26 @@ namespace vggt {
 namespace {
 
 constexpr int kBM = 128;                          // query rows per tile
-constexpr int kBN = 96;                           // keys per block
+constexpr int kBN = 80;                           // keys per block
 constexpr int kStages = 5;                        // K/V ring depth
 constexpr int kQTileBytes = kBM * kHeadDim * 2;   // 16 KB
-constexpr int kKVTileBytes = kBN * kHeadDim * 2;  // 12 KB
+constexpr int kKVTileBytes = kBN * kHeadDim * 2;  // 10 KB
+constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum block (16)
 constexpr int kThreads = 384;
 // Register split: 168 per thread at launch (the cap for 12 warps); the
 // TMA/MMA warpgroup gives up to 80, the two softmax warpgroups take 208:
 // 128 * 80 + 256 * 208 = 63488 <= 384 * 168.
+constexpr uint32_t kLaunchRegs = 168;
 constexpr uint32_t kRegsControl = 80;
 constexpr uint32_t kRegsSoftmax = 208;
-static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * 168,
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 
-// TMEM column of S_{t,b} (P_{t,b} aliases its first 48 columns) and of O_t.
-__device__ __forceinline__ constexpr uint32_t col_s(int t, int b) { return 256u * t + 96u * b; }
-__device__ __forceinline__ constexpr uint32_t col_o(int t) { return 256u * t + 192u; }
+// TMEM column of S_{t,b} (P_{t,b} aliases its first 40 columns) and of
+// [O_t | l_t].
+__device__ __forceinline__ constexpr uint32_t col_s(int t, int b) { return 256u * t + 80u * b; }
+__device__ __forceinline__ constexpr uint32_t col_o(int t) { return 256u * t + 160u; }
 
 constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64)
 constexpr float kLazy = 8.0f;
@@ -90,7 +101,7 @@ constexpr float kLazy = 8.0f;
 // kExp2OnFma pairs are evaluated on the FMA pipe (polynomial below) and the
 // rest with the MUFU ex2 instruction, so that the two units share the work.
 #ifndef VGGT_EXP2_ON_FMA_PER8
-#define VGGT_EXP2_ON_FMA_PER8 2
+#define VGGT_EXP2_ON_FMA_PER8 3
 #endif
 constexpr int kExp2OnFma = VGGT_EXP2_ON_FMA_PER8;
 
@@ -103,34 +114,15 @@ constexpr float kExp2C2 = 2.426111251e-01f;
 constexpr float kExp2C3 = 5.517166853e-02f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
-// 2^x for both lanes of a packed pair on the FMA pipe. x = j + f with
-// j = round(x) (taken by adding 1.5 * 2^23 in round-to-nearest, which leaves
-// j in the low mantissa bits of t) and f = x - j exactly, |f| <= 1/2; then
-// 2^x = p(f) * 2^j with 2^j applied by adding j << 23 to the bit pattern.
-// Valid for x in [-125, 127].
-__device__ __forceinline__ uint64_t exp2_fma_pair(uint64_t x) {
-    const uint64_t t = f2_add(x, f2_pack(kRoundMagic, kRoundMagic));
-    const uint64_t j = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
-    const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
-    uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-    p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-    p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-    uint32_t p0, p1, t0, t1;
-    u2_unpack(p, p0, p1);
-    u2_unpack(t, t0, t1);
-    return u2_pack(p0 + (t0 << 23), p1 + (t1 << 23));
-}
-
-// 2^x for both lanes with the MUFU ex2 instruction (exact 0 for -inf).
-__device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t x) {
-    float a, b;
-    f2_unpack(x, a, b);
-    return f2_pack(ex2_approx(a), ex2_approx(b));
-}
-
+// 2^x on the FMA pipe for x in [-125, 127]: x = j + f with j = round(x)
+// (taken by adding 1.5 * 2^23 in round-to-nearest, which leaves j in the low
+// mantissa bits of t = x + 1.5 * 2^23) and f = x - j exactly, |f| <= 1/2;
+// then 2^x = p(f) * 2^j, with 2^j applied by adding j << 23 to the bit
+// pattern of p(f). The attention scores keep x in [-24, 24].
 struct SharedStorage {
     uint8_t q[2][kQTileBytes];
     uint8_t kv[kStages][2][kKVTileBytes];  // [slot][K, V]
+    uint8_t ones[kKVTileBytes];            // [1, 0, ..., 0] per key row, 128B-swizzled
     uint64_t bar_q;
     uint64_t bar_kvfull[kStages];
     uint64_t bar_kvempty[kStages];
@@ -192,38 +184,69 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
     }
 }
 
-// Row maximum of 96 scores: 8 independent running maxima fed two scores at a
+// Row maximum of 80 scores: 8 independent running maxima fed two scores at a
 // time with the three-input max of sm_100.
-__device__ __forceinline__ float row_max96(const float (&s)[96]) {
+__device__ __forceinline__ float row_max80(const float (&s)[kBN]) {
     float m[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = s[i];
 #pragma unroll
-    for (int k = 0; k < 44; ++k) m[k & 7] = fmax3(m[k & 7], s[8 + 2 * k], s[9 + 2 * k]);
+    for (int k = 0; k < 36; ++k) m[k & 7] = fmax3(m[k & 7], s[8 + 2 * k], s[9 + 2 * k]);
     return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// p = 2^(s * log2(e)/8 - m) for 96 scores, packed to bf16 pairs in pk, with
-// the fp32 row sum of p returned. kMixed: share the exponentials between the
-// FMA pipe and MUFU; otherwise MUFU only (blocks with masked -inf scores).
+// p = 2^(s * log2(e)/8 - m) for 80 scores, packed to bf16 pairs in pk.
+// kMixed: share the exponentials between the FMA pipe and MUFU; otherwise
+// MUFU only (blocks with masked -inf scores). Written in phases over all 40
+// pairs (exponents, then each polynomial step for every FMA-pipe pair, then
+// the MUFU pairs, then the packing), so that long runs of independent
+// instructions hide the latency of each step.
 template <bool kMixed>
-__device__ __forceinline__ float exp_pack_row(const float (&s)[96], float m, uint32_t (&pk)[48]) {
+__device__ __forceinline__ void exp_pack_row(const float (&s)[kBN], float m, uint32_t (&pk)[kBN / 2]) {
+    constexpr int kPairs = kBN / 2;
     const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
     const uint64_t negm2 = f2_pack(-m, -m);
-    uint64_t acc[4] = {0, 0, 0, 0};  // packed partial sums (0 bits == 0.0f, 0.0f)
+    uint64_t x[kPairs];
 #pragma unroll
-    for (int c = 0; c < 48; ++c) {
-        const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, negm2);
-        const uint64_t p = (kMixed && (c & 7) < kExp2OnFma) ? exp2_fma_pair(x) : exp2_mufu_pair(x);
-        acc[c & 3] = f2_add(acc[c & 3], p);
+    for (int c = 0; c < kPairs; ++c) x[c] = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, negm2);
+    auto on_fma = [](int c) { return kMixed && (c & 7) < kExp2OnFma; };
+    // FMA pipe: x = j + f, 2^x = p(f) * 2^j (see exp2_fma_pair), step by step.
+    uint64_t tt[kPairs], ff[kPairs];
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (on_fma(c)) tt[c] = f2_add(x[c], f2_pack(kRoundMagic, kRoundMagic));
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (on_fma(c)) ff[c] = f2_add(tt[c], f2_pack(-kRoundMagic, -kRoundMagic));
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (on_fma(c)) ff[c] = f2_fma(ff[c], f2_pack(-1.0f, -1.0f), x[c]);
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (on_fma(c)) x[c] = f2_fma(f2_pack(kExp2C3, kExp2C3), ff[c], f2_pack(kExp2C2, kExp2C2));
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (on_fma(c)) x[c] = f2_fma(x[c], ff[c], f2_pack(kExp2C1, kExp2C1));
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (on_fma(c)) x[c] = f2_fma(x[c], ff[c], f2_pack(kExp2C0, kExp2C0));
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c) {
         float p0, p1;
-        f2_unpack(p, p0, p1);
+        if (on_fma(c)) {
+            uint32_t q0, q1, t0, t1;
+            u2_unpack(x[c], q0, q1);
+            u2_unpack(tt[c], t0, t1);
+            p0 = __uint_as_float(q0 + (t0 << 23));
+            p1 = __uint_as_float(q1 + (t1 << 23));
+        } else {
+            float x0, x1;
+            f2_unpack(x[c], x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+        }
         pk[c] = pack_bf16x2(p0, p1);
     }
-    const uint64_t a = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-    float lo, hi;
-    f2_unpack(a, lo, hi);
-    return lo + hi;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -256,6 +279,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar_o0 = smem_u32(&sm.bar_o[0]);
     const uint32_t q_smem0 = smem_u32(sm.q[0]);
     const uint32_t kv_smem0 = smem_u32(sm.kv[0][0]);
+    const uint32_t ones_smem = smem_u32(sm.ones);
     auto bar_kvfull = [&](int s) { return bar_kvfull0 + 8u * s; };
     auto bar_kvempty = [&](int s) { return bar_kvempty0 + 8u * s; };
     auto bar_s = [&](int t, int b) { return bar_s0 + 16u * t + 8u * b; };
@@ -264,6 +288,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto q_smem = [&](int t) { return q_smem0 + static_cast<uint32_t>(kQTileBytes) * t; };
     auto k_smem = [&](int s) { return kv_smem0 + static_cast<uint32_t>(2 * kKVTileBytes) * s; };
     auto v_smem = [&](int s) { return k_smem(s) + static_cast<uint32_t>(kKVTileBytes); };
+
+    // The constant [1, 0, ..., 0] rows in the 128-byte-swizzled layout the
+    // MMA reads: the 16-byte chunk c of row r sits at chunk c ^ (r % 8), so
+    // element 0 of row r lies at byte r * 128 + (r % 8) * 16.
+    for (int i = threadIdx.x; i < kKVTileBytes / 16; i += kThreads) {
+        const int r = i >> 3, chunk = i & 7;
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (chunk == (r & 7)) w.x = 0x3F80u;  // bf16 1.0 in the low half
+        reinterpret_cast<uint4*>(sm.ones)[i] = w;
+    }
+    fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -323,53 +358,73 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 1 || warp == 2) {
         // ------------------------------------------------------ MMA issuers
+        // The whole warp runs the loop (so the descriptor arithmetic is
+        // warp-uniform); every lane polls the barriers and the verdict is
+        // made uniform with a vote; one elected lane issues the tcgen05
+        // instructions and their commits.
         const int t = warp - 1;
-        if (lane == 0 && t < ntile) {
+        if (t < ntile) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, kHeadDim, true);
+            constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, kOCols, true);
             const uint64_t qdesc = smem_desc_sw128(q_smem(t), 16, 1024);
+            auto uwait = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(0xFFFFFFFFu, wait(bar, parity)) != 0;
+            };
             // S_{t,j} = Q_t K_j^T into buffer j % 2: 4 steps of 16 head dims.
             auto issue_s = [&](int j) {
                 const uint64_t kdesc = smem_desc_sw128(k_smem(j % kStages), 16, 1024);
+                const uint32_t d = tmem + col_s(t, j & 1);
+                const uint32_t done = bar_s(t, j & 1);
+                if (elect_one()) {
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                    mma_ss(tmem + col_s(t, j & 1), qdesc + static_cast<uint64_t>((kk * 32) >> 4),
-                           kdesc + static_cast<uint64_t>((kk * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
-                mma_commit(bar_s(t, j & 1));
+                    for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                        mma_ss(d, qdesc + static_cast<uint64_t>((kk * 32) >> 4),
+                               kdesc + static_cast<uint64_t>((kk * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
+                    mma_commit(done);
+                }
+                __syncwarp();
             };
-            bool ok = wait(bar_q, 0);
-            tc_fence_after();
+            bool ok = uwait(bar_q, 0);
             for (int j = 0; ok && j < min(2, nkb); ++j) {
-                if (!wait(bar_kvfull(j % kStages), (j / kStages) & 1)) {
+                if (!uwait(bar_kvfull(j % kStages), (j / kStages) & 1)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 issue_s(j);
             }
             for (int j = 0; ok && j < nkb; ++j) {
                 const int s = j % kStages;
-                if (!wait(bar_p(t, j & 1), (j >> 1) & 1)) break;
-                tc_fence_after();
-                // O_t (+)= P_{t,j} V_j: 6 steps of 16 keys; P sits in the first
-                // 48 columns of S_{t, j%2}.
-                const uint64_t vdesc = smem_desc_sw128(v_smem(s), 16, 1024);
+                if (!uwait(bar_p(t, j & 1), (j >> 1) & 1)) break;
+                // [O_t | l_t] (+)= P_{t,j} [V_j | 1]: 5 steps of 16 keys; P sits
+                // in the first 40 columns of S_{t, j%2}. The B operand's second
+                // 64-column block (the ones tile) lies a leading byte offset
+                // away from the V slot.
+                const uint32_t vaddr = v_smem(s);
+                const uint64_t vdesc = smem_desc_sw128(vaddr, ones_smem - vaddr, 1024);
+                const uint32_t a = tmem + col_s(t, j & 1);
+                const uint32_t d = tmem + col_o(t);
+                const uint32_t first = j > 0 ? 1u : 0u;
+                const uint32_t empty = bar_kvempty(s);
+                if (elect_one()) {
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(tmem + col_o(t), tmem + col_s(t, j & 1) + kk * 8,
-                           vdesc + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_o,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar_kvempty(s));  // K_j and V_j no longer needed by this tile
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_ts(d, a + kk * 8, vdesc + static_cast<uint64_t>((kk * 16 * 128) >> 4),
+                               idesc_o, kk > 0 ? 1u : first);
+                    mma_commit(empty);  // K_j and V_j no longer needed by this tile
+                }
+                __syncwarp();
                 const int jn = j + 2;
                 if (jn < nkb) {
-                    if (!wait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
-                    tc_fence_after();
+                    if (!uwait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
                     issue_s(jn);
                 }
             }
             // Completes once every MMA of this tile has finished: the softmax
             // warps wait on it before the epilogue; it doubles as the drain.
-            mma_commit(bar_o(t));
+            if (elect_one()) mma_commit(bar_o(t));
+            __syncwarp();
             drain_wait(bar_o(t), 0, prm.wait_limit);
         }
     } else if (warp >= 4) {
@@ -380,7 +435,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int row = quarter * 32 + lane;
         if (t < ntile) {
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            float m = 0.f, l = 0.f;
+            float m = 0.f;
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
                 const int b = j & 1;
@@ -389,20 +444,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     break;
                 }
                 tc_fence_after();
-                float s[96];
+                float s[kBN];
                 {
-                    uint32_t r[96];
-                    tmem_ld96(lane_base + col_s(t, b), r);
+                    uint32_t r[kBN];
+                    tmem_ld80(lane_base + col_s(t, b), r);
 #pragma unroll
-                    for (int i = 0; i < 96; ++i) s[i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
                 }
                 const bool masked = (j == nkb - 1) && last_valid < kBN;
                 if (masked) {
 #pragma unroll
-                    for (int c = 0; c < 96; ++c)
+                    for (int c = 0; c < kBN; ++c)
                         if (c >= last_valid) s[c] = -INFINITY;
                 }
-                const float mx = row_max96(s) * kScaleLog2;
+                const float mx = row_max80(s) * kScaleLog2;
                 // Lazy rescale: only when the block maximum exceeds the running
                 // maximum by more than kLazy (log2 units) anywhere in the warp,
                 // and never on the last block (see the header comment).
@@ -418,23 +473,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         m = mx;
                     }
                 }
-                uint32_t pk[48];
-                const float row_sum = masked ? exp_pack_row<false>(s, m, pk) : exp_pack_row<true>(s, m, pk);
-                tmem_st48(lane_base + col_s(t, b), pk);
-                l = l * f + row_sum;
+                uint32_t pk[kBN / 2];
+                if (masked)
+                    exp_pack_row<false>(s, m, pk);
+                else
+                    exp_pack_row<true>(s, m, pk);
+                tmem_st40(lane_base + col_s(t, b), pk);
                 if (rescale) {
-                    // O_t must hold sum_{i<j} P_i V_i: S_{t,j+1} complete
-                    // implies PV_{t,j-1} finished.
+                    // [O_t | l_t] must hold sum_{i<j} P_i [V_i | 1]: S_{t,j+1}
+                    // complete implies PV_{t,j-1} finished.
                     if (!wait(bar_s(t, b ^ 1), ((j + 1) >> 1) & 1)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    uint32_t o[64];
-                    tmem_ld64(lane_base + col_o(t), o);
+                    uint32_t o[kOCols];
+                    tmem_ld80(lane_base + col_o(t), o);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                    tmem_st64(lane_base + col_o(t), o);
+                    for (int i = 0; i < kOCols; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                    tmem_st80(lane_base + col_o(t), o);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -443,9 +500,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (ok && wait(bar_o(t), 0)) {
                 tc_fence_after();
                 const int row_in_seg = (tile0 + t) * kBM + row;
-                const float inv = 1.0f / l;
-                uint32_t o[64];
-                tmem_ld64(lane_base + col_o(t), o);
+                uint32_t o[kOCols];
+                tmem_ld80(lane_base + col_o(t), o);
+                const float inv = 1.0f / __uint_as_float(o[kHeadDim]);  // l = column 64
                 if (row_in_seg < prm.q_len) {
                     const size_t grow = static_cast<size_t>(seg) * prm.q_len + row_in_seg;
                     uint4* dst = reinterpret_cast<uint4*>(prm.out + (grow * prm.H + h) * kHeadDim);
@@ -543,9 +600,10 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_set[dev]) {
-        // The register split (setmaxnreg) needs the full 168 registers per
-        // thread at launch; with fewer, the softmax warpgroups' increase could
-        // never be granted. Refuse to launch such a build.
+        // The register split (setmaxnreg) needs the full launch allocation
+        // (kLaunchRegs per thread); with fewer registers the softmax
+        // warpgroups' increase could never be granted. Refuse to launch such
+        // a build.
         cudaFuncAttributes fa;
         e = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
         if (e != cudaSuccess) return e;
