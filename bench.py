@@ -351,37 +351,60 @@ def run_gpu(args):
     pro_ms = p0.elapsed_time(p1) / reps
     pro_bytes = 2 * w.n_q * H * 64 * 2 + w.n_q * 8  # read x + pos, write x_hat
 
-    # ---- end to end through the public call with host buffers
+    # ---- end to end through the public call with host buffers: every step
+    # uploads its inputs from pinned host memory and reads its output back.
+    # Two device buffer sets and a copy stream let step i+1's upload run while
+    # step i computes, as a caller streaming scenes through the library would.
     e2e = None
     if not args.skip_e2e:
         hq, hk, hv, hp = (t.pin_memory() for t in (q_h, k_h, v_h, pos_h))
-        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        dq, dk, dv, dp = (torch.empty_like(t) for t in (q, k, v, pos))
-        dout = torch.empty_like(out)
+        hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        dev_in = [[torch.empty_like(t) for t in (q, k, v, pos)] for _ in range(2)]
+        dev_out = [torch.empty_like(out) for _ in range(2)]
+        copy_stream = torch.cuda.Stream(dev)
+        uploaded = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dp.copy_(hp, non_blocking=True)
-            fn(dq, dk, dv, dp, dout, S=w.S, T=w.T, kv_down=w.kv_down)
-            hout.copy_(dout, non_blocking=True)
+        def upload(i):
+            b = i % 2
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(computed[b])  # buffer b's previous step is done
+                for d, hsrc in zip(dev_in[b], (hq, hk, hv, hp)):
+                    d.copy_(hsrc, non_blocking=True)
+                uploaded[b].record(copy_stream)
 
-        for _ in range(2):
-            e2e_step()
+        def compute(i):
+            b = i % 2
+            stream.wait_event(uploaded[b])
+            dq, dk, dv, dp = dev_in[b]
+            fn(dq, dk, dv, dp, dev_out[b], S=w.S, T=w.T, kv_down=w.kv_down)
+            hout[b].copy_(dev_out[b], non_blocking=True)
+            computed[b].record(stream)
+
+        def run_e2e(n):
+            copy_stream.wait_stream(stream)  # no upload starts before the start event
+            upload(0)
+            for i in range(n):
+                if i + 1 < n:
+                    upload(i + 1)
+                compute(i)
+
+        for b in range(2):
+            computed[b].record(stream)
+        run_e2e(3)
         torch.cuda.synchronize(dev)
         n_e2e = max(3, min(args.steps, 30))
         barrier(world, dev)
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
+        run_e2e(n_e2e)
+        stream.wait_stream(copy_stream)
         x1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, dev) / n_e2e
         e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size(),
-               "ms_per_step": e2e_ms}
+               "ms_per_step": e2e_ms, "overlap": "uploads double-buffered on a copy stream"}
 
     status2 = F.vggt_get_device_status()
 

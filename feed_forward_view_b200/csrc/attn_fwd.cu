@@ -198,19 +198,29 @@ __device__ __forceinline__ float row_max80(const float (&s)[kBN]) {
 // p = 2^(s * log2(e)/8 - m) for 80 scores, packed to bf16 pairs in pk.
 // kMixed: share the exponentials between the FMA pipe and MUFU; otherwise
 // MUFU only (blocks with masked -inf scores). Written in phases over all 40
-// pairs (exponents, then each polynomial step for every FMA-pipe pair, then
-// the MUFU pairs, then the packing), so that long runs of independent
-// instructions hide the latency of each step.
+// pairs -- exponents, every MUFU ex2, then each polynomial step for every
+// FMA-pipe pair, then the packing -- so that long runs of independent
+// instructions hide the latency of each step (the MUFU results are not
+// needed until the end).
 template <bool kMixed>
 __device__ __forceinline__ void exp_pack_row(const float (&s)[kBN], float m, uint32_t (&pk)[kBN / 2]) {
     constexpr int kPairs = kBN / 2;
     const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
     const uint64_t negm2 = f2_pack(-m, -m);
+    auto on_fma = [](int c) { return kMixed && (c & 7) < kExp2OnFma; };
     uint64_t x[kPairs];
 #pragma unroll
     for (int c = 0; c < kPairs; ++c) x[c] = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, negm2);
-    auto on_fma = [](int c) { return kMixed && (c & 7) < kExp2OnFma; };
-    // FMA pipe: x = j + f, 2^x = p(f) * 2^j (see exp2_fma_pair), step by step.
+    float p[kBN];
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c)
+        if (!on_fma(c)) {
+            float x0, x1;
+            f2_unpack(x[c], x0, x1);
+            p[2 * c] = ex2_approx(x0);
+            p[2 * c + 1] = ex2_approx(x1);
+        }
+    // FMA pipe: x = j + f, 2^x = p(f) * 2^j (see above), one step at a time.
     uint64_t tt[kPairs], ff[kPairs];
 #pragma unroll
     for (int c = 0; c < kPairs; ++c)
@@ -231,22 +241,16 @@ __device__ __forceinline__ void exp_pack_row(const float (&s)[kBN], float m, uin
     for (int c = 0; c < kPairs; ++c)
         if (on_fma(c)) x[c] = f2_fma(x[c], ff[c], f2_pack(kExp2C0, kExp2C0));
 #pragma unroll
-    for (int c = 0; c < kPairs; ++c) {
-        float p0, p1;
+    for (int c = 0; c < kPairs; ++c)
         if (on_fma(c)) {
             uint32_t q0, q1, t0, t1;
             u2_unpack(x[c], q0, q1);
             u2_unpack(tt[c], t0, t1);
-            p0 = __uint_as_float(q0 + (t0 << 23));
-            p1 = __uint_as_float(q1 + (t1 << 23));
-        } else {
-            float x0, x1;
-            f2_unpack(x[c], x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+            p[2 * c] = __uint_as_float(q0 + (t0 << 23));
+            p[2 * c + 1] = __uint_as_float(q1 + (t1 << 23));
         }
-        pk[c] = pack_bf16x2(p0, p1);
-    }
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

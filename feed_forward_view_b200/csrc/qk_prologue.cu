@@ -43,66 +43,102 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&b);
 }
 
-__device__ __forceinline__ void process_token(const PrologueJob& job, int t, int H, int lane,
-                                              float my_freq) {
-    // --- angles: lane l -> (half l/16, frequency l%16)
+// Up to 16 heads of one token per pass: the lane's two 8-byte pieces of every
+// head group are loaded before any arithmetic, so each warp keeps 2 KB of
+// loads in flight.
+constexpr int kMaxGroups = 4;
+
+struct TokenLoad {
+    uint2 w1[kMaxGroups], w2[kMaxGroups];
+};
+
+__device__ __forceinline__ void load_token(const PrologueJob& job, int t, int H, int h0, int lane,
+                                           int d1, TokenLoad& ld) {
+    const uint16_t* xt = job.x + static_cast<size_t>(t) * H * kHeadDim;
+#pragma unroll
+    for (int g = 0; g < kMaxGroups; ++g) {
+        const int h = h0 + 4 * g + (lane >> 3);
+        ld.w1[g] = make_uint2(0, 0);
+        ld.w2[g] = make_uint2(0, 0);
+        if (h < H) {
+            ld.w1[g] = __ldg(reinterpret_cast<const uint2*>(xt + h * kHeadDim + d1));
+            ld.w2[g] = __ldg(reinterpret_cast<const uint2*>(xt + h * kHeadDim + d1 + 16));
+        }
+    }
+}
+
+// LayerNorm + rotation of one head group (8 lanes = one head), stored
+// head-major. Every lane runs it (the shuffles need the whole warp); lanes
+// past the last head (live == false) hold zeros and store nothing.
+__device__ __forceinline__ void finish_group(const PrologueJob& job, int t, int h, bool live, int d1,
+                                             uint2 w1, uint2 w2, const float (&sv)[4],
+                                             const float (&cv)[4]) {
+    float x1[4] = {bf16_lo(w1.x), bf16_hi(w1.x), bf16_lo(w1.y), bf16_hi(w1.y)};
+    float x2[4] = {bf16_lo(w2.x), bf16_hi(w2.x), bf16_lo(w2.y), bf16_hi(w2.y)};
+    float sum = (x1[0] + x1[1]) + (x1[2] + x1[3]) + ((x2[0] + x2[1]) + (x2[2] + x2[3]));
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+    const float mean = sum * (1.0f / kHeadDim);
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x1[i] -= mean;
+        x2[i] -= mean;
+        sq = fmaf(x1[i], x1[i], sq);
+        sq = fmaf(x2[i], x2[i], sq);
+    }
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 4);
+    const float rstd = rsqrtf(sq * (1.0f / kHeadDim) + kEps);
+    float o1[4], o2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float y1 = x1[i] * rstd, y2 = x2[i] * rstd;
+        o1[i] = y1 * cv[i] - y2 * sv[i];
+        o2[i] = y2 * cv[i] + y1 * sv[i];
+    }
+    if (live) {
+        uint16_t* dst = job.x_hat + (static_cast<size_t>(h) * job.n + t) * kHeadDim;
+        *reinterpret_cast<uint2*>(dst + d1) = make_uint2(pack2(o1[0], o1[1]), pack2(o1[2], o1[3]));
+        *reinterpret_cast<uint2*>(dst + d1 + 16) =
+            make_uint2(pack2(o2[0], o2[1]), pack2(o2[2], o2[3]));
+    }
+}
+
+// (sin, cos) of the token's 8 angles this lane needs: lane l computes the
+// pair of (half l/16, frequency l%16) and the values are shuffled to the lanes
+// that own those dims.
+__device__ __forceinline__ void token_angles(const PrologueJob& job, int t, int lane, float my_freq,
+                                             float (&sv)[4], float (&cv)[4]) {
     const float2 p = reinterpret_cast<const float2*>(job.pos)[t];
     const float my_pos = (lane < 16) ? p.x : p.y;
     float sn, cs;
     sincosf(my_pos * my_freq, &sn, &cs);
-
-    const int sub = lane & 7;     // position inside the head's 8-lane group
-    const int a = sub >> 2;       // half
-    const int u = sub & 3;        // quarter of the half
-    float sv[4], cv[4];
+    const int sub = lane & 7, a = sub >> 2, u = sub & 3;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int src = a * 16 + 4 * u + i;
         sv[i] = __shfl_sync(0xFFFFFFFFu, sn, src);
         cv[i] = __shfl_sync(0xFFFFFFFFu, cs, src);
     }
+}
 
-    const int d1 = a * 32 + 4 * u;  // first dim of the x1 group; x2 at d1 + 16
-    const uint16_t* xt = job.x + static_cast<size_t>(t) * H * kHeadDim;
-    for (int hg = 0; hg < H; hg += 4) {
-        const int h = hg + (lane >> 3);
-        const bool live = h < H;
-        uint2 w1 = make_uint2(0, 0), w2 = make_uint2(0, 0);
-        if (live) {
-            w1 = *reinterpret_cast<const uint2*>(xt + h * kHeadDim + d1);
-            w2 = *reinterpret_cast<const uint2*>(xt + h * kHeadDim + d1 + 16);
-        }
-        float x1[4] = {bf16_lo(w1.x), bf16_hi(w1.x), bf16_lo(w1.y), bf16_hi(w1.y)};
-        float x2[4] = {bf16_lo(w2.x), bf16_hi(w2.x), bf16_lo(w2.y), bf16_hi(w2.y)};
-        float sum = (x1[0] + x1[1]) + (x1[2] + x1[3]) + ((x2[0] + x2[1]) + (x2[2] + x2[3]));
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-        const float mean = sum * (1.0f / kHeadDim);
-        float sq = 0.f;
+__device__ __forceinline__ void process_token(const PrologueJob& job, int t, int H, int lane,
+                                              float my_freq) {
+    const int sub = lane & 7;
+    const int d1 = (sub >> 2) * 32 + 4 * (sub & 3);  // first dim of the x1 group; x2 at d1 + 16
+    for (int h0 = 0; h0 < H; h0 += 4 * kMaxGroups) {
+        TokenLoad ld;
+        load_token(job, t, H, h0, lane, d1, ld);
+        float sv[4], cv[4];
+        token_angles(job, t, lane, my_freq, sv, cv);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x1[i] -= mean;
-            x2[i] -= mean;
-            sq = fmaf(x1[i], x1[i], sq);
-            sq = fmaf(x2[i], x2[i], sq);
-        }
-        sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
-        sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
-        sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 4);
-        const float rstd = rsqrtf(sq * (1.0f / kHeadDim) + kEps);
-        float o1[4], o2[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float y1 = x1[i] * rstd, y2 = x2[i] * rstd;
-            o1[i] = y1 * cv[i] - y2 * sv[i];
-            o2[i] = y2 * cv[i] + y1 * sv[i];
-        }
-        if (live) {
-            uint16_t* dst = job.x_hat + (static_cast<size_t>(h) * job.n + t) * kHeadDim;
-            *reinterpret_cast<uint2*>(dst + d1) = make_uint2(pack2(o1[0], o1[1]), pack2(o1[2], o1[3]));
-            *reinterpret_cast<uint2*>(dst + d1 + 16) =
-                make_uint2(pack2(o2[0], o2[1]), pack2(o2[2], o2[3]));
+        for (int g = 0; g < kMaxGroups; ++g) {
+            const int h = h0 + 4 * g + (lane >> 3);
+            if (h0 + 4 * g < H)  // warp-uniform
+                finish_group(job, t, h, h < H, d1, ld.w1[g], ld.w2[g], sv, cv);
         }
     }
 }
