@@ -21,7 +21,7 @@ using vggt::PrologueJob;
 constexpr long long kDefaultWaitLimit = 1LL << 32;  // SM cycles (~2 s at 2 GHz)
 constexpr int kMaxDevices = 64;
 
-__device__ int g_device_status;  // non-zero once a bounded device wait ran out
+__device__ int g_device_status;  // kStatusTimeout / kStatusRange bits, 0 when clear
 
 struct DeviceState {
     int* status = nullptr;  // device address of g_device_status
@@ -239,7 +239,7 @@ int vggt_get_device_status(cudaStream_t stream) {
         const int zero = 0;
         if (cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
             return VGGT_ERR_CUDA;
-        return VGGT_ERR_TIMEOUT;
+        return (h & vggt::kStatusTimeout) ? VGGT_ERR_TIMEOUT : VGGT_ERR_RANGE;
     }
     return VGGT_OK;
 }
@@ -253,6 +253,9 @@ const char* vggt_status_string(int status) {
         case VGGT_ERR_ALLOC: return "VGGT_ERR_ALLOC: scratch allocation failed";
         case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA: CUDA call or launch failed";
         case VGGT_ERR_TIMEOUT: return "VGGT_ERR_TIMEOUT: a bounded device wait ran out";
+        case VGGT_ERR_RANGE:
+            return "VGGT_ERR_RANGE: an attention row sum was not a positive finite number "
+                   "(q_hat/k_hat outside the core's norm bound)";
         default: return "unknown vggt_status";
     }
 }

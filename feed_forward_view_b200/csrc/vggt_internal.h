@@ -11,6 +11,10 @@ namespace vggt {
 constexpr int kNSpecial = 5;
 constexpr int kHeadDim = 64;
 
+// Bits of the device status word.
+constexpr int kStatusTimeout = 1;  // a bounded device wait ran out
+constexpr int kStatusRange = 2;    // an attention row sum was not a positive finite number
+
 // One tensor to normalise and rotate: x [n, H, 64] token-major in, x_hat
 // [H, n, 64] head-major out, positions pos [n, 2] (row, col).
 struct PrologueJob {

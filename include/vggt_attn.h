@@ -67,7 +67,11 @@ typedef enum vggt_status {
                                   size beyond the library's limits                */
     VGGT_ERR_ALLOC = -4,       /* scratch allocation failed                        */
     VGGT_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed             */
-    VGGT_ERR_TIMEOUT = -6      /* a bounded device-side wait ran out (reported by
+    VGGT_ERR_TIMEOUT = -6,     /* a bounded device-side wait ran out (reported by
+                                  vggt_get_device_status)                          */
+    VGGT_ERR_RANGE = -7        /* an attention row's softmax sum was not a positive
+                                  finite number: vggt_attn_core was given vectors
+                                  outside its norm bound (reported by
                                   vggt_get_device_status)                          */
 } vggt_status;
 
@@ -132,6 +136,14 @@ VGGT_API int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x
  * Frame attention is n_seg = S, q_len = k_len = T; global attention is
  * n_seg = 1, q_len = k_len = S*T. Takes no scratch. n_seg, q_len or k_len
  * == 0, or H == 0, is a no-op.
+ * Norm bound: the softmax is evaluated as exp(score) with no row maximum
+ * subtracted, which is exact up to rounding because softmax ignores a common
+ * factor, and safe because the prologue's vectors have norm below 8 (so
+ * |score| < 8). Every head vector of q_hat and k_hat must have Euclidean norm
+ * at most 16 (|score| <= 32, exponentials within 2^+-46); beyond that the
+ * fp32/bf16 exponentials and sums may overflow. A row whose sum of exponentials is not a positive finite number
+ * sets VGGT_ERR_RANGE for vggt_get_device_status (best effort: results of
+ * out-of-bound inputs are undefined either way).
  */
 VGGT_API int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
                             vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
@@ -185,8 +197,10 @@ VGGT_API int vggt_attn_global_noalloc(const vggt_bf16* q, const vggt_bf16* k, co
 VGGT_API int vggt_kv_pool_tokens(int T, int kv_down);
 
 /* Synchronises `stream`, then returns and clears the device status word of
-   the current device: VGGT_OK, or VGGT_ERR_TIMEOUT when a bounded device wait
-   ran out since the last call; VGGT_ERR_CUDA if the synchronisation failed. */
+   the current device: VGGT_OK; VGGT_ERR_TIMEOUT when a bounded device wait
+   ran out since the last call; else VGGT_ERR_RANGE when an attention row sum
+   was out of range (see vggt_attn_core); VGGT_ERR_CUDA if the
+   synchronisation failed. */
 VGGT_API int vggt_get_device_status(cudaStream_t stream);
 
 /* Human-readable name of a vggt_status value (static storage). */

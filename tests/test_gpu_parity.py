@@ -235,3 +235,54 @@ def test_bounded_wait_reports_timeout_and_context_survives(F):
     finally:
         F.vggt_set_wait_limit(prev)
     check_attention(F, "global", 1, 15, 1, seed=17)
+
+
+def _head_major(x: torch.Tensor) -> torch.Tensor:
+    """[N, H, D] token-major -> [H, N, D] head-major, contiguous."""
+    return x.permute(1, 0, 2).contiguous()
+
+
+def test_core_scores_at_the_norm_bound(F):
+    # The kernel takes exp(score) with no row maximum subtracted; the LayerNorm
+    # caps |q_hat| and |k_hat| at 8, so the scores of prologue outputs lie in
+    # [-8, 8]. Sweep the keys across that whole range: every query is 7.99 u
+    # (u a unit vector per head) and key j is 7.99 (cos a_j u + sin a_j w_j)
+    # with a_j evenly spaced in [0, pi] and w_j orthogonal to u, so the
+    # scores run from +7.98 to -7.98 and one row's weights span e^16
+    # (about 2^23). The oracle's max-subtracted softmax must agree.
+    gen = torch.Generator().manual_seed(31)
+    H, nq, nk = 2, 200, 520
+    u = torch.randn(H, 64, generator=gen, dtype=torch.float64)
+    u = u / u.norm(dim=-1, keepdim=True)
+    w = torch.randn(nk, H, 64, generator=gen, dtype=torch.float64)
+    w = w - (w * u).sum(-1, keepdim=True) * u
+    w = w / w.norm(dim=-1, keepdim=True)
+    a = torch.linspace(0.0, np.pi, nk, dtype=torch.float64)[:, None, None]
+    qh = (7.99 * u).expand(nq, H, 64).to(torch.bfloat16)
+    kh = (7.99 * (torch.cos(a) * u + torch.sin(a) * w)).to(torch.bfloat16)
+    v = torch.randn(nk, H, 64, generator=gen).to(torch.bfloat16)
+    out = torch.empty(nq, H, 64, dtype=torch.bfloat16, device="cuda")
+    F.vggt_attn_core(_head_major(qh).cuda(), _head_major(kh).cuda(), v.cuda(), out, 1, nq, nk, H=H)
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    ref = O.cross_attention(f64(qh), f64(kh), f64(v))
+    s_max = float((f64(qh)[0] * f64(kh)).sum(-1).max() / 8.0)
+    assert s_max > 7.9  # the sweep really reaches the edge
+    mx, rf = errors(f64(out.cpu()), ref)
+    assert mx <= MAX_ABS and rf <= REL_FRO, (mx, rf)
+
+
+def test_core_reports_inputs_beyond_the_norm_bound(F):
+    # Vectors far outside the core's bound (norm ~1600): the exponentials
+    # overflow, the kernel flags it in the status word without faulting, and
+    # the next read finds the word clear again.
+    S, g = 1, 10
+    q, k, v, pos = synth.make_qkv(S, g, seed=32)
+    qd, kd_, vd, pd = (t.cuda() for t in (q, k, v, pos))
+    qh = F.vggt_qk_prologue(qd, pd)
+    kh = F.vggt_qk_prologue(kd_, pd)
+    out = torch.empty_like(qd)
+    F.vggt_attn_core((qh.float() * 200.0).to(torch.bfloat16), kh, vd, out, 1, qd.shape[0], qd.shape[0])
+    assert F.vggt_get_device_status() == -7
+    assert F.vggt_get_device_status() == 0
+    check_attention(F, "global", 1, 10, 1, seed=32)
