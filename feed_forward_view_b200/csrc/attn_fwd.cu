@@ -45,23 +45,29 @@
 // per row, two per column), S_t [256t + 32, +96) (fp32), P_t [256t + 128, +48)
 // (96 bf16), [O_t | l_t] [256t + 176, +80) (fp32).
 //
-// One S buffer suffices: the issuer computes S_{t,j+1} as soon as the softmax
-// warps have *read* S_{t,j} (bar_sfree), at the start of their work on block
-// j, and has that whole block's exponentials to finish it in. PV_{t,j-1} is
-// issued as soon as P_{t,j-1} is written and has the same time to finish
-// before P_{t,j} overwrites P_t (bar_pfree).
+// One S buffer suffices, and the softmax warps and the issuer meet once per
+// block. Right after loading S_{t,j+1} into registers the softmax warps arrive
+// on bar_c[t]: P_{t,j} (written at the end of their previous block) is ready
+// and S_t is free. On that signal the issuer issues PV_{t,j} and S_{t,j+2}
+// back to back. Both have a whole block of exponentials to finish in:
+// PV_{t,j} before P_{t,j+1} overwrites P_t (bar_pfree), S_{t,j+2} before the
+// softmax warps come to block j+2 (bar_s). One handshake per block matters
+// because every instruction of the issuer competes with two busy softmax warps
+// for its scheduler.
 //
-// Issue order for tile t: [Q_t in TMEM, K_0 loaded] S_{t,0}, commit bar_s[t];
-// then for every block j: [S_{t,j} read, K_{j+1} loaded] S_{t,j+1}, commit
-// bar_s[t]; [P_{t,j} written] PV_{t,j}, commit bar_pfree[t] and kv_empty[j's
-// slot]; at the end, commit bar_o[t].
+// bar_c[t] phases: 0 = S_{t,0} read; j + 1 = P_{t,j} written and S_{t,j+1}
+// read (only P_{t,j} for the last block). Issue order for tile t: [Q_t in
+// TMEM, K_0 loaded] S_{t,0}; [bar_c 0, K_1 loaded] S_{t,1}; then for every
+// block j: [bar_c j+1] PV_{t,j}, commit bar_pfree[t] and kv_empty[j's slot];
+// [K_{j+2} loaded] S_{t,j+2}, commit bar_s[t]; at the end, commit bar_o[t].
 //
 // Barrier phases: a parity wait is unambiguous only while the barrier is at
-// most one phase away from the awaited one, in either direction. The per-tile
-// barriers complete once per block and strictly alternate with their
-// counterpart (bar_s / bar_sfree, bar_p / bar_pfree): neither side can get a
-// second phase ahead. The K/V ring: slot s is refilled only after both tiles
-// committed kv_empty for its previous block.
+// most one phase away from the awaited one, in either direction. bar_c,
+// bar_s and bar_pfree each complete once per step and the two sides advance
+// in lock step: bar_c phase j + 2 needs S_{t,j+2}, which the issuer issues
+// only after seeing phase j + 1; bar_s and bar_pfree phases follow issues that
+// each need the previous bar_c phase. The K/V ring: slot s is refilled only
+// after both tiles committed kv_empty for its previous block.
 //
 // Every wait is bounded; on timeout the CTA records the timeout in the device
 // status word, stops issuing work, drains what it has in flight and frees its
@@ -125,8 +131,7 @@ struct SharedStorage {
     uint64_t bar_kvempty[kStages];
     uint64_t bar_q[2];      // [tile]: Q_t copied into TMEM
     uint64_t bar_s[2];      // [tile]: S_{t,j} computed
-    uint64_t bar_sfree[2];  // [tile]: S_{t,j} read by the softmax warps
-    uint64_t bar_p[2];      // [tile]: P_{t,j} written
+    uint64_t bar_c[2];      // [tile]: P_{t,j-1} written and S_{t,j} read
     uint64_t bar_pfree[2];  // [tile]: PV_{t,j} finished (P_t free, O_t updated)
     uint64_t bar_o[2];      // [tile]: every MMA of the tile finished (once)
     uint32_t tmem_base;
@@ -187,77 +192,90 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
     }
 }
 
-// p = 2^(s * log2(e)/8) for the score pairs [kC0, kC0 + kNP) of a row, packed
-// to bf16 pairs in pk. kMixed: share the exponentials between the FMA pipe and
-// MUFU; otherwise MUFU only (the last block, whose masked scores are -inf).
-// Written in phases over the pairs -- every MUFU ex2 first, then each
-// polynomial step for every FMA-pipe pair, then the packing -- so that runs
-// of independent instructions hide the latency of each step.
+// Which score pairs of a row go to which unit: of every 8 consecutive pairs,
+// the first kExp2OnFma are evaluated on the FMA pipe, the rest with MUFU.
+constexpr int kPairs = kBN / 2;
+constexpr int kFmaPairs = kPairs / 8 * kExp2OnFma;
+constexpr int kMufuPairs = kPairs - kFmaPairs;
+static_assert(kPairs % 8 == 0, "pairs come in groups of 8");
+__device__ __forceinline__ constexpr int fma_pair(int k) {
+    return 8 * (k / kExp2OnFma) + k % kExp2OnFma;
+}
+__device__ __forceinline__ constexpr int mufu_pair(int k) {
+    return 8 * (k / (8 - kExp2OnFma)) + kExp2OnFma + k % (8 - kExp2OnFma);
+}
+
+// p = 2^(s * log2(e)/8) for all kBN scores of a row, packed to bf16 pairs.
 //
 // 2^x on the FMA pipe, x = s * log2(e)/8 in [-125, 125]: t = x + 1.5 * 2^23
 // rounds x to the nearest integer j and leaves j in the low mantissa bits of
 // t; -j = 1.5 * 2^23 - t exactly; f = x - j (one fused multiply-add from s,
 // so |f| <= 1/2 up to one rounding); 2^x = p(f) * 2^j, with 2^j applied by
-// adding j << 23 to the bit pattern of p(f).
-template <bool kMixed, int kC0, int kNP>
-__device__ __forceinline__ void exp_pack_pairs(const float (&s)[kBN], uint32_t (&pk)[kBN / 2]) {
+// adding j << 23 to the bit pattern of p(f). Six packed FMAs per pair.
+//
+// Instruction order. A warp issues in order; MUFU accepts one warp-wide ex2
+// every 8 cycles and a packed FMA holds the FMA pipe for 2. Emitting all the
+// MUFU work of a row and then all the polynomial work would leave one unit
+// idle at a time. Instead the row is software-pipelined: step k issues the
+// ex2 pair of MUFU pair k, then stage d of FMA pair k - d for every stage
+// d = 6..0 in flight, then packs MUFU pair k - 2 (whose results have landed
+// by then). Every step feeds both units, and each value is used a step after
+// it was produced, which hides the units' latencies.
+__device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kBN], uint32_t (&pk)[kPairs]) {
     const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
     const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
-    auto on_fma = [](int c) { return kMixed && (c & 7) < kExp2OnFma; };
-    float p[2 * kNP];
+    constexpr int kStagesFma = 7;  // t, -j, f, three Horner steps, combine + pack
+    constexpr int kSteps = (kMufuPairs + 2 > kFmaPairs + kStagesFma - 1)
+                               ? kMufuPairs + 2
+                               : kFmaPairs + kStagesFma - 1;
+    float p[kBN];
+    uint64_t tt[kFmaPairs > 0 ? kFmaPairs : 1], ff[kFmaPairs > 0 ? kFmaPairs : 1],
+        y[kFmaPairs > 0 ? kFmaPairs : 1];
 #pragma unroll
-    for (int i = 0; i < kNP; ++i) {
-        const int c = kC0 + i;
-        if (!on_fma(c)) {
+    for (int k = 0; k < kSteps; ++k) {
+        if (k < kMufuPairs) {
+            const int c = mufu_pair(k);
             float x0, x1;
             f2_unpack(f2_mul(f2_pack(s[2 * c], s[2 * c + 1]), scale2), x0, x1);
-            p[2 * i] = ex2_approx(x0);
-            p[2 * i + 1] = ex2_approx(x1);
+            p[2 * c] = ex2_approx(x0);
+            p[2 * c + 1] = ex2_approx(x1);
+        }
+#pragma unroll
+        for (int d = kStagesFma - 1; d >= 0; --d) {
+            const int i = k - d;
+            if (i < 0 || i >= kFmaPairs) continue;
+            const int c = fma_pair(i);
+            switch (d) {
+                case 0: tt[i] = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, magic2); break;
+                case 1: ff[i] = f2_fma(tt[i], f2_pack(-1.0f, -1.0f), magic2); break;  // -j
+                case 2: ff[i] = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, ff[i]); break;  // f
+                case 3: y[i] = f2_fma(f2_pack(kExp2C3, kExp2C3), ff[i], f2_pack(kExp2C2, kExp2C2)); break;
+                case 4: y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C1, kExp2C1)); break;
+                case 5: y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C0, kExp2C0)); break;
+                default: {
+                    uint32_t q0, q1, t0, t1;
+                    u2_unpack(y[i], q0, q1);
+                    u2_unpack(tt[i], t0, t1);
+                    pk[c] = pack_bf16x2(__uint_as_float(q0 + (t0 << 23)), __uint_as_float(q1 + (t1 << 23)));
+                }
+            }
+        }
+        if (k >= 2 && k - 2 < kMufuPairs) {
+            const int c = mufu_pair(k - 2);
+            pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
         }
     }
-    uint64_t tt[kNP], ff[kNP], y[kNP];
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i))
-            tt[i] = f2_fma(f2_pack(s[2 * (kC0 + i)], s[2 * (kC0 + i) + 1]), scale2, magic2);
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i)) ff[i] = f2_fma(tt[i], f2_pack(-1.0f, -1.0f), magic2);  // -j
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i))
-            ff[i] = f2_fma(f2_pack(s[2 * (kC0 + i)], s[2 * (kC0 + i) + 1]), scale2, ff[i]);  // f
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i)) y[i] = f2_fma(f2_pack(kExp2C3, kExp2C3), ff[i], f2_pack(kExp2C2, kExp2C2));
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i)) y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C1, kExp2C1));
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i)) y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C0, kExp2C0));
-#pragma unroll
-    for (int i = 0; i < kNP; ++i)
-        if (on_fma(kC0 + i)) {
-            uint32_t q0, q1, t0, t1;
-            u2_unpack(y[i], q0, q1);
-            u2_unpack(tt[i], t0, t1);
-            p[2 * i] = __uint_as_float(q0 + (t0 << 23));
-            p[2 * i + 1] = __uint_as_float(q1 + (t1 << 23));
-        }
-#pragma unroll
-    for (int i = 0; i < kNP; ++i) pk[kC0 + i] = pack_bf16x2(p[2 * i], p[2 * i + 1]);
 }
 
-// The whole row of kBN scores, 16 pairs at a time (keeps the live registers
-// of the polynomial steps bounded).
-template <bool kMixed>
-__device__ __forceinline__ void exp_pack_row(const float (&s)[kBN], uint32_t (&pk)[kBN / 2]) {
-    static_assert(kBN % 32 == 0 && kBN <= 128, "the row is processed in chunks of 16 pairs");
-    exp_pack_pairs<kMixed, 0, 16>(s, pk);
-    if constexpr (kBN / 2 > 16) exp_pack_pairs<kMixed, 16, 16>(s, pk);
-    if constexpr (kBN / 2 > 32) exp_pack_pairs<kMixed, 32, 16>(s, pk);
-    if constexpr (kBN / 2 > 48) exp_pack_pairs<kMixed, 48, 16>(s, pk);
+// MUFU only: the last block, whose masked scores are -inf (2^-inf = 0).
+__device__ __forceinline__ void exp_pack_row_mufu(const float (&s)[kBN], uint32_t (&pk)[kPairs]) {
+    const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c) {
+        float x0, x1;
+        f2_unpack(f2_mul(f2_pack(s[2 * c], s[2 * c + 1]), scale2), x0, x1);
+        pk[c] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -291,8 +309,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t bar_kvempty0 = smem_u32(&sm.bar_kvempty[0]);
     const uint32_t bar_q0 = smem_u32(&sm.bar_q[0]);
     const uint32_t bar_s0 = smem_u32(&sm.bar_s[0]);
-    const uint32_t bar_sfree0 = smem_u32(&sm.bar_sfree[0]);
-    const uint32_t bar_p0 = smem_u32(&sm.bar_p[0]);
+    const uint32_t bar_c0 = smem_u32(&sm.bar_c[0]);
     const uint32_t bar_pfree0 = smem_u32(&sm.bar_pfree[0]);
     const uint32_t bar_o0 = smem_u32(&sm.bar_o[0]);
     const uint32_t kv_smem0 = smem_u32(sm.kv[0][0]);
@@ -301,8 +318,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     auto bar_kvempty = [&](int s) { return bar_kvempty0 + 8u * s; };
     auto bar_q = [&](int t) { return bar_q0 + 8u * t; };
     auto bar_s = [&](int t) { return bar_s0 + 8u * t; };
-    auto bar_sfree = [&](int t) { return bar_sfree0 + 8u * t; };
-    auto bar_p = [&](int t) { return bar_p0 + 8u * t; };
+    auto bar_c = [&](int t) { return bar_c0 + 8u * t; };
     auto bar_pfree = [&](int t) { return bar_pfree0 + 8u * t; };
     auto bar_o = [&](int t) { return bar_o0 + 8u * t; };
     auto k_smem = [&](int s) { return kv_smem0 + static_cast<uint32_t>(2 * kKVTileBytes) * s; };
@@ -327,8 +343,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar_q(t), 4);  // one arrival per softmax warp
             mbar_init(bar_s(t), 1);
-            mbar_init(bar_sfree(t), 4);
-            mbar_init(bar_p(t), 4);
+            mbar_init(bar_c(t), 4);
             mbar_init(bar_pfree(t), 1);
             mbar_init(bar_o(t), 1);
         }
@@ -402,16 +417,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             };
             bool ok = uwait(bar_q(t), 0) && uwait(bar_kvfull(0), 0);
             if (ok) issue_s(0);
+            // Phase 0 (S_{t,0} read) is consumed even when there is no S_{t,1}:
+            // the loop below waits on phases 1, 2, ... by parity.
+            ok = ok && uwait(bar_c(t), 0);
+            if (ok && nkb > 1) {
+                ok = uwait(bar_kvfull(1 % kStages), (1 / kStages) & 1);
+                if (ok) issue_s(1);
+            }
             for (int j = 0; ok && j < nkb; ++j) {
                 const int s = j % kStages;
-                const int jn = j + 1;
-                if (jn < nkb) {
-                    // S_t is free once the softmax warps have read S_{t,j}.
-                    if (!uwait(bar_sfree(t), j & 1)) break;
-                    if (!uwait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
-                    issue_s(jn);
-                }
-                if (!uwait(bar_p(t), j & 1)) break;
+                if (!uwait(bar_c(t), (j + 1) & 1)) break;
                 // [O_t | l_t] (+)= P_{t,j} [V_j | 1]: 6 steps of 16 keys. The B
                 // operand's second 64-column block (the ones tile) lies a
                 // leading byte offset away from the V slot.
@@ -432,6 +447,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     mma_commit(empty);  // K_j and V_j no longer needed by this tile
                 }
                 __syncwarp();
+                const int jn = j + 2;
+                if (jn < nkb) {
+                    if (!uwait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
+                    issue_s(jn);
+                }
             }
             // Completes once every MMA of this tile has finished: the softmax
             // warps wait on it before the epilogue; it doubles as the drain.
@@ -490,18 +510,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                     for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
                 }
-                // The scores are in registers: S_t may take S_{t,j+1}.
+                // The scores are in registers and P_{t,j-1} is in TMEM: S_t may
+                // take S_{t,j+2} and PV_{t,j-1} may run.
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_sfree(t));
+                if (lane == 0) mbar_arrive(bar_c(t));
                 uint32_t pk[kBN / 2];
                 if (j == nkb - 1 && last_valid < kBN) {
 #pragma unroll
                     for (int c = 0; c < kBN; ++c)
                         if (c >= last_valid) s[c] = -INFINITY;
-                    exp_pack_row<false>(s, pk);
+                    exp_pack_row_mufu(s, pk);
                 } else {
-                    exp_pack_row<true>(s, pk);
+                    exp_pack_row_mixed(s, pk);
                 }
                 // P_t is free once PV_{t,j-1} has finished.
                 if (j > 0 && !wait(bar_pfree(t), (j - 1) & 1)) {
@@ -510,9 +531,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
                 tc_fence_after();
                 tmem_st48(lane_base + col_p(t), pk);
+            }
+            if (ok) {
+                // P of the last block is in TMEM (there is no next S to read).
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_p(t));
+                if (lane == 0) mbar_arrive(bar_c(t));
             }
             if (ok && wait(bar_o(t), 0)) {
                 tc_fence_after();
