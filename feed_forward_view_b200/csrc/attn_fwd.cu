@@ -426,6 +426,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             for (int j = 0; ok && j < nkb; ++j) {
                 const int s = j % kStages;
+                const int jn = j + 2;
+                // K_{j+2} has long landed by now (the ring runs kStages blocks
+                // ahead): check it first, so that once the softmax warps signal,
+                // PV_{t,j} and S_{t,j+2} go to the tensor core back to back.
+                if (jn < nkb && !uwait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
                 if (!uwait(bar_c(t), (j + 1) & 1)) break;
                 // [O_t | l_t] (+)= P_{t,j} [V_j | 1]: 6 steps of 16 keys. The B
                 // operand's second 64-column block (the ones tile) lies a
@@ -447,11 +452,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     mma_commit(empty);  // K_j and V_j no longer needed by this tile
                 }
                 __syncwarp();
-                const int jn = j + 2;
-                if (jn < nkb) {
-                    if (!uwait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
-                    issue_s(jn);
-                }
+                if (jn < nkb) issue_s(jn);
             }
             // Completes once every MMA of this tile has finished: the softmax
             // warps wait on it before the epilogue; it doubles as the drain.
