@@ -290,15 +290,23 @@ def run_gpu(args):
     def step():
         fn(q, k, v, pos, out, S=w.S, T=w.T, kv_down=w.kv_down)
 
-    # ---- warm-up, then the timed region: K steps between two barriers
-    for _ in range(args.warmup):
+    # ---- warm-up, then the timed region: K steps between two barriers. The
+    # clock sampler starts first; the warm-up (at least W steps, continued until
+    # the sampler has run 0.3 s) keeps the GPU busy meanwhile, so that the timed
+    # steps start at load clocks and not at clocks ramping up from idle.
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_warm = time.perf_counter()
+    warmed = 0
+    while warmed < args.warmup or time.perf_counter() - t_warm < 0.3:
         step()
+        warmed += 1
+        if warmed % 4 == 0:
+            torch.cuda.synchronize(dev)
     torch.cuda.synchronize(dev)
     if F.vggt_get_device_status() != 0:
         raise RuntimeError("device wait timeout during warm-up")
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
+    warmed = int(max_over_ranks(float(warmed), world, dev))  # same count on every rank's line
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -350,6 +358,24 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     pro_ms = p0.elapsed_time(p1) / reps
     pro_bytes = 2 * w.n_q * H * 64 * 2 + w.n_q * 8  # read x + pos, write x_hat
+    pool = None
+    if w.kind == "descriptor":
+        # K/V pooling alone: reads k, v and pos of every token, writes the
+        # pooled k, v and positions.
+        kp_o, vp_o, pp_o = (torch.empty_like(t) for t in (kp, vp, pp))
+        for _ in range(3):
+            F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
+        torch.cuda.synchronize(dev)
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for _ in range(reps):
+            F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
+        k1.record(stream)
+        torch.cuda.synchronize(dev)
+        pool_ms = k0.elapsed_time(k1) / reps
+        pool_bytes = 2 * (w.n_q + w.n_k) * H * 64 * 2 + (w.n_q + w.n_k) * 8
+        pool = {"ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"])}
 
     # ---- end to end through the public call with host buffers: every step
     # uploads its inputs from pinned host memory and reads its output back.
@@ -419,12 +445,14 @@ def run_gpu(args):
     if rank == 0:
         peaks, peak_src = load_peaks()
         attn_tf = flops / (attn_ms * 1e-3) / 1e12
+        scores = flops / (4.0 * w.D)  # query-key pairs x heads
+        sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
         peak = float(peaks["bf16_tflops"])
         traffic = profiled_traffic(w)
         clk = clocks.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "steps": args.steps, "warmup": warmed, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
@@ -440,7 +468,13 @@ def run_gpu(args):
                          "traffic": traffic, "kernel_ms": attn_ms,
                          "share_of_step": attn_ms / ms_step},
             "kernels": {"qk_prologue": {"ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
-                                        "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"])}},
+                                        "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+                        **({"kv_pool": pool} if pool else {})},
+            # every score costs one exponential: exponentials per second in
+            # the attention kernel, and per SM per clock at the sampled clock
+            "exp_per_s": scores / (attn_ms * 1e-3),
+            "exp_per_sm_clk": (scores / (attn_ms * 1e-3) / (sm_count * clk["sm_mhz"] * 1e6)
+                               if clk.get("sm_mhz") else None),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches * args.steps,
@@ -462,7 +496,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--cpu-rows", type=int, default=768)
+    ap.add_argument("--cpu-rows", type=int, default=2048)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle leg")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")

@@ -82,9 +82,14 @@ WORKLOADS = {
     )
 }
 
-# A smaller dense-global case whose inputs (151 MB) still exceed the 126 MB L2,
-# used for hardware-counter captures of the attention kernel.
-PROFILE_WORKLOADS = {w.name: w for w in (Workload("global_s6_g64", "global", S=6, g=64),)}
+# Smaller cases for hardware-counter captures, whose inputs still exceed the
+# 126 MB L2: dense global attention over 24 606 tokens (151 MB of q, k, v) for
+# the attention kernel and the prologue, and 40 frames of the descriptor
+# workload (k and v: 225 MB) for the pooling kernel.
+PROFILE_WORKLOADS = {w.name: w for w in (
+    Workload("global_s6_g64", "global", S=6, g=64),
+    Workload("descriptor_s40_g37_kd4", "descriptor", S=40, g=37, kv_down=4),
+)}
 ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS}
 
 
