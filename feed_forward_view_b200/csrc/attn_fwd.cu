@@ -18,11 +18,18 @@
 //               so shared memory only feeds the K and V tiles and every MMA
 //               runs at the tensor core's full rate even at these small N.
 //   warp 3      idle (completes the first warpgroup).
-//   warps 4-7   softmax for tile 0, warps 8-11 softmax for tile 1: each thread
-//               owns one query row (its TMEM lane). It first copies its row of
-//               q_hat from global memory into TMEM; then, per key block, reads
-//               the row's 96 scores from TMEM, exponentiates them in fp32,
-//               writes P as bf16 to TMEM; finally it normalises O and stores it.
+//   warps 4-11  softmax for tile 0, warps 12-19 for tile 1. A warp may only
+//               reach the 32 TMEM lanes of its lane quarter (warp % 4), so each
+//               quarter of a tile has two warps that split the key columns:
+//               warps 4-7 take score columns 0-47, warps 8-11 columns 48-95
+//               (likewise 12-15 / 16-19). Each thread owns one query row (its
+//               TMEM lane) and half of its columns: it first copies its half of
+//               the row of q_hat from global memory into TMEM; per key block it
+//               reads its 48 scores from TMEM, exponentiates them in fp32 and
+//               writes P as bf16 to TMEM; finally it normalises its 32 of the
+//               64 output dims and stores them. Four softmax warps per scheduler
+//               keep the exponential units busier than two, and fill one warp's
+//               waits with another's work.
 //
 // Softmax without a running maximum. softmax is invariant to a common factor
 // on every p of a row, so p = 2^(score * log2(e)) with score = q.k / 8 is as
@@ -48,18 +55,23 @@
 // One S buffer suffices, and the softmax warps and the issuer meet once per
 // block. Right after loading S_{t,j+1} into registers the softmax warps arrive
 // on bar_c[t]: P_{t,j} (written at the end of their previous block) is ready
-// and S_t is free. On that signal the issuer issues PV_{t,j} and S_{t,j+2}
-// back to back. Both have a whole block of exponentials to finish in:
-// PV_{t,j} before P_{t,j+1} overwrites P_t (bar_pfree), S_{t,j+2} before the
-// softmax warps come to block j+2 (bar_s). One handshake per block matters
-// because every instruction of the issuer competes with two busy softmax warps
-// for its scheduler.
+// and S_t is free; the tile's first softmax warp also checks, before it
+// arrives, that K_{j+2} has landed. On that signal the issuer issues PV_{t,j}
+// and S_{t,j+2} back to back. Both have a whole block of exponentials to
+// finish in: PV_{t,j} before P_{t,j+1} overwrites P_t (bar_pfree), S_{t,j+2}
+// before the softmax warps come to block j+2 (bar_s). The issuer waits on
+// nothing else, because every instruction it executes competes with four busy
+// softmax warps for its scheduler: measured, each extra wait there cost
+// hundreds of cycles per block even when its barrier had long completed.
 //
-// bar_c[t] phases: 0 = S_{t,0} read; j + 1 = P_{t,j} written and S_{t,j+1}
-// read (only P_{t,j} for the last block). Issue order for tile t: [Q_t in
-// TMEM, K_0 loaded] S_{t,0}; [bar_c 0, K_1 loaded] S_{t,1}; then for every
-// block j: [bar_c j+1] PV_{t,j}, commit bar_pfree[t] and kv_empty[j's slot];
-// [K_{j+2} loaded] S_{t,j+2}, commit bar_s[t]; at the end, commit bar_o[t].
+// bar_c[t] phases: 0 = S_{t,0} read (and K_1 loaded); j + 1 = P_{t,j} written,
+// S_{t,j+1} read and K_{j+2} loaded (only P_{t,j} for the last block). Issue
+// order for tile t: [Q_t in TMEM, K_0 loaded] S_{t,0}; [bar_c 0] S_{t,1}; then
+// for every block j: [bar_c j+1] PV_{t,j}, commit bar_pfree[t] and kv_empty[j's
+// slot]; S_{t,j+2}, commit bar_s[t]; at the end, commit bar_o[t]. (K_{j+2}
+// reaches the issuer through a chain: the TMA completes its full barrier, the
+// checking softmax warp observes it and then releases bar_c, the issuer
+// acquires bar_c and only then issues the MMA that reads the tile.)
 //
 // Barrier phases: a parity wait is unambiguous only while the barrier is at
 // most one phase away from the awaited one, in either direction. bar_c,
@@ -86,14 +98,16 @@ constexpr int kBN = 96;                           // keys per block
 constexpr int kStages = 8;                        // K/V ring depth
 constexpr int kKVTileBytes = kBN * kHeadDim * 2;  // 12 KB
 constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum block (16)
-constexpr int kThreads = 384;
-// Register split: 168 per thread at launch (the cap for 12 warps); the
-// TMA/MMA warpgroup gives up to 80, the two softmax warpgroups take 208:
-// 128 * 80 + 256 * 208 = 63488 <= 384 * 168.
-constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kRegsControl = 80;
-constexpr uint32_t kRegsSoftmax = 208;
-static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
+constexpr int kSoftmaxWarps = 16;                 // per CTA: 2 tiles x 4 lane quarters x 2 column halves
+constexpr int kThreads = 128 + 32 * kSoftmaxWarps;  // 640
+constexpr int kCols = kBN / 2;                      // score columns per softmax thread
+// Register split: 96 per thread at launch (the cap for 20 warps); the
+// TMA/MMA warpgroup gives up to 56, the four softmax warpgroups take 104:
+// 128 * 56 + 512 * 104 = 60416 <= 640 * 96.
+constexpr uint32_t kLaunchRegs = 96;
+constexpr uint32_t kRegsControl = 56;
+constexpr uint32_t kRegsSoftmax = 104;
+static_assert(128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 
@@ -111,7 +125,7 @@ constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64
 // kExp2OnFma pairs are evaluated on the FMA pipe (polynomial below) and the
 // rest with the MUFU ex2 instruction, so that the two units share the work.
 #ifndef VGGT_EXP2_ON_FMA_PER8
-#define VGGT_EXP2_ON_FMA_PER8 4
+#define VGGT_EXP2_ON_FMA_PER8 3
 #endif
 constexpr int kExp2OnFma = VGGT_EXP2_ON_FMA_PER8;
 
@@ -194,7 +208,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
 
 // Which score pairs of a row go to which unit: of every 8 consecutive pairs,
 // the first kExp2OnFma are evaluated on the FMA pipe, the rest with MUFU.
-constexpr int kPairs = kBN / 2;
+constexpr int kPairs = kCols / 2;
 constexpr int kFmaPairs = kPairs / 8 * kExp2OnFma;
 constexpr int kMufuPairs = kPairs - kFmaPairs;
 static_assert(kPairs % 8 == 0, "pairs come in groups of 8");
@@ -205,7 +219,7 @@ __device__ __forceinline__ constexpr int mufu_pair(int k) {
     return 8 * (k / (8 - kExp2OnFma)) + kExp2OnFma + k % (8 - kExp2OnFma);
 }
 
-// p = 2^(s * log2(e)/8) for all kBN scores of a row, packed to bf16 pairs.
+// p = 2^(s * log2(e)/8) for a thread's kCols scores, packed to bf16 pairs.
 //
 // 2^x on the FMA pipe, x = s * log2(e)/8 in [-125, 125]: t = x + 1.5 * 2^23
 // rounds x to the nearest integer j and leaves j in the low mantissa bits of
@@ -221,14 +235,14 @@ __device__ __forceinline__ constexpr int mufu_pair(int k) {
 // d = 6..0 in flight, then packs MUFU pair k - 2 (whose results have landed
 // by then). Every step feeds both units, and each value is used a step after
 // it was produced, which hides the units' latencies.
-__device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kBN], uint32_t (&pk)[kPairs]) {
+__device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint32_t (&pk)[kPairs]) {
     const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
     const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
     constexpr int kStagesFma = 7;  // t, -j, f, three Horner steps, combine + pack
     constexpr int kSteps = (kMufuPairs + 2 > kFmaPairs + kStagesFma - 1)
                                ? kMufuPairs + 2
                                : kFmaPairs + kStagesFma - 1;
-    float p[kBN];
+    float p[kCols];
     uint64_t tt[kFmaPairs > 0 ? kFmaPairs : 1], ff[kFmaPairs > 0 ? kFmaPairs : 1],
         y[kFmaPairs > 0 ? kFmaPairs : 1];
 #pragma unroll
@@ -268,7 +282,7 @@ __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kBN], uint32
 }
 
 // MUFU only: the last block, whose masked scores are -inf (2^-inf = 0).
-__device__ __forceinline__ void exp_pack_row_mufu(const float (&s)[kBN], uint32_t (&pk)[kPairs]) {
+__device__ __forceinline__ void exp_pack_row_mufu(const float (&s)[kCols], uint32_t (&pk)[kPairs]) {
     const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
 #pragma unroll
     for (int c = 0; c < kPairs; ++c) {
@@ -341,9 +355,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_init(bar_kvempty(s), ntile);  // one commit per tile issuer
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_q(t), 4);  // one arrival per softmax warp
+            mbar_init(bar_q(t), kSoftmaxWarps / 2);  // one arrival per softmax warp of the tile
             mbar_init(bar_s(t), 1);
-            mbar_init(bar_c(t), 4);
+            mbar_init(bar_c(t), kSoftmaxWarps / 2);
             mbar_init(bar_pfree(t), 1);
             mbar_init(bar_o(t), 1);
         }
@@ -419,18 +433,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (ok) issue_s(0);
             // Phase 0 (S_{t,0} read) is consumed even when there is no S_{t,1}:
             // the loop below waits on phases 1, 2, ... by parity.
+            // bar_c phase j also vouches for K_{j+1}: one softmax warp checks
+            // that block's full barrier before arriving, so the issuer's one
+            // wait per block is this one.
             ok = ok && uwait(bar_c(t), 0);
-            if (ok && nkb > 1) {
-                ok = uwait(bar_kvfull(1 % kStages), (1 / kStages) & 1);
-                if (ok) issue_s(1);
-            }
+            if (ok && nkb > 1) issue_s(1);
             for (int j = 0; ok && j < nkb; ++j) {
                 const int s = j % kStages;
                 const int jn = j + 2;
-                // K_{j+2} has long landed by now (the ring runs kStages blocks
-                // ahead): check it first, so that once the softmax warps signal,
-                // PV_{t,j} and S_{t,j+2} go to the tensor core back to back.
-                if (jn < nkb && !uwait(bar_kvfull(jn % kStages), (jn / kStages) & 1)) break;
                 if (!uwait(bar_c(t), (j + 1) & 1)) break;
                 // [O_t | l_t] (+)= P_{t,j} [V_j | 1]: 6 steps of 16 keys. The B
                 // operand's second 64-column block (the ones tile) lies a
@@ -463,25 +473,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else if (warp >= 4) {
         // ------------------------------------------------------ softmax
         regs_inc<kRegsSoftmax>();
-        const int t = (warp >> 2) - 1;
+        const int t = (warp - 4) >> 3;
+        const int half = ((warp - 4) >> 2) & 1;  // score columns [kCols*half, +kCols)
         const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
         const int row = quarter * 32 + lane;
         if (t < ntile) {
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            // Waits are made warp-uniform with a vote: the tcgen05 loads and
+            // stores after them need the whole warp.
+            auto uwait = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(0xFFFFFFFFu, wait(bar, parity)) != 0;
+            };
             const int row_in_seg = (tile0 + t) * kBM + row;
             const bool row_live = row_in_seg < prm.q_len;
             const long long grow = static_cast<long long>(seg) * prm.q_len + row_in_seg;
-            // Q_t into TMEM: this thread's row of q_hat (64 bf16 = 32 words,
-            // two head dims per word, low half first) into its lane, the
-            // layout the MMA reads an M x K operand in. Rows past the
-            // segment are zeros and never stored.
+            // Q_t into TMEM: this thread's half of its row of q_hat (32 bf16
+            // = 16 words, two head dims per word, low half first) into its
+            // lane, the layout the MMA reads an M x K operand in. Rows past
+            // the segment are zeros and never stored.
             {
-                uint32_t qr[32];
+                uint32_t qr[16];
                 if (row_live) {
                     const uint4* src = reinterpret_cast<const uint4*>(
-                        prm.q_hat + (static_cast<long long>(h) * prm.n_q + grow) * kHeadDim);
+                        prm.q_hat + (static_cast<long long>(h) * prm.n_q + grow) * kHeadDim + 32 * half);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int i = 0; i < 4; ++i) {
                         const uint4 w = __ldg(src + i);
                         qr[4 * i] = w.x;
                         qr[4 * i + 1] = w.y;
@@ -490,48 +506,60 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) qr[i] = 0u;
+                    for (int i = 0; i < 16; ++i) qr[i] = 0u;
                 }
-                tmem_st32(lane_base + col_q(t), qr);
+                tmem_st16(lane_base + col_q(t) + 16 * half, qr);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_q(t));
             }
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
-                if (!wait(bar_s(t), j & 1)) {
+                if (!uwait(bar_s(t), j & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                float s[kBN];
+                float s[kCols];
                 {
-                    uint32_t r[kBN];
-                    tmem_ld96(lane_base + col_s(t), r);
+                    uint32_t r[kCols];
+                    tmem_ld48(lane_base + col_s(t) + kCols * half, r);
 #pragma unroll
-                    for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < kCols; ++i) s[i] = __uint_as_float(r[i]);
                 }
                 // The scores are in registers and P_{t,j-1} is in TMEM: S_t may
-                // take S_{t,j+2} and PV_{t,j-1} may run.
+                // take S_{t,j+1} and PV_{t,j-1} may run. S_{t,j+1} reads K_{j+1}:
+                // the tile's first warp makes sure it has landed before
+                // arriving (the ring runs kStages blocks ahead, so this is
+                // normally satisfied at once), so that a completed bar_c phase
+                // implies it. The issuer, whose every instruction competes with
+                // busy softmax warps for its scheduler, then has one barrier
+                // per block to wait for.
+                if (quarter == 0 && half == 0 && j + 1 < nkb &&
+                    !uwait(bar_kvfull((j + 1) % kStages), ((j + 1) / kStages) & 1)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_c(t));
-                uint32_t pk[kBN / 2];
+                uint32_t pk[kPairs];
                 if (j == nkb - 1 && last_valid < kBN) {
+                    const int valid = last_valid - kCols * half;  // of this thread's columns
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c)
-                        if (c >= last_valid) s[c] = -INFINITY;
+                    for (int c = 0; c < kCols; ++c)
+                        if (c >= valid) s[c] = -INFINITY;
                     exp_pack_row_mufu(s, pk);
                 } else {
                     exp_pack_row_mixed(s, pk);
                 }
                 // P_t is free once PV_{t,j-1} has finished.
-                if (j > 0 && !wait(bar_pfree(t), (j - 1) & 1)) {
+                if (j > 0 && !uwait(bar_pfree(t), (j - 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                tmem_st48(lane_base + col_p(t), pk);
+                tmem_st24(lane_base + col_p(t) + kPairs * half, pk);
             }
             if (ok) {
                 // P of the last block is in TMEM (there is no next S to read).
@@ -539,19 +567,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_c(t));
             }
-            if (ok && wait(bar_o(t), 0)) {
+            if (ok && uwait(bar_o(t), 0)) {
                 tc_fence_after();
-                uint32_t o[kOCols];
-                tmem_ld80(lane_base + col_o(t), o);
-                const float l = __uint_as_float(o[kHeadDim]);  // column 64
+                // This thread's 32 of the 64 output dims, and l (column 64).
+                uint32_t o[33];
+                tmem_ld32_1(lane_base + col_o(t) + 32 * half, lane_base + col_o(t) + kHeadDim, o);
+                const float l = __uint_as_float(o[32]);
                 const float inv = 1.0f / l;
                 if (row_live) {
                     // Inputs outside the core's contract can overflow the
                     // max-free softmax; say so instead of storing silently.
                     if (!(l > 0.0f && l <= 3.0e38f)) atomicOr(prm.status, kStatusRange);
-                    uint4* dst = reinterpret_cast<uint4*>(prm.out + (grow * prm.H + h) * kHeadDim);
+                    uint4* dst = reinterpret_cast<uint4*>(prm.out + (grow * prm.H + h) * kHeadDim + 32 * half);
 #pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4) {
+                    for (int v4 = 0; v4 < 4; ++v4) {
                         uint4 w;
                         w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv,
                                           __uint_as_float(o[8 * v4 + 1]) * inv);
@@ -649,7 +678,7 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
         cudaFuncAttributes fa;
         e = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
         if (e != cudaSuccess) return e;
-        if (static_cast<uint32_t>(fa.numRegs) * kThreads < 128 * kRegsControl + 256 * kRegsSoftmax)
+        if (static_cast<uint32_t>(fa.numRegs) * kThreads < 128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax)
             return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes));
