@@ -119,6 +119,9 @@ __device__ __forceinline__ constexpr uint32_t col_o(int t) { return 256u * t + 1
 static_assert(32 + kBN <= 128 && 128 + kBN / 2 <= 176 && 176 + kOCols <= 256,
               "TMEM columns of one tile overlap");
 
+static_assert(kBN / 16 == 6 && kHeadDim / 16 == 4,
+              "the MMA group helpers issue 6 PV steps and 4 S steps");
+
 constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64)
 
 // Exponentials per key block: of every 8 consecutive score pairs,
@@ -414,55 +417,66 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             };
             // S_{t,j} = Q_t K_j^T: 4 steps of 16 head dims; Q_t's 16 dims are
             // 8 TMEM columns, K_j's 32 bytes of each 128-byte row.
-            auto issue_s = [&](int j) {
-                const uint64_t kdesc = smem_desc_sw128(k_smem(j % kStages), 16, 1024);
-                const uint32_t a = tmem + col_q(t);
-                const uint32_t d = tmem + col_s(t);
-                const uint32_t done = bar_s(t);
+            const uint32_t q_tm = tmem + col_q(t);
+            const uint32_t s_tm = tmem + col_s(t);
+            const uint32_t p_tm = tmem + col_p(t);
+            const uint32_t o_tm = tmem + col_o(t);
+            auto k_descs = [&](int j, uint64_t (&kd)[4]) {
+                const uint64_t base = smem_desc_sw128(k_smem(j % kStages), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) kd[kk] = base + static_cast<uint64_t>((kk * 32) >> 4);
+            };
+            auto issue_s = [&](const uint64_t (&kd)[4]) {
                 if (elect_one()) {
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                        mma_ts(d, a + kk * 8, kdesc + static_cast<uint64_t>((kk * 32) >> 4), idesc_s,
-                               kk > 0 ? 1u : 0u);
-                    mma_commit(done);
+                    mma_ts4_commit(s_tm, q_tm, kd, idesc_s, bar_s(t));
                 }
                 __syncwarp();
             };
             bool ok = uwait(bar_q(t), 0) && uwait(bar_kvfull(0), 0);
-            if (ok) issue_s(0);
+            if (ok) {
+                uint64_t kd[4];
+                k_descs(0, kd);
+                issue_s(kd);
+            }
             // Phase 0 (S_{t,0} read) is consumed even when there is no S_{t,1}:
             // the loop below waits on phases 1, 2, ... by parity.
             // bar_c phase j also vouches for K_{j+1}: one softmax warp checks
             // that block's full barrier before arriving, so the issuer's one
             // wait per block is this one.
             ok = ok && uwait(bar_c(t), 0);
-            if (ok && nkb > 1) issue_s(1);
+            if (ok && nkb > 1) {
+                uint64_t kd[4];
+                k_descs(1, kd);
+                issue_s(kd);
+            }
             for (int j = 0; ok && j < nkb; ++j) {
                 const int s = j % kStages;
                 const int jn = j + 2;
-                if (!uwait(bar_c(t), (j + 1) & 1)) break;
+                // Every operand of this block's MMAs is ready before the wait,
+                // so that once the softmax warps signal, the elected thread
+                // only has the MMAs and commits to emit.
                 // [O_t | l_t] (+)= P_{t,j} [V_j | 1]: 6 steps of 16 keys. The B
                 // operand's second 64-column block (the ones tile) lies a
                 // leading byte offset away from the V slot.
                 const uint32_t vaddr = v_smem(s);
-                const uint64_t vdesc = smem_desc_sw128(vaddr, ones_smem - vaddr, 1024);
-                const uint32_t a = tmem + col_p(t);
-                const uint32_t d = tmem + col_o(t);
-                const uint32_t first = j > 0 ? 1u : 0u;
+                const uint64_t vbase = smem_desc_sw128(vaddr, ones_smem - vaddr, 1024);
+                uint64_t vd[6];
+#pragma unroll
+                for (int kk = 0; kk < 6; ++kk) vd[kk] = vbase + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+                uint64_t kd[4];
+                k_descs(jn, kd);
                 const uint32_t pfree = bar_pfree(t);
                 const uint32_t empty = bar_kvempty(s);
+                if (!uwait(bar_c(t), (j + 1) & 1)) break;
                 if (elect_one()) {
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_ts(d, a + kk * 8, vdesc + static_cast<uint64_t>((kk * 16 * 128) >> 4),
-                               idesc_o, kk > 0 ? 1u : first);
-                    mma_commit(pfree);  // P_t free again, O_t includes block j
-                    mma_commit(empty);  // K_j and V_j no longer needed by this tile
+                    // P_t free again and O_t includes block j; K_j and V_j no
+                    // longer needed by this tile.
+                    mma_ts6_commit2(o_tm, p_tm, vd, idesc_o, j > 0 ? 1u : 0u, pfree, empty);
+                    if (jn < nkb) mma_ts4_commit(s_tm, q_tm, kd, idesc_s, bar_s(t));
                 }
                 __syncwarp();
-                if (jn < nkb) issue_s(jn);
             }
             // Completes once every MMA of this tile has finished: the softmax
             // warps wait on it before the epilogue; it doubles as the drain.

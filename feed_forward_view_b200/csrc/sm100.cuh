@@ -151,6 +151,46 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 
 // Arrives once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
+// Six kind::f16 MMAs with A in TMEM, back to back in one asm block, then two
+// commits: D (+)= sum over k of A_k B_k, A_k at TMEM address a + 8k (16 bf16
+// columns), B_k described by b[k]. The first step accumulates onto D only if
+// acc_first != 0. Every operand is prepared before the block, so the issuing
+// thread emits nothing but the MMAs and their commits.
+__device__ __forceinline__ void mma_ts6_commit2(uint32_t d, uint32_t a, const uint64_t (&b)[6], uint32_t idesc,
+                                                uint32_t acc_first, uint32_t bar0, uint32_t bar1) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t"
+        "setp.ne.b32 pf, %9, 0;\n\t"
+        "setp.eq.b32 pt, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %3, %2, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%10], %4, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%11], %5, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%12], %6, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%13], %7, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%14], %8, %2, pt;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%15];\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%16];\n\t}"
+        ::"r"(d), "r"(a), "r"(idesc), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]),
+        "r"(acc_first), "r"(a + 8), "r"(a + 16), "r"(a + 24), "r"(a + 32), "r"(a + 40), "r"(bar0), "r"(bar1)
+        : "memory");
+}
+// Four kind::f16 MMAs with A in TMEM (D = sum over k of A_k B_k, overwriting
+// D), back to back, then one commit.
+__device__ __forceinline__ void mma_ts4_commit(uint32_t d, uint32_t a, const uint64_t (&b)[4], uint32_t idesc,
+                                               uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t"
+        "setp.ne.b32 pf, %2, %2;\n\t"
+        "setp.eq.b32 pt, %2, %2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %3, %2, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %4, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %5, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %6, %2, pt;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%10];\n\t}"
+        ::"r"(d), "r"(a), "r"(idesc), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+        "r"(a + 8), "r"(a + 16), "r"(a + 24), "r"(bar)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
