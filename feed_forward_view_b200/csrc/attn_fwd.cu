@@ -209,6 +209,17 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
     }
 }
 
+// Two bf16 (low half first) times log2(e)/8, rounded back to bf16 (nearest,
+// ties to even). Scaling Q once per tile saves a multiply per score pair in
+// every key block; the extra rounding (relative 2^-9 per element of Q) moves
+// a score by ~0.002 (log2 units) rms, well inside the rounding P already
+// takes when it is stored as bf16.
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w) {
+    const float lo = __uint_as_float(w << 16) * kScaleLog2;
+    const float hi = __uint_as_float(w & 0xFFFF0000u) * kScaleLog2;
+    return pack_bf16x2(lo, hi);
+}
+
 // Which score pairs of a row go to which unit: of every 8 consecutive pairs,
 // the first kExp2OnFma are evaluated on the FMA pipe, the rest with MUFU.
 constexpr int kPairs = kCols / 2;
@@ -222,13 +233,15 @@ __device__ __forceinline__ constexpr int mufu_pair(int k) {
     return 8 * (k / (8 - kExp2OnFma)) + kExp2OnFma + k % (8 - kExp2OnFma);
 }
 
-// p = 2^(s * log2(e)/8) for a thread's kCols scores, packed to bf16 pairs.
+// p = 2^x for a thread's kCols scores x, packed to bf16 pairs. The scores
+// are already in log2 units (Q was scaled by log2(e)/8 when it was copied to
+// TMEM): x = q.k * log2(e) / 8.
 //
-// 2^x on the FMA pipe, x = s * log2(e)/8 in [-125, 125]: t = x + 1.5 * 2^23
-// rounds x to the nearest integer j and leaves j in the low mantissa bits of
-// t; -j = 1.5 * 2^23 - t exactly; f = x - j (one fused multiply-add from s,
-// so |f| <= 1/2 up to one rounding); 2^x = p(f) * 2^j, with 2^j applied by
-// adding j << 23 to the bit pattern of p(f). Six packed FMAs per pair.
+// 2^x on the FMA pipe, x in [-125, 125]: t = x + 1.5 * 2^23 rounds x to the
+// nearest integer j and leaves j in the low mantissa bits of t; -j =
+// 1.5 * 2^23 - t exactly; f = x - j exactly (|f| <= 1/2); 2^x = p(f) * 2^j,
+// with 2^j applied by adding j << 23 to the bit pattern of p(f). Six packed
+// adds and FMAs per pair.
 //
 // Instruction order. A warp issues in order; MUFU accepts one warp-wide ex2
 // every 8 cycles and a packed FMA holds the FMA pipe for 2. Emitting all the
@@ -239,7 +252,6 @@ __device__ __forceinline__ constexpr int mufu_pair(int k) {
 // by then). Every step feeds both units, and each value is used a step after
 // it was produced, which hides the units' latencies.
 __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint32_t (&pk)[kPairs]) {
-    const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
     const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
     constexpr int kStagesFma = 7;  // t, -j, f, three Horner steps, combine + pack
     constexpr int kSteps = (kMufuPairs + 2 > kFmaPairs + kStagesFma - 1)
@@ -252,10 +264,8 @@ __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint
     for (int k = 0; k < kSteps; ++k) {
         if (k < kMufuPairs) {
             const int c = mufu_pair(k);
-            float x0, x1;
-            f2_unpack(f2_mul(f2_pack(s[2 * c], s[2 * c + 1]), scale2), x0, x1);
-            p[2 * c] = ex2_approx(x0);
-            p[2 * c + 1] = ex2_approx(x1);
+            p[2 * c] = ex2_approx(s[2 * c]);
+            p[2 * c + 1] = ex2_approx(s[2 * c + 1]);
         }
 #pragma unroll
         for (int d = kStagesFma - 1; d >= 0; --d) {
@@ -263,9 +273,9 @@ __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint
             if (i < 0 || i >= kFmaPairs) continue;
             const int c = fma_pair(i);
             switch (d) {
-                case 0: tt[i] = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, magic2); break;
+                case 0: tt[i] = f2_add(f2_pack(s[2 * c], s[2 * c + 1]), magic2); break;
                 case 1: ff[i] = f2_fma(tt[i], f2_pack(-1.0f, -1.0f), magic2); break;  // -j
-                case 2: ff[i] = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), scale2, ff[i]); break;  // f
+                case 2: ff[i] = f2_add(f2_pack(s[2 * c], s[2 * c + 1]), ff[i]); break;  // f
                 case 3: y[i] = f2_fma(f2_pack(kExp2C3, kExp2C3), ff[i], f2_pack(kExp2C2, kExp2C2)); break;
                 case 4: y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C1, kExp2C1)); break;
                 case 5: y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C0, kExp2C0)); break;
@@ -286,13 +296,8 @@ __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint
 
 // MUFU only: the last block, whose masked scores are -inf (2^-inf = 0).
 __device__ __forceinline__ void exp_pack_row_mufu(const float (&s)[kCols], uint32_t (&pk)[kPairs]) {
-    const uint64_t scale2 = f2_pack(kScaleLog2, kScaleLog2);
 #pragma unroll
-    for (int c = 0; c < kPairs; ++c) {
-        float x0, x1;
-        f2_unpack(f2_mul(f2_pack(s[2 * c], s[2 * c + 1]), scale2), x0, x1);
-        pk[c] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
-    }
+    for (int c = 0; c < kPairs; ++c) pk[c] = pack_bf16x2(ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -503,8 +508,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const long long grow = static_cast<long long>(seg) * prm.q_len + row_in_seg;
             // Q_t into TMEM: this thread's half of its row of q_hat (32 bf16
             // = 16 words, two head dims per word, low half first) into its
-            // lane, the layout the MMA reads an M x K operand in. Rows past
-            // the segment are zeros and never stored.
+            // lane, the layout the MMA reads an M x K operand in, each value
+            // multiplied by log2(e)/8 on the way (so that S comes out of the
+            // MMA in log2 units and the exponentials need no multiply). Rows
+            // past the segment are zeros and never stored.
             {
                 uint32_t qr[16];
                 if (row_live) {
@@ -513,10 +520,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const uint4 w = __ldg(src + i);
-                        qr[4 * i] = w.x;
-                        qr[4 * i + 1] = w.y;
-                        qr[4 * i + 2] = w.z;
-                        qr[4 * i + 3] = w.w;
+                        qr[4 * i] = scale_bf16x2(w.x);
+                        qr[4 * i + 1] = scale_bf16x2(w.y);
+                        qr[4 * i + 2] = scale_bf16x2(w.z);
+                        qr[4 * i + 3] = scale_bf16x2(w.w);
                     }
                 } else {
 #pragma unroll
