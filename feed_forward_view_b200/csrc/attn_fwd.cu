@@ -98,15 +98,23 @@ constexpr int kBN = 96;                           // keys per block
 constexpr int kStages = 8;                        // K/V ring depth
 constexpr int kKVTileBytes = kBN * kHeadDim * 2;  // 12 KB
 constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum block (16)
-constexpr int kSoftmaxWarps = 16;                 // per CTA: 2 tiles x 4 lane quarters x 2 column halves
-constexpr int kThreads = 128 + 32 * kSoftmaxWarps;  // 640
-constexpr int kCols = kBN / 2;                      // score columns per softmax thread
-// Register split: 96 per thread at launch (the cap for 20 warps); the
-// TMA/MMA warpgroup gives up to 56, the four softmax warpgroups take 104:
-// 128 * 56 + 512 * 104 = 60416 <= 640 * 96.
-constexpr uint32_t kLaunchRegs = 96;
-constexpr uint32_t kRegsControl = 56;
-constexpr uint32_t kRegsSoftmax = 104;
+// Softmax warps per lane quarter of a tile: 2 = each takes half the score
+// columns (16 softmax warps), 1 = one warp takes the whole row (8 warps).
+#ifndef VGGT_COL_SPLIT
+#define VGGT_COL_SPLIT 2
+#endif
+constexpr int kColSplit = VGGT_COL_SPLIT;
+static_assert(kColSplit == 1 || kColSplit == 2, "one or two softmax warps per lane quarter");
+constexpr int kSoftmaxWarps = 8 * kColSplit;         // per CTA: 2 tiles x 4 lane quarters x kColSplit
+constexpr int kThreads = 128 + 32 * kSoftmaxWarps;   // 640 or 384
+constexpr int kCols = kBN / kColSplit;               // score columns per softmax thread
+// Register split: the cap for the CTA's warps at launch; the TMA/MMA
+// warpgroup gives registers up, the softmax warpgroups take them:
+// 2 halves: 128 * 56 + 512 * 104 = 60416 <= 640 * 96;
+// 1 half:   128 * 80 + 256 * 208 = 63488 <= 384 * 168.
+constexpr uint32_t kLaunchRegs = kColSplit == 2 ? 96 : 168;
+constexpr uint32_t kRegsControl = kColSplit == 2 ? 56 : 80;
+constexpr uint32_t kRegsSoftmax = kColSplit == 2 ? 104 : 208;
 static_assert(128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
@@ -207,6 +215,30 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > limit) return;
     }
+}
+
+// TMEM loads and stores of the widths the two column splits use, picked by
+// array size.
+template <int N>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 48 || N == 96, "unsupported width");
+    if constexpr (N == 48) tmem_ld48(taddr, r);
+    if constexpr (N == 96) tmem_ld96(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 24 || N == 32 || N == 48, "unsupported width");
+    if constexpr (N == 16) tmem_st16(taddr, r);
+    if constexpr (N == 24) tmem_st24(taddr, r);
+    if constexpr (N == 32) tmem_st32(taddr, r);
+    if constexpr (N == 48) tmem_st48(taddr, r);
+}
+// O columns [first, first + N - 1) and l (column 64) of [O | l].
+template <int N>
+__device__ __forceinline__ void tmem_load_o(uint32_t o_base, uint32_t first, uint32_t (&r)[N]) {
+    static_assert(N == 33 || N == 80, "unsupported width");
+    if constexpr (N == 33) tmem_ld32_1(o_base + first, o_base + kHeadDim, r);
+    if constexpr (N == 80) tmem_ld80(o_base, r);
 }
 
 // Two bf16 (low half first) times log2(e)/8, rounded back to bf16 (nearest,
@@ -492,8 +524,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else if (warp >= 4) {
         // ------------------------------------------------------ softmax
         regs_inc<kRegsSoftmax>();
-        const int t = (warp - 4) >> 3;
-        const int half = ((warp - 4) >> 2) & 1;  // score columns [kCols*half, +kCols)
+        const int t = (warp - 4) / (4 * kColSplit);
+        const int half = ((warp - 4) >> 2) % kColSplit;  // score columns [kCols*half, +kCols)
         const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
         const int row = quarter * 32 + lane;
         if (t < ntile) {
@@ -513,12 +545,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // MMA in log2 units and the exponentials need no multiply). Rows
             // past the segment are zeros and never stored.
             {
-                uint32_t qr[16];
+                constexpr int kQWords = 32 / kColSplit;  // this thread's 2-dim words of the row
+                uint32_t qr[kQWords];
                 if (row_live) {
                     const uint4* src = reinterpret_cast<const uint4*>(
-                        prm.q_hat + (static_cast<long long>(h) * prm.n_q + grow) * kHeadDim + 32 * half);
+                        prm.q_hat + (static_cast<long long>(h) * prm.n_q + grow) * kHeadDim + 2 * kQWords * half);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < kQWords / 4; ++i) {
                         const uint4 w = __ldg(src + i);
                         qr[4 * i] = scale_bf16x2(w.x);
                         qr[4 * i + 1] = scale_bf16x2(w.y);
@@ -527,9 +560,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) qr[i] = 0u;
+                    for (int i = 0; i < kQWords; ++i) qr[i] = 0u;
                 }
-                tmem_st16(lane_base + col_q(t) + 16 * half, qr);
+                tmem_store(lane_base + col_q(t) + kQWords * half, qr);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_q(t));
@@ -544,7 +577,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 float s[kCols];
                 {
                     uint32_t r[kCols];
-                    tmem_ld48(lane_base + col_s(t) + kCols * half, r);
+                    tmem_load(lane_base + col_s(t) + kCols * half, r);
 #pragma unroll
                     for (int i = 0; i < kCols; ++i) s[i] = __uint_as_float(r[i]);
                 }
@@ -580,7 +613,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     break;
                 }
                 tc_fence_after();
-                tmem_st24(lane_base + col_p(t) + kPairs * half, pk);
+                tmem_store(lane_base + col_p(t) + kPairs * half, pk);
             }
             if (ok) {
                 // P of the last block is in TMEM (there is no next S to read).
@@ -591,17 +624,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (ok && uwait(bar_o(t), 0)) {
                 tc_fence_after();
                 // This thread's 32 of the 64 output dims, and l (column 64).
-                uint32_t o[33];
-                tmem_ld32_1(lane_base + col_o(t) + 32 * half, lane_base + col_o(t) + kHeadDim, o);
-                const float l = __uint_as_float(o[32]);
+                constexpr int kODims = kHeadDim / kColSplit;  // this thread's output dims
+                uint32_t o[kColSplit == 2 ? 33 : kOCols];
+                tmem_load_o(lane_base + col_o(t), kODims * half, o);
+                const float l = __uint_as_float(o[kODims]);
                 const float inv = 1.0f / l;
                 if (row_live) {
                     // Inputs outside the core's contract can overflow the
                     // max-free softmax; say so instead of storing silently.
                     if (!(l > 0.0f && l <= 3.0e38f)) atomicOr(prm.status, kStatusRange);
-                    uint4* dst = reinterpret_cast<uint4*>(prm.out + (grow * prm.H + h) * kHeadDim + 32 * half);
+                    uint4* dst = reinterpret_cast<uint4*>(prm.out + (grow * prm.H + h) * kHeadDim + kODims * half);
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
+                    for (int v4 = 0; v4 < kODims / 8; ++v4) {
                         uint4 w;
                         w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv,
                                           __uint_as_float(o[8 * v4 + 1]) * inv);
