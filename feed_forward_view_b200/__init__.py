@@ -29,6 +29,7 @@ __all__ = [
     "vggt_attn_core",
     "vggt_attn_global_noalloc",
     "vggt_get_device_status",
+    "vggt_release_scratch",
     "vggt_status_string",
     "vggt_set_wait_limit",
     "vggt_debug_wait_timeout",
@@ -46,6 +47,7 @@ EXPORTED_SYMBOLS = (
     "vggt_kv_pool",
     "vggt_kv_pool_tokens",
     "vggt_get_device_status",
+    "vggt_release_scratch",
     "vggt_status_string",
     "vggt_set_wait_limit",
     "vggt_debug_wait_timeout",
@@ -73,6 +75,8 @@ lib.vggt_attn_core.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.vggt_attn_core.restype = _i
 lib.vggt_kv_pool_tokens.argtypes = [_i, _i]
 lib.vggt_kv_pool_tokens.restype = _i
+lib.vggt_release_scratch.argtypes = []
+lib.vggt_release_scratch.restype = _i
 lib.vggt_get_device_status.argtypes = [_p]
 lib.vggt_get_device_status.restype = _i
 lib.vggt_status_string.argtypes = [_i]
@@ -201,6 +205,11 @@ def vggt_kv_pool(k, v, pos, k_out=None, v_out=None, pos_out=None, S=None, T=None
 
 def vggt_get_device_status(stream=None) -> int:
     return int(lib.vggt_get_device_status(_stream(stream)))
+
+
+def vggt_release_scratch() -> None:
+    """Return the library's unused scratch memory on the current device."""
+    _check(lib.vggt_release_scratch(), "vggt_release_scratch")
 
 
 def vggt_set_wait_limit(cycles: int) -> int:

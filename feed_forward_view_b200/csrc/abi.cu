@@ -1,9 +1,13 @@
 // abi.cu -- the extern "C" entry points declared in include/vggt_attn.h.
 //
 // Each call validates every argument on the host (nothing is launched for an
-// invalid call), takes its scratch with cudaMallocAsync on the caller's
-// stream, launches the kernels in stream order and frees the scratch with
-// cudaFreeAsync on the same stream. No call synchronises the stream.
+// invalid call), takes its scratch from the library's stream-ordered memory
+// pool on the caller's stream, launches the kernels in stream order and frees
+// the scratch with cudaFreeAsync on the same stream. No call synchronises the
+// stream. The pool keeps freed memory for the next call (the device's default
+// pool returns it to the system at every synchronisation, and taking a
+// gigabyte back costs milliseconds of host time per call, during which the
+// GPU idles); vggt_release_scratch hands it back on request.
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -26,6 +30,7 @@ __device__ int g_device_status;  // kStatusTimeout / kStatusRange bits, 0 when c
 struct DeviceState {
     int* status = nullptr;  // device address of g_device_status
     long long wait_limit = kDefaultWaitLimit;
+    cudaMemPool_t pool = nullptr;  // scratch pool, release threshold at its maximum
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -39,6 +44,24 @@ DeviceState* device_state() {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
         st.status = static_cast<int*>(p);
+    }
+    if (!st.pool) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            cudaGetLastError();
+            cudaMemPoolDestroy(pool);
+            return nullptr;
+        }
+        st.pool = pool;
     }
     return &st;
 }
@@ -90,8 +113,8 @@ int run_attention(const uint16_t* q, const float* pos, const uint16_t* k, const 
     const long long nq = static_cast<long long>(n_seg) * q_len;
     const long long nk = static_cast<long long>(n_seg) * k_len;
     void* scratch = nullptr;
-    if (cudaMallocAsync(&scratch, head_plane_bytes(nq, H) + head_plane_bytes(nk, H), stream) !=
-        cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&scratch, head_plane_bytes(nq, H) + head_plane_bytes(nk, H), st->pool,
+                                stream) != cudaSuccess) {
         cudaGetLastError();
         if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
         return VGGT_ERR_ALLOC;
@@ -210,8 +233,10 @@ int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16
     // pooled k, pooled v, pooled positions
     const size_t kv_bytes = head_plane_bytes(nk, H);
     const size_t pos_bytes = static_cast<size_t>(nk) * 2 * sizeof(float);
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
     void* pooled = nullptr;
-    if (cudaMallocAsync(&pooled, 2 * kv_bytes + pos_bytes, stream) != cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&pooled, 2 * kv_bytes + pos_bytes, st->pool, stream) != cudaSuccess) {
         cudaGetLastError();
         return VGGT_ERR_ALLOC;
     }
@@ -226,6 +251,16 @@ int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16
     // Every query row attends to all S*Tk descriptors: one segment.
     return run_attention(q, pos, kp, pp, vp, out, 1, S * T, static_cast<int>(nk), H, pooled,
                          stream);
+}
+
+int vggt_release_scratch(void) {
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    if (cudaMemPoolTrimTo(st->pool, 0) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_CUDA;
+    }
+    return VGGT_OK;
 }
 
 int vggt_get_device_status(cudaStream_t stream) {

@@ -33,8 +33,13 @@
  *   - Every pointer must be 16-byte aligned (TMA and 16-byte vector access).
  *   - S == 0 or H == 0 is an empty problem: VGGT_OK, nothing is launched.
  *   - Everything is asynchronous on `stream`; no call synchronises it.
- *   - Scratch (normalised q/k, pooled k/v) is taken with cudaMallocAsync and
- *     released with cudaFreeAsync on `stream`.
+ *   - Scratch (normalised q/k, pooled k/v) comes from a stream-ordered memory
+ *     pool the library owns (one per device) and is released to it with
+ *     cudaFreeAsync on `stream`. The pool keeps that memory for later calls
+ *     instead of returning it to the system at every synchronisation (which
+ *     would cost milliseconds of host time per call to take it back), so
+ *     after a call the library holds up to the largest scratch any call
+ *     needed -- about 4 * S*T * H * D bytes; vggt_release_scratch returns it.
  *   - Outputs must not overlap inputs.
  *   - Every argument is checked on the host before any launch; an invalid call
  *     returns a negative vggt_status and launches nothing.
@@ -202,6 +207,13 @@ VGGT_API int vggt_kv_pool_tokens(int T, int kv_down);
    was out of range (see vggt_attn_core); VGGT_ERR_CUDA if the
    synchronisation failed. */
 VGGT_API int vggt_get_device_status(cudaStream_t stream);
+
+/* Returns the library's unused scratch memory on the current device to the
+   system (memory whose cudaFreeAsync has not yet executed in its stream stays
+   reserved: synchronise those streams first). Later calls take it back as
+   they need it. VGGT_OK, or VGGT_ERR_CUDA. Host only. (No counterpart on the
+   pages: memory management of this library.) */
+VGGT_API int vggt_release_scratch(void);
 
 /* Human-readable name of a vggt_status value (static storage). */
 VGGT_API const char* vggt_status_string(int status);

@@ -286,3 +286,19 @@ def test_core_reports_inputs_beyond_the_norm_bound(F):
     assert F.vggt_get_device_status() == -7
     assert F.vggt_get_device_status() == 0
     check_attention(F, "global", 1, 10, 1, seed=32)
+
+
+def test_scratch_pool_release_and_reuse(F):
+    # Scratch comes from the library's pool, which keeps it between calls;
+    # vggt_release_scratch hands it back and later calls take it again. The
+    # results do not depend on where the scratch came from.
+    S, g, kd = 3, 9, 3
+    q, k, v, pos = synth.make_qkv(S, g, seed=33)
+    T = 5 + g * g
+    a = run_gpu(F, "descriptor", q, k, v, pos, S, T, kd)
+    b = run_gpu(F, "global", q, k, v, pos, S, T, 1)
+    torch.cuda.synchronize()
+    F.vggt_release_scratch()
+    F.vggt_release_scratch()  # nothing left to release: still fine
+    assert torch.equal(run_gpu(F, "descriptor", q, k, v, pos, S, T, kd), a)
+    assert torch.equal(run_gpu(F, "global", q, k, v, pos, S, T, 1), b)
