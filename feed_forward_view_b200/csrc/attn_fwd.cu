@@ -64,6 +64,13 @@
 // softmax warps for its scheduler: measured, each extra wait there cost
 // hundreds of cycles per block even when its barrier had long completed.
 //
+// The two tiles' issuers take turns (bar_tok): tile 0 issues its group for
+// block j after tile 1 issued its group for block j-1, tile 1 after tile 0's
+// group j. Left alone, the two tiles drift into step and their groups reach
+// the tensor core together, each then waiting behind the other's; taking
+// turns offsets the tiles by about one group, so that each group finds the
+// tensor core idle and its results come back sooner (measured +4-5%).
+//
 // bar_c[t] phases: 0 = S_{t,0} read (and K_1 loaded); j + 1 = P_{t,j} written,
 // S_{t,j+1} read and K_{j+2} loaded (only P_{t,j} for the last block). Issue
 // order for tile t: [Q_t in TMEM, K_0 loaded] S_{t,0}; [bar_c 0] S_{t,1}; then
@@ -159,6 +166,7 @@ struct SharedStorage {
     uint64_t bar_c[2];      // [tile]: P_{t,j-1} written and S_{t,j} read
     uint64_t bar_pfree[2];  // [tile]: PV_{t,j} finished (P_t free, O_t updated)
     uint64_t bar_o[2];      // [tile]: every MMA of the tile finished (once)
+    uint64_t bar_tok[2];    // [tile]: the other tile issued its previous MMA group
     uint32_t tmem_base;
     int abort;
 };
@@ -366,6 +374,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t bar_c0 = smem_u32(&sm.bar_c[0]);
     const uint32_t bar_pfree0 = smem_u32(&sm.bar_pfree[0]);
     const uint32_t bar_o0 = smem_u32(&sm.bar_o[0]);
+    const uint32_t bar_tok0 = smem_u32(&sm.bar_tok[0]);
     const uint32_t kv_smem0 = smem_u32(sm.kv[0][0]);
     const uint32_t ones_smem = smem_u32(sm.ones);
     auto bar_kvfull = [&](int s) { return bar_kvfull0 + 8u * s; };
@@ -375,6 +384,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     auto bar_c = [&](int t) { return bar_c0 + 8u * t; };
     auto bar_pfree = [&](int t) { return bar_pfree0 + 8u * t; };
     auto bar_o = [&](int t) { return bar_o0 + 8u * t; };
+    auto bar_tok = [&](int t) { return bar_tok0 + 8u * t; };
     auto k_smem = [&](int s) { return kv_smem0 + static_cast<uint32_t>(2 * kKVTileBytes) * s; };
     auto v_smem = [&](int s) { return k_smem(s) + static_cast<uint32_t>(kKVTileBytes); };
 
@@ -400,6 +410,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_init(bar_c(t), kSoftmaxWarps / 2);
             mbar_init(bar_pfree(t), 1);
             mbar_init(bar_o(t), 1);
+            mbar_init(bar_tok(t), 1);
         }
         sm.abort = 0;
         fence_barrier_init();
@@ -506,12 +517,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const uint32_t pfree = bar_pfree(t);
                 const uint32_t empty = bar_kvempty(s);
                 if (!uwait(bar_c(t), (j + 1) & 1)) break;
+                // The two tiles take turns: tile 0's group j follows tile 1's
+                // group j-1, tile 1's group j follows tile 0's group j.
+                if (ntile == 2 && (t == 1 || j > 0) &&
+                    !uwait(bar_tok(t), (t == 0 ? j - 1 : j) & 1))
+                    break;
                 if (elect_one()) {
                     tc_fence_after();
                     // P_t free again and O_t includes block j; K_j and V_j no
                     // longer needed by this tile.
                     mma_ts6_commit2(o_tm, p_tm, vd, idesc_o, j > 0 ? 1u : 0u, pfree, empty);
                     if (jn < nkb) mma_ts4_commit(s_tm, q_tm, kd, idesc_s, bar_s(t));
+                    if (ntile == 2) mbar_arrive(bar_tok(1 - t));
                 }
                 __syncwarp();
             }
