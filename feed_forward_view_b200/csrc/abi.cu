@@ -121,11 +121,11 @@ int run_attention(const uint16_t* q, const float* pos, const uint16_t* k, const 
     }
     uint16_t* q_hat = static_cast<uint16_t*>(scratch);
     uint16_t* k_hat = q_hat + head_plane_bytes(nq, H) / sizeof(uint16_t);
-    PrologueJob jq{q, pos, q_hat, static_cast<int>(nq)};
-    PrologueJob jk{k, pos_k, k_hat, static_cast<int>(nk)};
+    PrologueJob jq{q, pos, q_hat, static_cast<int>(nq), nq};
+    PrologueJob jk{k, pos_k, k_hat, static_cast<int>(nk), nk};
     int rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
     if (rc == VGGT_OK) {
-        AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H};
+        AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H, nq, nk};
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -174,8 +174,8 @@ int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int
     if (N == 0 || H == 0) return VGGT_OK;
     if (!x || !pos || !x_hat) return VGGT_ERR_NULL;
     if (!aligned16(x) || !aligned16(pos) || !aligned16(x_hat)) return VGGT_ERR_UNSUPPORTED;
-    PrologueJob j{x, pos, x_hat, N};
-    PrologueJob none{nullptr, nullptr, nullptr, 0};
+    PrologueJob j{x, pos, x_hat, N, N};
+    PrologueJob none{nullptr, nullptr, nullptr, 0, 0};
     return to_status(vggt::launch_qk_prologue(j, none, H, stream));
 }
 
@@ -193,7 +193,8 @@ int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf
         return VGGT_ERR_UNSUPPORTED;
     DeviceState* st = device_state();
     if (!st) return VGGT_ERR_CUDA;
-    AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H};
+    AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H,
+                  static_cast<long long>(n_seg) * q_len, static_cast<long long>(n_seg) * k_len};
     return to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
 }
 

@@ -175,11 +175,11 @@ constexpr size_t kSmemBytes = sizeof(SharedStorage) + 1024;  // + alignment slac
 static_assert(kSmemBytes <= 227 * 1024, "shared memory beyond the per-CTA limit");
 
 struct Params {
-    const uint16_t* q_hat;  // [H, n_q, 64] head-major
-    uint16_t* out;          // [n_q, H, 64]
+    const uint16_t* q_hat;  // head-major, head planes q_stride rows apart
+    uint16_t* out;          // [n_seg*q_len, H, 64]
     int* status;            // device status word
     long long wait_limit;
-    long long n_q;          // n_seg * q_len
+    long long q_stride;     // rows per head plane of q_hat
     int q_len, k_len, H;
     int pairs_per_seg;
 };
@@ -566,7 +566,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 uint32_t qr[kQWords];
                 if (row_live) {
                     const uint4* src = reinterpret_cast<const uint4*>(
-                        prm.q_hat + (static_cast<long long>(h) * prm.n_q + grow) * kHeadDim + 2 * kQWords * half);
+                        prm.q_hat + (static_cast<long long>(h) * prm.q_stride + grow) * kHeadDim + 2 * kQWords * half);
 #pragma unroll
                     for (int i = 0; i < kQWords / 4; ++i) {
                         const uint4 w = __ldg(src + i);
@@ -730,9 +730,11 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     if (p.n_seg <= 0 || p.H <= 0 || p.q_len <= 0 || p.k_len <= 0) return cudaSuccess;
     const uint64_t nk = static_cast<uint64_t>(p.n_seg) * p.k_len;
     const uint64_t row_bytes = kHeadDim * 2;
+    const uint64_t ks = static_cast<uint64_t>(p.k_stride);
     CUtensorMap tm_k, tm_v;
-    // k_hat: [H][nk][64] -> dims {64, nk, H}, box {64, kBN, 1}
-    if (!make_map(&tm_k, p.k_hat, nk, p.H, row_bytes, nk * row_bytes, kBN, 1) ||
+    // k_hat: head planes k_stride rows apart -> dims {64, k_stride, H}, box
+    // {64, kBN, 1} (rows past a segment's keys are masked in the kernel)
+    if (!make_map(&tm_k, p.k_hat, ks, p.H, row_bytes, ks * row_bytes, kBN, 1) ||
         // v: [nk][H][64] -> dims {64, H, nk}, box {64, 1, kBN}
         !make_map(&tm_v, p.v, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
         return cudaErrorInvalidValue;
@@ -762,7 +764,7 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     prm.out = p.out;
     prm.status = status;
     prm.wait_limit = wait_limit;
-    prm.n_q = static_cast<long long>(p.n_seg) * p.q_len;
+    prm.q_stride = p.q_stride;
     prm.q_len = p.q_len;
     prm.k_len = p.k_len;
     prm.H = p.H;

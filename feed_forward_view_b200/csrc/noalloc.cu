@@ -88,10 +88,10 @@ extern "C" int vggt_attn_global_noalloc(const vggt_bf16* q, const vggt_bf16* k,
     uint16_t* q_hat = static_cast<uint16_t*>(scratch);
     uint16_t* k_hat = q_hat + plane / sizeof(uint16_t);
     const int N = static_cast<int>(n);
-    vggt::PrologueJob jq{q, pos, q_hat, N};
-    vggt::PrologueJob jk{k, pos, k_hat, N};
+    vggt::PrologueJob jq{q, pos, q_hat, N, N};
+    vggt::PrologueJob jk{k, pos, k_hat, N, N};
     if (vggt::launch_qk_prologue(jq, jk, H, stream) != cudaSuccess) return VGGT_ERR_CUDA;
-    vggt::AttnProblem p{q_hat, k_hat, v, out, 1, N, N, H};
+    vggt::AttnProblem p{q_hat, k_hat, v, out, 1, N, N, H, N, N};
     if (vggt::launch_attention(p, status, wait_limit, stream) != cudaSuccess) return VGGT_ERR_CUDA;
     return VGGT_OK;
 }

@@ -100,7 +100,7 @@ __device__ __forceinline__ void finish_group(const PrologueJob& job, int t, int 
         o2[i] = y2 * cv[i] + y1 * sv[i];
     }
     if (live) {
-        uint16_t* dst = job.x_hat + (static_cast<size_t>(h) * job.n + t) * kHeadDim;
+        uint16_t* dst = job.x_hat + (static_cast<size_t>(h) * job.out_stride + t) * kHeadDim;
         *reinterpret_cast<uint2*>(dst + d1) = make_uint2(pack2(o1[0], o1[1]), pack2(o1[2], o1[3]));
         *reinterpret_cast<uint2*>(dst + d1 + 16) =
             make_uint2(pack2(o2[0], o2[1]), pack2(o2[2], o2[3]));

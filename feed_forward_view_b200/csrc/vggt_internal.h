@@ -15,13 +15,16 @@ constexpr int kHeadDim = 64;
 constexpr int kStatusTimeout = 1;  // a bounded device wait ran out
 constexpr int kStatusRange = 2;    // an attention row sum was not a positive finite number
 
-// One tensor to normalise and rotate: x [n, H, 64] token-major in, x_hat
-// [H, n, 64] head-major out, positions pos [n, 2] (row, col).
+// One tensor to normalise and rotate: x [n, H, 64] token-major in, positions
+// pos [n, 2] (row, col); out head-major: row t of head h goes to
+// x_hat + (h * out_stride + t) * 64 (out_stride = n for a [H, n, 64] array;
+// larger to write n rows into a bigger head-major array at x_hat's row).
 struct PrologueJob {
     const uint16_t* x;
     const float* pos;
     uint16_t* x_hat;
     int n;
+    long long out_stride;
 };
 
 // LayerNorm (eps 1e-5, no affine) + 2D RoPE (base 100) over one or two jobs in
@@ -37,7 +40,9 @@ cudaError_t launch_kv_pool(const uint16_t* k, const uint16_t* v, const float* po
 
 // Attention over segments: segment s has queries rows [s*q_len, (s+1)*q_len)
 // of q_hat and keys rows [s*k_len, (s+1)*k_len) of k_hat / v.
-//   q_hat [H, n_seg*q_len, 64] and k_hat [H, n_seg*k_len, 64] head-major,
+//   q_hat and k_hat head-major: row r of head h at q_hat + (h * q_stride + r)
+//   * 64 (likewise k_hat with k_stride); q_stride >= n_seg*q_len, k_stride >=
+//   n_seg*k_len (equal for plain [H, n, 64] arrays);
 //   v [n_seg*k_len, H, 64] and out [n_seg*q_len, H, 64] token-major.
 struct AttnProblem {
     const uint16_t* q_hat;
@@ -48,6 +53,8 @@ struct AttnProblem {
     int q_len;
     int k_len;
     int H;
+    long long q_stride;
+    long long k_stride;
 };
 
 // Returns cudaSuccess, or an error from tensor-map encoding or the launch.

@@ -30,7 +30,13 @@ What it computes, per head, for bf16 inputs widened exactly to float64:
      five special tokens unchanged plus one average per ``kd x kd`` cell of the
      patch grid (ceil mode), at the cell's mean position (FlashVGGT README,
      Overview: cross-attention between all image tokens and the per-frame
-     descriptor set; Key Arguments: ``--kv_downfactor`` 4).
+     descriptor set; Key Arguments: ``--kv_downfactor`` 4);
+   * streaming descriptor attention: frames arrive in chunks of ``chunk``
+     frames; every query of chunk ``c`` sees the descriptors of all frames of
+     chunks ``0..c`` -- the cached descriptors of earlier chunks and its own
+     chunk's (FlashVGGT README, Overview: a chunk-recursive mechanism that
+     reuses cached descriptors from previous chunks; streaming inference with
+     ``--chunksize``, default 10).
 
 Evaluating a subset of query rows is the same definition restricted to those
 rows: every output row depends only on its own query and the key set, so
@@ -322,6 +328,28 @@ def attn_descriptor(q, k, v, pos, S: int, T: int, kd: int, rows=None) -> np.ndar
     q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows])
     k_hat = qk_prologue(kp, pp)
     return cross_attention(q_hat, k_hat, vp)
+
+
+def attn_descriptor_stream(q, k, v, pos, S: int, T: int, kd: int, chunk: int, rows=None) -> np.ndarray:
+    """Streaming descriptor attention: a query of frame ``f`` sees the
+    descriptors of frames ``0 .. min(S, (f // chunk + 1) * chunk) - 1``. The
+    descriptors are the per-frame pooled tokens of ``attn_descriptor``; their
+    keys go through the prologue at their cell-mean positions."""
+    if chunk < 1:
+        raise ValueError("chunk must be >= 1")
+    kp, vp, pp = kv_pool(k, v, pos, S, T, kd)
+    k_hat = qk_prologue(kp, pp)
+    tk = pooled_tokens_per_frame(T, kd)
+    rows = _rows(S * T, rows)
+    out = np.empty((rows.size,) + np.asarray(q).shape[1:])
+    chunk_of_row = (rows // T) // chunk
+    for c in np.unique(chunk_of_row):
+        sel = np.nonzero(chunk_of_row == c)[0]
+        r = rows[sel]
+        n_keys = min(S, (int(c) + 1) * chunk) * tk
+        q_hat = qk_prologue(np.asarray(q)[r], np.asarray(pos)[r])
+        out[sel] = cross_attention(q_hat, k_hat[:n_keys], vp[:n_keys])
+    return out
 
 
 def flops(kind: str, S: int, T: int, Tk: int, H: int, D: int, n_rows=None) -> float:

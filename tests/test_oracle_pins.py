@@ -414,3 +414,69 @@ def test_pool_reference_kd1_is_bit_identity():
     assert np.array_equal(kb, _bits(k).reshape(kb.shape))
     assert np.array_equal(vb, _bits(v).reshape(vb.shape))
     assert np.array_equal(pb, pos)
+
+
+# ----------------------------------------------------- streaming descriptors
+
+
+def test_stream_one_chunk_covering_all_frames_is_descriptor_attention():
+    S = 3
+    q, k, v, pos, T = _scene(S, 4, seed=41)
+    full = O.attn_descriptor(q, k, v, pos, S, T, 2)
+    for chunk in (3, 5):
+        got = O.attn_descriptor_stream(q, k, v, pos, S, T, 2, chunk)
+        np.testing.assert_allclose(got, full, rtol=0, atol=1e-13)
+
+
+def test_stream_chunk_one_is_a_causal_prefix_over_frames():
+    # chunk = 1: frame f sees the descriptors of frames 0..f, i.e. it is the
+    # descriptor attention of the scene cut after frame f.
+    S = 4
+    q, k, v, pos, T = _scene(S, 3, seed=42)
+    got = O.attn_descriptor_stream(q, k, v, pos, S, T, 2, 1)
+    for f in range(S):
+        n = (f + 1) * T
+        prefix = O.attn_descriptor(q[:n], k[:n], v[:n], pos[:n], f + 1, T, 2)
+        np.testing.assert_allclose(got[f * T:(f + 1) * T], prefix[f * T:], rtol=0, atol=1e-13)
+
+
+def test_stream_earlier_chunks_ignore_later_frames():
+    S = 5
+    q, k, v, pos, T = _scene(S, 3, seed=43)
+    a = O.attn_descriptor_stream(q, k, v, pos, S, T, 2, 2)
+    k2, v2 = k.copy(), v.copy()
+    k2[4 * T:] += 3.0  # frame 4: chunk 2 only
+    v2[4 * T:] -= 5.0
+    b = O.attn_descriptor_stream(q, k2, v2, pos, S, T, 2, 2)
+    np.testing.assert_array_equal(a[:4 * T], b[:4 * T])
+    assert np.abs(a[4 * T:] - b[4 * T:]).max() > 1e-3
+
+
+def test_stream_brute_force_tiny():
+    # Explicit loops: pooled descriptors per frame, the visible frames of each
+    # query listed by hand (chunk 2 of S = 3: frames {0,1} see {0,1}; frame 2
+    # sees {0,1,2}), exp-and-normalise in math.exp.
+    S = 3
+    q, k, v, pos, T = _scene(S, 2, H=1, seed=44)
+    kd = 1
+    kp, vp, pp = O.kv_pool(k, v, pos, S, T, kd)
+    kh = O.qk_prologue(kp, pp)
+    qh = O.qk_prologue(q, pos)
+    tk = O.pooled_tokens_per_frame(T, kd)
+    visible = {0: [0, 1], 1: [0, 1], 2: [0, 1, 2]}
+    got = O.attn_descriptor_stream(q, k, v, pos, S, T, kd, 2)
+    for r in range(S * T):
+        keys = [f * tk + i for f in visible[r // T] for i in range(tk)]
+        s = [sum(qh[r, 0, d] * kh[j, 0, d] for d in range(64)) / 8.0 for j in keys]
+        m = max(s)
+        w = [math.exp(x - m) for x in s]
+        z = sum(w)
+        want = [sum(w[i] * vp[keys[i], 0, d] for i in range(len(keys))) / z for d in range(64)]
+        np.testing.assert_allclose(got[r, 0], want, rtol=0, atol=1e-12)
+
+
+def test_stream_rejects_empty_chunks():
+    S = 2
+    q, k, v, pos, T = _scene(S, 2, seed=45)
+    with pytest.raises(ValueError):
+        O.attn_descriptor_stream(q, k, v, pos, S, T, 1, 0)
