@@ -19,6 +19,7 @@ from .build import LIB_PATH
 
 __all__ = [
     "VggtError",
+    "DescCache",
     "lib",
     "vggt_attn_frame",
     "vggt_attn_global",
@@ -30,6 +31,11 @@ __all__ = [
     "vggt_attn_global_noalloc",
     "vggt_get_device_status",
     "vggt_release_scratch",
+    "vggt_desc_cache_create",
+    "vggt_desc_cache_destroy",
+    "vggt_desc_cache_frames",
+    "vggt_desc_cache_reset",
+    "vggt_attn_descriptor_chunk",
     "vggt_status_string",
     "vggt_set_wait_limit",
     "vggt_debug_wait_timeout",
@@ -48,6 +54,11 @@ EXPORTED_SYMBOLS = (
     "vggt_kv_pool_tokens",
     "vggt_get_device_status",
     "vggt_release_scratch",
+    "vggt_desc_cache_create",
+    "vggt_desc_cache_destroy",
+    "vggt_desc_cache_frames",
+    "vggt_desc_cache_reset",
+    "vggt_attn_descriptor_chunk",
     "vggt_status_string",
     "vggt_set_wait_limit",
     "vggt_debug_wait_timeout",
@@ -75,6 +86,16 @@ lib.vggt_attn_core.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.vggt_attn_core.restype = _i
 lib.vggt_kv_pool_tokens.argtypes = [_i, _i]
 lib.vggt_kv_pool_tokens.restype = _i
+lib.vggt_desc_cache_create.argtypes = [ctypes.POINTER(_p), _i, _i, _i, _i, _i]
+lib.vggt_desc_cache_create.restype = _i
+lib.vggt_desc_cache_destroy.argtypes = [_p]
+lib.vggt_desc_cache_destroy.restype = _i
+lib.vggt_desc_cache_frames.argtypes = [_p]
+lib.vggt_desc_cache_frames.restype = _i
+lib.vggt_desc_cache_reset.argtypes = [_p]
+lib.vggt_desc_cache_reset.restype = _i
+lib.vggt_attn_descriptor_chunk.argtypes = [_p, _p, _p, _p, _p, _p, _i, _p]
+lib.vggt_attn_descriptor_chunk.restype = _i
 lib.vggt_release_scratch.argtypes = []
 lib.vggt_release_scratch.restype = _i
 lib.vggt_get_device_status.argtypes = [_p]
@@ -205,6 +226,57 @@ def vggt_kv_pool(k, v, pos, k_out=None, v_out=None, pos_out=None, S=None, T=None
 
 def vggt_get_device_status(stream=None) -> int:
     return int(lib.vggt_get_device_status(_stream(stream)))
+
+
+class DescCache:
+    """A streaming descriptor cache (see include/vggt_attn.h): holds the
+    normalised pooled keys, values and positions of the frames seen so far
+    of one sequence, on the device that was current at creation."""
+
+    def __init__(self, max_frames: int, T: int, H: int = 16, D: int = 64, kv_down: int = 4):
+        self._h = _p()
+        _check(lib.vggt_desc_cache_create(ctypes.byref(self._h), int(max_frames), int(T), int(H),
+                                          int(D), int(kv_down)), "vggt_desc_cache_create")
+        self.T, self.H, self.D = int(T), int(H), int(D)
+
+    @property
+    def frames(self) -> int:
+        n = lib.vggt_desc_cache_frames(self._h)
+        _check(min(n, 0), "vggt_desc_cache_frames")
+        return int(n)
+
+    def reset(self) -> None:
+        _check(lib.vggt_desc_cache_reset(self._h), "vggt_desc_cache_reset")
+
+    def attend(self, q, k, v, pos, out=None, C=None, stream=None):
+        """One chunk of C frames: q, k, v [C*T, H, D] bf16, pos [C*T, 2] fp32.
+        Appends the chunk's descriptors and returns ``out`` (the chunk's
+        tokens attending to every cached descriptor)."""
+        C = q.shape[0] // self.T if C is None else C
+        if out is None:
+            out = torch.empty_like(q)
+        rc = lib.vggt_attn_descriptor_chunk(self._h, _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                            _ptr(v, torch.bfloat16, "v"), _ptr(pos, torch.float32, "pos"),
+                                            _ptr(out, torch.bfloat16, "out"), int(C), _stream(stream))
+        _check(rc, "vggt_attn_descriptor_chunk")
+        return out
+
+    def close(self) -> None:
+        if self._h:
+            _check(lib.vggt_desc_cache_destroy(self._h), "vggt_desc_cache_destroy")
+            self._h = _p()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def vggt_release_scratch() -> None:

@@ -9,6 +9,7 @@
 // gigabyte back costs milliseconds of host time per call, during which the
 // GPU idles); vggt_release_scratch hands it back on request.
 #include <cmath>
+#include <new>
 #include <cstdint>
 #include <cstdio>
 
@@ -78,6 +79,10 @@ int grid_side(int T) {
 // Every tensor is read or written with 16-byte vector accesses or by TMA,
 // which needs 16-byte aligned global addresses.
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Positions are read as float2 and written as floats: 8 bytes suffice (a
+// frame-aligned slice of a positions array is only 8-byte aligned when its
+// first token index is odd).
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
 // Shared checks. Returns VGGT_OK to proceed, 1 for an empty problem, or an
 // error status.
@@ -90,7 +95,7 @@ int check_common(const void* q, const void* k, const void* v, const void* pos, c
     if (H > 65535) return VGGT_ERR_SHAPE;
     if (S == 0 || H == 0) return 1;
     if (!q || !k || !v || !pos || !out) return VGGT_ERR_NULL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(pos) || !aligned16(out))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned8(pos) || !aligned16(out))
         return VGGT_ERR_UNSUPPORTED;
     return VGGT_OK;
 }
@@ -173,7 +178,7 @@ int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int
     if (N > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
     if (N == 0 || H == 0) return VGGT_OK;
     if (!x || !pos || !x_hat) return VGGT_ERR_NULL;
-    if (!aligned16(x) || !aligned16(pos) || !aligned16(x_hat)) return VGGT_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned8(pos) || !aligned16(x_hat)) return VGGT_ERR_UNSUPPORTED;
     PrologueJob j{x, pos, x_hat, N, N};
     PrologueJob none{nullptr, nullptr, nullptr, 0, 0};
     return to_status(vggt::launch_qk_prologue(j, none, H, stream));
@@ -215,8 +220,8 @@ int vggt_kv_pool(const vggt_bf16* k, const vggt_bf16* v, const float* pos, vggt_
     if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
     if (S == 0 || H == 0) return VGGT_OK;
     if (!k || !v || !pos || !k_out || !v_out || !pos_out) return VGGT_ERR_NULL;
-    if (!aligned16(k) || !aligned16(v) || !aligned16(pos) || !aligned16(k_out) ||
-        !aligned16(v_out) || !aligned16(pos_out))
+    if (!aligned16(k) || !aligned16(v) || !aligned8(pos) || !aligned16(k_out) ||
+        !aligned16(v_out) || !aligned8(pos_out))
         return VGGT_ERR_UNSUPPORTED;
     return to_status(vggt::launch_kv_pool(k, v, pos, k_out, v_out, pos_out, S, T, g, kv_down, H,
                                           stream));
@@ -254,6 +259,129 @@ int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16
                          stream);
 }
 
+// ------------------------------------------------------------- streaming
+
+struct vggt_desc_cache {
+    int device;
+    int max_frames, T, H, kv_down, g, Tk;
+    long long capacity;  // max_frames * Tk descriptor rows
+    int frames;          // frames appended so far
+    uint16_t* k_hat;     // [H][capacity][64] normalised pooled keys, head-major
+    uint16_t* v;         // [capacity][H][64] pooled values, token-major
+    float* pos;          // [capacity][2] cell-mean positions
+};
+
+int vggt_desc_cache_create(vggt_desc_cache** cache, int max_frames, int T, int H, int D,
+                           int kv_down) {
+    if (!cache) return VGGT_ERR_NULL;
+    *cache = nullptr;
+    if (max_frames < 1 || T < 1 || H < 1 || kv_down < 1 || H > 65535) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    const int g = grid_side(T);
+    const int Tk = vggt_kv_pool_tokens(T, kv_down);
+    if (g < 0 || Tk < 0) return VGGT_ERR_SHAPE;
+    const long long capacity = static_cast<long long>(max_frames) * Tk;
+    if (capacity > VGGT_MAX_TOKENS) return VGGT_ERR_SHAPE;
+    vggt_desc_cache* c = new (std::nothrow) vggt_desc_cache();
+    if (!c) return VGGT_ERR_ALLOC;
+    if (cudaGetDevice(&c->device) != cudaSuccess) {
+        delete c;
+        return VGGT_ERR_CUDA;
+    }
+    c->max_frames = max_frames;
+    c->T = T;
+    c->H = H;
+    c->kv_down = kv_down;
+    c->g = g;
+    c->Tk = Tk;
+    c->capacity = capacity;
+    c->frames = 0;
+    const size_t plane = head_plane_bytes(capacity, H);
+    void* mem = nullptr;
+    if (cudaMalloc(&mem, 2 * plane + static_cast<size_t>(capacity) * 2 * sizeof(float)) != cudaSuccess) {
+        cudaGetLastError();
+        delete c;
+        return VGGT_ERR_ALLOC;
+    }
+    c->k_hat = static_cast<uint16_t*>(mem);
+    c->v = c->k_hat + plane / sizeof(uint16_t);
+    c->pos = reinterpret_cast<float*>(c->v + plane / sizeof(uint16_t));
+    *cache = c;
+    return VGGT_OK;
+}
+
+int vggt_desc_cache_destroy(vggt_desc_cache* cache) {
+    if (!cache) return VGGT_OK;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return VGGT_ERR_CUDA;
+    if (cur != cache->device && cudaSetDevice(cache->device) != cudaSuccess) return VGGT_ERR_CUDA;
+    const cudaError_t e = cudaFree(cache->k_hat);
+    if (cur != cache->device) cudaSetDevice(cur);
+    delete cache;
+    return e == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+int vggt_desc_cache_frames(const vggt_desc_cache* cache) {
+    return cache ? cache->frames : VGGT_ERR_NULL;
+}
+
+int vggt_desc_cache_reset(vggt_desc_cache* cache) {
+    if (!cache) return VGGT_ERR_NULL;
+    cache->frames = 0;
+    return VGGT_OK;
+}
+
+int vggt_attn_descriptor_chunk(vggt_desc_cache* cache, const vggt_bf16* q, const vggt_bf16* k,
+                               const vggt_bf16* v, const float* pos, vggt_bf16* out, int C,
+                               cudaStream_t stream) {
+    if (!cache) return VGGT_ERR_NULL;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return VGGT_ERR_CUDA;
+    if (cur != cache->device) return VGGT_ERR_UNSUPPORTED;
+    if (C < 0) return VGGT_ERR_SHAPE;
+    int rc = check_common(q, k, v, pos, out, C, cache->T, cache->H, VGGT_HEAD_DIM);
+    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
+    if (cache->frames + C > cache->max_frames) return VGGT_ERR_SHAPE;
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    const int H = cache->H, T = cache->T, Tk = cache->Tk;
+    const long long n_q = static_cast<long long>(C) * T;
+    const long long row0 = static_cast<long long>(cache->frames) * Tk;  // first new descriptor
+    const long long n_new = static_cast<long long>(C) * Tk;
+    // Scratch: the chunk's pooled raw keys [C*Tk, H, 64] and q_hat [H, C*T, 64].
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, head_plane_bytes(n_new, H) + head_plane_bytes(n_q, H),
+                                st->pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_ALLOC;
+    }
+    uint16_t* k_raw = static_cast<uint16_t*>(scratch);
+    uint16_t* q_hat = k_raw + head_plane_bytes(n_new, H) / sizeof(uint16_t);
+    uint16_t* v_new = cache->v + row0 * H * VGGT_HEAD_DIM;
+    float* pos_new = cache->pos + row0 * 2;
+    // 1. The chunk's descriptors: pooled values and positions straight into
+    //    the cache, pooled keys into scratch ...
+    rc = to_status(vggt::launch_kv_pool(k, v, pos, k_raw, v_new, pos_new, C, T, cache->g,
+                                        cache->kv_down, H, stream));
+    // 2. ... then normalised into the cache's key planes (row0 onwards of
+    //    each head's plane), together with the chunk's queries.
+    if (rc == VGGT_OK) {
+        PrologueJob jq{q, pos, q_hat, static_cast<int>(n_q), n_q};
+        PrologueJob jk{k_raw, pos_new, cache->k_hat + row0 * VGGT_HEAD_DIM, static_cast<int>(n_new),
+                       cache->capacity};
+        rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
+    }
+    // 3. Every query of the chunk attends to every cached descriptor.
+    if (rc == VGGT_OK) {
+        AttnProblem p{q_hat, cache->k_hat, cache->v, out, 1, static_cast<int>(n_q),
+                      static_cast<int>(row0 + n_new), H, n_q, cache->capacity};
+        rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
+    }
+    cudaFreeAsync(scratch, stream);
+    if (rc == VGGT_OK) cache->frames += C;
+    return rc;
+}
+
 int vggt_release_scratch(void) {
     DeviceState* st = device_state();
     if (!st) return VGGT_ERR_CUDA;
@@ -284,7 +412,9 @@ const char* vggt_status_string(int status) {
     switch (status) {
         case VGGT_OK: return "VGGT_OK";
         case VGGT_ERR_NULL: return "VGGT_ERR_NULL: a required pointer is NULL";
-        case VGGT_ERR_UNSUPPORTED: return "VGGT_ERR_UNSUPPORTED: head dimension must be 64";
+        case VGGT_ERR_UNSUPPORTED:
+            return "VGGT_ERR_UNSUPPORTED: head dimension must be 64, pointers aligned (16 bytes; "
+                   "positions 8), and the current device the cache's";
         case VGGT_ERR_SHAPE: return "VGGT_ERR_SHAPE: invalid sizes";
         case VGGT_ERR_ALLOC: return "VGGT_ERR_ALLOC: scratch allocation failed";
         case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA: CUDA call or launch failed";

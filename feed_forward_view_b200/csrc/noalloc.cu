@@ -76,7 +76,8 @@ extern "C" int vggt_attn_global_noalloc(const vggt_bf16* q, const vggt_bf16* k,
     if (2ull * plane > VGGT_NOALLOC_SCRATCH_BYTES) return VGGT_ERR_SHAPE;
     if (S == 0 || H == 0) return VGGT_OK;
     if (!q || !k || !v || !pos || !out) return VGGT_ERR_NULL;
-    if (!is_aligned16(q) || !is_aligned16(k) || !is_aligned16(v) || !is_aligned16(pos) ||
+    if (!is_aligned16(q) || !is_aligned16(k) || !is_aligned16(v) ||
+        (reinterpret_cast<uintptr_t>(pos) & 7u) != 0 ||
         !is_aligned16(out))
         return VGGT_ERR_UNSUPPORTED;
 

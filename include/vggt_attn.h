@@ -30,7 +30,8 @@
  *
  * Common rules:
  *   - D must be 64 (VGGT: 16 heads x 64 dims). H >= 1 is free.
- *   - Every pointer must be 16-byte aligned (TMA and 16-byte vector access).
+ *   - Every bf16 pointer must be 16-byte aligned (TMA and 16-byte vector
+ *     access); positions (pos, pos_out) 8-byte aligned (read as pairs).
  *   - S == 0 or H == 0 is an empty problem: VGGT_OK, nothing is launched.
  *   - Everything is asynchronous on `stream`; no call synchronises it.
  *   - Scratch (normalised q/k, pooled k/v) comes from a stream-ordered memory
@@ -67,7 +68,8 @@ typedef uint16_t vggt_bf16; /* raw bf16 bits */
 typedef enum vggt_status {
     VGGT_OK = 0,
     VGGT_ERR_NULL = -1,        /* a required pointer is NULL                      */
-    VGGT_ERR_UNSUPPORTED = -2, /* D != 64, or a pointer not 16-byte aligned        */
+    VGGT_ERR_UNSUPPORTED = -2, /* D != 64, a misaligned pointer, or a cache used on
+                                  another device than its own                      */
     VGGT_ERR_SHAPE = -3,       /* negative sizes, T != 5 + g*g, bad kv_down, or a
                                   size beyond the library's limits                */
     VGGT_ERR_ALLOC = -4,       /* scratch allocation failed                        */
@@ -170,6 +172,61 @@ VGGT_API int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, cons
 VGGT_API int vggt_kv_pool(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                  vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out,
                  int S, int T, int H, int D, int kv_down, cudaStream_t stream);
+
+/*
+ * Streaming (chunk-recursive) descriptor attention -- the FlashVGGTStream
+ * mode: "the compactness of the descriptors enables online inference over
+ * long sequences via a chunk-recursive mechanism that reuses cached
+ * descriptors from previous chunks" (FlashVGGT README, Overview; streaming
+ * inference with --chunksize, default 10, Key Arguments). Frames arrive in
+ * chunks; every query of a chunk attends to the descriptors of all frames
+ * seen so far -- the cached descriptors of earlier chunks and its own
+ * chunk's (pooled exactly as vggt_kv_pool, keys normalised by the prologue
+ * at their cell-mean positions).
+ *
+ * A vggt_desc_cache holds those descriptors on one device: normalised keys,
+ * values and positions of up to max_frames frames. It is owned by the caller
+ * (create / destroy) and used by one sequence at a time (reset starts a new
+ * one). Calls that use a cache must be ordered by the caller (one stream, or
+ * streams synchronised with each other).
+ */
+typedef struct vggt_desc_cache vggt_desc_cache;
+
+/* Creates a cache on the current device for up to max_frames frames of T =
+   5 + g*g tokens, H heads of D = 64 dims, pooled kv_down x kv_down. Takes
+   max_frames * T_k * H * D * 2 * 2 + max_frames * T_k * 8 bytes with
+   cudaMalloc (T_k = vggt_kv_pool_tokens(T, kv_down)). On failure *cache is
+   NULL and a negative vggt_status is returned (VGGT_ERR_NULL, _SHAPE,
+   _UNSUPPORTED for D != 64, _ALLOC, _CUDA). Host only; synchronous. */
+VGGT_API int vggt_desc_cache_create(vggt_desc_cache** cache, int max_frames, int T, int H, int D,
+                                    int kv_down);
+
+/* Frees the cache's memory (cudaFree, on the cache's device) and the cache.
+   NULL is a no-op. Make sure no call that uses it is still running. */
+VGGT_API int vggt_desc_cache_destroy(vggt_desc_cache* cache);
+
+/* Frames the cache holds (>= 0), or VGGT_ERR_NULL. Host only. */
+VGGT_API int vggt_desc_cache_frames(const vggt_desc_cache* cache);
+
+/* Forgets every cached frame (a new sequence). Host only; no device work. */
+VGGT_API int vggt_desc_cache_reset(vggt_desc_cache* cache);
+
+/*
+ * One chunk of C frames of the sequence:
+ *   1. pools the chunk's K/V per frame (as vggt_kv_pool) and appends the
+ *      descriptors to the cache, their keys normalised once, in the cache;
+ *   2. every token of the chunk attends to all descriptors now in the cache.
+ * q, k, v, out: [C, T, H, D] bf16; pos [C, T, 2] fp32 (the cache's T, H, D).
+ * out is the same as vggt_attn_descriptor over all frames cached so far,
+ * restricted to the chunk's queries. Runs on the cache's device (else
+ * VGGT_ERR_UNSUPPORTED); fails with VGGT_ERR_SHAPE, launching nothing and
+ * leaving the cache unchanged, if the chunk does not fit. C == 0 is a no-op.
+ * The cache's frame count grows by C when the call returns VGGT_OK.
+ * Scratch: the chunk's q_hat and pooled raw keys, from the scratch pool.
+ */
+VGGT_API int vggt_attn_descriptor_chunk(vggt_desc_cache* cache, const vggt_bf16* q,
+                                        const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                                        vggt_bf16* out, int C, cudaStream_t stream);
 
 /* Size of the fixed scratch array vggt_attn_global_noalloc draws on. */
 #define VGGT_NOALLOC_SCRATCH_BYTES (16u << 20)

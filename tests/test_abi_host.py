@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol_and_nothing_else():
 
 
 def test_status_strings():
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert F.vggt_status_string(code).startswith("VGGT_")
     assert "unknown" in F.vggt_status_string(7)
 
@@ -73,7 +73,7 @@ def test_attention_argument_checks(name):
         assert fn(*q, 2, 261, 16, 64, kd, None) == E_NULL
     for i in range(5):
         q = list(p)
-        q[i] = FAKE + 8  # not 16-byte aligned
+        q[i] = FAKE + (4 if i == 3 else 8)  # bf16 arrays need 16 bytes, positions 8
         assert fn(*q, 2, 261, 16, 64, kd, None) == E_UNSUP
     # empty problems succeed without touching any pointer
     assert fn(None, None, None, None, None, 0, 261, 16, 64, kd, None) == OK
@@ -117,3 +117,21 @@ def test_binding_rejects_host_tensors():
     pos = torch.zeros(261 * 2, 2)
     with pytest.raises(ValueError):
         F.vggt_attn_global(q, q, q, pos, q.clone(), S=2, T=261)
+
+
+def test_descriptor_cache_argument_checks():
+    import ctypes
+
+    h = ctypes.c_void_p()
+    create = F.lib.vggt_desc_cache_create
+    assert create(None, 4, 41, 16, 64, 4) == E_NULL
+    assert create(ctypes.byref(h), 0, 41, 16, 64, 4) == E_SHAPE and not h.value
+    assert create(ctypes.byref(h), 4, 40, 16, 64, 4) == E_SHAPE  # 40 - 5 is not a square
+    assert create(ctypes.byref(h), 4, 41, 16, 64, 0) == E_SHAPE
+    assert create(ctypes.byref(h), 4, 41, 16, 32, 4) == E_UNSUP
+    assert create(ctypes.byref(h), 1 << 20, 1374, 16, 64, 4) == E_SHAPE  # beyond VGGT_MAX_TOKENS
+    assert F.lib.vggt_desc_cache_frames(None) == E_NULL
+    assert F.lib.vggt_desc_cache_reset(None) == E_NULL
+    assert F.lib.vggt_desc_cache_destroy(None) == OK
+    fake = ctypes.c_void_p(0x1000)
+    assert F.lib.vggt_attn_descriptor_chunk(None, fake, fake, fake, fake, fake, 1, None) == E_NULL

@@ -302,3 +302,73 @@ def test_scratch_pool_release_and_reuse(F):
     F.vggt_release_scratch()  # nothing left to release: still fine
     assert torch.equal(run_gpu(F, "descriptor", q, k, v, pos, S, T, kd), a)
     assert torch.equal(run_gpu(F, "global", q, k, v, pos, S, T, 1), b)
+
+
+# ------------------------------------------------------ streaming descriptors
+
+
+def _stream_gpu(F, q, k, v, pos, S, T, kd, chunk, H=16):
+    """Feed the scene chunk by chunk through one descriptor cache."""
+    dev = torch.device("cuda:0")
+    qd, kd_, vd, pd = (t.to(dev) for t in (q, k, v, pos))
+    out = torch.empty_like(qd)
+    with F.DescCache(S, T, H=H, kv_down=kd) as cache:
+        for f0 in range(0, S, chunk):
+            c = min(chunk, S - f0)
+            r0, r1 = f0 * T, (f0 + c) * T
+            cache.attend(qd[r0:r1], kd_[r0:r1], vd[r0:r1], pd[r0:r1], out[r0:r1], C=c)
+            assert cache.frames == f0 + c
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    return out.cpu()
+
+
+@pytest.mark.parametrize("S,g,kd,chunk", [(6, 9, 3, 2), (5, 11, 4, 2), (4, 6, 1, 3), (3, 7, 2, 1)])
+def test_stream_chunks_match_oracle(F, S, g, kd, chunk):
+    q, k, v, pos = synth.make_qkv(S, g, seed=50 + S)
+    T = 5 + g * g
+    got = f64(_stream_gpu(F, q, k, v, pos, S, T, kd, chunk))
+    ref = O.attn_descriptor_stream(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, kd, chunk)
+    mx, rf = errors(got, ref)
+    assert np.isfinite(got).all()
+    assert mx <= MAX_ABS and rf <= REL_FRO, (S, g, kd, chunk, mx, rf)
+
+
+def test_stream_single_chunk_equals_descriptor_call(F):
+    S, g, kd = 4, 10, 3
+    q, k, v, pos = synth.make_qkv(S, g, seed=60)
+    T = 5 + g * g
+    a = _stream_gpu(F, q, k, v, pos, S, T, kd, S)
+    b = run_gpu(F, "descriptor", q, k, v, pos, S, T, kd)
+    assert torch.equal(a, b)
+
+
+def test_stream_cache_capacity_and_reset(F):
+    S, g, kd = 3, 6, 2
+    q, k, v, pos = (t.cuda() for t in synth.make_qkv(S, g, seed=61))
+    T = 5 + g * g
+    out1 = torch.empty_like(q)
+    out2 = torch.empty_like(q)
+    with F.DescCache(2, T, kv_down=kd) as cache:
+        cache.attend(q[:2 * T], k[:2 * T], v[:2 * T], pos[:2 * T], out1[:2 * T], C=2)
+        with pytest.raises(F.VggtError):
+            cache.attend(q[2 * T:], k[2 * T:], v[2 * T:], pos[2 * T:], out1[2 * T:], C=1)  # 3 > 2 frames
+        assert cache.frames == 2
+        cache.reset()
+        assert cache.frames == 0
+        cache.attend(q[:2 * T], k[:2 * T], v[:2 * T], pos[:2 * T], out2[:2 * T], C=2)
+    torch.cuda.synchronize()
+    assert torch.equal(out1[:2 * T], out2[:2 * T])
+
+
+def test_stream_full_size_sampled_rows(F):
+    # The descriptor workload's scene (200 frames of 1374 tokens, 4x4 pooling)
+    # streamed in chunks of 10 frames, checked on rows sampled across chunks.
+    w = synth.WORKLOADS["descriptor_s200_g37_kd4"]
+    q, k, v, pos = synth.make_workload(w, 1)
+    got = _stream_gpu(F, q, k, v, pos, w.S, w.T, w.kv_down, 10)
+    rows = synth.sample_rows(w.n_q, 160, seed=5).numpy()
+    ref = O.attn_descriptor_stream(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), w.S, w.T,
+                                   w.kv_down, 10, rows=rows)
+    mx, rf = errors(f64(got)[rows], ref)
+    assert mx <= MAX_ABS and rf <= REL_FRO, (mx, rf)
