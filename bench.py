@@ -199,12 +199,18 @@ class OracleLeg:
 
     def run(self, n_rows: int, seed: int = 0):
         """Returns (TFLOP/s, seconds, rows)."""
+        import numpy
+
         w, O = self.w, self.O
         rows = self.synth.sample_rows(w.n_q, n_rows, seed).numpy()
         t0 = time.perf_counter()
         if w.kind == "frame":
             O.attn_frame(self.q, self.k, self.v, self.pos, w.S, w.T, rows=rows)
             keys = w.T
+        elif w.kind == "stream":
+            O.attn_descriptor_stream(self.q, self.k, self.v, self.pos, w.S, w.T, w.kv_down, w.chunk, rows=rows)
+            chunk_of = rows // (w.T * w.chunk)
+            keys = float((numpy.minimum(w.S, (chunk_of + 1) * w.chunk) * w.T_k).mean())
         else:
             O.cross_attention(O.qk_prologue(self.q[rows], self.pos[rows]), self.k_hat, self.vv)
             keys = w.n_k
@@ -247,8 +253,10 @@ def run_reference(args):
         times.append(dt)
     threads = blas_threads()
     value = statistics.median(vals)
-    sample = (f"{rows} query rows x all {w.n_k if w.kind != 'frame' else w.T} keys x {w.H} heads per step "
-              f"(of {w.n_q} rows), key prologue precomputed")
+    keys_desc = ({"frame": f"all {w.T}", "stream": "the cached-prefix"}.get(w.kind, f"all {w.n_k}"))
+    sample = (f"{rows} query rows x {keys_desc} keys x {w.H} heads per step "
+              f"(of {w.n_q} rows)" + ("; pooling and key prologue redone each step" if w.kind == "stream"
+                                       else ", key prologue precomputed"))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -278,8 +286,6 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.ALL_WORKLOADS[args.workload]
-    fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
-          "descriptor": F.vggt_attn_descriptor}[w.kind]
 
     q_h, k_h, v_h, pos_h = synth.make_workload(w, seed=rank)
     q, k, v, pos = (t.to(dev) for t in (q_h, k_h, v_h, pos_h))
@@ -287,8 +293,25 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, pos))
 
+    if w.kind == "stream":
+        # the whole sequence through one descriptor cache, chunk by chunk
+        cache = F.DescCache(w.S, w.T, H=w.H, kv_down=w.kv_down)
+        chunks = [(f0 * w.T, (f0 + min(w.chunk, w.S - f0)) * w.T, min(w.chunk, w.S - f0))
+                  for f0 in range(0, w.S, w.chunk)]
+
+        def call(qq, kk, vv, pp, oo):
+            cache.reset()
+            for r0, r1, c in chunks:
+                cache.attend(qq[r0:r1], kk[r0:r1], vv[r0:r1], pp[r0:r1], oo[r0:r1], C=c)
+    else:
+        fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
+              "descriptor": F.vggt_attn_descriptor}[w.kind]
+
+        def call(qq, kk, vv, pp, oo):
+            fn(qq, kk, vv, pp, oo, S=w.S, T=w.T, kv_down=w.kv_down)
+
     def step():
-        fn(q, k, v, pos, out, S=w.S, T=w.T, kv_down=w.kv_down)
+        call(q, k, v, pos, out)
 
     # ---- warm-up, then the timed region: K steps between two barriers. The
     # clock sampler starts first; the warm-up (at least W steps, continued until
@@ -320,17 +343,21 @@ def run_gpu(args):
     ms_local = e0.elapsed_time(e1)
     status = F.vggt_get_device_status()
     ms_total = max_over_ranks(ms_local, world, dev)
-    launches = 2 + (1 if w.kind == "descriptor" else 0)  # prologue + attention (+ pool)
+    # prologue + attention (+ pool), per call or per chunk
+    launches = 3 * len(chunks) if w.kind == "stream" else 2 + (1 if w.kind == "descriptor" else 0)
     ms_step = ms_total / args.steps
     flops = w.flops()
     value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
     tokens_s = world * w.n_q * args.steps / (ms_total * 1e-3)
 
-    # ---- kernel-only timings (same kernels, launched one by one with events)
+    # ---- kernel-only timings (same kernels, launched one by one with events);
+    # a streamed sequence is many calls of growing size: there the step itself
+    # stands for the attention kernel
     H = w.H
+    kind_core = "descriptor" if w.kind == "stream" else w.kind
     q_hat = torch.empty((H, w.n_q, 64), dtype=torch.bfloat16, device=dev)
     k_hat = torch.empty((H, w.n_k, 64), dtype=torch.bfloat16, device=dev)
-    if w.kind == "descriptor":
+    if kind_core == "descriptor":
         kp, vp, pp = F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down)
         F.vggt_qk_prologue(kp, pp, k_hat)
         v_use = vp
@@ -340,16 +367,19 @@ def run_gpu(args):
     F.vggt_qk_prologue(q, pos, q_hat)
     n_seg, q_len, k_len = (w.S, w.T, w.T) if w.kind == "frame" else (1, w.n_q, w.n_k)
     reps = max(5, min(args.steps, 50))
-    for _ in range(3):
-        F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
-    torch.cuda.synchronize(dev)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(reps):
-        F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
-    a1.record(stream)
-    torch.cuda.synchronize(dev)
-    attn_ms = a0.elapsed_time(a1) / reps
+    if w.kind == "stream":
+        attn_ms = ms_step
+    else:
+        for _ in range(3):
+            F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
+        torch.cuda.synchronize(dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        attn_ms = a0.elapsed_time(a1) / reps
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     for _ in range(reps):
@@ -359,7 +389,7 @@ def run_gpu(args):
     pro_ms = p0.elapsed_time(p1) / reps
     pro_bytes = 2 * w.n_q * H * 64 * 2 + w.n_q * 8  # read x + pos, write x_hat
     pool = None
-    if w.kind == "descriptor":
+    if kind_core == "descriptor":
         # K/V pooling alone: reads k, v and pos of every token, writes the
         # pooled k, v and positions.
         kp_o, vp_o, pp_o = (torch.empty_like(t) for t in (kp, vp, pp))
@@ -403,7 +433,7 @@ def run_gpu(args):
             b = i % 2
             stream.wait_event(uploaded[b])
             dq, dk, dv, dp = dev_in[b]
-            fn(dq, dk, dv, dp, dev_out[b], S=w.S, T=w.T, kv_down=w.kv_down)
+            call(dq, dk, dv, dp, dev_out[b])
             hout[b].copy_(dev_out[b], non_blocking=True)
             computed[b].record(stream)
 
@@ -439,8 +469,11 @@ def run_gpu(args):
     if world == 1 and not args.skip_cpu:
         tf, dt, rows = OracleLeg(w).run(args.cpu_rows)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{rows} of {w.n_q} query rows x all keys x {w.H} heads, fp64 numpy, "
-                         f"{dt:.1f} s; key prologue precomputed"}
+               "sample": f"{rows} of {w.n_q} query rows x "
+                         f"{'the cached-prefix' if w.kind == 'stream' else 'all'} keys x {w.H} heads, "
+                         f"fp64 numpy, {dt:.1f} s"
+                         + ("; pooling and key prologue redone" if w.kind == "stream"
+                            else "; key prologue precomputed")}
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -461,7 +494,10 @@ def run_gpu(args):
                        "l2": f"inputs {in_bytes / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
             "tokens_per_s": tokens_s,
             "pct_of_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tf,
+            "roofline": {"bound": "tensor",
+                         "kernel": ("stream step: per chunk pool + prologue + attn_fwd_kernel"
+                                    if w.kind == "stream" else "attn_fwd_kernel"),
+                         "achieved": attn_tf,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
                          "peak_source": f"{peak_src} bf16 burst",
                          "frac_of_sustained": attn_tf / float(peaks.get("bf16_tflops_sustained", peak)),

@@ -34,12 +34,13 @@ class Workload:
     """One attention workload: kind, frame count, grid side and pooling factor."""
 
     name: str
-    kind: str  # "global" | "frame" | "descriptor"
+    kind: str  # "global" | "frame" | "descriptor" | "stream" (descriptors, chunk by chunk)
     S: int
     g: int
     kv_down: int = 1
     H: int = HEADS
     D: int = HEAD_DIM
+    chunk: int = 0  # frames per chunk ("stream")
 
     @property
     def T(self) -> int:
@@ -51,7 +52,7 @@ class Workload:
 
     @property
     def T_k(self) -> int:
-        if self.kind != "descriptor":
+        if self.kind not in ("descriptor", "stream"):
             return self.T
         nc = -(-self.g // self.kv_down) if self.g > 0 else 0
         return N_SPECIAL + nc * nc
@@ -64,6 +65,10 @@ class Workload:
         """Algorithmic attention FLOPs: 4 * H * D per (query, key) pair."""
         if self.kind == "frame":
             pairs = self.S * self.T * self.T
+        elif self.kind == "stream":
+            # chunk c's queries see the descriptors of chunks 0..c
+            pairs = sum(min(self.chunk, self.S - f0) * self.T * min(self.S, f0 + self.chunk) * self.T_k
+                        for f0 in range(0, self.S, self.chunk))
         else:
             pairs = self.n_q * self.n_k
         return 4.0 * self.H * self.D * pairs
@@ -90,7 +95,13 @@ PROFILE_WORKLOADS = {w.name: w for w in (
     Workload("global_s6_g64", "global", S=6, g=64),
     Workload("descriptor_s40_g37_kd4", "descriptor", S=40, g=37, kv_down=4),
 )}
-ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS}
+
+# The descriptor workload streamed in chunks of 10 frames (FlashVGGTStream's
+# default chunk size), for measurement.
+STREAM_WORKLOADS = {w.name: w for w in (
+    Workload("stream_s200_g37_kd4_c10", "stream", S=200, g=37, kv_down=4, chunk=10),
+)}
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS}
 
 
 def grid_side(T: int) -> int:
