@@ -38,6 +38,18 @@ What it computes, per head, for bf16 inputs widened exactly to float64:
      reuses cached descriptors from previous chunks; streaming inference with
      ``--chunksize``, default 10).
 
+Options beyond the pages' default reading (both off by default):
+
+* ``layout = (n_front, grid_h, grid_w, n_back)``: a frame of ``n_front``
+  special tokens, a rectangular patch grid (vggt-jax README: its two-image
+  benchmark feeds 350 x 518 images, a 25 x 37 grid) and ``n_back`` trailing
+  tokens (the VGGT-Omega page appends its register tokens after the patches).
+  Pooling copies front and trailing tokens and averages the grid's cells.
+* ``ln = (q_gamma, q_beta, k_gamma, k_beta)``: a per-dim scale and shift after
+  each QK LayerNorm, shared by the heads, applied before the rotation (a
+  trained LayerNorm carries them; the pages give no values, so the default is
+  the identity).
+
 Evaluating a subset of query rows is the same definition restricted to those
 rows: every output row depends only on its own query and the key set, so
 ``rows=`` changes nothing about any row that is computed.
@@ -103,14 +115,21 @@ def softmax(x: np.ndarray, axis: int = -1) -> np.ndarray:
     return e / np.sum(e, axis=axis, keepdims=True)
 
 
-def layer_norm(x: np.ndarray, eps: float = LN_EPS) -> np.ndarray:
+def layer_norm(x: np.ndarray, eps: float = LN_EPS, gamma=None, beta=None) -> np.ndarray:
     """``(x - mu) / sqrt(var + eps)`` over the last axis; biased variance,
-    computed from the centered values; no scale or shift."""
+    computed from the centered values. With ``gamma`` / ``beta`` (vectors of
+    the last axis' length) the result is then scaled by ``gamma`` and shifted
+    by ``beta``, element by element; by default there is no scale or shift."""
     x = np.asarray(x, dtype=np.float64)
     mu = x.mean(axis=-1, keepdims=True)
     c = x - mu
     var = (c * c).mean(axis=-1, keepdims=True)
-    return c / np.sqrt(var + eps)
+    y = c / np.sqrt(var + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, dtype=np.float64)
+    if beta is not None:
+        y = y + np.asarray(beta, dtype=np.float64)
+    return y
 
 
 def rope_frequencies(base: float, d: int) -> np.ndarray:
@@ -156,9 +175,19 @@ def rope_2d(x: np.ndarray, pos: np.ndarray, base: float = ROPE_BASE) -> np.ndarr
     return out
 
 
-def qk_prologue(x: np.ndarray, pos: np.ndarray) -> np.ndarray:
-    """LayerNorm then 2D RoPE for ``x[N, H, D]`` at ``pos[N, 2]``."""
-    return rope_2d(layer_norm(x), np.asarray(pos)[:, None, :])
+def qk_prologue(x: np.ndarray, pos: np.ndarray, gamma=None, beta=None) -> np.ndarray:
+    """LayerNorm (with the optional per-dim ``gamma`` / ``beta``, shared by all
+    heads) then 2D RoPE for ``x[N, H, D]`` at ``pos[N, 2]``."""
+    return rope_2d(layer_norm(x, gamma=gamma, beta=beta), np.asarray(pos)[:, None, :])
+
+
+def _ln(ln, which: str):
+    """``(gamma, beta)`` of the query (``which == "q"``) or key LayerNorm from
+    ``ln = (q_gamma, q_beta, k_gamma, k_beta)`` (entries may be None), or no
+    affine when ``ln`` is None."""
+    if ln is None:
+        return None, None
+    return (ln[0], ln[1]) if which == "q" else (ln[2], ln[3])
 
 
 # --------------------------------------------------------------------------
@@ -175,54 +204,84 @@ def grid_side(T: int) -> int:
     return g if g * g == p else -1
 
 
-def pool_cells(g: int, kd: int):
-    """Ceil-mode ``kd x kd`` cells of a ``g x g`` grid, row-major.
+def frame_layout(T: int, layout=None):
+    """The token layout of one frame as ``(n_front, grid_h, grid_w, n_back)``:
+    ``n_front`` special tokens, then the ``grid_h x grid_w`` patch grid in
+    row-major order, then ``n_back`` trailing tokens (the VGGT-Omega page puts
+    its register tokens after each frame's patches). Without ``layout`` the
+    frame is VGGT-1B's: 5 special tokens in front of a square grid."""
+    if layout is None:
+        g = grid_side(T)
+        if g < 0:
+            raise ValueError(f"T={T} is not 5 + g*g")
+        return (N_SPECIAL, g, g, 0)
+    nf, gh, gw, nb = (int(x) for x in layout)
+    if min(nf, gh, gw, nb) < 0 or nf + gh * gw + nb != T:
+        raise ValueError(f"layout {layout} does not describe T={T} tokens")
+    return (nf, gh, gw, nb)
 
-    Each cell is a list of member patch indices ``r*g + c`` in row-major
+
+def pool_cells_rect(gh: int, gw: int, kd: int):
+    """Ceil-mode ``kd x kd`` cells of a ``gh x gw`` grid, row-major.
+
+    Each cell is a list of member patch indices ``r*gw + c`` in row-major
     order; edge cells keep only the members that lie inside the grid.
     """
-    nc = -(-g // kd) if g > 0 else 0
+    nch = -(-gh // kd) if gh > 0 else 0
+    ncw = -(-gw // kd) if gw > 0 else 0
     cells = []
-    for cr in range(nc):
-        for cc in range(nc):
-            rows = range(cr * kd, min(cr * kd + kd, g))
-            cols = range(cc * kd, min(cc * kd + kd, g))
-            cells.append([r * g + c for r in rows for c in cols])
+    for cr in range(nch):
+        for cc in range(ncw):
+            rows = range(cr * kd, min(cr * kd + kd, gh))
+            cols = range(cc * kd, min(cc * kd + kd, gw))
+            cells.append([r * gw + c for r in rows for c in cols])
     return cells
 
 
-def pooled_tokens_per_frame(T: int, kd: int) -> int:
-    g = grid_side(T)
-    nc = -(-g // kd) if g > 0 else 0
-    return N_SPECIAL + nc * nc
+def pool_cells(g: int, kd: int):
+    """The cells of a square ``g x g`` grid (``pool_cells_rect(g, g, kd)``)."""
+    return pool_cells_rect(g, g, kd)
 
 
-def kv_pool(k: np.ndarray, v: np.ndarray, pos: np.ndarray, S: int, T: int, kd: int):
-    """Per-frame descriptors in float64: the 5 special tokens unchanged, then
-    the mean of each ceil-mode ``kd x kd`` cell of the patch grid (K, V and
-    position alike). Inputs are ``[S*T, H, D]`` and ``[S*T, 2]``."""
-    g = grid_side(T)
-    cells = pool_cells(g, kd)
-    Tk = N_SPECIAL + len(cells)
+def pooled_tokens_per_frame(T: int, kd: int, layout=None) -> int:
+    nf, gh, gw, nb = frame_layout(T, layout)
+    return nf + len(pool_cells_rect(gh, gw, kd)) + nb
+
+
+def _pooled_sources(T: int, kd: int, layout):
+    """For every pooled token of a frame, in order, ``(sources, is_special)``:
+    front specials and trailing tokens are their own single source and are
+    copied; each cell lists its patches in row-major order."""
+    nf, gh, gw, nb = frame_layout(T, layout)
+    src = [([t], True) for t in range(nf)]
+    src += [([nf + m for m in members], False) for members in pool_cells_rect(gh, gw, kd)]
+    src += [([nf + gh * gw + t], True) for t in range(nb)]
+    return src
+
+
+def kv_pool(k: np.ndarray, v: np.ndarray, pos: np.ndarray, S: int, T: int, kd: int, layout=None):
+    """Per-frame descriptors in float64: the special (front and trailing)
+    tokens unchanged, and the mean of each ceil-mode ``kd x kd`` cell of the
+    patch grid (K, V and position alike), ordered front specials, cells
+    (row-major), trailing tokens. Inputs are ``[S*T, H, D]`` and ``[S*T, 2]``."""
+    src = _pooled_sources(T, kd, layout)
+    Tk = len(src)
     k = np.asarray(k, dtype=np.float64).reshape(S, T, *k.shape[1:])
     v = np.asarray(v, dtype=np.float64).reshape(S, T, *v.shape[1:])
     pos = np.asarray(pos, dtype=np.float64).reshape(S, T, 2)
     kp = np.empty((S, Tk) + k.shape[2:])
     vp = np.empty((S, Tk) + v.shape[2:])
     pp = np.empty((S, Tk, 2))
-    kp[:, :N_SPECIAL] = k[:, :N_SPECIAL]
-    vp[:, :N_SPECIAL] = v[:, :N_SPECIAL]
-    pp[:, :N_SPECIAL] = pos[:, :N_SPECIAL]
-    for ci, members in enumerate(cells):
-        idx = N_SPECIAL + np.asarray(members)
-        kp[:, N_SPECIAL + ci] = k[:, idx].mean(axis=1)
-        vp[:, N_SPECIAL + ci] = v[:, idx].mean(axis=1)
-        pp[:, N_SPECIAL + ci] = pos[:, idx].mean(axis=1)
+    for i, (members, _) in enumerate(src):
+        idx = np.asarray(members)
+        kp[:, i] = k[:, idx].mean(axis=1)
+        vp[:, i] = v[:, idx].mean(axis=1)
+        pp[:, i] = pos[:, idx].mean(axis=1)
     return (kp.reshape(S * Tk, *k.shape[2:]), vp.reshape(S * Tk, *v.shape[2:]),
             pp.reshape(S * Tk, 2))
 
 
-def kv_pool_bf16_reference(k_bits, v_bits, pos, S: int, T: int, kd: int):
+def kv_pool_bf16_reference(k_bits, v_bits, pos, S: int, T: int, kd: int, layout=None):
     """The stored form of the pooled descriptors, bit for bit.
 
     For every cell and channel: float32 sum of the members in row-major order
@@ -231,9 +290,8 @@ def kv_pool_bf16_reference(k_bits, v_bits, pos, S: int, T: int, kd: int):
     sum and division, kept in float32. Special tokens are copied unchanged.
     Returns ``(k_bits, v_bits, pos_f32)``.
     """
-    g = grid_side(T)
-    cells = pool_cells(g, kd)
-    Tk = N_SPECIAL + len(cells)
+    src = _pooled_sources(T, kd, layout)
+    Tk = len(src)
     k32 = bf16_bits_to_f32(k_bits).reshape(S, T, -1)
     v32 = bf16_bits_to_f32(v_bits).reshape(S, T, -1)
     p32 = np.asarray(pos, dtype=np.float32).reshape(S, T, 2)
@@ -242,22 +300,23 @@ def kv_pool_bf16_reference(k_bits, v_bits, pos, S: int, T: int, kd: int):
     ko = np.empty((S, Tk, kb.shape[2]), dtype=np.uint16)
     vo = np.empty((S, Tk, vb.shape[2]), dtype=np.uint16)
     po = np.empty((S, Tk, 2), dtype=np.float32)
-    ko[:, :N_SPECIAL] = kb[:, :N_SPECIAL]
-    vo[:, :N_SPECIAL] = vb[:, :N_SPECIAL]
-    po[:, :N_SPECIAL] = p32[:, :N_SPECIAL]
-    for ci, members in enumerate(cells):
+    for i, (members, special) in enumerate(src):
+        if special:  # copied as it is (a one-member cell is still summed: -0 becomes +0)
+            ko[:, i] = kb[:, members[0]]
+            vo[:, i] = vb[:, members[0]]
+            po[:, i] = p32[:, members[0]]
+            continue
         ak = np.zeros((S, k32.shape[2]), dtype=np.float32)
         av = np.zeros((S, v32.shape[2]), dtype=np.float32)
         ap = np.zeros((S, 2), dtype=np.float32)
-        for m in members:  # row-major member order
-            t = N_SPECIAL + m
+        for t in members:  # row-major member order
             ak = ak + k32[:, t]
             av = av + v32[:, t]
             ap = ap + p32[:, t]
         n = np.float32(len(members))
-        ko[:, N_SPECIAL + ci] = f32_to_bf16_bits(ak / n)
-        vo[:, N_SPECIAL + ci] = f32_to_bf16_bits(av / n)
-        po[:, N_SPECIAL + ci] = ap / n
+        ko[:, i] = f32_to_bf16_bits(ak / n)
+        vo[:, i] = f32_to_bf16_bits(av / n)
+        po[:, i] = ap / n
     return ko.reshape(S * Tk, -1), vo.reshape(S * Tk, -1), po.reshape(S * Tk, 2)
 
 
@@ -295,16 +354,19 @@ def _rows(n: int, rows):
     return np.arange(n) if rows is None else np.asarray(rows)
 
 
-def attn_global(q, k, v, pos, S: int, T: int, rows=None) -> np.ndarray:
-    """Global attention: all ``S*T`` tokens attend to all ``S*T`` tokens."""
+def attn_global(q, k, v, pos, S: int, T: int, rows=None, ln=None) -> np.ndarray:
+    """Global attention: all ``S*T`` tokens attend to all ``S*T`` tokens.
+    ``ln = (q_gamma, q_beta, k_gamma, k_beta)`` gives the QK LayerNorms an
+    affine (any entry may be None); by default they have none."""
     rows = _rows(S * T, rows)
-    q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows])
-    k_hat = qk_prologue(k, pos)
+    q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows], *_ln(ln, "q"))
+    k_hat = qk_prologue(k, pos, *_ln(ln, "k"))
     return cross_attention(q_hat, k_hat, np.asarray(v, dtype=np.float64))
 
 
-def attn_frame(q, k, v, pos, S: int, T: int, rows=None) -> np.ndarray:
-    """Frame attention: each token attends to the ``T`` tokens of its frame."""
+def attn_frame(q, k, v, pos, S: int, T: int, rows=None, ln=None) -> np.ndarray:
+    """Frame attention: each token attends to the ``T`` tokens of its frame
+    (``ln`` as for ``attn_global``)."""
     rows = _rows(S * T, rows)
     q, k, pos = np.asarray(q), np.asarray(k), np.asarray(pos)
     v = np.asarray(v, dtype=np.float64)
@@ -313,33 +375,36 @@ def attn_frame(q, k, v, pos, S: int, T: int, rows=None) -> np.ndarray:
     for s in np.unique(frames):
         sel = np.nonzero(frames == s)[0]
         lo, hi = s * T, (s + 1) * T
-        q_hat = qk_prologue(q[rows[sel]], pos[rows[sel]])
-        k_hat = qk_prologue(k[lo:hi], pos[lo:hi])
+        q_hat = qk_prologue(q[rows[sel]], pos[rows[sel]], *_ln(ln, "q"))
+        k_hat = qk_prologue(k[lo:hi], pos[lo:hi], *_ln(ln, "k"))
         out[sel] = cross_attention(q_hat, k_hat, v[lo:hi])
     return out
 
 
-def attn_descriptor(q, k, v, pos, S: int, T: int, kd: int, rows=None) -> np.ndarray:
+def attn_descriptor(q, k, v, pos, S: int, T: int, kd: int, rows=None, layout=None,
+                    ln=None) -> np.ndarray:
     """Descriptor attention: every query attends to all frames' pooled
     descriptors; the pooled keys go through the prologue at their cell-mean
-    positions, pooled values are used as they are."""
-    kp, vp, pp = kv_pool(k, v, pos, S, T, kd)
+    positions, pooled values are used as they are. ``layout`` is the frame
+    layout of ``frame_layout``; ``ln`` as for ``attn_global``."""
+    kp, vp, pp = kv_pool(k, v, pos, S, T, kd, layout)
     rows = _rows(S * T, rows)
-    q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows])
-    k_hat = qk_prologue(kp, pp)
+    q_hat = qk_prologue(np.asarray(q)[rows], np.asarray(pos)[rows], *_ln(ln, "q"))
+    k_hat = qk_prologue(kp, pp, *_ln(ln, "k"))
     return cross_attention(q_hat, k_hat, vp)
 
 
-def attn_descriptor_stream(q, k, v, pos, S: int, T: int, kd: int, chunk: int, rows=None) -> np.ndarray:
+def attn_descriptor_stream(q, k, v, pos, S: int, T: int, kd: int, chunk: int, rows=None, layout=None,
+                           ln=None) -> np.ndarray:
     """Streaming descriptor attention: a query of frame ``f`` sees the
     descriptors of frames ``0 .. min(S, (f // chunk + 1) * chunk) - 1``. The
     descriptors are the per-frame pooled tokens of ``attn_descriptor``; their
     keys go through the prologue at their cell-mean positions."""
     if chunk < 1:
         raise ValueError("chunk must be >= 1")
-    kp, vp, pp = kv_pool(k, v, pos, S, T, kd)
-    k_hat = qk_prologue(kp, pp)
-    tk = pooled_tokens_per_frame(T, kd)
+    kp, vp, pp = kv_pool(k, v, pos, S, T, kd, layout)
+    k_hat = qk_prologue(kp, pp, *_ln(ln, "k"))
+    tk = pooled_tokens_per_frame(T, kd, layout)
     rows = _rows(S * T, rows)
     out = np.empty((rows.size,) + np.asarray(q).shape[1:])
     chunk_of_row = (rows // T) // chunk
@@ -347,7 +412,7 @@ def attn_descriptor_stream(q, k, v, pos, S: int, T: int, kd: int, chunk: int, ro
         sel = np.nonzero(chunk_of_row == c)[0]
         r = rows[sel]
         n_keys = min(S, (int(c) + 1) * chunk) * tk
-        q_hat = qk_prologue(np.asarray(q)[r], np.asarray(pos)[r])
+        q_hat = qk_prologue(np.asarray(q)[r], np.asarray(pos)[r], *_ln(ln, "q"))
         out[sel] = cross_attention(q_hat, k_hat[:n_keys], vp[:n_keys])
     return out
 

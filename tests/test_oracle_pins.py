@@ -480,3 +480,153 @@ def test_stream_rejects_empty_chunks():
     q, k, v, pos, T = _scene(S, 2, seed=45)
     with pytest.raises(ValueError):
         O.attn_descriptor_stream(q, k, v, pos, S, T, 1, 0)
+
+
+# ----------------------------------------------------------------- frame layouts and LN affine
+
+
+def _layout_scene(S, nf, gh, gw, nb, H=2, seed=0):
+    """Random q/k/v of ``S`` frames laid out as ``nf`` specials, a ``gh x gw``
+    grid at (r+1, c+1), ``nb`` trailing tokens; specials and trailing tokens
+    at the origin."""
+    T = nf + gh * gw + nb
+    rng = np.random.default_rng(seed)
+    q, k, v = (rng.normal(size=(S * T, H, 64)) for _ in range(3))
+    pos = np.zeros((S * T, 2))
+    for s in range(S):
+        for r in range(gh):
+            for c in range(gw):
+                pos[s * T + nf + r * gw + c] = (r + 1, c + 1)
+    return q, k, v, pos, T
+
+
+def test_default_layout_is_five_specials_and_a_square_grid():
+    assert O.frame_layout(5 + 37 * 37) == (5, 37, 37, 0)
+    with pytest.raises(ValueError):
+        O.frame_layout(5 + 25 * 37)
+    with pytest.raises(ValueError):
+        O.frame_layout(10, (5, 2, 2, 0))
+    S, g = 2, 6
+    q, k, v, pos, T = _scene(S, g, seed=31)
+    a = O.kv_pool(k, v, pos, S, T, 4)
+    b = O.kv_pool(k, v, pos, S, T, 4, layout=(5, g, g, 0))
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_rect_pool_brute_force_with_trailing_tokens():
+    # every grid element is assigned to cell (r // kd, c // kd) by a direct
+    # scan, independent of the oracle's range construction
+    S, nf, gh, gw, nb, kd = 2, 2, 3, 5, 3, 2
+    q, k, v, pos, T = _layout_scene(S, nf, gh, gw, nb, seed=32)
+    kp, vp, pp = O.kv_pool(k, v, pos, S, T, kd, layout=(nf, gh, gw, nb))
+    nch, ncw = -(-gh // kd), -(-gw // kd)
+    Tk = nf + nch * ncw + nb
+    assert O.pooled_tokens_per_frame(T, kd, (nf, gh, gw, nb)) == Tk == 2 + 6 + 3
+    assert kp.shape == (S * Tk, 2, 64)
+    for s in range(S):
+        base, out = s * T, s * Tk
+        for i in range(nf):
+            assert np.array_equal(kp[out + i], k[base + i])
+            assert np.array_equal(pp[out + i], pos[base + i])
+        for cr in range(nch):
+            for cc in range(ncw):
+                members = [base + nf + r * gw + c for r in range(gh) for c in range(gw)
+                           if r // kd == cr and c // kd == cc]
+                i = out + nf + cr * ncw + cc
+                assert np.allclose(kp[i], k[members].mean(axis=0), rtol=0, atol=1e-14)
+                assert np.allclose(vp[i], v[members].mean(axis=0), rtol=0, atol=1e-14)
+                assert np.allclose(pp[i], pos[members].mean(axis=0), rtol=0, atol=1e-14)
+        for j in range(nb):
+            assert np.array_equal(vp[out + nf + nch * ncw + j], v[base + nf + gh * gw + j])
+    # the 1x1 corner cell (row 2, cols 4) is its single member
+    assert np.array_equal(kp[nf + 1 * ncw + 2], k[nf + 2 * gw + 4])
+
+
+def test_rect_pool_kd1_is_identity_and_bits_reference_agrees():
+    S, nf, gh, gw, nb = 2, 1, 3, 4, 2
+    _, k, v, pos, T = _layout_scene(S, nf, gh, gw, nb, seed=33)
+    lay = (nf, gh, gw, nb)
+    kp, vp, pp = O.kv_pool(k, v, pos, S, T, 1, layout=lay)
+    assert np.array_equal(kp, k) and np.array_equal(vp, v) and np.array_equal(pp, pos)
+    kb = torch.from_numpy(k.astype(np.float32)).to(torch.bfloat16)
+    vb = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
+    ko, vo, po = O.kv_pool_bf16_reference(_bits(kb).reshape(S * T, -1), _bits(vb).reshape(S * T, -1),
+                                         pos, S, T, 1, layout=lay)
+    assert np.array_equal(ko, _bits(kb).reshape(S * T, -1))
+    # kd = 2 (counts 4 and 2): correctly rounded means, where the float32 sums
+    # are exact (values on a coarse dyadic grid) and division by a power of
+    # two is exact, so there is no double rounding
+    kq = np.round(k * 8) / 8 + 0.0  # + 0.0: no negative zeros (a copied -0 keeps its sign)
+    kqb = torch.from_numpy(kq.astype(np.float32)).to(torch.bfloat16)
+    ko, _, po = O.kv_pool_bf16_reference(_bits(kqb).reshape(S * T, -1), _bits(vb).reshape(S * T, -1),
+                                        pos, S, T, 2, layout=lay)
+    kp, _, pp = O.kv_pool(_f64(kqb), v, pos, S, T, 2, layout=lay)
+    want = torch.from_numpy(kp.reshape(ko.shape)).to(torch.bfloat16)
+    assert np.array_equal(ko, _bits(want))
+    assert np.array_equal(po, pp.astype(np.float32))
+
+
+def test_layernorm_affine_matches_torch_layer_norm():
+    rng = np.random.default_rng(34)
+    x = rng.normal(scale=3.0, size=(50, 64)) + rng.normal(size=(50, 1)) * 5
+    gamma, beta = rng.normal(size=64), rng.normal(size=64)
+    want = torch.nn.functional.layer_norm(torch.from_numpy(x), (64,), torch.from_numpy(gamma),
+                                          torch.from_numpy(beta), eps=O.LN_EPS).numpy()
+    assert np.allclose(O.layer_norm(x, gamma=gamma, beta=beta), want, rtol=0, atol=1e-12)
+    # the identity affine is the plain LayerNorm
+    assert np.array_equal(O.layer_norm(x, gamma=np.ones(64), beta=np.zeros(64)), O.layer_norm(x))
+
+
+def test_affine_comes_before_the_rotation():
+    # RoPE keeps scores a function of position differences only if the affine
+    # is applied before it: shifting every position leaves the output alone
+    S, g = 2, 3
+    q, k, v, pos, T = _scene(S, g, seed=35)
+    rng = np.random.default_rng(36)
+    ln = (rng.uniform(0.5, 1.5, 64), rng.normal(scale=0.2, size=64),
+          rng.uniform(0.5, 1.5, 64), rng.normal(scale=0.2, size=64))
+    a = O.attn_global(q, k, v, pos, S, T, ln=ln)
+    b = O.attn_global(q, k, v, pos + np.array([3.0, -7.0]), S, T, ln=ln)
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
+    # and the affine is not a no-op
+    c = O.attn_global(q, k, v, pos, S, T)
+    assert np.abs(a - c).max() > 1e-3
+    # a query affine that scales every dim by c is a softmax temperature c
+    ln2 = (np.full(64, 2.0), None, None, None)
+    qh = O.qk_prologue(q, pos) * 2.0
+    kh = O.qk_prologue(k, pos)
+    want = O.cross_attention(qh, kh, v)
+    assert np.allclose(O.attn_global(q, k, v, pos, S, T, ln=ln2), want, rtol=0, atol=1e-12)
+
+
+def test_descriptor_with_rect_layout_brute_force_tiny():
+    S, nf, gh, gw, nb, kd, H = 2, 1, 2, 3, 1, 2, 1
+    q, k, v, pos, T = _layout_scene(S, nf, gh, gw, nb, H=H, seed=37)
+    lay = (nf, gh, gw, nb)
+    rng = np.random.default_rng(38)
+    ln = (rng.uniform(0.5, 1.5, 64), rng.normal(scale=0.2, size=64), None, rng.normal(scale=0.2, size=64))
+    got = O.attn_descriptor(q, k, v, pos, S, T, kd, layout=lay, ln=ln)
+    # brute force: pooled keys by a direct scan, then scalar softmax loops
+    keys = []
+    for s in range(S):
+        base = s * T
+        keys.append([base])
+        for cc in range(2):
+            keys.append([base + nf + r * gw + c for r in range(gh) for c in range(gw) if c // kd == cc])
+        keys.append([base + nf + gh * gw])
+    for i in range(S * T):
+        x = q[i, 0]
+        xq = (x - x.mean()) / math.sqrt(((x - x.mean()) ** 2).mean() + 1e-5) * ln[0] + ln[1]
+        qh = O.rope_2d(xq, pos[i])
+        sc, vals = [], []
+        for members in keys:
+            kbar = k[members, 0].mean(axis=0)
+            pbar = pos[members].mean(axis=0)
+            xk = (kbar - kbar.mean()) / math.sqrt(((kbar - kbar.mean()) ** 2).mean() + 1e-5) + ln[3]
+            sc.append(float(qh @ O.rope_2d(xk, pbar)) / 8.0)
+            vals.append(v[members, 0].mean(axis=0))
+        m = max(sc)
+        w = [math.exp(t - m) for t in sc]
+        want = sum(wi * vi for wi, vi in zip(w, vals)) / sum(w)
+        assert np.allclose(got[i, 0], want, rtol=0, atol=1e-12)
