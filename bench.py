@@ -343,7 +343,8 @@ def run_gpu(args):
     ms_local = e0.elapsed_time(e1)
     status = F.vggt_get_device_status()
     ms_total = max_over_ranks(ms_local, world, dev)
-    # prologue + attention (+ pool), per call or per chunk
+    # per call or chunk: the prologue, the pooling fused with the key
+    # prologue (descriptors only), the attention
     launches = 3 * len(chunks) if w.kind == "stream" else 2 + (1 if w.kind == "descriptor" else 0)
     ms_step = ms_total / args.steps
     flops = w.flops()
@@ -359,7 +360,7 @@ def run_gpu(args):
     k_hat = torch.empty((H, w.n_k, 64), dtype=torch.bfloat16, device=dev)
     if kind_core == "descriptor":
         kp, vp, pp = F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down)
-        F.vggt_qk_prologue(kp, pp, k_hat)
+        F.vggt_descriptor_keys(k, v, pos, k_hat, vp, pp, S=w.S, T=w.T, kv_down=w.kv_down)
         v_use = vp
     else:
         F.vggt_qk_prologue(k, pos, k_hat)
@@ -388,7 +389,7 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     pro_ms = p0.elapsed_time(p1) / reps
     pro_bytes = 2 * w.n_q * H * 64 * 2 + w.n_q * 8  # read x + pos, write x_hat
-    pool = None
+    pool = fused_keys = None
     if kind_core == "descriptor":
         # K/V pooling alone: reads k, v and pos of every token, writes the
         # pooled k, v and positions.
@@ -406,6 +407,19 @@ def run_gpu(args):
         pool_bytes = 2 * (w.n_q + w.n_k) * H * 64 * 2 + (w.n_q + w.n_k) * 8
         pool = {"ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
                 "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"])}
+        # the pooling fused with the key prologue (what the call runs): the
+        # same bytes, with normalised keys written instead of pooled ones
+        for _ in range(3):
+            F.vggt_descriptor_keys(k, v, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
+        torch.cuda.synchronize(dev)
+        k0.record(stream)
+        for _ in range(reps):
+            F.vggt_descriptor_keys(k, v, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
+        k1.record(stream)
+        torch.cuda.synchronize(dev)
+        fk_ms = k0.elapsed_time(k1) / reps
+        fused_keys = {"ms": fk_ms, "gbs": pool_bytes / (fk_ms * 1e-3) / 1e9,
+                      "frac_hbm": pool_bytes / (fk_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"])}
 
     # ---- end to end through the public call with host buffers: every step
     # uploads its inputs from pinned host memory and reads its output back.
@@ -505,7 +519,8 @@ def run_gpu(args):
                          "share_of_step": attn_ms / ms_step},
             "kernels": {"qk_prologue": {"ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
                                         "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
-                        **({"kv_pool": pool} if pool else {})},
+                        **({"kv_pool": pool} if pool else {}),
+                        **({"descriptor_keys": fused_keys} if fused_keys else {})},
             # every score costs one exponential: exponentials per second in
             # the attention kernel, and per SM per clock at the sampled clock
             "exp_per_s": scores / (attn_ms * 1e-3),

@@ -39,6 +39,16 @@ __all__ = [
     "vggt_status_string",
     "vggt_set_wait_limit",
     "vggt_debug_wait_timeout",
+    "vggt_attn_frame_ex",
+    "vggt_attn_global_ex",
+    "vggt_attn_descriptor_ex",
+    "vggt_kv_pool_ex",
+    "vggt_kv_pool_tokens_ex",
+    "vggt_qk_prologue_ex",
+    "vggt_descriptor_keys",
+    "vggt_desc_cache_create_ex",
+    "FrameLayout",
+    "QKNorm",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -62,6 +72,14 @@ EXPORTED_SYMBOLS = (
     "vggt_status_string",
     "vggt_set_wait_limit",
     "vggt_debug_wait_timeout",
+    "vggt_attn_frame_ex",
+    "vggt_attn_global_ex",
+    "vggt_attn_descriptor_ex",
+    "vggt_kv_pool_ex",
+    "vggt_kv_pool_tokens_ex",
+    "vggt_qk_prologue_ex",
+    "vggt_descriptor_keys",
+    "vggt_desc_cache_create_ex",
 )
 
 if not os.path.exists(LIB_PATH):
@@ -106,6 +124,40 @@ lib.vggt_set_wait_limit.argtypes = [ctypes.c_longlong]
 lib.vggt_set_wait_limit.restype = ctypes.c_longlong
 lib.vggt_debug_wait_timeout.argtypes = [_p]
 lib.vggt_debug_wait_timeout.restype = _i
+
+
+class FrameLayout(ctypes.Structure):
+    """``vggt_frame_layout``: n_front special tokens, a grid_h x grid_w patch
+    grid (row-major), n_back trailing tokens per frame."""
+    _fields_ = [("n_front", _i), ("grid_h", _i), ("grid_w", _i), ("n_back", _i)]
+
+
+_f32p = ctypes.POINTER(ctypes.c_float)
+
+
+class QKNorm(ctypes.Structure):
+    """``vggt_qk_norm``: host fp32 arrays of D values (or NULL) for the QK
+    LayerNorm affine."""
+    _fields_ = [("q_weight", _f32p), ("q_bias", _f32p), ("k_weight", _f32p), ("k_bias", _f32p)]
+
+
+_LP = ctypes.POINTER(FrameLayout)
+_NP = ctypes.POINTER(QKNorm)
+for _name in ("vggt_attn_frame_ex", "vggt_attn_global_ex"):
+    getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _NP, _p]
+    getattr(lib, _name).restype = _i
+lib.vggt_attn_descriptor_ex.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _LP, _NP, _p]
+lib.vggt_attn_descriptor_ex.restype = _i
+lib.vggt_kv_pool_ex.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _LP, _p]
+lib.vggt_kv_pool_ex.restype = _i
+lib.vggt_kv_pool_tokens_ex.argtypes = [_i, _i, _LP]
+lib.vggt_kv_pool_tokens_ex.restype = _i
+lib.vggt_qk_prologue_ex.argtypes = [_p, _p, _p, _i, _i, _i, _f32p, _f32p, _p]
+lib.vggt_qk_prologue_ex.restype = _i
+lib.vggt_descriptor_keys.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _LP, _f32p, _f32p, _p]
+lib.vggt_descriptor_keys.restype = _i
+lib.vggt_desc_cache_create_ex.argtypes = [ctypes.POINTER(_p), _i, _i, _i, _i, _i, _LP, _NP]
+lib.vggt_desc_cache_create_ex.restype = _i
 
 
 class VggtError(RuntimeError):
@@ -224,6 +276,140 @@ def vggt_kv_pool(k, v, pos, k_out=None, v_out=None, pos_out=None, S=None, T=None
     return k_out, v_out, pos_out
 
 
+# ----------------------------------------------------------------- _ex calls
+
+
+def _host_f32(x, name):
+    """A host fp32 array for an affine argument (None stays NULL); returns
+    (ctypes pointer, owner to keep alive during the call)."""
+    if x is None:
+        return None, None
+    if isinstance(x, torch.Tensor):
+        x = x.detach().to("cpu", torch.float32).contiguous()
+        if x.numel() != 64:
+            raise ValueError(f"{name} must hold 64 values")
+        return ctypes.cast(x.data_ptr(), _f32p), x
+    arr = (ctypes.c_float * 64)(*[float(t) for t in x])
+    return ctypes.cast(arr, _f32p), arr
+
+
+def _layout(layout):
+    if layout is None:
+        return None
+    if isinstance(layout, FrameLayout):
+        return ctypes.pointer(layout)
+    return ctypes.pointer(FrameLayout(*[int(t) for t in layout]))
+
+
+def _norm(ln):
+    """``ln = (q_weight, q_bias, k_weight, k_bias)`` (entries may be None) ->
+    (pointer to QKNorm or None, owners)."""
+    if ln is None:
+        return None, ()
+    parts = [_host_f32(x, n) for x, n in zip(ln, ("q_weight", "q_bias", "k_weight", "k_bias"))]
+    return ctypes.pointer(QKNorm(*[p for p, _ in parts])), tuple(o for _, o in parts)
+
+
+def _attn_ex(fn, q, k, v, pos, out, S, T, H, D, ln, stream):
+    if out is None:
+        out = torch.empty_like(q)
+    norm, keep = _norm(ln)
+    rc = fn(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+            _ptr(pos, torch.float32, "pos"), _ptr(out, torch.bfloat16, "out"),
+            int(S), int(T), int(H), int(D), norm, _stream(stream))
+    del keep
+    _check(rc, fn.__name__)
+    return out
+
+
+def vggt_attn_frame_ex(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
+    """Frame attention, any T, optional QK LayerNorm affine ``ln = (q_weight,
+    q_bias, k_weight, k_bias)`` (host values; entries may be None)."""
+    return _attn_ex(lib.vggt_attn_frame_ex, q, k, v, pos, out, S, T, H, D, ln, stream)
+
+
+def vggt_attn_global_ex(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
+    """Global attention, any T, optional QK LayerNorm affine."""
+    return _attn_ex(lib.vggt_attn_global_ex, q, k, v, pos, out, S, T, H, D, ln, stream)
+
+
+def vggt_attn_descriptor_ex(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, kv_down=4, layout=None,
+                            ln=None, stream=None):
+    """Descriptor attention with a frame layout ``(n_front, grid_h, grid_w,
+    n_back)`` and an optional QK LayerNorm affine."""
+    if out is None:
+        out = torch.empty_like(q)
+    norm, keep = _norm(ln)
+    rc = lib.vggt_attn_descriptor_ex(
+        _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+        _ptr(pos, torch.float32, "pos"), _ptr(out, torch.bfloat16, "out"), int(S), int(T), int(H), int(D),
+        int(kv_down), _layout(layout), norm, _stream(stream))
+    del keep
+    _check(rc, "vggt_attn_descriptor_ex")
+    return out
+
+
+def vggt_kv_pool_tokens_ex(T: int, kv_down: int, layout=None) -> int:
+    return int(lib.vggt_kv_pool_tokens_ex(int(T), int(kv_down), _layout(layout)))
+
+
+def _pooled_shapes(T, kv_down, layout, where):
+    Tk = vggt_kv_pool_tokens_ex(T, kv_down, layout)
+    if Tk < 0:
+        raise VggtError(Tk, where)
+    return Tk
+
+
+def vggt_kv_pool_ex(k, v, pos, k_out=None, v_out=None, pos_out=None, S=None, T=None, H=16, D=64,
+                    kv_down=4, layout=None, stream=None):
+    """Pooled descriptors for a frame layout. Returns ``(k_out, v_out, pos_out)``."""
+    Tk = _pooled_shapes(T, kv_down, layout, "vggt_kv_pool_tokens_ex")
+    k_out = torch.empty((S * Tk, H, D), dtype=torch.bfloat16, device=k.device) if k_out is None else k_out
+    v_out = torch.empty((S * Tk, H, D), dtype=torch.bfloat16, device=k.device) if v_out is None else v_out
+    pos_out = torch.empty((S * Tk, 2), dtype=torch.float32, device=k.device) if pos_out is None else pos_out
+    rc = lib.vggt_kv_pool_ex(_ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+                             _ptr(pos, torch.float32, "pos"), _ptr(k_out, torch.bfloat16, "k_out"),
+                             _ptr(v_out, torch.bfloat16, "v_out"), _ptr(pos_out, torch.float32, "pos_out"),
+                             int(S), int(T), int(H), int(D), int(kv_down), _layout(layout), _stream(stream))
+    _check(rc, "vggt_kv_pool_ex")
+    return k_out, v_out, pos_out
+
+
+def vggt_qk_prologue_ex(x, pos, x_hat=None, N=None, H=16, D=64, ln_weight=None, ln_bias=None, stream=None):
+    """LayerNorm (+ optional host affine) + 2D RoPE; returns x_hat [H, N, D]."""
+    N = x.shape[0] if N is None else N
+    if x_hat is None:
+        x_hat = torch.empty((H, N, D), dtype=torch.bfloat16, device=x.device)
+    w, kw = _host_f32(ln_weight, "ln_weight")
+    b, kb = _host_f32(ln_bias, "ln_bias")
+    rc = lib.vggt_qk_prologue_ex(_ptr(x, torch.bfloat16, "x"), _ptr(pos, torch.float32, "pos"),
+                                 _ptr(x_hat, torch.bfloat16, "x_hat"), int(N), int(H), int(D), w, b,
+                                 _stream(stream))
+    del kw, kb
+    _check(rc, "vggt_qk_prologue_ex")
+    return x_hat
+
+
+def vggt_descriptor_keys(k, v, pos, k_hat=None, v_out=None, pos_out=None, S=None, T=None, H=16, D=64,
+                         kv_down=4, layout=None, ln_weight=None, ln_bias=None, stream=None):
+    """Pooling fused with the key prologue. Returns ``(k_hat [H, S*T_k, D],
+    v_out [S*T_k, H, D], pos_out [S*T_k, 2])``."""
+    Tk = _pooled_shapes(T, kv_down, layout, "vggt_kv_pool_tokens_ex")
+    k_hat = torch.empty((H, S * Tk, D), dtype=torch.bfloat16, device=k.device) if k_hat is None else k_hat
+    v_out = torch.empty((S * Tk, H, D), dtype=torch.bfloat16, device=k.device) if v_out is None else v_out
+    pos_out = torch.empty((S * Tk, 2), dtype=torch.float32, device=k.device) if pos_out is None else pos_out
+    w, kw = _host_f32(ln_weight, "ln_weight")
+    b, kb = _host_f32(ln_bias, "ln_bias")
+    rc = lib.vggt_descriptor_keys(_ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+                                  _ptr(pos, torch.float32, "pos"), _ptr(k_hat, torch.bfloat16, "k_hat"),
+                                  _ptr(v_out, torch.bfloat16, "v_out"), _ptr(pos_out, torch.float32, "pos_out"),
+                                  int(S), int(T), int(H), int(D), int(kv_down), _layout(layout), w, b,
+                                  _stream(stream))
+    del kw, kb
+    _check(rc, "vggt_descriptor_keys")
+    return k_hat, v_out, pos_out
+
+
 def vggt_get_device_status(stream=None) -> int:
     return int(lib.vggt_get_device_status(_stream(stream)))
 
@@ -233,10 +419,14 @@ class DescCache:
     normalised pooled keys, values and positions of the frames seen so far
     of one sequence, on the device that was current at creation."""
 
-    def __init__(self, max_frames: int, T: int, H: int = 16, D: int = 64, kv_down: int = 4):
-        self._h = _p()
-        _check(lib.vggt_desc_cache_create(ctypes.byref(self._h), int(max_frames), int(T), int(H),
-                                          int(D), int(kv_down)), "vggt_desc_cache_create")
+    def __init__(self, max_frames: int, T: int, H: int = 16, D: int = 64, kv_down: int = 4,
+                 layout=None, ln=None):
+        """``layout = (n_front, grid_h, grid_w, n_back)`` and ``ln = (q_weight,
+        q_bias, k_weight, k_bias)`` (host values) select the _ex form."""
+        if layout is None and ln is None:
+            self._h = vggt_desc_cache_create(max_frames, T, H, D, kv_down)
+        else:
+            self._h = vggt_desc_cache_create_ex(max_frames, T, H, D, kv_down, layout, ln)
         self.T, self.H, self.D = int(T), int(H), int(D)
 
     @property
@@ -255,15 +445,11 @@ class DescCache:
         C = q.shape[0] // self.T if C is None else C
         if out is None:
             out = torch.empty_like(q)
-        rc = lib.vggt_attn_descriptor_chunk(self._h, _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
-                                            _ptr(v, torch.bfloat16, "v"), _ptr(pos, torch.float32, "pos"),
-                                            _ptr(out, torch.bfloat16, "out"), int(C), _stream(stream))
-        _check(rc, "vggt_attn_descriptor_chunk")
-        return out
+        return vggt_attn_descriptor_chunk(self._h, q, k, v, pos, out, C, stream)
 
     def close(self) -> None:
         if self._h:
-            _check(lib.vggt_desc_cache_destroy(self._h), "vggt_desc_cache_destroy")
+            vggt_desc_cache_destroy(self._h)
             self._h = _p()
 
     def __enter__(self):
@@ -277,6 +463,49 @@ class DescCache:
             self.close()
         except Exception:
             pass
+
+
+def vggt_desc_cache_create(max_frames: int, T: int, H: int = 16, D: int = 64, kv_down: int = 4):
+    """Returns an opaque cache handle (see :class:`DescCache` for the managed form)."""
+    h = _p()
+    _check(lib.vggt_desc_cache_create(ctypes.byref(h), int(max_frames), int(T), int(H), int(D), int(kv_down)),
+           "vggt_desc_cache_create")
+    return h
+
+
+def vggt_desc_cache_create_ex(max_frames: int, T: int, H: int = 16, D: int = 64, kv_down: int = 4,
+                              layout=None, ln=None):
+    """Cache handle with a frame layout and a QK LayerNorm affine (either may be None)."""
+    h = _p()
+    norm, keep = _norm(ln)
+    rc = lib.vggt_desc_cache_create_ex(ctypes.byref(h), int(max_frames), int(T), int(H), int(D), int(kv_down),
+                                       _layout(layout), norm)
+    del keep
+    _check(rc, "vggt_desc_cache_create_ex")
+    return h
+
+
+def vggt_desc_cache_destroy(h) -> None:
+    _check(lib.vggt_desc_cache_destroy(h), "vggt_desc_cache_destroy")
+
+
+def vggt_desc_cache_frames(h) -> int:
+    n = lib.vggt_desc_cache_frames(h)
+    _check(min(n, 0), "vggt_desc_cache_frames")
+    return int(n)
+
+
+def vggt_desc_cache_reset(h) -> None:
+    _check(lib.vggt_desc_cache_reset(h), "vggt_desc_cache_reset")
+
+
+def vggt_attn_descriptor_chunk(h, q, k, v, pos, out, C, stream=None):
+    """One chunk of C frames through cache ``h``; returns ``out``."""
+    rc = lib.vggt_attn_descriptor_chunk(h, _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                        _ptr(v, torch.bfloat16, "v"), _ptr(pos, torch.float32, "pos"),
+                                        _ptr(out, torch.bfloat16, "out"), int(C), _stream(stream))
+    _check(rc, "vggt_attn_descriptor_chunk")
+    return out
 
 
 def vggt_release_scratch() -> None:

@@ -88,9 +88,8 @@ bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0
 // error status.
 int check_common(const void* q, const void* k, const void* v, const void* pos, const void* out,
                  int S, int T, int H, int D) {
-    if (S < 0 || T < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (S < 0 || T < 1 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
     if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
-    if (grid_side(T) < 0) return VGGT_ERR_SHAPE;
     if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS) return VGGT_ERR_SHAPE;
     if (H > 65535) return VGGT_ERR_SHAPE;
     if (S == 0 || H == 0) return 1;
@@ -100,43 +99,104 @@ int check_common(const void* q, const void* k, const void* v, const void* pos, c
     return VGGT_OK;
 }
 
+// Frame layout of a call: the caller's, checked against T, or VGGT-1B's
+// (5 specials + a square grid) when layout is NULL.
+int make_layout(const vggt_frame_layout* layout, int T, vggt::FrameLayout* out) {
+    if (!layout) {
+        const int g = grid_side(T);
+        if (g < 0) return VGGT_ERR_SHAPE;
+        *out = vggt::FrameLayout{VGGT_N_SPECIAL, g, g, 0};
+        return VGGT_OK;
+    }
+    const vggt_frame_layout& l = *layout;
+    if (l.n_front < 0 || l.grid_h < 0 || l.grid_w < 0 || l.n_back < 0) return VGGT_ERR_SHAPE;
+    const long long t = static_cast<long long>(l.n_front) + static_cast<long long>(l.grid_h) * l.grid_w +
+                        l.n_back;
+    if (t != T) return VGGT_ERR_SHAPE;
+    *out = vggt::FrameLayout{l.n_front, l.grid_h, l.grid_w, l.n_back};
+    return VGGT_OK;
+}
+
+// One LayerNorm affine from host arrays (NULL weight = 1, NULL bias = 0);
+// *bound receives max|weight| * 8 + ||bias||_2, a bound on the norm of the
+// normalised vector (the unscaled LayerNorm output has norm below 8).
+bool make_affine(const float* w, const float* b, vggt::LnAffine* a, double* bound) {
+    *a = vggt::LnAffine{};
+    a->on = (w || b) ? 1 : 0;
+    double wmax = w ? 0.0 : 1.0, b2 = 0.0;
+    for (int d = 0; d < VGGT_HEAD_DIM; ++d) {
+        const float wd = w ? w[d] : 1.0f, bd = b ? b[d] : 0.0f;
+        if (!std::isfinite(wd) || !std::isfinite(bd)) return false;
+        a->gamma[d] = wd;
+        a->beta[d] = bd;
+        wmax = std::fmax(wmax, std::fabs(static_cast<double>(wd)));
+        b2 += static_cast<double>(bd) * bd;
+    }
+    *bound = 8.0 * wmax + std::sqrt(b2);
+    return true;
+}
+
+// The query and key affines of a call. The attention kernel evaluates
+// exp(score) without subtracting a row maximum (exact up to rounding, as
+// softmax ignores a common factor), which needs every score bounded: with
+// |q_hat| <= Bq and |k_hat| <= Bk the score in log2 units is at most
+// Bq * Bk / 8 * log2(e) (+1% for the bf16 roundings), and this stays below
+// kMaxLog2Score so that exponentials, their sums over up to 2^21 keys and the
+// weighted value sums keep far from the fp32 limits. Beyond it: UNSUPPORTED.
+constexpr double kMaxLog2Score = 64.0;
+struct Norms {
+    vggt::LnAffine q, k;
+};
+int make_norms(const vggt_qk_norm* n, Norms* out) {
+    double bq = 8.0, bk = 8.0;
+    if (!make_affine(n ? n->q_weight : nullptr, n ? n->q_bias : nullptr, &out->q, &bq) ||
+        !make_affine(n ? n->k_weight : nullptr, n ? n->k_bias : nullptr, &out->k, &bk))
+        return VGGT_ERR_UNSUPPORTED;
+    if (bq * bk / 8.0 * 1.4426950408889634 * 1.01 > kMaxLog2Score) return VGGT_ERR_UNSUPPORTED;
+    return VGGT_OK;
+}
+
 size_t head_plane_bytes(long long n_tokens, int H) {
     return static_cast<size_t>(n_tokens) * H * VGGT_HEAD_DIM * sizeof(uint16_t);
 }
 
 int to_status(cudaError_t e) { return e == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA; }
 
-// Prologue on (q, pos) and (k, pos_k), then attention; frees the scratch.
-int run_attention(const uint16_t* q, const float* pos, const uint16_t* k, const float* pos_k,
-                  const uint16_t* v, uint16_t* out, int n_seg, int q_len, int k_len, int H,
-                  void* extra_scratch, cudaStream_t stream) {
+// Frame (n_seg = S, q_len = k_len = T) or global (n_seg = 1, q_len = k_len
+// = S*T) attention: prologue on q and k (one launch), then attention; the
+// scratch q_hat | k_hat is freed on the stream.
+int run_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* pos,
+                  uint16_t* out, int n_seg, int len, int H, const Norms& norms, cudaStream_t stream) {
     DeviceState* st = device_state();
-    if (!st) {
-        if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
-        return VGGT_ERR_CUDA;
-    }
-    const long long nq = static_cast<long long>(n_seg) * q_len;
-    const long long nk = static_cast<long long>(n_seg) * k_len;
+    if (!st) return VGGT_ERR_CUDA;
+    const long long n = static_cast<long long>(n_seg) * len;
     void* scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, head_plane_bytes(nq, H) + head_plane_bytes(nk, H), st->pool,
-                                stream) != cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&scratch, 2 * head_plane_bytes(n, H), st->pool, stream) != cudaSuccess) {
         cudaGetLastError();
-        if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
         return VGGT_ERR_ALLOC;
     }
     uint16_t* q_hat = static_cast<uint16_t*>(scratch);
-    uint16_t* k_hat = q_hat + head_plane_bytes(nq, H) / sizeof(uint16_t);
-    PrologueJob jq{q, pos, q_hat, static_cast<int>(nq), nq};
-    PrologueJob jk{k, pos_k, k_hat, static_cast<int>(nk), nk};
+    uint16_t* k_hat = q_hat + head_plane_bytes(n, H) / sizeof(uint16_t);
+    PrologueJob jq{q, pos, q_hat, static_cast<int>(n), n, norms.q};
+    PrologueJob jk{k, pos, k_hat, static_cast<int>(n), n, norms.k};
     int rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
     if (rc == VGGT_OK) {
-        AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H, nq, nk};
+        AttnProblem p{q_hat, k_hat, v, out, n_seg, len, len, H, n, n};
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
-    if (extra_scratch) cudaFreeAsync(extra_scratch, stream);
     return rc;
 }
+
+// Frame, global and descriptor calls, with or without the _ex options.
+enum class Kind { kFrame, kGlobal, kDescriptor };
+
+// plain == true: the original calls, whose frames are VGGT-1B's (T = 5 +
+// g*g). The _ex calls take any T for frame and global attention (they do not
+// look at the token order) and the caller's layout for the descriptor.
+int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+              const float* pos, uint16_t* out, int S, int T, int H, int D, int kv_down,
+              const vggt_frame_layout* layout, const vggt_qk_norm* norm, cudaStream_t stream);
 
 }  // namespace
 
@@ -152,35 +212,182 @@ bool device_status_word(int** status, long long* wait_limit) {
 
 }  // namespace vggt
 
+namespace {
+
+// The descriptor paths' two memory passes: the query prologue of (q, q_pos,
+// nq tokens) into q_hat (skipped when nq == 0), then the pooling fused with
+// the key prologue -- pools the S frames of k/v/pos into v_out / pos_out and
+// writes the normalised pooled keys head-major into k_hat (row r of head h at
+// k_hat + (h * k_stride + r) * 64).
+int pool_and_prologue(const uint16_t* k, const uint16_t* v, const float* pos, int S, int T,
+                      const vggt::FrameLayout& L, int kd, int H, uint16_t* k_hat, long long k_stride,
+                      uint16_t* v_out, float* pos_out, const uint16_t* q, const float* q_pos,
+                      long long nq, uint16_t* q_hat, const Norms& norms, cudaStream_t stream) {
+    vggt::PoolJob job{};
+    job.k = k;
+    job.v = v;
+    job.pos = pos;
+    job.k_out = nullptr;
+    job.k_hat = k_hat;
+    job.k_hat_stride = k_stride;
+    job.v_out = v_out;
+    job.pos_out = pos_out;
+    job.S = S;
+    job.T = T;
+    job.layout = L;
+    job.kd = kd;
+    job.H = H;
+    job.k_ln = norms.k;
+    if (nq > 0) {
+        PrologueJob jq{q, q_pos, q_hat, static_cast<int>(nq), nq, norms.q};
+        PrologueJob none{};
+        const int rc = to_status(vggt::launch_qk_prologue(jq, none, H, stream));
+        if (rc != VGGT_OK) return rc;
+    }
+    return to_status(vggt::launch_kv_pool(job, stream));
+}
+
+int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+              const float* pos, uint16_t* out, int S, int T, int H, int D, int kv_down,
+              const vggt_frame_layout* layout, const vggt_qk_norm* norm, cudaStream_t stream) {
+    int rc = check_common(q, k, v, pos, out, S, T, H, D);
+    vggt::FrameLayout L{};
+    if ((rc == VGGT_OK || rc == 1) && (plain || kind == Kind::kDescriptor)) {
+        const int lrc = make_layout(layout, T, &L);
+        if (lrc != VGGT_OK) rc = lrc;
+    }
+    if ((rc == VGGT_OK || rc == 1) && kind != Kind::kDescriptor && kv_down != 0 && kv_down != 1)
+        rc = VGGT_ERR_SHAPE;
+    if ((rc == VGGT_OK || rc == 1) && kind == Kind::kDescriptor && kv_down < 1) rc = VGGT_ERR_SHAPE;
+    Norms norms;
+    if (rc == VGGT_OK || rc == 1) {
+        const int nrc = make_norms(norm, &norms);
+        if (nrc != VGGT_OK) rc = nrc;
+    }
+    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
+    if (kind == Kind::kFrame) return run_attention(q, k, v, pos, out, S, T, H, norms, stream);
+    if (kind == Kind::kGlobal) return run_attention(q, k, v, pos, out, 1, S * T, H, norms, stream);
+
+    const int Tk = L.pooled(kv_down);
+    const long long nq = static_cast<long long>(S) * T;
+    const long long nk = static_cast<long long>(S) * Tk;
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    // scratch: q_hat [H, nq, 64] | k_hat [H, nk, 64] | pooled v [nk, H, 64] | pooled pos [nk, 2]
+    const size_t q_bytes = head_plane_bytes(nq, H), k_bytes = head_plane_bytes(nk, H);
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, q_bytes + 2 * k_bytes + static_cast<size_t>(nk) * 2 * sizeof(float),
+                                st->pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_ALLOC;
+    }
+    uint16_t* q_hat = static_cast<uint16_t*>(scratch);
+    uint16_t* k_hat = q_hat + q_bytes / sizeof(uint16_t);
+    uint16_t* vp = k_hat + k_bytes / sizeof(uint16_t);
+    float* pp = reinterpret_cast<float*>(vp + k_bytes / sizeof(uint16_t));
+    rc = pool_and_prologue(k, v, pos, S, T, L, kv_down, H, k_hat, nk, vp, pp, q, pos, nq, q_hat, norms,
+                           stream);
+    if (rc == VGGT_OK) {
+        // every query row attends to all S*Tk descriptors: one segment
+        AttnProblem p{q_hat, k_hat, vp, out, 1, static_cast<int>(nq), static_cast<int>(nk), H, nq, nk};
+        rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
+    }
+    cudaFreeAsync(scratch, stream);
+    return rc;
+}
+
+int kv_pool_call(const uint16_t* k, const uint16_t* v, const float* pos, uint16_t* k_out,
+                 uint16_t* v_out, float* pos_out, int S, int T, int H, int D, int kv_down,
+                 const vggt_frame_layout* layout, cudaStream_t stream) {
+    if (S < 0 || T < 1 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    vggt::FrameLayout L{};
+    const int lrc = make_layout(layout, T, &L);
+    if (lrc != VGGT_OK) return lrc;
+    if (kv_down < 1) return VGGT_ERR_SHAPE;
+    if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
+    if (S == 0 || H == 0) return VGGT_OK;
+    if (!k || !v || !pos || !k_out || !v_out || !pos_out) return VGGT_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned8(pos) || !aligned16(k_out) || !aligned16(v_out) ||
+        !aligned8(pos_out))
+        return VGGT_ERR_UNSUPPORTED;
+    vggt::PoolJob job{};
+    job.k = k;
+    job.v = v;
+    job.pos = pos;
+    job.k_out = k_out;
+    job.k_hat = nullptr;
+    job.v_out = v_out;
+    job.pos_out = pos_out;
+    job.S = S;
+    job.T = T;
+    job.layout = L;
+    job.kd = kv_down;
+    job.H = H;
+    return to_status(vggt::launch_kv_pool(job, stream));
+}
+
+}  // namespace
+
 extern "C" {
 
 int vggt_attn_frame(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                     vggt_bf16* out, int S, int T, int H, int D, int kv_down, cudaStream_t stream) {
-    int rc = check_common(q, k, v, pos, out, S, T, H, D);
-    if (rc == VGGT_OK && kv_down != 0 && kv_down != 1) rc = VGGT_ERR_SHAPE;
-    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
-    return run_attention(q, pos, k, pos, v, out, S, T, T, H, nullptr, stream);
+    return attn_call(Kind::kFrame, true, q, k, v, pos, out, S, T, H, D, kv_down, nullptr, nullptr,
+                     stream);
 }
 
 int vggt_attn_global(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                      vggt_bf16* out, int S, int T, int H, int D, int kv_down, cudaStream_t stream) {
-    int rc = check_common(q, k, v, pos, out, S, T, H, D);
-    if (rc == VGGT_OK && kv_down != 0 && kv_down != 1) rc = VGGT_ERR_SHAPE;
-    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
-    const int n = S * T;
-    return run_attention(q, pos, k, pos, v, out, 1, n, n, H, nullptr, stream);
+    return attn_call(Kind::kGlobal, true, q, k, v, pos, out, S, T, H, D, kv_down, nullptr, nullptr,
+                     stream);
+}
+
+int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                         const float* pos, vggt_bf16* out, int S, int T, int H, int D, int kv_down,
+                         cudaStream_t stream) {
+    return attn_call(Kind::kDescriptor, true, q, k, v, pos, out, S, T, H, D, kv_down, nullptr, nullptr,
+                     stream);
+}
+
+int vggt_attn_frame_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                       vggt_bf16* out, int S, int T, int H, int D, const vggt_qk_norm* norm,
+                       cudaStream_t stream) {
+    return attn_call(Kind::kFrame, false, q, k, v, pos, out, S, T, H, D, 1, nullptr, norm, stream);
+}
+
+int vggt_attn_global_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                        vggt_bf16* out, int S, int T, int H, int D, const vggt_qk_norm* norm,
+                        cudaStream_t stream) {
+    return attn_call(Kind::kGlobal, false, q, k, v, pos, out, S, T, H, D, 1, nullptr, norm, stream);
+}
+
+int vggt_attn_descriptor_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                            const float* pos, vggt_bf16* out, int S, int T, int H, int D, int kv_down,
+                            const vggt_frame_layout* layout, const vggt_qk_norm* norm,
+                            cudaStream_t stream) {
+    return attn_call(Kind::kDescriptor, false, q, k, v, pos, out, S, T, H, D, kv_down, layout, norm,
+                     stream);
 }
 
 int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int N, int H, int D,
                      cudaStream_t stream) {
+    return vggt_qk_prologue_ex(x, pos, x_hat, N, H, D, nullptr, nullptr, stream);
+}
+
+int vggt_qk_prologue_ex(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int N, int H, int D,
+                        const float* ln_weight, const float* ln_bias, cudaStream_t stream) {
     if (N < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
     if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
     if (N > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
+    vggt::LnAffine ln;
+    double bound = 0.0;
+    if (!make_affine(ln_weight, ln_bias, &ln, &bound)) return VGGT_ERR_UNSUPPORTED;
     if (N == 0 || H == 0) return VGGT_OK;
     if (!x || !pos || !x_hat) return VGGT_ERR_NULL;
     if (!aligned16(x) || !aligned8(pos) || !aligned16(x_hat)) return VGGT_ERR_UNSUPPORTED;
-    PrologueJob j{x, pos, x_hat, N, N};
-    PrologueJob none{nullptr, nullptr, nullptr, 0, 0};
+    PrologueJob j{x, pos, x_hat, N, N, ln};
+    PrologueJob none{};
     return to_status(vggt::launch_qk_prologue(j, none, H, stream));
 }
 
@@ -203,67 +410,59 @@ int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf
     return to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
 }
 
-int vggt_kv_pool_tokens(int T, int kv_down) {
-    const int g = grid_side(T);
-    if (g < 0 || kv_down < 1) return VGGT_ERR_SHAPE;
-    const int nc = g > 0 ? (g + kv_down - 1) / kv_down : 0;
-    return VGGT_N_SPECIAL + nc * nc;
+int vggt_kv_pool_tokens(int T, int kv_down) { return vggt_kv_pool_tokens_ex(T, kv_down, nullptr); }
+
+int vggt_kv_pool_tokens_ex(int T, int kv_down, const vggt_frame_layout* layout) {
+    vggt::FrameLayout L{};
+    if (T < 1 || kv_down < 1) return VGGT_ERR_SHAPE;
+    const int rc = make_layout(layout, T, &L);
+    return rc != VGGT_OK ? rc : L.pooled(kv_down);
 }
 
 int vggt_kv_pool(const vggt_bf16* k, const vggt_bf16* v, const float* pos, vggt_bf16* k_out,
                  vggt_bf16* v_out, float* pos_out, int S, int T, int H, int D, int kv_down,
                  cudaStream_t stream) {
-    if (S < 0 || T < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
-    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
-    const int g = grid_side(T);
-    if (g < 0 || kv_down < 1) return VGGT_ERR_SHAPE;
-    if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
-    if (S == 0 || H == 0) return VGGT_OK;
-    if (!k || !v || !pos || !k_out || !v_out || !pos_out) return VGGT_ERR_NULL;
-    if (!aligned16(k) || !aligned16(v) || !aligned8(pos) || !aligned16(k_out) ||
-        !aligned16(v_out) || !aligned8(pos_out))
-        return VGGT_ERR_UNSUPPORTED;
-    return to_status(vggt::launch_kv_pool(k, v, pos, k_out, v_out, pos_out, S, T, g, kv_down, H,
-                                          stream));
+    return kv_pool_call(k, v, pos, k_out, v_out, pos_out, S, T, H, D, kv_down, nullptr, stream);
 }
 
-int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
-                         const float* pos, vggt_bf16* out, int S, int T, int H, int D, int kv_down,
+int vggt_kv_pool_ex(const vggt_bf16* k, const vggt_bf16* v, const float* pos, vggt_bf16* k_out,
+                    vggt_bf16* v_out, float* pos_out, int S, int T, int H, int D, int kv_down,
+                    const vggt_frame_layout* layout, cudaStream_t stream) {
+    return kv_pool_call(k, v, pos, k_out, v_out, pos_out, S, T, H, D, kv_down, layout, stream);
+}
+
+int vggt_descriptor_keys(const vggt_bf16* k, const vggt_bf16* v, const float* pos, vggt_bf16* k_hat,
+                         vggt_bf16* v_out, float* pos_out, int S, int T, int H, int D, int kv_down,
+                         const vggt_frame_layout* layout, const float* ln_weight, const float* ln_bias,
                          cudaStream_t stream) {
-    int rc = check_common(q, k, v, pos, out, S, T, H, D);
-    if (rc == VGGT_OK && kv_down < 1) rc = VGGT_ERR_SHAPE;
-    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
-    const int g = grid_side(T);
-    const int Tk = vggt_kv_pool_tokens(T, kv_down);
-    const long long nk = static_cast<long long>(S) * Tk;
-    // pooled k, pooled v, pooled positions
-    const size_t kv_bytes = head_plane_bytes(nk, H);
-    const size_t pos_bytes = static_cast<size_t>(nk) * 2 * sizeof(float);
-    DeviceState* st = device_state();
-    if (!st) return VGGT_ERR_CUDA;
-    void* pooled = nullptr;
-    if (cudaMallocFromPoolAsync(&pooled, 2 * kv_bytes + pos_bytes, st->pool, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return VGGT_ERR_ALLOC;
-    }
-    uint16_t* kp = static_cast<uint16_t*>(pooled);
-    uint16_t* vp = kp + kv_bytes / sizeof(uint16_t);
-    float* pp = reinterpret_cast<float*>(vp + kv_bytes / sizeof(uint16_t));
-    rc = to_status(vggt::launch_kv_pool(k, v, pos, kp, vp, pp, S, T, g, kv_down, H, stream));
-    if (rc != VGGT_OK) {
-        cudaFreeAsync(pooled, stream);
-        return rc;
-    }
-    // Every query row attends to all S*Tk descriptors: one segment.
-    return run_attention(q, pos, kp, pp, vp, out, 1, S * T, static_cast<int>(nk), H, pooled,
-                         stream);
+    if (S < 0 || T < 1 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    vggt::FrameLayout L{};
+    const int lrc = make_layout(layout, T, &L);
+    if (lrc != VGGT_OK) return lrc;
+    if (kv_down < 1) return VGGT_ERR_SHAPE;
+    if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
+    Norms norms{};
+    double bound = 0.0;
+    if (!make_affine(ln_weight, ln_bias, &norms.k, &bound)) return VGGT_ERR_UNSUPPORTED;
+    if (S == 0 || H == 0) return VGGT_OK;
+    if (!k || !v || !pos || !k_hat || !v_out || !pos_out) return VGGT_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned8(pos) || !aligned16(k_hat) || !aligned16(v_out) ||
+        !aligned8(pos_out))
+        return VGGT_ERR_UNSUPPORTED;
+    const long long nk = static_cast<long long>(S) * L.pooled(kv_down);
+    return pool_and_prologue(k, v, pos, S, T, L, kv_down, H, k_hat, nk, v_out, pos_out, nullptr, nullptr,
+                             0, nullptr, norms, stream);
 }
-
 // ------------------------------------------------------------- streaming
+
+}  // extern "C"
 
 struct vggt_desc_cache {
     int device;
-    int max_frames, T, H, kv_down, g, Tk;
+    int max_frames, T, H, kv_down, Tk;
+    vggt::FrameLayout layout;
+    Norms norms;
     long long capacity;  // max_frames * Tk descriptor rows
     int frames;          // frames appended so far
     uint16_t* k_hat;     // [H][capacity][64] normalised pooled keys, head-major
@@ -271,17 +470,29 @@ struct vggt_desc_cache {
     float* pos;          // [capacity][2] cell-mean positions
 };
 
+extern "C" {
+
 int vggt_desc_cache_create(vggt_desc_cache** cache, int max_frames, int T, int H, int D,
                            int kv_down) {
+    return vggt_desc_cache_create_ex(cache, max_frames, T, H, D, kv_down, nullptr, nullptr);
+}
+
+int vggt_desc_cache_create_ex(vggt_desc_cache** cache, int max_frames, int T, int H, int D, int kv_down,
+                              const vggt_frame_layout* layout, const vggt_qk_norm* norm) {
     if (!cache) return VGGT_ERR_NULL;
     *cache = nullptr;
     if (max_frames < 1 || T < 1 || H < 1 || kv_down < 1 || H > 65535) return VGGT_ERR_SHAPE;
     if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
-    const int g = grid_side(T);
-    const int Tk = vggt_kv_pool_tokens(T, kv_down);
-    if (g < 0 || Tk < 0) return VGGT_ERR_SHAPE;
+    vggt::FrameLayout L{};
+    const int lrc = make_layout(layout, T, &L);
+    if (lrc != VGGT_OK) return lrc;
+    Norms norms;
+    const int nrc = make_norms(norm, &norms);
+    if (nrc != VGGT_OK) return nrc;
+    const int Tk = L.pooled(kv_down);
     const long long capacity = static_cast<long long>(max_frames) * Tk;
-    if (capacity > VGGT_MAX_TOKENS) return VGGT_ERR_SHAPE;
+    if (capacity > VGGT_MAX_TOKENS || static_cast<long long>(max_frames) * T > VGGT_MAX_TOKENS)
+        return VGGT_ERR_SHAPE;
     vggt_desc_cache* c = new (std::nothrow) vggt_desc_cache();
     if (!c) return VGGT_ERR_ALLOC;
     if (cudaGetDevice(&c->device) != cudaSuccess) {
@@ -292,8 +503,9 @@ int vggt_desc_cache_create(vggt_desc_cache** cache, int max_frames, int T, int H
     c->T = T;
     c->H = H;
     c->kv_down = kv_down;
-    c->g = g;
     c->Tk = Tk;
+    c->layout = L;
+    c->norms = norms;
     c->capacity = capacity;
     c->frames = 0;
     const size_t plane = head_plane_bytes(capacity, H);
@@ -348,30 +560,21 @@ int vggt_attn_descriptor_chunk(vggt_desc_cache* cache, const vggt_bf16* q, const
     const long long n_q = static_cast<long long>(C) * T;
     const long long row0 = static_cast<long long>(cache->frames) * Tk;  // first new descriptor
     const long long n_new = static_cast<long long>(C) * Tk;
-    // Scratch: the chunk's pooled raw keys [C*Tk, H, 64] and q_hat [H, C*T, 64].
+    // Scratch: the chunk's q_hat [H, C*T, 64].
     void* scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, head_plane_bytes(n_new, H) + head_plane_bytes(n_q, H),
-                                st->pool, stream) != cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&scratch, head_plane_bytes(n_q, H), st->pool, stream) != cudaSuccess) {
         cudaGetLastError();
         return VGGT_ERR_ALLOC;
     }
-    uint16_t* k_raw = static_cast<uint16_t*>(scratch);
-    uint16_t* q_hat = k_raw + head_plane_bytes(n_new, H) / sizeof(uint16_t);
-    uint16_t* v_new = cache->v + row0 * H * VGGT_HEAD_DIM;
-    float* pos_new = cache->pos + row0 * 2;
-    // 1. The chunk's descriptors: pooled values and positions straight into
-    //    the cache, pooled keys into scratch ...
-    rc = to_status(vggt::launch_kv_pool(k, v, pos, k_raw, v_new, pos_new, C, T, cache->g,
-                                        cache->kv_down, H, stream));
-    // 2. ... then normalised into the cache's key planes (row0 onwards of
-    //    each head's plane), together with the chunk's queries.
-    if (rc == VGGT_OK) {
-        PrologueJob jq{q, pos, q_hat, static_cast<int>(n_q), n_q};
-        PrologueJob jk{k_raw, pos_new, cache->k_hat + row0 * VGGT_HEAD_DIM, static_cast<int>(n_new),
-                       cache->capacity};
-        rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
-    }
-    // 3. Every query of the chunk attends to every cached descriptor.
+    uint16_t* q_hat = static_cast<uint16_t*>(scratch);
+    // 1. The chunk's queries through the prologue, and its descriptors
+    //    straight into the cache (values and positions at row0, normalised
+    //    keys at row0 of every head's plane).
+    rc = pool_and_prologue(k, v, pos, C, T, cache->layout, cache->kv_down, H,
+                           cache->k_hat + row0 * VGGT_HEAD_DIM, cache->capacity,
+                           cache->v + row0 * H * VGGT_HEAD_DIM, cache->pos + row0 * 2, q, pos, n_q, q_hat,
+                           cache->norms, stream);
+    // 2. Every query of the chunk attends to every cached descriptor.
     if (rc == VGGT_OK) {
         AttnProblem p{q_hat, cache->k_hat, cache->v, out, 1, static_cast<int>(n_q),
                       static_cast<int>(row0 + n_new), H, n_q, cache->capacity};
@@ -414,7 +617,8 @@ const char* vggt_status_string(int status) {
         case VGGT_ERR_NULL: return "VGGT_ERR_NULL: a required pointer is NULL";
         case VGGT_ERR_UNSUPPORTED:
             return "VGGT_ERR_UNSUPPORTED: head dimension must be 64, pointers aligned (16 bytes; "
-                   "positions 8), and the current device the cache's";
+                   "positions 8), the current device the cache's, and a QK LayerNorm affine finite "
+                   "and within the score bound";
         case VGGT_ERR_SHAPE: return "VGGT_ERR_SHAPE: invalid sizes";
         case VGGT_ERR_ALLOC: return "VGGT_ERR_ALLOC: scratch allocation failed";
         case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA: CUDA call or launch failed";

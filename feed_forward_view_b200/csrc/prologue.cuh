@@ -1,0 +1,182 @@
+// prologue.cuh -- the per-head QK LayerNorm + 2D RoPE arithmetic, shared by
+// the prologue kernel (qk_prologue.cu) and the fused pooling + key prologue
+// kernel (kv_pool.cu) so that both produce the same bits for the same input.
+//
+// For one head vector x (64 dims) at position (row, col):
+//   y = (x - mean) / sqrt(var + 1e-5)          (biased variance, centered)
+//   y = y * gamma + beta                       (optional per-dim affine)
+//   half a in {0: dims 0-31 by row, 1: dims 32-63 by col}:
+//     (y[j], y[j+16]) of the half turn by theta_j = p_a * 100^(-j/16)
+// (LayerNorm: "Norm: Layer Normalization" slide of the VGGT paper-report
+//  slides and layer_norm_eps 1e-05 of the VGGT-Omega config.json table; RoPE
+//  base: rope_base 100.0 in the same table; frequency schedule: "Positional
+//  Encoding (4/6)" slide.)
+//
+// Lane layout: 8 lanes per head. Lane sub = lane % 8 owns dims
+// {d1 .. d1+3} and {d1+16 .. d1+19} with d1 = 32*(sub/4) + 4*(sub%4), so both
+// members of every rotation pair stay in one thread. A warp covers 4 heads.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "vggt_internal.h"
+
+namespace vggt {
+namespace prologue {
+
+constexpr float kEps = 1e-5f;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// First dim of a lane's low group; the high group is at d1 + 16.
+__device__ __forceinline__ int lane_dim(int lane) {
+    const int sub = lane & 7;
+    return (sub >> 2) * 32 + 4 * (sub & 3);
+}
+
+// The affine of a job, staged in shared memory by the block (so that no
+// registers hold it): gamma then beta, 64 floats each; null when the job has
+// none.
+struct SmemAffine {
+    float v[2 * kHeadDim];
+};
+
+// Copies job affine a into s (all threads of the block call it, followed by
+// a __syncthreads before use); returns the staged values.
+__device__ __forceinline__ const float* stage_affine(const LnAffine& a, SmemAffine& s) {
+    for (int i = threadIdx.x; i < 2 * kHeadDim; i += blockDim.x)
+        s.v[i] = i < kHeadDim ? a.gamma[i] : a.beta[i - kHeadDim];
+    return s.v;
+}
+
+// (sin, cos) of the 8 angles a lane needs at position p = (row, col): lane l
+// computes the pair of (half l/16, frequency l%16) and the values are
+// shuffled to the lanes that own those dims. Every lane of the warp calls it.
+__device__ __forceinline__ void token_angles(float2 p, int lane, float my_freq, float (&sv)[4],
+                                             float (&cv)[4]) {
+    const float my_pos = (lane < 16) ? p.x : p.y;
+    float sn, cs;
+    sincosf(my_pos * my_freq, &sn, &cs);
+    const int sub = lane & 7, a = sub >> 2, u = sub & 3;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int src = a * 16 + 4 * u + i;
+        sv[i] = __shfl_sync(0xFFFFFFFFu, sn, src);
+        cv[i] = __shfl_sync(0xFFFFFFFFu, cs, src);
+    }
+}
+
+// LayerNorm (+ affine) and rotation of one head (8 lanes) whose 8 dims per
+// lane are x1 (dims d1..d1+3) and x2 (d1+16..d1+19); the result is stored at
+// dst + d1 and dst + d1 + 16 (dst = the head vector's 64 outputs). Every lane
+// of the warp runs it (the shuffles need the whole warp); lanes with
+// live == false hold zeros and store nothing. kAffine: apply the affine
+// staged at aff (gamma[64] then beta[64] in shared memory).
+template <bool kAffine>
+__device__ __forceinline__ void norm_rotate_store(float (&x1)[4], float (&x2)[4], const float* aff,
+                                                  const float (&sv)[4], const float (&cv)[4], bool live,
+                                                  uint16_t* dst, int d1) {
+    float sum = (x1[0] + x1[1]) + (x1[2] + x1[3]) + ((x2[0] + x2[1]) + (x2[2] + x2[3]));
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+    const float mean = sum * (1.0f / kHeadDim);
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x1[i] -= mean;
+        x2[i] -= mean;
+        sq = fmaf(x1[i], x1[i], sq);
+        sq = fmaf(x2[i], x2[i], sq);
+    }
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 4);
+    const float rstd = rsqrtf(sq * (1.0f / kHeadDim) + kEps);
+    float y1[4], y2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        y1[i] = x1[i] * rstd;
+        y2[i] = x2[i] * rstd;
+    }
+    if (kAffine) {
+        // volatile: read from shared memory at each use, so the compiler
+        // does not hoist 16 affine values per lane into registers for the
+        // whole token loop
+        const volatile float* va = aff;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            y1[i] = fmaf(y1[i], va[d1 + i], va[kHeadDim + d1 + i]);
+            y2[i] = fmaf(y2[i], va[d1 + 16 + i], va[kHeadDim + d1 + 16 + i]);
+        }
+    }
+    float o1[4], o2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o1[i] = y1[i] * cv[i] - y2[i] * sv[i];
+        o2[i] = y2[i] * cv[i] + y1[i] * sv[i];
+    }
+    if (live) {
+        *reinterpret_cast<uint2*>(dst + d1) = make_uint2(pack2(o1[0], o1[1]), pack2(o1[2], o1[3]));
+        *reinterpret_cast<uint2*>(dst + d1 + 16) = make_uint2(pack2(o2[0], o2[1]), pack2(o2[2], o2[3]));
+    }
+}
+
+// This lane's RoPE frequency 100^(-(lane%16)/16), chosen from the table with
+// constant indices (no local memory).
+__device__ __forceinline__ float lane_freq(const FreqTable& freq, int lane) {
+    float f = freq.f[0];
+#pragma unroll
+    for (int i = 1; i < 16; ++i)
+        if ((lane & 15) == i) f = freq.f[i];
+    return f;
+}
+
+// Up to 16 heads of one token per pass: the lane's two 8-byte pieces of every
+// head group are loaded before any arithmetic, so each warp keeps 2 KB of
+// loads in flight.
+constexpr int kMaxGroups = 4;
+
+// Token t of job: normalise and rotate all H heads, store head-major. One
+// warp per token; every lane of the warp calls it. aff: the job's staged
+// affine, or nullptr.
+template <bool kAffine>
+__device__ __forceinline__ void process_token(const PrologueJob& job, const float* aff, int t, int H,
+                                              int lane, float my_freq) {
+    const int d1 = lane_dim(lane);
+    const uint16_t* xt = job.x + static_cast<size_t>(t) * H * kHeadDim;
+    for (int h0 = 0; h0 < H; h0 += 4 * kMaxGroups) {
+        uint2 w1[kMaxGroups], w2[kMaxGroups];
+#pragma unroll
+        for (int g = 0; g < kMaxGroups; ++g) {
+            const int h = h0 + 4 * g + (lane >> 3);
+            w1[g] = make_uint2(0, 0);
+            w2[g] = make_uint2(0, 0);
+            if (h < H) {
+                w1[g] = __ldg(reinterpret_cast<const uint2*>(xt + h * kHeadDim + d1));
+                w2[g] = __ldg(reinterpret_cast<const uint2*>(xt + h * kHeadDim + d1 + 16));
+            }
+        }
+        float sv[4], cv[4];
+        token_angles(reinterpret_cast<const float2*>(job.pos)[t], lane, my_freq, sv, cv);
+#pragma unroll
+        for (int g = 0; g < kMaxGroups; ++g) {
+            const int h = h0 + 4 * g + (lane >> 3);
+            if (h0 + 4 * g < H) {  // warp-uniform
+                float x1[4] = {bf16_lo(w1[g].x), bf16_hi(w1[g].x), bf16_lo(w1[g].y), bf16_hi(w1[g].y)};
+                float x2[4] = {bf16_lo(w2[g].x), bf16_hi(w2[g].x), bf16_lo(w2[g].y), bf16_hi(w2[g].y)};
+                uint16_t* dst = job.x_hat + (static_cast<size_t>(h) * job.out_stride + t) * kHeadDim;
+                norm_rotate_store<kAffine>(x1, x2, aff, sv, cv, h < H, dst, d1);
+            }
+        }
+    }
+}
+
+}  // namespace prologue
+}  // namespace vggt

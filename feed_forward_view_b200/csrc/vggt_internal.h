@@ -6,6 +6,12 @@
 #include <cstdint>
 #include <cuda_runtime_api.h>
 
+#ifdef __CUDACC__
+#define VGGT_HD __host__ __device__
+#else
+#define VGGT_HD
+#endif
+
 namespace vggt {
 
 constexpr int kNSpecial = 5;
@@ -14,6 +20,20 @@ constexpr int kHeadDim = 64;
 // Bits of the device status word.
 constexpr int kStatusTimeout = 1;  // a bounded device wait ran out
 constexpr int kStatusRange = 2;    // an attention row sum was not a positive finite number
+
+// RoPE frequencies 100^(-j/16), j = 0..15, in fp32, passed by value.
+struct FreqTable {
+    float f[16];
+};
+FreqTable rope_freq_table();
+
+// Optional per-dim scale and shift after a QK LayerNorm (shared by the
+// heads), passed by value; on == 0 means none.
+struct LnAffine {
+    float gamma[kHeadDim];
+    float beta[kHeadDim];
+    int on;
+};
 
 // One tensor to normalise and rotate: x [n, H, 64] token-major in, positions
 // pos [n, 2] (row, col); out head-major: row t of head h goes to
@@ -25,18 +45,49 @@ struct PrologueJob {
     uint16_t* x_hat;
     int n;
     long long out_stride;
+    LnAffine ln;
 };
 
-// LayerNorm (eps 1e-5, no affine) + 2D RoPE (base 100) over one or two jobs in
-// a single launch. Returns the launch's cudaError_t.
+// LayerNorm (eps 1e-5, optional affine) + 2D RoPE (base 100) over one or two
+// jobs in a single launch. Returns the launch's cudaError_t.
 cudaError_t launch_qk_prologue(const PrologueJob& a, const PrologueJob& b, int H,
                                cudaStream_t stream);
 
+// Token layout of one frame: n_front special tokens, a grid_h x grid_w patch
+// grid in row-major order, n_back trailing tokens.
+struct FrameLayout {
+    int n_front, grid_h, grid_w, n_back;
+    VGGT_HD int tokens() const { return n_front + grid_h * grid_w + n_back; }
+    // tokens per pooled frame for kd x kd ceil-mode cells
+    VGGT_HD int pooled(int kd) const {
+        const int nch = grid_h > 0 ? (grid_h + kd - 1) / kd : 0;
+        const int ncw = grid_w > 0 ? (grid_w + kd - 1) / kd : 0;
+        return n_front + nch * ncw + n_back;
+    }
+};
+
 // Ceil-mode kd x kd average pooling of the patch grid of every frame, special
-// tokens copied. k,v [S*T, H, 64] -> [S*Tk, H, 64]; pos [S*T,2] -> [S*Tk,2].
-cudaError_t launch_kv_pool(const uint16_t* k, const uint16_t* v, const float* pos,
-                           uint16_t* k_out, uint16_t* v_out, float* pos_out,
-                           int S, int T, int g, int kd, int H, cudaStream_t stream);
+// tokens copied; pooled frame = front specials, cells row-major, trailing
+// tokens. v [S*T, H, 64] -> v_out [S*Tk, H, 64]; pos [S*T,2] -> pos_out
+// [S*Tk,2]. Keys either pooled the same way into k_out (k_hat == nullptr), or
+// (k_out == nullptr) pooled, normalised (k_ln) and rotated at their pooled
+// position, and written head-major: pooled row r of head h at
+// k_hat + (h * k_hat_stride + r) * 64.
+struct PoolJob {
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* pos;
+    uint16_t* k_out;
+    uint16_t* k_hat;
+    long long k_hat_stride;
+    uint16_t* v_out;
+    float* pos_out;
+    int S, T;
+    FrameLayout layout;
+    int kd, H;
+    LnAffine k_ln;
+};
+cudaError_t launch_kv_pool(const PoolJob& job, cudaStream_t stream);
 
 // Attention over segments: segment s has queries rows [s*q_len, (s+1)*q_len)
 // of q_hat and keys rows [s*k_len, (s+1)*k_len) of k_hat / v.

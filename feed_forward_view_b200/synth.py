@@ -146,6 +146,38 @@ def make_qkv(S: int, g: int, seed: int, H: int = HEADS, D: int = HEAD_DIM):
     return q, k, v, grid_positions(S, g)
 
 
+def layout_positions(S: int, layout) -> torch.Tensor:
+    """``[S*T, 2]`` fp32 for frames laid out ``(n_front, grid_h, grid_w,
+    n_back)``: front and trailing tokens at (0,0), patch (r,c) at
+    (r+1,c+1)."""
+    nf, gh, gw, nb = (int(x) for x in layout)
+    one = torch.zeros(nf + gh * gw + nb, 2, dtype=torch.float32)
+    if gh > 0 and gw > 0:
+        one[nf:nf + gh * gw, 0] = torch.arange(gh, dtype=torch.float32).repeat_interleave(gw) + 1.0
+        one[nf:nf + gh * gw, 1] = torch.arange(gw, dtype=torch.float32).repeat(gh) + 1.0
+    return one.repeat(S, 1).contiguous()
+
+
+def make_layout_qkv(S: int, layout, seed: int, H: int = HEADS, D: int = HEAD_DIM):
+    """``make_qkv`` for frames laid out ``(n_front, grid_h, grid_w, n_back)``."""
+    nf, gh, gw, nb = (int(x) for x in layout)
+    n = S * (nf + gh * gw + nb)
+    q = normal_bf16((n, H, D), 3 * seed)
+    k = normal_bf16((n, H, D), 3 * seed + 1)
+    v = normal_bf16((n, H, D), 3 * seed + 2)
+    return q, k, v, layout_positions(S, layout)
+
+
+def ln_affine(seed: int, scale: float = 0.5, shift: float = 0.2, D: int = HEAD_DIM):
+    """A seeded QK LayerNorm affine ``(q_weight, q_bias, k_weight, k_bias)``:
+    weights 1 + U(-scale, scale), biases N(0, shift^2), fp32 CPU tensors."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(20_000 + int(seed))
+    w = lambda: 1.0 + scale * (2.0 * torch.rand(D, generator=gen) - 1.0)  # noqa: E731
+    b = lambda: shift * torch.randn(D, generator=gen)  # noqa: E731
+    return (w(), b(), w(), b())
+
+
 def make_workload(w: Workload, seed: int):
     return make_qkv(w.S, w.g, seed, w.H, w.D)
 

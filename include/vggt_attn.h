@@ -26,7 +26,9 @@
  *                  (r + 1, c + 1); the library uses whatever pos holds.
  *   Each frame holds T = 5 + g*g tokens: the 5 special tokens first, then the
  *   g x g patch grid row-major. Only the descriptor pooling depends on this
- *   order; frame and global attention use pos alone.
+ *   order; frame and global attention use pos alone. The _ex calls lift this:
+ *   frame and global attention take any T >= 1, and the descriptor calls
+ *   take a vggt_frame_layout (rectangular grid, trailing tokens).
  *
  * Common rules:
  *   - D must be 64 (VGGT: 16 heads x 64 dims). H >= 1 is free.
@@ -68,10 +70,13 @@ typedef uint16_t vggt_bf16; /* raw bf16 bits */
 typedef enum vggt_status {
     VGGT_OK = 0,
     VGGT_ERR_NULL = -1,        /* a required pointer is NULL                      */
-    VGGT_ERR_UNSUPPORTED = -2, /* D != 64, a misaligned pointer, or a cache used on
-                                  another device than its own                      */
-    VGGT_ERR_SHAPE = -3,       /* negative sizes, T != 5 + g*g, bad kv_down, or a
-                                  size beyond the library's limits                */
+    VGGT_ERR_UNSUPPORTED = -2, /* D != 64, a misaligned pointer, a cache used on
+                                  another device than its own, or a QK LayerNorm
+                                  affine that is not finite or exceeds the score
+                                  bound (see vggt_qk_norm)                         */
+    VGGT_ERR_SHAPE = -3,       /* negative sizes, T != 5 + g*g (plain calls) or a
+                                  layout that does not add up to T, bad kv_down, or
+                                  a size beyond the library's limits              */
     VGGT_ERR_ALLOC = -4,       /* scratch allocation failed                        */
     VGGT_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed             */
     VGGT_ERR_TIMEOUT = -6,     /* a bounded device-side wait ran out (reported by
@@ -222,11 +227,105 @@ VGGT_API int vggt_desc_cache_reset(vggt_desc_cache* cache);
  * VGGT_ERR_UNSUPPORTED); fails with VGGT_ERR_SHAPE, launching nothing and
  * leaving the cache unchanged, if the chunk does not fit. C == 0 is a no-op.
  * The cache's frame count grows by C when the call returns VGGT_OK.
- * Scratch: the chunk's q_hat and pooled raw keys, from the scratch pool.
+ * Scratch: the chunk's q_hat, from the scratch pool. Three launches: the
+ * query prologue, the pooling fused with the prologue of the new keys, then
+ * the attention.
  */
 VGGT_API int vggt_attn_descriptor_chunk(vggt_desc_cache* cache, const vggt_bf16* q,
                                         const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                                         vggt_bf16* out, int C, cudaStream_t stream);
+
+/* ------------------------------------------------------------------ _ex calls
+ *
+ * Frame layout: every frame holds n_front special tokens, then a
+ * grid_h x grid_w patch grid in row-major order, then n_back trailing tokens:
+ * T = n_front + grid_h * grid_w + n_back. VGGT-1B frames are {5, g, g, 0}
+ * (the default wherever a layout pointer may be NULL); the vggt-jax README's
+ * two-image benchmark feeds 350 x 518 images, a 25 x 37 grid; the VGGT-Omega
+ * page appends its 16 register tokens after each frame's patches
+ * ({0, 32, 32, 16} at 512 px, patch 16). Pooling copies front and trailing
+ * tokens and averages the grid's cells: a pooled frame is the n_front
+ * tokens, the ceil(grid_h/kv_down) x ceil(grid_w/kv_down) cells row-major,
+ * then the n_back tokens.
+ */
+typedef struct vggt_frame_layout {
+    int n_front;
+    int grid_h;
+    int grid_w;
+    int n_back;
+} vggt_frame_layout;
+
+/*
+ * QK LayerNorm affine: after the per-head LayerNorm, y = y * weight + bias per
+ * dim, the same D = 64 values for every head (the scale and shift a trained
+ * LayerNorm carries; the pages give none, so without it there is no affine).
+ * Separate arrays for queries and keys; each is a HOST array of D fp32
+ * values or NULL (weight 1, bias 0), read during the call (no reference is
+ * kept). Values must be finite.
+ * Score bound: the attention kernel evaluates exp(score) without a row
+ * maximum (exact up to rounding: softmax ignores a common factor), which
+ * needs every score bounded. With Bq = 8 * max|q_weight| + ||q_bias||_2 (a
+ * bound on the norm of a normalised query, the plain LayerNorm's being below
+ * 8) and Bk likewise, a call needs Bq * Bk / 8 * log2(e) * 1.01 <= 64 (e.g.
+ * weights up to 2.3 with zero bias); beyond it returns VGGT_ERR_UNSUPPORTED.
+ */
+typedef struct vggt_qk_norm {
+    const float* q_weight;
+    const float* q_bias;
+    const float* k_weight;
+    const float* k_bias;
+} vggt_qk_norm;
+
+/* vggt_attn_frame / vggt_attn_global with any T >= 1 (these do not look at
+   the token order) and an optional QK LayerNorm affine (norm may be NULL). */
+VGGT_API int vggt_attn_frame_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                                const float* pos, vggt_bf16* out, int S, int T, int H, int D,
+                                const vggt_qk_norm* norm, cudaStream_t stream);
+VGGT_API int vggt_attn_global_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                                 const float* pos, vggt_bf16* out, int S, int T, int H, int D,
+                                 const vggt_qk_norm* norm, cudaStream_t stream);
+
+/* vggt_attn_descriptor with a frame layout (NULL: {5, g, g, 0}) and an
+   optional QK LayerNorm affine (NULL: none). */
+VGGT_API int vggt_attn_descriptor_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                                     const float* pos, vggt_bf16* out, int S, int T, int H, int D,
+                                     int kv_down, const vggt_frame_layout* layout,
+                                     const vggt_qk_norm* norm, cudaStream_t stream);
+
+/* vggt_kv_pool and vggt_kv_pool_tokens with a frame layout (NULL: default). */
+VGGT_API int vggt_kv_pool_ex(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                             vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out, int S, int T, int H,
+                             int D, int kv_down, const vggt_frame_layout* layout, cudaStream_t stream);
+VGGT_API int vggt_kv_pool_tokens_ex(int T, int kv_down, const vggt_frame_layout* layout);
+
+/* vggt_qk_prologue with an optional affine (HOST arrays of D fp32 values or
+   NULL, as in vggt_qk_norm; no score bound applies here). */
+VGGT_API int vggt_qk_prologue_ex(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int N, int H,
+                                 int D, const float* ln_weight, const float* ln_bias,
+                                 cudaStream_t stream);
+
+/*
+ * The descriptor keys in one memory pass: pools k/v/pos exactly as
+ * vggt_kv_pool_ex, and instead of storing the pooled keys normalises and
+ * rotates them at their pooled positions (the prologue, with the optional
+ * key affine) -- the inputs the attention kernel reads. Bit-identical to
+ * vggt_kv_pool_ex followed by vggt_qk_prologue_ex on the pooled keys, with
+ * one less write and read of the pooled keys. The descriptor calls and the
+ * streaming cache use this pass internally.
+ *   k_hat [H, S*T_k, D] bf16 head-major; v_out [S, T_k, H, D] bf16;
+ *   pos_out [S, T_k, 2] fp32; T_k = vggt_kv_pool_tokens_ex(T, kv_down, layout).
+ */
+VGGT_API int vggt_descriptor_keys(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                                  vggt_bf16* k_hat, vggt_bf16* v_out, float* pos_out, int S, int T,
+                                  int H, int D, int kv_down, const vggt_frame_layout* layout,
+                                  const float* ln_weight, const float* ln_bias, cudaStream_t stream);
+
+/* vggt_desc_cache_create with a frame layout and a QK LayerNorm affine
+   (either may be NULL); the cache keeps copies of both and applies them to
+   every chunk. */
+VGGT_API int vggt_desc_cache_create_ex(vggt_desc_cache** cache, int max_frames, int T, int H, int D,
+                                       int kv_down, const vggt_frame_layout* layout,
+                                       const vggt_qk_norm* norm);
 
 /* Size of the fixed scratch array vggt_attn_global_noalloc draws on. */
 #define VGGT_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -135,3 +135,88 @@ def test_descriptor_cache_argument_checks():
     assert F.lib.vggt_desc_cache_destroy(None) == OK
     fake = ctypes.c_void_p(0x1000)
     assert F.lib.vggt_attn_descriptor_chunk(None, fake, fake, fake, fake, fake, 1, None) == E_NULL
+
+
+# ----------------------------------------------------------------- _ex calls (layouts, LN affine)
+
+
+def test_pool_token_counts_for_layouts():
+    assert F.vggt_kv_pool_tokens_ex(5 + 25 * 37, 4, (5, 25, 37, 0)) == 5 + 7 * 10
+    assert F.vggt_kv_pool_tokens_ex(32 * 32 + 16, 4, (0, 32, 32, 16)) == 64 + 16
+    assert F.vggt_kv_pool_tokens_ex(1374, 4, None) == 105
+    assert F.vggt_kv_pool_tokens_ex(1374, 4, (5, 37, 37, 0)) == 105
+    assert F.vggt_kv_pool_tokens_ex(2 + 3 * 5 + 3, 2, (2, 3, 5, 3)) == 2 + 6 + 3
+    assert F.vggt_kv_pool_tokens_ex(5 + 25 * 37, 4, (5, 37, 25, 1)) == E_SHAPE  # does not add up to T
+    assert F.vggt_kv_pool_tokens_ex(10, 4, (-1, 3, 3, 2)) == E_SHAPE
+    assert F.vggt_kv_pool_tokens_ex(10, 0, (1, 3, 3, 0)) == E_SHAPE
+
+
+def _ex_call(fn, T, ln=None, layout=None, kd=None, S=0):
+    """An empty problem (S = 0): validation runs, nothing is launched."""
+    norm, keep = F._norm(ln)
+    if fn is F.lib.vggt_attn_descriptor_ex:
+        return fn(FAKE, FAKE, FAKE, FAKE, FAKE, S, T, 16, 64, 4 if kd is None else kd, F._layout(layout), norm, None)
+    return fn(FAKE, FAKE, FAKE, FAKE, FAKE, S, T, 16, 64, norm, None)
+
+
+def test_ex_frame_and_global_take_any_frame_length():
+    for plain, ex in ((F.lib.vggt_attn_frame, F.lib.vggt_attn_frame_ex),
+                      (F.lib.vggt_attn_global, F.lib.vggt_attn_global_ex)):
+        assert plain(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 100, 16, 64, 0, None) == E_SHAPE
+        assert _ex_call(ex, 100) == OK
+        assert _ex_call(ex, 0) == E_SHAPE
+        assert ex(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 100, 16, 32, None, None) == E_UNSUP
+
+
+def test_ex_descriptor_layout_checks():
+    d = F.lib.vggt_attn_descriptor_ex
+    assert _ex_call(d, 5 + 25 * 37, layout=(5, 25, 37, 0)) == OK
+    assert _ex_call(d, 5 + 25 * 37) == E_SHAPE              # default layout wants a square grid
+    assert _ex_call(d, 5 + 25 * 37, layout=(5, 25, 36, 0)) == E_SHAPE
+    assert _ex_call(d, 1374, kd=0) == E_SHAPE
+
+
+def test_ln_affine_bound_and_finiteness():
+    g = F.lib.vggt_attn_global_ex
+    w = lambda c: [c] * 64  # noqa: E731
+    assert _ex_call(g, 100, ln=(w(2.0), None, w(2.0), None)) == OK
+    assert _ex_call(g, 100, ln=(w(2.3), None, w(2.3), None)) == OK
+    assert _ex_call(g, 100, ln=(w(2.4), None, w(2.4), None)) == E_UNSUP
+    assert _ex_call(g, 100, ln=(w(-2.4), None, None, None)) == OK        # only the product is bounded
+    # one side alone: Bq * 8 / 8 * log2(e) * 1.01 <= 64 up to Bq = 43.9
+    assert _ex_call(g, 100, ln=(w(5.0), None, None, None)) == OK          # Bq = 40
+    assert _ex_call(g, 100, ln=(w(6.0), None, None, None)) == E_UNSUP     # Bq = 48
+    assert _ex_call(g, 100, ln=(None, w(4.0), None, None)) == OK          # Bq = 8 + ||bias|| = 40
+    assert _ex_call(g, 100, ln=(None, w(5.0), None, None)) == E_UNSUP     # Bq = 48
+    assert _ex_call(g, 100, ln=(w(float("nan")), None, None, None)) == E_UNSUP
+    assert _ex_call(g, 100, ln=(None, None, None, w(float("inf")))) == E_UNSUP
+    # the prologue alone has no score bound, only finiteness
+    wp, keep = F._host_f32(w(50.0), "w")
+    assert F.lib.vggt_qk_prologue_ex(FAKE, FAKE, FAKE, 0, 16, 64, wp, None, None) == OK
+    nanp, keep2 = F._host_f32(w(float("nan")), "w")
+    assert F.lib.vggt_qk_prologue_ex(FAKE, FAKE, FAKE, 0, 16, 64, nanp, None, None) == E_UNSUP
+
+
+def test_descriptor_keys_and_pool_ex_argument_checks():
+    lay = F._layout((5, 25, 37, 0))
+    T = 5 + 25 * 37
+    k = F.lib.vggt_descriptor_keys
+    assert k(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, T, 16, 64, 4, lay, None, None, None) == OK
+    assert k(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, T, 16, 64, 4, None, None, None, None) == E_SHAPE
+    assert k(FAKE, FAKE, FAKE, None, FAKE, FAKE, 1, T, 16, 64, 4, lay, None, None, None) == E_NULL
+    assert k(FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, 1, T, 16, 64, 4, lay, None, None, None) == E_UNSUP
+    p = F.lib.vggt_kv_pool_ex
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, T, 16, 64, 4, lay, None) == OK
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, T, 16, 64, 4, None, None) == E_SHAPE
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, T, 16, 64, 0, lay, None) == E_SHAPE
+
+
+def test_descriptor_cache_ex_checks_before_allocating():
+    import ctypes
+    h = ctypes.c_void_p()
+    c = F.lib.vggt_desc_cache_create_ex
+    assert c(ctypes.byref(h), 10, 5 + 25 * 37, 16, 64, 4, None, None) == E_SHAPE
+    assert not h.value
+    norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
+    assert c(ctypes.byref(h), 10, 5 + 25 * 37, 16, 64, 4, F._layout((5, 25, 37, 0)), norm) == E_UNSUP
+    assert not h.value

@@ -1,0 +1,195 @@
+"""GPU parity of the _ex calls -- frame layouts with a rectangular grid and
+trailing tokens, the QK LayerNorm affine, and the pooling pass fused with the
+key prologue -- against the fp64 CPU oracle (same bars as the plain calls:
+max-abs <= 2e-2 and relative Frobenius <= 5e-3 for attention outputs,
+bit-exact pooled K/V)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vggt_oracle as O
+from feed_forward_view_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_FRO = 5e-3
+
+
+@pytest.fixture(scope="module")
+def F():
+    import feed_forward_view_b200 as F
+
+    return F
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return O.bf16_bits_to_f64(bits(t)).reshape(t.shape)
+
+
+def ln64(ln):
+    return None if ln is None else tuple(None if x is None else x.numpy().astype(np.float64) for x in ln)
+
+
+def check(got: torch.Tensor, ref: np.ndarray, what):
+    g = f64(got)
+    assert np.isfinite(g).all(), what
+    d = g - ref
+    mx = float(np.abs(d).max())
+    rf = float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30))
+    assert mx <= MAX_ABS and rf <= REL_FRO, (what, mx, rf)
+
+
+def status_ok(F):
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+
+
+LAYOUTS = [
+    ((5, 25, 37, 0), 4),   # vggt-jax two-image benchmark grid (350 x 518 images)
+    ((0, 32, 32, 16), 4),  # registers after the patches, 32 x 32 grid
+    ((2, 3, 5, 3), 2),
+    ((1, 7, 4, 2), 3),
+    ((3, 0, 0, 2), 2),     # no grid at all
+]
+
+
+@pytest.mark.parametrize("layout,kd", LAYOUTS)
+def test_kv_pool_ex_bit_exact(F, layout, kd):
+    S = 3
+    q, k, v, pos = synth.make_layout_qkv(S, layout, seed=41)
+    T = k.shape[0] // S
+    ko, vo, po = F.vggt_kv_pool_ex(k.cuda(), v.cuda(), pos.cuda(), S=S, T=T, kv_down=kd, layout=layout)
+    status_ok(F)
+    rk, rv, rp = O.kv_pool_bf16_reference(bits(k).reshape(S * T, -1), bits(v).reshape(S * T, -1),
+                                          pos.numpy(), S, T, kd, layout=layout)
+    assert np.array_equal(bits(ko).reshape(rk.shape), rk)
+    assert np.array_equal(bits(vo).reshape(rv.shape), rv)
+    assert np.array_equal(po.cpu().numpy(), rp)
+
+
+@pytest.mark.parametrize("H", [16, 5, 20])
+@pytest.mark.parametrize("affine", [False, True])
+def test_fused_descriptor_keys_equal_pool_then_prologue(F, H, affine):
+    S, layout, kd = 3, (5, 9, 11, 2), 3
+    q, k, v, pos = synth.make_layout_qkv(S, layout, seed=42, H=H)
+    T = k.shape[0] // S
+    w, b = (synth.ln_affine(7)[2:]) if affine else (None, None)
+    kd_, vd, pd = k.cuda(), v.cuda(), pos.cuda()
+    kh, vo, po = F.vggt_descriptor_keys(kd_, vd, pd, S=S, T=T, H=H, kv_down=kd, layout=layout,
+                                        ln_weight=w, ln_bias=b)
+    kp, vp, pp = F.vggt_kv_pool_ex(kd_, vd, pd, S=S, T=T, H=H, kv_down=kd, layout=layout)
+    kh2 = F.vggt_qk_prologue_ex(kp, pp, H=H, ln_weight=w, ln_bias=b)
+    status_ok(F)
+    assert np.array_equal(bits(vo), bits(vp))
+    assert np.array_equal(po.cpu().numpy(), pp.cpu().numpy())
+    assert np.array_equal(bits(kh), bits(kh2))
+    # and the keys are the oracle's within one bf16 rounding
+    rk, _, rp = O.kv_pool(f64(k), f64(v), pos.numpy().astype(np.float64), S, T, kd, layout=layout)
+    ref = O.qk_prologue(f64(kp.cpu()), pp.cpu().numpy().astype(np.float64),
+                        None if w is None else w.numpy().astype(np.float64),
+                        None if b is None else b.numpy().astype(np.float64)).transpose(1, 0, 2)
+    got = f64(kh)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-4)
+
+
+def test_prologue_ex_affine_matches_oracle(F):
+    S, g, H = 2, 9, 16
+    x, _, _, pos = synth.make_qkv(S, g, seed=43, H=H)
+    w, b, _, _ = synth.ln_affine(8, scale=1.5, shift=1.0)
+    xh = F.vggt_qk_prologue_ex(x.cuda(), pos.cuda(), H=H, ln_weight=w, ln_bias=b)
+    status_ok(F)
+    ref = O.qk_prologue(f64(x), pos.numpy().astype(np.float64), w.numpy().astype(np.float64),
+                        b.numpy().astype(np.float64)).transpose(1, 0, 2)
+    assert np.all(np.abs(f64(xh) - ref) <= 2.0 ** -8 * np.abs(ref) + 5e-4)
+
+
+@pytest.mark.parametrize("kind,S,layout,affine", [
+    ("frame", 3, (0, 10, 30, 0), True),     # T = 300: not 5 + g*g
+    ("frame", 2, (5, 25, 37, 0), False),
+    ("global", 2, (5, 11, 19, 3), True),
+    ("global", 1, (0, 13, 13, 0), False),
+])
+def test_frame_and_global_ex_match_oracle(F, kind, S, layout, affine):
+    q, k, v, pos = synth.make_layout_qkv(S, layout, seed=44)
+    T = q.shape[0] // S
+    ln = synth.ln_affine(9) if affine else None
+    fn = F.vggt_attn_frame_ex if kind == "frame" else F.vggt_attn_global_ex
+    out = fn(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), S=S, T=T, ln=ln)
+    status_ok(F)
+    oracle = O.attn_frame if kind == "frame" else O.attn_global
+    ref = oracle(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, ln=ln64(ln))
+    check(out, ref, (kind, S, layout, affine))
+
+
+@pytest.mark.parametrize("layout,kd,affine", [
+    ((5, 25, 37, 0), 4, False),
+    ((0, 32, 32, 16), 4, True),
+    ((2, 7, 12, 3), 3, True),
+    ((5, 25, 37, 0), 1, False),
+])
+def test_descriptor_ex_matches_oracle(F, layout, kd, affine):
+    S = 4
+    q, k, v, pos = synth.make_layout_qkv(S, layout, seed=45)
+    T = q.shape[0] // S
+    ln = synth.ln_affine(10) if affine else None
+    out = F.vggt_attn_descriptor_ex(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), S=S, T=T, kv_down=kd,
+                                    layout=layout, ln=ln)
+    status_ok(F)
+    ref = O.attn_descriptor(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, kd,
+                            layout=layout, ln=ln64(ln))
+    check(out, ref, (layout, kd, affine))
+
+
+def test_descriptor_ex_default_layout_equals_plain_call(F):
+    S, g = 3, 9
+    q, k, v, pos = synth.make_qkv(S, g, seed=46)
+    T = 5 + g * g
+    args = [t.cuda() for t in (q, k, v, pos)]
+    a = F.vggt_attn_descriptor(*args, S=S, T=T, kv_down=4)
+    b = F.vggt_attn_descriptor_ex(*args, S=S, T=T, kv_down=4, layout=None, ln=None)
+    c = F.vggt_attn_descriptor_ex(*args, S=S, T=T, kv_down=4, layout=(5, g, g, 0),
+                                  ln=(torch.ones(64), torch.zeros(64), None, None))
+    status_ok(F)
+    assert torch.equal(a, b)
+    check(c, f64(a), "identity affine")
+
+
+def test_stream_with_layout_and_affine(F):
+    S, layout, kd, chunk = 5, (0, 12, 16, 4), 4, 2
+    q, k, v, pos = synth.make_layout_qkv(S, layout, seed=47)
+    T = q.shape[0] // S
+    ln = synth.ln_affine(11)
+    dev = [t.cuda() for t in (q, k, v, pos)]
+    out = torch.empty_like(dev[0])
+    with F.DescCache(S, T, kv_down=kd, layout=layout, ln=ln) as cache:
+        for f0 in range(0, S, chunk):
+            c = min(chunk, S - f0)
+            r0, r1 = f0 * T, (f0 + c) * T
+            cache.attend(dev[0][r0:r1], dev[1][r0:r1], dev[2][r0:r1], dev[3][r0:r1], out[r0:r1], C=c)
+        status_ok(F)
+        assert cache.frames == S
+    ref = O.attn_descriptor_stream(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, kd, chunk,
+                                   layout=layout, ln=ln64(ln))
+    check(out, ref, "stream ex")
+
+
+def test_affine_at_the_score_bound(F):
+    # weights 2.3 on queries and keys (the largest the bound admits with no
+    # bias) and k = q: every query's own key scores |q_hat|^2 / 8 ~ 42, about
+    # 61 in log2 units -- exponentials near 2^61 without a row maximum
+    S, g = 2, 9
+    q, _, v, pos = synth.make_qkv(S, g, seed=48)
+    T = 5 + g * g
+    w = torch.full((64,), 2.3)
+    ln = (w, None, w, None)
+    out = F.vggt_attn_global_ex(q.cuda(), q.cuda(), v.cuda(), pos.cuda(), S=S, T=T, ln=ln)
+    status_ok(F)
+    ref = O.attn_global(f64(q), f64(q), f64(v), pos.numpy().astype(np.float64), S, T, ln=ln64(ln))
+    check(out, ref, "bound")
+    # the diagonal dominates: each output is close to its own value row
+    assert np.abs(ref - f64(v)).max() < 0.05
