@@ -50,6 +50,15 @@ Options beyond the pages' default reading (both off by default):
   trained LayerNorm carries them; the pages give no values, so the default is
   the identity).
 
+* token subsets (``attn_subset``): frames whose last ``n_skip_back`` tokens
+  take no part in a call, plus ``n_extra`` sequence tokens after the frames
+  that take part in global attention only -- the VGGT-Omega page's register
+  tokens (after the patches, attending only at register_attention_block_
+  indices [2, 6, 9, 14, 20]), storage tokens (4, shared by the sequence) and
+  camera token (one for all frames). How the storage and camera tokens attend
+  is not on the page; the reading here: as ordinary tokens of the global
+  sequence, outside every frame.
+
 Evaluating a subset of query rows is the same definition restricted to those
 rows: every output row depends only on its own query and the key set, so
 ``rows=`` changes nothing about any row that is computed.
@@ -414,6 +423,59 @@ def attn_descriptor_stream(q, k, v, pos, S: int, T: int, kd: int, chunk: int, ro
         n_keys = min(S, (int(c) + 1) * chunk) * tk
         q_hat = qk_prologue(np.asarray(q)[r], np.asarray(pos)[r], *_ln(ln, "q"))
         out[sel] = cross_attention(q_hat, k_hat[:n_keys], vp[:n_keys])
+    return out
+
+
+def subset_rows(S: int, T: int, n_skip_back: int, n_extra: int) -> np.ndarray:
+    """The token rows that take part in a subset call, in order: the first
+    ``T - n_skip_back`` tokens of each of the ``S`` frames, then the
+    ``n_extra`` sequence tokens that follow the frames (rows ``S*T ..``)."""
+    keep = T - n_skip_back
+    if not (0 <= n_skip_back <= T and n_extra >= 0):
+        raise ValueError("need 0 <= n_skip_back <= T and n_extra >= 0")
+    rows = [s * T + np.arange(keep) for s in range(S)] + [S * T + np.arange(n_extra)]
+    return np.concatenate(rows).astype(np.int64)
+
+
+def attn_subset(q, k, v, pos, S: int, T: int, n_skip_back: int, n_extra: int, kind: str,
+                rows=None, ln=None) -> np.ndarray:
+    """Attention over a subset of the tokens -- the VGGT-Omega layout, whose
+    register tokens sit after each frame's patches and take part only in some
+    blocks, and whose storage and camera tokens belong to the whole sequence
+    (VGGT-Omega page: num_register_tokens, register_attention_block_indices,
+    num_storage_tokens, camera_token).
+
+    Tokens: ``S`` frames of ``T`` rows, then ``n_extra`` sequence rows. The
+    last ``n_skip_back`` rows of every frame take no part (neither query nor
+    key). ``kind == "frame"``: every kept row of frame ``s`` attends to the kept
+    rows of frame ``s``; the sequence rows take no part. ``kind == "global"``:
+    every kept row and every sequence row attends to all of them. Returns the
+    outputs of the selected kept rows (``rows``: indices into the original
+    token rows, all kept by default), in that order.
+    """
+    keep_rows = subset_rows(S, T, n_skip_back, n_extra if kind == "global" else 0)
+    q, k, pos = np.asarray(q), np.asarray(k), np.asarray(pos)
+    v = np.asarray(v, dtype=np.float64)
+    if rows is None:
+        rows = keep_rows
+    rows = np.asarray(rows, dtype=np.int64)
+    if not np.isin(rows, keep_rows).all():
+        raise ValueError("rows must be rows that take part")
+    if kind == "global":
+        q_hat = qk_prologue(q[rows], pos[rows], *_ln(ln, "q"))
+        k_hat = qk_prologue(k[keep_rows], pos[keep_rows], *_ln(ln, "k"))
+        return cross_attention(q_hat, k_hat, v[keep_rows])
+    if kind != "frame":
+        raise ValueError("kind must be 'frame' or 'global'")
+    keep = T - n_skip_back
+    out = np.empty((rows.size, q.shape[1], v.shape[2]))
+    frames = rows // T
+    for s in np.unique(frames):
+        sel = np.nonzero(frames == s)[0]
+        kr = s * T + np.arange(keep)
+        q_hat = qk_prologue(q[rows[sel]], pos[rows[sel]], *_ln(ln, "q"))
+        k_hat = qk_prologue(k[kr], pos[kr], *_ln(ln, "k"))
+        out[sel] = cross_attention(q_hat, k_hat, v[kr])
     return out
 
 

@@ -630,3 +630,80 @@ def test_descriptor_with_rect_layout_brute_force_tiny():
         w = [math.exp(t - m) for t in sc]
         want = sum(wi * vi for wi, vi in zip(w, vals)) / sum(w)
         assert np.allclose(got[i, 0], want, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------- token subsets (VGGT-Omega layout)
+
+
+def _seq_scene(S, T, E, H=2, seed=0):
+    rng = np.random.default_rng(seed)
+    n = S * T + E
+    q, k, v = (rng.normal(size=(n, H, 64)) for _ in range(3))
+    pos = rng.integers(0, 9, size=(n, 2)).astype(np.float64)
+    return q, k, v, pos
+
+
+def test_subset_rows_lists_kept_frame_rows_then_sequence_rows():
+    assert O.subset_rows(2, 5, 2, 3).tolist() == [0, 1, 2, 5, 6, 7, 10, 11, 12]
+    assert O.subset_rows(2, 3, 0, 0).tolist() == [0, 1, 2, 3, 4, 5]
+    assert O.subset_rows(1, 4, 4, 1).tolist() == [4]
+    with pytest.raises(ValueError):
+        O.subset_rows(2, 3, 4, 0)
+
+
+def test_subset_without_skips_or_extras_is_frame_and_global_attention():
+    S, T = 3, 7
+    q, k, v, pos = _seq_scene(S, T, 0, seed=51)
+    assert np.allclose(O.attn_subset(q, k, v, pos, S, T, 0, 0, "frame"), O.attn_frame(q, k, v, pos, S, T),
+                       rtol=0, atol=1e-14)
+    assert np.allclose(O.attn_subset(q, k, v, pos, S, T, 0, 0, "global"), O.attn_global(q, k, v, pos, S, T),
+                       rtol=0, atol=1e-14)
+
+
+def test_subset_ignores_skipped_tokens_and_frame_kind_ignores_sequence_tokens():
+    S, T, skip, E = 3, 6, 2, 2
+    q, k, v, pos = _seq_scene(S, T, E, seed=52)
+    base_g = O.attn_subset(q, k, v, pos, S, T, skip, E, "global")
+    base_f = O.attn_subset(q, k, v, pos, S, T, skip, E, "frame")
+    q2, k2, v2, p2 = (x.copy() for x in (q, k, v, pos))
+    skipped = [s * T + j for s in range(S) for j in range(T - skip, T)]
+    for x in (q2, k2, v2):
+        x[skipped] += 5.0
+    p2[skipped] += 3.0
+    assert np.array_equal(O.attn_subset(q2, k2, v2, p2, S, T, skip, E, "global"), base_g)
+    assert np.array_equal(O.attn_subset(q2, k2, v2, p2, S, T, skip, E, "frame"), base_f)
+    # sequence tokens: part of global attention, not of frame attention
+    k3, v3 = k.copy(), v.copy()
+    k3[S * T:] += 1.0
+    v3[S * T:] += 1.0
+    assert np.array_equal(O.attn_subset(q, k3, v3, pos, S, T, skip, E, "frame"), base_f)
+    assert np.abs(O.attn_subset(q, k3, v3, pos, S, T, skip, E, "global") - base_g).max() > 1e-6
+    with pytest.raises(ValueError):
+        O.attn_subset(q, k, v, pos, S, T, skip, E, "global", rows=[T - 1])
+
+
+def test_subset_brute_force_tiny():
+    S, T, skip, E, H = 2, 4, 1, 2, 1
+    q, k, v, pos = _seq_scene(S, T, E, H=H, seed=53)
+    n = S * T + E
+
+    def ln(x):
+        m = x.mean()
+        return (x - m) / math.sqrt(((x - m) ** 2).mean() + 1e-5)
+
+    def attend(i, keys):
+        qh = O.rope_2d(ln(q[i, 0]), pos[i])
+        sc = [float(qh @ O.rope_2d(ln(k[j, 0]), pos[j])) / 8.0 for j in keys]
+        m = max(sc)
+        w = [math.exp(x - m) for x in sc]
+        return sum(wi * v[j, 0] for wi, j in zip(w, keys)) / sum(w)
+
+    kept = [t for t in range(n) if t >= S * T or t % T < T - skip]
+    got = O.attn_subset(q, k, v, pos, S, T, skip, E, "global")
+    for r, i in enumerate(kept):
+        assert np.allclose(got[r, 0], attend(i, kept), rtol=0, atol=1e-12)
+    got = O.attn_subset(q, k, v, pos, S, T, skip, E, "frame")
+    frame_rows = [t for t in range(S * T) if t % T < T - skip]
+    for r, i in enumerate(frame_rows):
+        keys = [j for j in frame_rows if j // T == i // T]
+        assert np.allclose(got[r, 0], attend(i, keys), rtol=0, atol=1e-12)
