@@ -211,6 +211,11 @@ class OracleLeg:
             O.attn_descriptor_stream(self.q, self.k, self.v, self.pos, w.S, w.T, w.kv_down, w.chunk, rows=rows)
             chunk_of = rows // (w.T * w.chunk)
             keys = float((numpy.minimum(w.S, (chunk_of + 1) * w.chunk) * w.T_k).mean())
+        elif w.kind.startswith("subset"):
+            kind = w.kind[len("subset_"):]
+            kept = O.subset_rows(w.S, w.T, w.skip, w.n_extra if kind == "global" else 0)
+            O.attn_subset(self.q, self.k, self.v, self.pos, w.S, w.T, w.skip, w.n_extra, kind, rows=kept[rows])
+            keys = w.n_k if kind == "global" else w.T_k
         else:
             O.cross_attention(O.qk_prologue(self.q[rows], self.pos[rows]), self.k_hat, self.vv)
             keys = w.n_k
@@ -263,7 +268,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
-                   "keys": w.n_k if w.kind != "frame" else w.T, "H": w.H, "D": w.D,
+                   "keys": w.T if w.kind == "frame" else (w.T_k if w.kind == "subset_frame" else w.n_k), "H": w.H, "D": w.D,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
@@ -303,6 +308,10 @@ def run_gpu(args):
             cache.reset()
             for r0, r1, c in chunks:
                 cache.attend(qq[r0:r1], kk[r0:r1], vv[r0:r1], pp[r0:r1], oo[r0:r1], C=c)
+    elif w.kind.startswith("subset"):
+        def call(qq, kk, vv, pp, oo):
+            F.vggt_attn_subset(qq, kk, vv, pp, oo, S=w.S, T=w.T, n_skip_back=w.skip, n_extra=w.n_extra,
+                               kind=w.kind[len("subset_"):])
     else:
         fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
               "descriptor": F.vggt_attn_descriptor}[w.kind]
@@ -344,8 +353,12 @@ def run_gpu(args):
     status = F.vggt_get_device_status()
     ms_total = max_over_ranks(ms_local, world, dev)
     # per call or chunk: the prologue, the pooling fused with the key
-    # prologue (descriptors only), the attention
-    launches = 3 * len(chunks) if w.kind == "stream" else 2 + (1 if w.kind == "descriptor" else 0)
+    # prologue (descriptors) or the value gather (subsets that leave tokens
+    # out), the attention
+    if w.kind == "stream":
+        launches = 3 * len(chunks)
+    else:
+        launches = 2 + (1 if w.kind == "descriptor" or (w.kind.startswith("subset") and w.skip) else 0)
     ms_step = ms_total / args.steps
     flops = w.flops()
     value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
@@ -363,10 +376,17 @@ def run_gpu(args):
         F.vggt_descriptor_keys(k, v, pos, k_hat, vp, pp, S=w.S, T=w.T, kv_down=w.kv_down)
         v_use = vp
     else:
-        F.vggt_qk_prologue(k, pos, k_hat)
-        v_use = v
-    F.vggt_qk_prologue(q, pos, q_hat)
-    n_seg, q_len, k_len = (w.S, w.T, w.T) if w.kind == "frame" else (1, w.n_q, w.n_k)
+        # (subsets: the first n_k rows stand in for the kept ones -- the same
+        # sizes, so the same kernel time)
+        F.vggt_qk_prologue(k[:w.n_k], pos[:w.n_k], k_hat)
+        v_use = v[:w.n_k]
+    F.vggt_qk_prologue(q[:w.n_q], pos[:w.n_q], q_hat)
+    if w.kind == "frame":
+        n_seg, q_len, k_len = w.S, w.T, w.T
+    elif w.kind == "subset_frame":
+        n_seg, q_len, k_len = w.S, w.T_k, w.T_k
+    else:
+        n_seg, q_len, k_len = 1, w.n_q, w.n_k
     reps = max(5, min(args.steps, 50))
     if w.kind == "stream":
         attn_ms = ms_step
@@ -384,7 +404,7 @@ def run_gpu(args):
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     for _ in range(reps):
-        F.vggt_qk_prologue(q, pos, q_hat)
+        F.vggt_qk_prologue(q[:w.n_q], pos[:w.n_q], q_hat)
     p1.record(stream)
     torch.cuda.synchronize(dev)
     pro_ms = p0.elapsed_time(p1) / reps
@@ -503,7 +523,7 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
-                       "keys": w.n_k if w.kind != "frame" else w.T, "H": w.H, "D": w.D,
+                       "keys": w.T if w.kind == "frame" else (w.T_k if w.kind == "subset_frame" else w.n_k), "H": w.H, "D": w.D,
                        "kv_down": w.kv_down, "parallelism": f"replicas x{world}",
                        "l2": f"inputs {in_bytes / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
             "tokens_per_s": tokens_s,

@@ -47,6 +47,7 @@ __all__ = [
     "vggt_qk_prologue_ex",
     "vggt_descriptor_keys",
     "vggt_desc_cache_create_ex",
+    "vggt_attn_subset",
     "FrameLayout",
     "QKNorm",
     "EXPORTED_SYMBOLS",
@@ -80,6 +81,7 @@ EXPORTED_SYMBOLS = (
     "vggt_qk_prologue_ex",
     "vggt_descriptor_keys",
     "vggt_desc_cache_create_ex",
+    "vggt_attn_subset",
 )
 
 if not os.path.exists(LIB_PATH):
@@ -156,6 +158,8 @@ lib.vggt_qk_prologue_ex.argtypes = [_p, _p, _p, _i, _i, _i, _f32p, _f32p, _p]
 lib.vggt_qk_prologue_ex.restype = _i
 lib.vggt_descriptor_keys.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _LP, _f32p, _f32p, _p]
 lib.vggt_descriptor_keys.restype = _i
+lib.vggt_attn_subset.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _NP, _p]
+lib.vggt_attn_subset.restype = _i
 lib.vggt_desc_cache_create_ex.argtypes = [ctypes.POINTER(_p), _i, _i, _i, _i, _i, _LP, _NP]
 lib.vggt_desc_cache_create_ex.restype = _i
 
@@ -346,6 +350,24 @@ def vggt_attn_descriptor_ex(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, 
         int(kv_down), _layout(layout), norm, _stream(stream))
     del keep
     _check(rc, "vggt_attn_descriptor_ex")
+    return out
+
+
+def vggt_attn_subset(q, k, v, pos, out=None, S=None, T=None, n_skip_back=0, n_extra=0, H=16, D=64,
+                     kind="global", ln=None, stream=None):
+    """Attention over a token subset (VGGT-Omega layout): S frames of T tokens
+    whose last ``n_skip_back`` take no part, then ``n_extra`` sequence tokens
+    (global attention only). ``kind``: "frame" or "global". Rows that take no
+    part are left as they are in ``out``. Returns ``out``."""
+    if out is None:
+        out = torch.zeros_like(q)
+    norm, keep = _norm(ln)
+    rc = lib.vggt_attn_subset(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                              _ptr(v, torch.bfloat16, "v"), _ptr(pos, torch.float32, "pos"),
+                              _ptr(out, torch.bfloat16, "out"), int(S), int(T), int(n_skip_back), int(n_extra),
+                              int(H), int(D), {"frame": 0, "global": 1}[kind], norm, _stream(stream))
+    del keep
+    _check(rc, "vggt_attn_subset")
     return out
 
 

@@ -410,6 +410,65 @@ int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf
     return to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
 }
 
+int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                     vggt_bf16* out, int S, int T, int n_skip_back, int n_extra, int H, int D, int global,
+                     const vggt_qk_norm* norm, cudaStream_t stream) {
+    if (S < 0 || T < 1 || H < 0 || D < 0 || n_skip_back < 0 || n_skip_back > T || n_extra < 0)
+        return VGGT_ERR_SHAPE;
+    if (global != 0 && global != 1) return VGGT_ERR_SHAPE;
+    if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
+    if (static_cast<long long>(S) * T + n_extra > VGGT_MAX_TOKENS || H > 65535) return VGGT_ERR_SHAPE;
+    Norms norms;
+    const int nrc = make_norms(norm, &norms);
+    if (nrc != VGGT_OK) return nrc;
+    const int keep = T - n_skip_back;
+    // rows that take part: the kept tokens of every frame, then (global) the
+    // sequence tokens after the frames
+    const long long n_frames_rows = static_cast<long long>(S) * keep;
+    const long long n = n_frames_rows + (global ? n_extra : 0);
+    if (n == 0 || H == 0) return VGGT_OK;
+    if (!q || !k || !v || !pos || !out) return VGGT_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned8(pos) || !aligned16(out))
+        return VGGT_ERR_UNSUPPORTED;
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    vggt::RowMap map;
+    if (n_skip_back > 0) {
+        map.group = keep;
+        map.stride = T;
+        map.n_grouped = n_frames_rows;
+    }
+    // scratch: q_hat | k_hat [H, n, 64] and, when rows are left out, the
+    // gathered values [n, H, 64]
+    const size_t plane = head_plane_bytes(n, H);
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, (n_skip_back > 0 ? 3 : 2) * plane, st->pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_ALLOC;
+    }
+    uint16_t* q_hat = static_cast<uint16_t*>(scratch);
+    uint16_t* k_hat = q_hat + plane / sizeof(uint16_t);
+    const uint16_t* v_use = v;
+    int rc = VGGT_OK;
+    if (n_skip_back > 0) {
+        uint16_t* v_c = k_hat + plane / sizeof(uint16_t);
+        rc = to_status(vggt::launch_gather_rows(v, v_c, n, H * VGGT_HEAD_DIM, map, stream));
+        v_use = v_c;
+    }
+    if (rc == VGGT_OK) {
+        PrologueJob jq{q, pos, q_hat, static_cast<int>(n), n, norms.q, map};
+        PrologueJob jk{k, pos, k_hat, static_cast<int>(n), n, norms.k, map};
+        rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
+    }
+    if (rc == VGGT_OK) {
+        AttnProblem p{q_hat, k_hat, v_use, out, global ? 1 : S, global ? static_cast<int>(n) : keep,
+                      global ? static_cast<int>(n) : keep, H, n, n, map};
+        rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
+    }
+    cudaFreeAsync(scratch, stream);
+    return rc;
+}
+
 int vggt_kv_pool_tokens(int T, int kv_down) { return vggt_kv_pool_tokens_ex(T, kv_down, nullptr); }
 
 int vggt_kv_pool_tokens_ex(int T, int kv_down, const vggt_frame_layout* layout) {

@@ -182,6 +182,7 @@ struct Params {
     long long q_stride;     // rows per head plane of q_hat
     int q_len, k_len, H;
     int pairs_per_seg;
+    RowMap out_map;         // query row r is stored at output row map_row(out_map, r)
 };
 
 // Bounded wait that also gives up once this CTA or any other CTA reported a
@@ -650,7 +651,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     // Inputs outside the core's contract can overflow the
                     // max-free softmax; say so instead of storing silently.
                     if (!(l > 0.0f && l <= 3.0e38f)) atomicOr(prm.status, kStatusRange);
-                    uint4* dst = reinterpret_cast<uint4*>(prm.out + (grow * prm.H + h) * kHeadDim + kODims * half);
+                    const long long orow = map_row(prm.out_map, grow);
+                    uint4* dst = reinterpret_cast<uint4*>(prm.out + (orow * prm.H + h) * kHeadDim + kODims * half);
 #pragma unroll
                     for (int v4 = 0; v4 < kODims / 8; ++v4) {
                         uint4 w;
@@ -768,6 +770,7 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     prm.q_len = p.q_len;
     prm.k_len = p.k_len;
     prm.H = p.H;
+    prm.out_map = p.out_map;
     const int n_qtiles = (p.q_len + kBM - 1) / kBM;
     prm.pairs_per_seg = (n_qtiles + 1) / 2;
     dim3 grid(p.n_seg * prm.pairs_per_seg, p.H);

@@ -150,7 +150,8 @@ template <bool kAffine>
 __device__ __forceinline__ void process_token(const PrologueJob& job, const float* aff, int t, int H,
                                               int lane, float my_freq) {
     const int d1 = lane_dim(lane);
-    const uint16_t* xt = job.x + static_cast<size_t>(t) * H * kHeadDim;
+    const long long src = map_row(job.in_map, t);
+    const uint16_t* xt = job.x + static_cast<size_t>(src) * H * kHeadDim;
     for (int h0 = 0; h0 < H; h0 += 4 * kMaxGroups) {
         uint2 w1[kMaxGroups], w2[kMaxGroups];
 #pragma unroll
@@ -164,7 +165,7 @@ __device__ __forceinline__ void process_token(const PrologueJob& job, const floa
             }
         }
         float sv[4], cv[4];
-        token_angles(reinterpret_cast<const float2*>(job.pos)[t], lane, my_freq, sv, cv);
+        token_angles(reinterpret_cast<const float2*>(job.pos)[src], lane, my_freq, sv, cv);
 #pragma unroll
         for (int g = 0; g < kMaxGroups; ++g) {
             const int h = h0 + 4 * g + (lane >> 3);

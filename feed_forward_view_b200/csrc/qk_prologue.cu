@@ -40,7 +40,34 @@ qk_prologue_kernel(const __grid_constant__ PrologueJob a, const __grid_constant_
     }
 }
 
+// One warp per destination row, 16 bytes per lane per step.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n, int chunks, RowMap m) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+    for (long long c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); c < n; c += warps) {
+        const uint4* s = src + map_row(m, c) * chunks;
+        uint4* d = dst + c * chunks;
+        for (int i = lane; i < chunks; i += 32) d[i] = __ldg(s + i);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, long long n, int row_elems,
+                               const RowMap& m, cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long blocks = (n + 7) / 8;
+    if (blocks > static_cast<long long>(sms) * 8) blocks = static_cast<long long>(sms) * 8;
+    gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n, row_elems / 8, m);
+    return cudaPeekAtLastError();
+}
 
 FreqTable rope_freq_table() {
     FreqTable freq;

@@ -21,6 +21,21 @@ constexpr int kHeadDim = 64;
 constexpr int kStatusTimeout = 1;  // a bounded device wait ran out
 constexpr int kStatusRange = 2;    // an attention row sum was not a positive finite number
 
+// Compact row c -> original token row. Identity when group == 0; otherwise
+// the first n_grouped compact rows come in groups of `group` rows whose
+// originals start `stride` rows apart (row c at (c / group) * stride + c %
+// group), and the rows from n_grouped on follow the last group's stride
+// contiguously. Used for calls where a frame's trailing tokens take no part:
+// group = kept tokens per frame, stride = T.
+struct RowMap {
+    long long group = 0, stride = 0, n_grouped = 0;
+};
+VGGT_HD inline long long map_row(const RowMap& m, long long c) {
+    if (m.group == 0) return c;
+    if (c < m.n_grouped) return (c / m.group) * m.stride + c % m.group;
+    return (m.n_grouped / m.group) * m.stride + (c - m.n_grouped);
+}
+
 // RoPE frequencies 100^(-j/16), j = 0..15, in fp32, passed by value.
 struct FreqTable {
     float f[16];
@@ -35,10 +50,11 @@ struct LnAffine {
     int on;
 };
 
-// One tensor to normalise and rotate: x [n, H, 64] token-major in, positions
-// pos [n, 2] (row, col); out head-major: row t of head h goes to
+// One tensor to normalise and rotate: x [., H, 64] token-major in, positions
+// pos [., 2] (row, col); n rows out, head-major: row t of head h goes to
 // x_hat + (h * out_stride + t) * 64 (out_stride = n for a [H, n, 64] array;
-// larger to write n rows into a bigger head-major array at x_hat's row).
+// larger to write n rows into a bigger head-major array at x_hat's row). Row
+// t reads token map_row(in_map, t) of x and pos (identity by default).
 struct PrologueJob {
     const uint16_t* x;
     const float* pos;
@@ -46,6 +62,7 @@ struct PrologueJob {
     int n;
     long long out_stride;
     LnAffine ln;
+    RowMap in_map;
 };
 
 // LayerNorm (eps 1e-5, optional affine) + 2D RoPE (base 100) over one or two
@@ -65,6 +82,11 @@ struct FrameLayout {
         return n_front + nch * ncw + n_back;
     }
 };
+
+// dst row c = src row map_row(m, c) for c < n; rows of `row_elems` bf16
+// values (a multiple of 8).
+cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, long long n, int row_elems,
+                               const RowMap& m, cudaStream_t stream);
 
 // Ceil-mode kd x kd average pooling of the patch grid of every frame, special
 // tokens copied; pooled frame = front specials, cells row-major, trailing
@@ -106,6 +128,7 @@ struct AttnProblem {
     int H;
     long long q_stride;
     long long k_stride;
+    RowMap out_map;  // output row of query row r: map_row(out_map, r)
 };
 
 // Returns cudaSuccess, or an error from tensor-map encoding or the launch.

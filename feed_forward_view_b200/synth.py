@@ -34,24 +34,47 @@ class Workload:
     """One attention workload: kind, frame count, grid side and pooling factor."""
 
     name: str
-    kind: str  # "global" | "frame" | "descriptor" | "stream" (descriptors, chunk by chunk)
+    # "global" | "frame" | "descriptor" | "stream" (descriptors, chunk by
+    # chunk) | "subset_global" | "subset_frame" (a frame's last `skip` tokens
+    # take no part; `n_extra` sequence tokens follow the frames)
+    kind: str
     S: int
     g: int
     kv_down: int = 1
     H: int = HEADS
     D: int = HEAD_DIM
     chunk: int = 0  # frames per chunk ("stream")
+    n_front: int = N_SPECIAL  # special tokens before the grid
+    n_back: int = 0           # tokens after the grid
+    skip: int = 0             # trailing tokens per frame left out ("subset_*")
+    n_extra: int = 0          # sequence tokens after the frames ("subset_*")
 
     @property
     def T(self) -> int:
-        return N_SPECIAL + self.g * self.g
+        return self.n_front + self.g * self.g + self.n_back
+
+    @property
+    def layout(self):
+        return (self.n_front, self.g, self.g, self.n_back)
+
+    @property
+    def rows(self) -> int:
+        """Token rows of the input tensors."""
+        return self.S * self.T + self.n_extra
 
     @property
     def n_q(self) -> int:
+        """Query rows that take part."""
+        if self.kind == "subset_global":
+            return self.S * (self.T - self.skip) + self.n_extra
+        if self.kind == "subset_frame":
+            return self.S * (self.T - self.skip)
         return self.S * self.T
 
     @property
     def T_k(self) -> int:
+        if self.kind in ("subset_global", "subset_frame"):
+            return self.T - self.skip
         if self.kind not in ("descriptor", "stream"):
             return self.T
         nc = -(-self.g // self.kv_down) if self.g > 0 else 0
@@ -59,12 +82,16 @@ class Workload:
 
     @property
     def n_k(self) -> int:
+        if self.kind == "subset_global":
+            return self.n_q
         return self.S * self.T_k
 
     def flops(self) -> float:
         """Algorithmic attention FLOPs: 4 * H * D per (query, key) pair."""
         if self.kind == "frame":
             pairs = self.S * self.T * self.T
+        elif self.kind == "subset_frame":
+            pairs = self.S * self.T_k * self.T_k
         elif self.kind == "stream":
             # chunk c's queries see the descriptors of chunks 0..c
             pairs = sum(min(self.chunk, self.S - f0) * self.T * min(self.S, f0 + self.chunk) * self.T_k
@@ -101,7 +128,15 @@ PROFILE_WORKLOADS = {w.name: w for w in (
 STREAM_WORKLOADS = {w.name: w for w in (
     Workload("stream_s200_g37_kd4_c10", "stream", S=200, g=37, kv_down=4, chunk=10),
 )}
-ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS}
+# The VGGT-Omega layout at 512 px (patch 16: a 32 x 32 grid, 16 register
+# tokens after the patches, 4 storage tokens + 1 camera token for the
+# sequence), 32 frames: global and frame attention of a block where the
+# registers take no part.
+SUBSET_WORKLOADS = {w.name: w for w in (
+    Workload("omega_global_s32_g32", "subset_global", S=32, g=32, n_front=0, n_back=16, skip=16, n_extra=5),
+    Workload("omega_frame_s32_g32", "subset_frame", S=32, g=32, n_front=0, n_back=16, skip=16, n_extra=5),
+)}
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS, **SUBSET_WORKLOADS}
 
 
 def grid_side(T: int) -> int:
@@ -178,7 +213,20 @@ def ln_affine(seed: int, scale: float = 0.5, shift: float = 0.2, D: int = HEAD_D
     return (w(), b(), w(), b())
 
 
+def make_sequence_qkv(S: int, layout, n_extra: int, seed: int, H: int = HEADS, D: int = HEAD_DIM):
+    """``make_layout_qkv`` plus ``n_extra`` sequence tokens after the frames
+    (positions (0,0)), drawn from their own generators."""
+    q, k, v, pos = make_layout_qkv(S, layout, seed, H, D)
+    if n_extra:
+        extra = [normal_bf16((n_extra, H, D), 900 + 3 * seed + i) for i in range(3)]
+        q, k, v = (torch.cat([a, b]) for a, b in zip((q, k, v), extra))
+        pos = torch.cat([pos, torch.zeros(n_extra, 2)])
+    return q, k, v, pos
+
+
 def make_workload(w: Workload, seed: int):
+    if w.kind.startswith("subset"):
+        return make_sequence_qkv(w.S, w.layout, w.n_extra, seed, w.H, w.D)
     return make_qkv(w.S, w.g, seed, w.H, w.D)
 
 

@@ -292,6 +292,33 @@ VGGT_API int vggt_attn_descriptor_ex(const vggt_bf16* q, const vggt_bf16* k, con
                                      int kv_down, const vggt_frame_layout* layout,
                                      const vggt_qk_norm* norm, cudaStream_t stream);
 
+/*
+ * Attention over a subset of the tokens -- the VGGT-Omega layout (VGGT-Omega
+ * page: 16 register tokens after each frame's patches that take part in
+ * attention only at blocks [2, 6, 9, 14, 20]; 4 storage tokens shared by the
+ * whole sequence; one camera token for all frames).
+ *   Tokens: S frames of T tokens, then n_extra sequence tokens (rows S*T ..
+ *   S*T + n_extra - 1) -- q, k, v, out [S*T + n_extra, H, D] bf16, pos
+ *   [S*T + n_extra, 2] fp32.
+ *   The last n_skip_back tokens of every frame take no part: they are neither
+ *   queries nor keys, and their output rows are not written (0 <= n_skip_back
+ *   <= T; at the register blocks n_skip_back = 0).
+ *   global == 0: frame attention over each frame's T - n_skip_back kept tokens;
+ *   the sequence tokens take no part (their output rows are not written).
+ *   global == 1: every kept token and every sequence token attends to all of
+ *   them. How the storage and camera tokens attend is not on the page; this
+ *   call treats them as ordinary tokens of the global sequence, outside every
+ *   frame.
+ * norm: optional QK LayerNorm affine (vggt_qk_norm, may be NULL). With
+ * n_skip_back == 0 and n_extra == 0 this is vggt_attn_frame_ex /
+ * vggt_attn_global_ex. Scratch: q_hat and k_hat of the kept rows, plus their
+ * gathered values when n_skip_back > 0.
+ */
+VGGT_API int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                              const float* pos, vggt_bf16* out, int S, int T, int n_skip_back,
+                              int n_extra, int H, int D, int global, const vggt_qk_norm* norm,
+                              cudaStream_t stream);
+
 /* vggt_kv_pool and vggt_kv_pool_tokens with a frame layout (NULL: default). */
 VGGT_API int vggt_kv_pool_ex(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                              vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out, int S, int T, int H,

@@ -220,3 +220,22 @@ def test_descriptor_cache_ex_checks_before_allocating():
     norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
     assert c(ctypes.byref(h), 10, 5 + 25 * 37, 16, 64, 4, F._layout((5, 25, 37, 0)), norm) == E_UNSUP
     assert not h.value
+
+
+def test_subset_argument_checks():
+    s = F.lib.vggt_attn_subset
+    args = lambda S, T, skip, E, H=16, D=64, g=1: (FAKE, FAKE, FAKE, FAKE, FAKE, S, T, skip, E, H, D, g, None, None)  # noqa: E731
+    assert s(*args(0, 1040, 16, 5, g=0)) == OK         # frame attention of no frames (the sequence
+                                                       # tokens take no part in frame attention)
+    assert s(*args(2, 10, 10, 0)) == OK                # every frame token left out, no sequence tokens
+    assert s(*args(2, 10, 11, 0)) == E_SHAPE
+    assert s(*args(2, 10, -1, 0)) == E_SHAPE
+    assert s(*args(2, 10, 0, -1)) == E_SHAPE
+    assert s(*args(2, 0, 0, 0)) == E_SHAPE
+    assert s(*args(2, 10, 0, 0, g=2)) == E_SHAPE
+    assert s(*args(2, 10, 0, 0, D=32)) == E_UNSUP
+    assert s(*args(2, 10, 0, 0, H=0)) == OK
+    assert s(FAKE, None, FAKE, FAKE, FAKE, 2, 10, 0, 0, 16, 64, 1, None, None) == E_NULL
+    assert s(FAKE, FAKE, FAKE + 8, FAKE, FAKE, 2, 10, 0, 0, 16, 64, 1, None, None) == E_UNSUP
+    norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
+    assert s(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 0, 0, 16, 64, 1, norm, None) == E_UNSUP

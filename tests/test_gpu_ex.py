@@ -193,3 +193,52 @@ def test_affine_at_the_score_bound(F):
     check(out, ref, "bound")
     # the diagonal dominates: each output is close to its own value row
     assert np.abs(ref - f64(v)).max() < 0.05
+
+
+# ----------------------------------------------------------------- token subsets (VGGT-Omega layout)
+
+
+def _omega_scene(S, layout, E, seed):
+    """Frames laid out per ``layout`` plus ``E`` sequence tokens at (0,0)."""
+    return synth.make_sequence_qkv(S, layout, E, seed)
+
+
+SENTINEL = 7.0
+
+
+@pytest.mark.parametrize("kind,S,layout,skip,E,affine", [
+    ("global", 3, (0, 6, 8, 2), 2, 3, False),
+    ("global", 3, (0, 6, 8, 2), 2, 3, True),
+    ("frame", 3, (0, 6, 8, 2), 2, 3, True),
+    ("global", 2, (1, 9, 13, 0), 0, 4, False),      # sequence tokens only
+    ("frame", 5, (0, 11, 12, 5), 5, 0, False),      # ragged frames (132 kept tokens)
+    ("global", 4, (0, 32, 32, 16), 16, 5, False),   # VGGT-Omega at 512 px, a block without registers
+    ("global", 4, (0, 32, 32, 16), 0, 5, True),     # ... a register block
+    ("frame", 4, (0, 32, 32, 16), 16, 5, False),
+])
+def test_subset_matches_oracle_and_leaves_other_rows(F, kind, S, layout, skip, E, affine):
+    q, k, v, pos = _omega_scene(S, layout, E, seed=61)
+    T = sum(layout[::3]) + layout[1] * layout[2]
+    ln = synth.ln_affine(12) if affine else None
+    out = torch.full(q.shape, SENTINEL, dtype=torch.bfloat16, device="cuda")
+    F.vggt_attn_subset(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), out, S=S, T=T, n_skip_back=skip, n_extra=E,
+                       kind=kind, ln=ln)
+    status_ok(F)
+    kept = O.subset_rows(S, T, skip, E if kind == "global" else 0)
+    ref = O.attn_subset(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, skip, E, kind,
+                        ln=ln64(ln))
+    got = out.cpu()
+    check(got[torch.from_numpy(kept)], ref, (kind, S, layout, skip, E, affine))
+    untouched = np.setdiff1d(np.arange(q.shape[0]), kept)
+    assert torch.all(got[torch.from_numpy(untouched)] == SENTINEL)
+
+
+def test_subset_without_skips_equals_the_ex_calls(F):
+    S, layout = 3, (5, 9, 9, 0)
+    q, k, v, pos = (t.cuda() for t in synth.make_layout_qkv(S, layout, seed=62))
+    T = 86
+    for kind, ex in (("frame", F.vggt_attn_frame_ex), ("global", F.vggt_attn_global_ex)):
+        a = F.vggt_attn_subset(q, k, v, pos, S=S, T=T, kind=kind)
+        b = ex(q, k, v, pos, S=S, T=T)
+        status_ok(F)
+        assert torch.equal(a, b), kind
