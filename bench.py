@@ -308,6 +308,11 @@ def run_gpu(args):
             cache.reset()
             for r0, r1, c in chunks:
                 cache.attend(qq[r0:r1], kk[r0:r1], vv[r0:r1], pp[r0:r1], oo[r0:r1], C=c)
+    elif w.kind.endswith("_f32"):
+        fn32 = F.vggt_attn_global_f32 if w.kind == "global_f32" else F.vggt_attn_frame_f32
+
+        def call(qq, kk, vv, pp, oo):
+            fn32(qq, kk, vv, pp, oo, S=w.S, T=w.T)
     elif w.kind.startswith("subset"):
         def call(qq, kk, vv, pp, oo):
             F.vggt_attn_subset(qq, kk, vv, pp, oo, S=w.S, T=w.T, n_skip_back=w.skip, n_extra=w.n_extra,
@@ -369,42 +374,47 @@ def run_gpu(args):
     # stands for the attention kernel
     H = w.H
     kind_core = "descriptor" if w.kind == "stream" else w.kind
+    f32 = w.kind.endswith("_f32")
     q_hat = torch.empty((H, w.n_q, 64), dtype=torch.bfloat16, device=dev)
     k_hat = torch.empty((H, w.n_k, 64), dtype=torch.bfloat16, device=dev)
+    # the bf16 kernels below time the same shapes (on bf16 copies in the fp32
+    # mode, whose own attention kernel is timed as the whole step)
+    qb, kb, vb = (t.to(torch.bfloat16) for t in (q, k, v)) if f32 else (q, k, v)
+    out_b = torch.empty_like(qb) if f32 else out
     if kind_core == "descriptor":
-        kp, vp, pp = F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down)
-        F.vggt_descriptor_keys(k, v, pos, k_hat, vp, pp, S=w.S, T=w.T, kv_down=w.kv_down)
+        kp, vp, pp = F.vggt_kv_pool(kb, vb, pos, S=w.S, T=w.T, kv_down=w.kv_down)
+        F.vggt_descriptor_keys(kb, vb, pos, k_hat, vp, pp, S=w.S, T=w.T, kv_down=w.kv_down)
         v_use = vp
     else:
         # (subsets: the first n_k rows stand in for the kept ones -- the same
         # sizes, so the same kernel time)
-        F.vggt_qk_prologue(k[:w.n_k], pos[:w.n_k], k_hat)
-        v_use = v[:w.n_k]
-    F.vggt_qk_prologue(q[:w.n_q], pos[:w.n_q], q_hat)
-    if w.kind == "frame":
+        F.vggt_qk_prologue(kb[:w.n_k], pos[:w.n_k], k_hat)
+        v_use = vb[:w.n_k]
+    F.vggt_qk_prologue(qb[:w.n_q], pos[:w.n_q], q_hat)
+    if w.kind in ("frame", "frame_f32"):
         n_seg, q_len, k_len = w.S, w.T, w.T
     elif w.kind == "subset_frame":
         n_seg, q_len, k_len = w.S, w.T_k, w.T_k
     else:
         n_seg, q_len, k_len = 1, w.n_q, w.n_k
     reps = max(5, min(args.steps, 50))
-    if w.kind == "stream":
+    if w.kind == "stream" or f32:
         attn_ms = ms_step
     else:
         for _ in range(3):
-            F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
+            F.vggt_attn_core(q_hat, k_hat, v_use, out_b, n_seg, q_len, k_len)
         torch.cuda.synchronize(dev)
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for _ in range(reps):
-            F.vggt_attn_core(q_hat, k_hat, v_use, out, n_seg, q_len, k_len)
+            F.vggt_attn_core(q_hat, k_hat, v_use, out_b, n_seg, q_len, k_len)
         a1.record(stream)
         torch.cuda.synchronize(dev)
         attn_ms = a0.elapsed_time(a1) / reps
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     for _ in range(reps):
-        F.vggt_qk_prologue(q[:w.n_q], pos[:w.n_q], q_hat)
+        F.vggt_qk_prologue(qb[:w.n_q], pos[:w.n_q], q_hat)
     p1.record(stream)
     torch.cuda.synchronize(dev)
     pro_ms = p0.elapsed_time(p1) / reps
@@ -415,12 +425,12 @@ def run_gpu(args):
         # pooled k, v and positions.
         kp_o, vp_o, pp_o = (torch.empty_like(t) for t in (kp, vp, pp))
         for _ in range(3):
-            F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
+            F.vggt_kv_pool(kb, vb, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
         torch.cuda.synchronize(dev)
         k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         k0.record(stream)
         for _ in range(reps):
-            F.vggt_kv_pool(k, v, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
+            F.vggt_kv_pool(kb, vb, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
         k1.record(stream)
         torch.cuda.synchronize(dev)
         pool_ms = k0.elapsed_time(k1) / reps
@@ -430,11 +440,11 @@ def run_gpu(args):
         # the pooling fused with the key prologue (what the call runs): the
         # same bytes, with normalised keys written instead of pooled ones
         for _ in range(3):
-            F.vggt_descriptor_keys(k, v, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
+            F.vggt_descriptor_keys(kb, vb, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
         torch.cuda.synchronize(dev)
         k0.record(stream)
         for _ in range(reps):
-            F.vggt_descriptor_keys(k, v, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
+            F.vggt_descriptor_keys(kb, vb, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
         k1.record(stream)
         torch.cuda.synchronize(dev)
         fk_ms = k0.elapsed_time(k1) / reps
@@ -520,7 +530,8 @@ def run_gpu(args):
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": warmed, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (bf16x3 tensor-core products)" if f32 else "bf16",
             "data": "synthetic",
             "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
                        "keys": w.T if w.kind == "frame" else (w.T_k if w.kind == "subset_frame" else w.n_k), "H": w.H, "D": w.D,
@@ -530,7 +541,9 @@ def run_gpu(args):
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor",
                          "kernel": ("stream step: per chunk pool + prologue + attn_fwd_kernel"
-                                    if w.kind == "stream" else "attn_fwd_kernel"),
+                                    if w.kind == "stream" else
+                                    "fp32-mode step: prologue, operand split, attn_fwd_f32_kernel (flops counted "
+                                    "once per pair; the tensor cores run 3 products)" if f32 else "attn_fwd_kernel"),
                          "achieved": attn_tf,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
                          "peak_source": f"{peak_src} bf16 burst",

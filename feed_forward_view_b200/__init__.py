@@ -48,6 +48,8 @@ __all__ = [
     "vggt_descriptor_keys",
     "vggt_desc_cache_create_ex",
     "vggt_attn_subset",
+    "vggt_attn_frame_f32",
+    "vggt_attn_global_f32",
     "FrameLayout",
     "QKNorm",
     "EXPORTED_SYMBOLS",
@@ -82,6 +84,8 @@ EXPORTED_SYMBOLS = (
     "vggt_descriptor_keys",
     "vggt_desc_cache_create_ex",
     "vggt_attn_subset",
+    "vggt_attn_frame_f32",
+    "vggt_attn_global_f32",
 )
 
 if not os.path.exists(LIB_PATH):
@@ -158,6 +162,9 @@ lib.vggt_qk_prologue_ex.argtypes = [_p, _p, _p, _i, _i, _i, _f32p, _f32p, _p]
 lib.vggt_qk_prologue_ex.restype = _i
 lib.vggt_descriptor_keys.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _LP, _f32p, _f32p, _p]
 lib.vggt_descriptor_keys.restype = _i
+for _name in ("vggt_attn_frame_f32", "vggt_attn_global_f32"):
+    getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _NP, _p]
+    getattr(lib, _name).restype = _i
 lib.vggt_attn_subset.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _NP, _p]
 lib.vggt_attn_subset.restype = _i
 lib.vggt_desc_cache_create_ex.argtypes = [ctypes.POINTER(_p), _i, _i, _i, _i, _i, _LP, _NP]
@@ -369,6 +376,28 @@ def vggt_attn_subset(q, k, v, pos, out=None, S=None, T=None, n_skip_back=0, n_ex
     del keep
     _check(rc, "vggt_attn_subset")
     return out
+
+
+def _attn_f32(fn, q, k, v, pos, out, S, T, H, D, ln, stream):
+    if out is None:
+        out = torch.empty_like(q)
+    norm, keep = _norm(ln)
+    rc = fn(_ptr(q, torch.float32, "q"), _ptr(k, torch.float32, "k"), _ptr(v, torch.float32, "v"),
+            _ptr(pos, torch.float32, "pos"), _ptr(out, torch.float32, "out"),
+            int(S), int(T), int(H), int(D), norm, _stream(stream))
+    del keep
+    _check(rc, fn.__name__)
+    return out
+
+
+def vggt_attn_frame_f32(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
+    """Frame attention in the fp32 mode: fp32 q, k, v [S*T, H, D] in, fp32 out."""
+    return _attn_f32(lib.vggt_attn_frame_f32, q, k, v, pos, out, S, T, H, D, ln, stream)
+
+
+def vggt_attn_global_f32(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
+    """Global attention in the fp32 mode: fp32 q, k, v [S*T, H, D] in, fp32 out."""
+    return _attn_f32(lib.vggt_attn_global_f32, q, k, v, pos, out, S, T, H, D, ln, stream)
 
 
 def vggt_kv_pool_tokens_ex(T: int, kv_down: int, layout=None) -> int:

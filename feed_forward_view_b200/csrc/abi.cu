@@ -469,6 +469,62 @@ int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
     return rc;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The fp32 mode: prologue (q fp32, k split into hi/lo), split v, attention.
+int attn_f32_call(bool global, const float* q, const float* k, const float* v, const float* pos, float* out,
+                  int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream) {
+    int rc = check_common(q, k, v, pos, out, S, T, H, D);
+    Norms norms;
+    if (rc == VGGT_OK || rc == 1) {
+        const int nrc = make_norms(norm, &norms);
+        if (nrc != VGGT_OK) rc = nrc;
+    }
+    if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
+    DeviceState* st = device_state();
+    if (!st) return VGGT_ERR_CUDA;
+    const long long n = static_cast<long long>(S) * T;
+    const size_t plane2 = head_plane_bytes(n, H);  // one bf16 [H, n, 64] plane
+    // scratch: q_hat fp32 | k_hi | k_lo | v_hi | v_lo
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, 6 * plane2, st->pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_ALLOC;
+    }
+    float* q_hat = static_cast<float*>(scratch);
+    uint16_t* k_hi = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(scratch) + 2 * plane2);
+    uint16_t* k_lo = k_hi + plane2 / 2;
+    uint16_t* v_hi = k_lo + plane2 / 2;
+    uint16_t* v_lo = v_hi + plane2 / 2;
+    vggt::PrologueJobF32 jq{q, pos, q_hat, nullptr, static_cast<int>(n), n, norms.q, 0};
+    vggt::PrologueJobF32 jk{k, pos, k_hi, k_lo, static_cast<int>(n), n, norms.k, 1};
+    rc = to_status(vggt::launch_qk_prologue_f32(jq, jk, H, stream));
+    if (rc == VGGT_OK) rc = to_status(vggt::launch_split_bf16(v, v_hi, v_lo, n * H * VGGT_HEAD_DIM, stream));
+    if (rc == VGGT_OK) {
+        vggt::AttnProblemF32 p{q_hat, k_hi, k_lo, v_hi, v_lo, out, global ? 1 : S,
+                               global ? static_cast<int>(n) : T, global ? static_cast<int>(n) : T, H, n, n};
+        rc = to_status(vggt::launch_attention_f32(p, st->status, st->wait_limit, stream));
+    }
+    cudaFreeAsync(scratch, stream);
+    return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vggt_attn_frame_f32(const float* q, const float* k, const float* v, const float* pos, float* out, int S, int T,
+                        int H, int D, const vggt_qk_norm* norm, cudaStream_t stream) {
+    return attn_f32_call(false, q, k, v, pos, out, S, T, H, D, norm, stream);
+}
+
+int vggt_attn_global_f32(const float* q, const float* k, const float* v, const float* pos, float* out, int S, int T,
+                         int H, int D, const vggt_qk_norm* norm, cudaStream_t stream) {
+    return attn_f32_call(true, q, k, v, pos, out, S, T, H, D, norm, stream);
+}
+
 int vggt_kv_pool_tokens(int T, int kv_down) { return vggt_kv_pool_tokens_ex(T, kv_down, nullptr); }
 
 int vggt_kv_pool_tokens_ex(int T, int kv_down, const vggt_frame_layout* layout) {

@@ -73,15 +73,13 @@ __device__ __forceinline__ void token_angles(float2 p, int lane, float my_freq, 
 }
 
 // LayerNorm (+ affine) and rotation of one head (8 lanes) whose 8 dims per
-// lane are x1 (dims d1..d1+3) and x2 (d1+16..d1+19); the result is stored at
-// dst + d1 and dst + d1 + 16 (dst = the head vector's 64 outputs). Every lane
-// of the warp runs it (the shuffles need the whole warp); lanes with
-// live == false hold zeros and store nothing. kAffine: apply the affine
+// lane are x1 (dims d1..d1+3) and x2 (d1+16..d1+19); the results, in fp32,
+// go to o1 and o2. Every lane of the warp runs it (the shuffles need the
+// whole warp); lanes that hold no head hold zeros. kAffine: apply the affine
 // staged at aff (gamma[64] then beta[64] in shared memory).
 template <bool kAffine>
-__device__ __forceinline__ void norm_rotate_store(float (&x1)[4], float (&x2)[4], const float* aff,
-                                                  const float (&sv)[4], const float (&cv)[4], bool live,
-                                                  uint16_t* dst, int d1) {
+__device__ __forceinline__ void norm_rotate(float (&x1)[4], float (&x2)[4], const float* aff, const float (&sv)[4],
+                                            const float (&cv)[4], int d1, float (&o1)[4], float (&o2)[4]) {
     float sum = (x1[0] + x1[1]) + (x1[2] + x1[3]) + ((x2[0] + x2[1]) + (x2[2] + x2[3]));
     sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
     sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
@@ -116,12 +114,21 @@ __device__ __forceinline__ void norm_rotate_store(float (&x1)[4], float (&x2)[4]
             y2[i] = fmaf(y2[i], va[d1 + 16 + i], va[kHeadDim + d1 + 16 + i]);
         }
     }
-    float o1[4], o2[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         o1[i] = y1[i] * cv[i] - y2[i] * sv[i];
         o2[i] = y2[i] * cv[i] + y1[i] * sv[i];
     }
+}
+
+// norm_rotate, then the bf16 results stored at dst + d1 and dst + d1 + 16
+// (dst = the head vector's 64 outputs) by lanes with live == true.
+template <bool kAffine>
+__device__ __forceinline__ void norm_rotate_store(float (&x1)[4], float (&x2)[4], const float* aff,
+                                                  const float (&sv)[4], const float (&cv)[4], bool live,
+                                                  uint16_t* dst, int d1) {
+    float o1[4], o2[4];
+    norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, o1, o2);
     if (live) {
         *reinterpret_cast<uint2*>(dst + d1) = make_uint2(pack2(o1[0], o1[1]), pack2(o1[2], o1[3]));
         *reinterpret_cast<uint2*>(dst + d1 + 16) = make_uint2(pack2(o2[0], o2[1]), pack2(o2[2], o2[3]));

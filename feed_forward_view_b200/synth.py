@@ -36,7 +36,8 @@ class Workload:
     name: str
     # "global" | "frame" | "descriptor" | "stream" (descriptors, chunk by
     # chunk) | "subset_global" | "subset_frame" (a frame's last `skip` tokens
-    # take no part; `n_extra` sequence tokens follow the frames)
+    # take no part; `n_extra` sequence tokens follow the frames) |
+    # "global_f32" | "frame_f32" (the fp32 mode)
     kind: str
     S: int
     g: int
@@ -88,7 +89,7 @@ class Workload:
 
     def flops(self) -> float:
         """Algorithmic attention FLOPs: 4 * H * D per (query, key) pair."""
-        if self.kind == "frame":
+        if self.kind in ("frame", "frame_f32"):
             pairs = self.S * self.T * self.T
         elif self.kind == "subset_frame":
             pairs = self.S * self.T_k * self.T_k
@@ -136,7 +137,13 @@ SUBSET_WORKLOADS = {w.name: w for w in (
     Workload("omega_global_s32_g32", "subset_global", S=32, g=32, n_front=0, n_back=16, skip=16, n_extra=5),
     Workload("omega_frame_s32_g32", "subset_frame", S=32, g=32, n_front=0, n_back=16, skip=16, n_extra=5),
 )}
-ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS, **SUBSET_WORKLOADS}
+# The fp32 mode on the dense global workload (9 frames of 1024^2 at patch 16)
+# and on eight 518^2 frames.
+F32_WORKLOADS = {w.name: w for w in (
+    Workload("global_s9_g64_f32", "global_f32", S=9, g=64),
+    Workload("frame_s8_g37_f32", "frame_f32", S=8, g=37),
+)}
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS, **SUBSET_WORKLOADS, **F32_WORKLOADS}
 
 
 def grid_side(T: int) -> int:
@@ -224,7 +231,22 @@ def make_sequence_qkv(S: int, layout, n_extra: int, seed: int, H: int = HEADS, D
     return q, k, v, pos
 
 
+def make_qkv_f32(S: int, layout, seed: int, H: int = HEADS, D: int = HEAD_DIM):
+    """fp32 q, k, v (N(0,1), not rounded) and positions for frames laid out
+    ``(n_front, grid_h, grid_w, n_back)``: the inputs of the fp32 mode."""
+    nf, gh, gw, nb = (int(x) for x in layout)
+    n = S * (nf + gh * gw + nb)
+    gens = []
+    for i in range(3):
+        g = torch.Generator(device="cpu")
+        g.manual_seed(3 * int(seed) + i + 50_000)
+        gens.append(torch.randn(n, H, D, generator=g, dtype=torch.float32))
+    return gens[0], gens[1], gens[2], layout_positions(S, layout)
+
+
 def make_workload(w: Workload, seed: int):
+    if w.kind.endswith("_f32"):
+        return make_qkv_f32(w.S, w.layout, seed, w.H, w.D)
     if w.kind.startswith("subset"):
         return make_sequence_qkv(w.S, w.layout, w.n_extra, seed, w.H, w.D)
     return make_qkv(w.S, w.g, seed, w.H, w.D)

@@ -319,6 +319,24 @@ VGGT_API int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt
                               int n_extra, int H, int D, int global, const vggt_qk_norm* norm,
                               cudaStream_t stream);
 
+/*
+ * The fp32 mode: frame / global attention (as vggt_attn_frame_ex /
+ * vggt_attn_global_ex, any T >= 1, optional QK LayerNorm affine) on fp32
+ * q, k, v [S*T, H, D] with fp32 out, to about fp32 accuracy -- the precision
+ * the vggt-jax README's FP32 parity runs use (its attention: TF32x3 Triton
+ * kernels). The prologue runs in fp32; both attention products run on the
+ * bf16 tensor cores with every fp32 operand x carried as x_hi = bf16(x) plus
+ * x_lo = bf16(x - x_hi): a b = a_hi b_hi + a_hi b_lo + a_lo b_hi (three MMAs,
+ * the dropped term is ~2^-18 a b), fp32 accumulation, exponentials to ~2^-22.
+ * Pointers: q, k, v, out 16-byte aligned (fp32 arrays), pos 8-byte aligned.
+ * Scratch: 12 bytes per (token, head, dim) -- fp32 q_hat and the bf16 hi/lo
+ * terms of k_hat and v. About 3x the tensor-core work of the bf16 path.
+ */
+VGGT_API int vggt_attn_frame_f32(const float* q, const float* k, const float* v, const float* pos, float* out,
+                                 int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream);
+VGGT_API int vggt_attn_global_f32(const float* q, const float* k, const float* v, const float* pos, float* out,
+                                  int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream);
+
 /* vggt_kv_pool and vggt_kv_pool_tokens with a frame layout (NULL: default). */
 VGGT_API int vggt_kv_pool_ex(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                              vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out, int S, int T, int H,

@@ -1,0 +1,99 @@
+"""GPU parity of the fp32 mode (fp32 q, k, v in, fp32 out; both attention
+products as three bf16 MMAs on hi/lo terms) against the fp64 oracle.
+
+Bar (from the arithmetic): hi + lo carries an fp32 operand to ~2^-17
+relative and the dropped lo*lo term is ~2^-18 of a product, so a score
+q_hat.k_hat/8 (|score| < 8) is off by ~1e-5 at most and p = 2^s (MUFU, ~2^-22)
+by ~1e-5 relative; an output, a weighted mean of N(0,1) values, is then off
+by ~1e-5 of the values' scale at worst -- against ~1e-2 for the bf16 path.
+The outputs themselves shrink like 1/sqrt(keys) (about 0.04 at 36 909 keys),
+so the relative Frobenius error of the same absolute error grows with the key
+count. The values themselves enter as v_hi + v_lo (2^-18 relative) with the
+p_lo * v_lo term dropped (~2^-18): with a single key the output is v to
+~1e-5 of |v|. Bars: max-abs <= 2e-5 * max|v|, relative Frobenius <= 2e-4,
+and at least 50x below the bf16 path on the same inputs rounded to bf16.
+Measured: max-abs 3.4e-6 and relative Frobenius 8.0e-5 at 36 909 keys;
+3.3e-5 (|v| up to ~4) with one key."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vggt_oracle as O
+from feed_forward_view_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS_PER_V = 2e-5
+REL_FRO = 2e-4
+
+
+@pytest.fixture(scope="module")
+def F():
+    import feed_forward_view_b200 as F
+
+    return F
+
+
+def f64(t):
+    return t.detach().cpu().double().numpy()
+
+
+def errs(got, ref):
+    d = got - ref
+    return float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(ref))
+
+
+def ln64(ln):
+    return None if ln is None else tuple(None if x is None else x.numpy().astype(np.float64) for x in ln)
+
+
+@pytest.mark.parametrize("kind,S,layout,affine", [
+    ("global", 2, (5, 16, 16, 0), False),   # 522 tokens: ragged tiles and key blocks
+    ("frame", 3, (0, 10, 30, 0), False),    # T = 300
+    ("global", 2, (5, 11, 19, 3), True),
+    ("frame", 8, (5, 37, 37, 0), False),    # 1374-token frames
+    ("global", 1, (0, 1, 1, 0), False),     # a single token
+])
+def test_f32_mode_matches_oracle(F, kind, S, layout, affine):
+    q, k, v, pos = synth.make_qkv_f32(S, layout, seed=71)
+    T = q.shape[0] // S
+    ln = synth.ln_affine(13) if affine else None
+    fn = F.vggt_attn_frame_f32 if kind == "frame" else F.vggt_attn_global_f32
+    out = fn(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), S=S, T=T, ln=ln)
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    oracle = O.attn_frame if kind == "frame" else O.attn_global
+    ref = oracle(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, ln=ln64(ln))
+    got = f64(out)
+    assert np.isfinite(got).all()
+    mx, rf = errs(got, ref)
+    assert mx <= MAX_ABS_PER_V * float(v.abs().max()) and rf <= REL_FRO, (kind, S, layout, mx, rf)
+
+
+def test_f32_mode_is_far_more_accurate_than_bf16(F):
+    S, layout = 2, (5, 16, 16, 0)
+    q, k, v, pos = synth.make_qkv_f32(S, layout, seed=72)
+    T = q.shape[0] // S
+    qb, kb, vb = (t.to(torch.bfloat16) for t in (q, k, v))
+    d = [t.cuda() for t in (q, k, v, pos)]
+    o32 = F.vggt_attn_global_f32(*d, S=S, T=T)
+    o16 = F.vggt_attn_global_ex(qb.cuda(), kb.cuda(), vb.cuda(), d[3], S=S, T=T)
+    torch.cuda.synchronize()
+    p = pos.numpy().astype(np.float64)
+    e32 = errs(f64(o32), O.attn_global(f64(q), f64(k), f64(v), p, S, T))[1]
+    e16 = errs(f64(o16.float()), O.attn_global(f64(qb.float()), f64(kb.float()), f64(vb.float()), p, S, T))[1]
+    assert e32 * 50 < e16, (e32, e16)
+
+
+def test_f32_mode_full_size_sampled_rows(F):
+    # the bench workload's shape (9 frames of 4101 tokens), rows sampled
+    S, layout = 9, (5, 64, 64, 0)
+    q, k, v, pos = synth.make_qkv_f32(S, layout, seed=73)
+    T = q.shape[0] // S
+    out = F.vggt_attn_global_f32(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), S=S, T=T)
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    rows = synth.sample_rows(S * T, 256, seed=5).numpy()
+    ref = O.attn_global(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), S, T, rows=rows)
+    mx, rf = errs(f64(out)[rows], ref)
+    assert mx <= MAX_ABS_PER_V * float(v.abs().max()) and rf <= REL_FRO, (mx, rf)
