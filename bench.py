@@ -33,7 +33,8 @@ DEFAULT_WORKLOAD = "global_s9_g64"
 L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_kernel_global_s6_g64.txt")
-KERNEL_SOURCES = ("feed_forward_view_b200/csrc/attn_fwd.cu", "feed_forward_view_b200/csrc/sm100.cuh")
+KERNEL_SOURCES = ("feed_forward_view_b200/csrc/attn_fwd.cu", "feed_forward_view_b200/csrc/attn_common.cuh",
+                  "feed_forward_view_b200/csrc/sm100.cuh")
 
 
 # ----------------------------------------------------------------------------- helpers

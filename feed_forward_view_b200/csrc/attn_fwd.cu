@@ -94,11 +94,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "sm100.cuh"
-#include "vggt_internal.h"
+#include "attn_common.cuh"
 
 namespace vggt {
 namespace {
+
+using attn::drain_wait;
+using attn::make_map;
+using attn::Waiter;
 
 constexpr int kBM = 128;                          // query rows per tile
 constexpr int kBN = 96;                           // keys per block
@@ -184,47 +187,6 @@ struct Params {
     int pairs_per_seg;
     RowMap out_map;         // query row r is stored at output row map_row(out_map, r)
 };
-
-// Bounded wait that also gives up once this CTA or any other CTA reported a
-// timeout; records a timeout of its own. The barrier is polled back to back
-// (try_wait itself suspends the thread for a while); the abort flag, the clock
-// and the global status word are only looked at every 256 polls, so that a
-// phase that completes is noticed within one poll and not one global-memory
-// round trip later.
-struct Waiter {
-    long long limit;
-    volatile int* abort;
-    int* status;
-
-    __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
-        if (mbar_try_wait(bar, parity)) return true;
-        const long long t0 = clock64();
-        for (uint32_t it = 1;; ++it) {
-            if (mbar_try_wait(bar, parity)) return true;
-            if ((it & 255u) == 0) {
-                if (*abort) return false;
-                if (*reinterpret_cast<volatile int*>(status) & kStatusTimeout) {
-                    *abort = 1;
-                    return false;
-                }
-                if (clock64() - t0 > limit) {
-                    *abort = 1;
-                    atomicOr(status, kStatusTimeout);
-                    return false;
-                }
-            }
-        }
-    }
-};
-
-// Wait used while draining on the way out: ignores the abort flags.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long long limit) {
-    if (mbar_try_wait(bar, parity)) return;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > limit) return;
-    }
-}
 
 // TMEM loads and stores of the widths the two column splits use, picked by
 // array size.
@@ -389,15 +351,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     auto k_smem = [&](int s) { return kv_smem0 + static_cast<uint32_t>(2 * kKVTileBytes) * s; };
     auto v_smem = [&](int s) { return k_smem(s) + static_cast<uint32_t>(kKVTileBytes); };
 
-    // The constant [1, 0, ..., 0] rows in the 128-byte-swizzled layout the
-    // MMA reads: the 16-byte chunk c of row r sits at chunk c ^ (r % 8), so
-    // element 0 of row r lies at byte r * 128 + (r % 8) * 16.
-    for (int i = threadIdx.x; i < kKVTileBytes / 16; i += kThreads) {
-        const int r = i >> 3, chunk = i & 7;
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (chunk == (r & 7)) w.x = 0x3F80u;  // bf16 1.0 in the low half
-        reinterpret_cast<uint4*>(sm.ones)[i] = w;
-    }
+    attn::fill_ones_tile(sm.ones, kKVTileBytes, kThreads);
     fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
 
     if (threadIdx.x == 0) {
@@ -680,38 +634,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }
 
 // ---------------------------------------------------------------- host
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 3-D bf16 tensor map with a {64, box1, box2} box and 128-byte swizzling.
-bool make_map(CUtensorMap* map, const void* base, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
-              uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), d1, d2};
-    const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kHeadDim), box1, box2};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 __global__ void wait_probe_kernel(int* status, long long limit) {
     __shared__ uint64_t bar;

@@ -31,15 +31,16 @@
 // Every wait is bounded; on timeout the CTA records it in the device status
 // word, stops issuing, drains what it has in flight and frees its tensor
 // memory.
-#include <cuda.h>
 #include <cuda_bf16.h>
-#include <cuda_runtime.h>
 
-#include "sm100.cuh"
-#include "vggt_internal.h"
+#include "attn_common.cuh"
 
 namespace vggt {
 namespace {
+
+using attn::drain_wait;
+using attn::make_map;
+using attn::Waiter;
 
 constexpr int kBM = 128;                          // query rows per CTA
 constexpr int kBN = 96;                           // keys per block
@@ -81,41 +82,6 @@ struct Params {
     int tiles_per_seg;
 };
 
-// Bounded wait; gives up once this CTA or another one reported a timeout.
-struct Waiter {
-    long long limit;
-    volatile int* abort;
-    int* status;
-
-    __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
-        if (mbar_try_wait(bar, parity)) return true;
-        const long long t0 = clock64();
-        for (uint32_t it = 1;; ++it) {
-            if (mbar_try_wait(bar, parity)) return true;
-            if ((it & 255u) == 0) {
-                if (*abort) return false;
-                if (*reinterpret_cast<volatile int*>(status) & kStatusTimeout) {
-                    *abort = 1;
-                    return false;
-                }
-                if (clock64() - t0 > limit) {
-                    *abort = 1;
-                    atomicOr(status, kStatusTimeout);
-                    return false;
-                }
-            }
-        }
-    }
-};
-
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long long limit) {
-    if (mbar_try_wait(bar, parity)) return;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > limit) return;
-    }
-}
-
 // hi/lo bf16 terms of two fp32 values, packed low half first.
 __device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
     const float ah = __bfloat162float(__float2bfloat16_rn(a));
@@ -155,13 +121,7 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
     // tile i (0 K_hi, 1 K_lo, 2 V_hi, 3 V_lo) of slot s
     auto tile_smem = [&](int s, int i) { return kv_smem0 + static_cast<uint32_t>(kTileBytes) * (4 * s + i); };
 
-    // the constant [1, 0, ..., 0] rows in the 128-byte-swizzled layout
-    for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads) {
-        const int r = i >> 3, chunk = i & 7;
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (chunk == (r & 7)) w.x = 0x3F80u;
-        reinterpret_cast<uint4*>(sm.ones)[i] = w;
-    }
+    attn::fill_ones_tile(sm.ones, kTileBytes, kThreads);
     fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
@@ -387,36 +347,6 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
 }
 
 // ---------------------------------------------------------------- host
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 3-D bf16 tensor map with a {64, box1, box2} box and 128-byte swizzling.
-bool make_map(CUtensorMap* map, const void* base, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
-              uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), d1, d2};
-    const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kHeadDim), box1, box2};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 }  // namespace
 
