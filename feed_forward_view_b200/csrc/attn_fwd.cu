@@ -184,7 +184,8 @@ struct Params {
     long long wait_limit;
     long long q_stride;     // rows per head plane of q_hat
     int q_len, k_len, H;
-    int pairs_per_seg;
+    int pairs_per_seg;      // CTAs per segment
+    int tiles_per_cta;      // query tiles a CTA owns: 2, or 1 for grids too small to fill the GPU
     RowMap out_map;         // query row r is stored at output row map_row(out_map, r)
 };
 
@@ -322,8 +323,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int pair = blockIdx.x - seg * prm.pairs_per_seg;
     const int h = blockIdx.y;
     const int n_qtiles = (prm.q_len + kBM - 1) / kBM;
-    const int tile0 = 2 * pair;                          // first tile in the segment
-    const int ntile = min(2, n_qtiles - tile0);          // 1 or 2
+    const int tile0 = prm.tiles_per_cta * pair;              // first tile in the segment
+    const int ntile = min(prm.tiles_per_cta, n_qtiles - tile0);  // 1 or 2
     const int k_row0 = seg * prm.k_len;
     const int nkb = (prm.k_len + kBN - 1) / kBN;
     const int last_valid = prm.k_len - (nkb - 1) * kBN;  // keys in the last block
@@ -694,7 +695,18 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     prm.H = p.H;
     prm.out_map = p.out_map;
     const int n_qtiles = (p.q_len + kBM - 1) / kBM;
-    prm.pairs_per_seg = (n_qtiles + 1) / 2;
+    // Two tiles per CTA share every K/V block and keep the tensor core busy
+    // while one tile's softmax runs; one tile per CTA doubles the CTA count,
+    // which pays when two-tile CTAs would not even fill the GPU once.
+#ifndef VGGT_TILES_PER_CTA
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long pair_ctas = static_cast<long long>(p.n_seg) * ((n_qtiles + 1) / 2) * p.H;
+    prm.tiles_per_cta = pair_ctas < sms ? 1 : 2;
+#else
+    prm.tiles_per_cta = VGGT_TILES_PER_CTA;
+#endif
+    prm.pairs_per_seg = (n_qtiles + prm.tiles_per_cta - 1) / prm.tiles_per_cta;
     dim3 grid(p.n_seg * prm.pairs_per_seg, p.H);
     attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_v, prm);
     return cudaPeekAtLastError();
