@@ -372,3 +372,31 @@ def test_stream_full_size_sampled_rows(F):
                                    w.kv_down, 10, rows=rows)
     mx, rf = errors(f64(got)[rows], ref)
     assert mx <= MAX_ABS and rf <= REL_FRO, (mx, rf)
+
+
+def test_frame_attention_at_the_token_limit(F):
+    # the largest call the library accepts: 1526 frames of 1374 tokens =
+    # 2 096 724 tokens <= VGGT_MAX_TOKENS (2^21); rows sampled over all frames,
+    # the first and the last row included
+    S, g = 1526, 37
+    T = 5 + g * g
+    assert S * T <= 1 << 21 < (S + 1) * T
+    q, k, v, pos = synth.make_qkv(S, g, seed=9)
+    dev = torch.device("cuda:0")
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    F.vggt_attn_frame(q.to(dev), k.to(dev), v.to(dev), pos.to(dev), out, S=S, T=T)
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    rows = synth.sample_rows(S * T, 256, seed=11).numpy()
+    # the oracle needs only the frames the sampled rows live in
+    frames = np.unique(rows // T)
+    sel = np.concatenate([np.arange(f * T, (f + 1) * T) for f in frames])
+    remap = {f: i for i, f in enumerate(frames)}
+    local_rows = np.array([remap[r // T] * T + r % T for r in rows])
+    ref = O.attn_frame(f64(q[torch.from_numpy(sel)]), f64(k[torch.from_numpy(sel)]),
+                       f64(v[torch.from_numpy(sel)]), pos.numpy()[sel].astype(np.float64),
+                       frames.size, T, rows=local_rows)
+    got = f64(out.cpu()[torch.from_numpy(rows)])
+    mx, rf = errors(got, ref)
+    assert np.isfinite(got).all()
+    assert mx <= MAX_ABS and rf <= REL_FRO, (mx, rf)
