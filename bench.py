@@ -189,13 +189,15 @@ class OracleLeg:
         q, k, v, pos = synth.make_workload(w, seed)
 
         def f64(t):
+            if t.dtype == torch.float32:  # the fp32 mode's inputs
+                return t.double().numpy()
             return O.bf16_bits_to_f64(t.contiguous().view(torch.int16).numpy().view(np.uint16)).reshape(t.shape)
 
         self.q, self.k, self.v, self.pos = f64(q), f64(k), f64(v), pos.numpy().astype(np.float64)
         if w.kind == "descriptor":
             kp, vp, pp = O.kv_pool(self.k, self.v, self.pos, w.S, w.T, w.kv_down)
             self.k_hat, self.vv = O.qk_prologue(kp, pp), vp
-        elif w.kind == "global":
+        elif w.kind in ("global", "global_f32"):
             self.k_hat, self.vv = O.qk_prologue(self.k, self.pos), self.v
 
     def run(self, n_rows: int, seed: int = 0):
@@ -205,7 +207,7 @@ class OracleLeg:
         w, O = self.w, self.O
         rows = self.synth.sample_rows(w.n_q, n_rows, seed).numpy()
         t0 = time.perf_counter()
-        if w.kind == "frame":
+        if w.kind in ("frame", "frame_f32"):
             O.attn_frame(self.q, self.k, self.v, self.pos, w.S, w.T, rows=rows)
             keys = w.T
         elif w.kind == "stream":
@@ -259,7 +261,8 @@ def run_reference(args):
         times.append(dt)
     threads = blas_threads()
     value = statistics.median(vals)
-    keys_desc = ({"frame": f"all {w.T}", "stream": "the cached-prefix"}.get(w.kind, f"all {w.n_k}"))
+    keys_desc = ({"frame": f"all {w.T}", "frame_f32": f"all {w.T}", "subset_frame": f"all {w.T_k}",
+                  "stream": "the cached-prefix"}.get(w.kind, f"all {w.n_k}"))
     sample = (f"{rows} query rows x {keys_desc} keys x {w.H} heads per step "
               f"(of {w.n_q} rows)" + ("; pooling and key prologue redone each step" if w.kind == "stream"
                                        else ", key prologue precomputed"))

@@ -78,11 +78,12 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic(w) is None
 
 
-@pytest.mark.parametrize("name", ["global_s2_g16", "frame_s8_g37", "descriptor_s200_g37_kd4"])
+@pytest.mark.parametrize("name", ["global_s2_g16", "frame_s8_g37", "descriptor_s200_g37_kd4",
+                                  "omega_frame_s32_g32", "omega_global_s32_g32", "frame_s8_g37_f32"])
 def test_oracle_leg_runs_on_a_small_sample(name):
     from feed_forward_view_b200 import synth
 
-    w = synth.WORKLOADS[name]
+    w = synth.ALL_WORKLOADS[name]
     if w.n_q > 50000:
         pytest.skip("large setup; covered by the reference arm")
     tf, dt, rows = bench.OracleLeg(w).run(8)
