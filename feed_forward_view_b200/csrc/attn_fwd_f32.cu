@@ -14,8 +14,11 @@
 //   S    = Q_hi K_hi^T + Q_hi K_lo^T + Q_lo K_hi^T          (3 x 4 K-steps, N = 96)
 //   [O|l] += P_hi [V_hi|1] + P_lo [V_hi|1] + P_hi [V_lo]    (3 x 6 K-steps, N = 80/80/64)
 // The row sum l comes from the ones column of the first two products (l =
-// sum of P_hi + P_lo, the P that multiplies V); the exponentials use MUFU ex2
-// only (relative error ~2^-22; the bf16 path's cubic polynomial would not do).
+// sum of P_hi + P_lo, the P that multiplies V). The exponentials must be good
+// to ~2^-22: 6 of every 8 score pairs go to MUFU ex2 (that accuracy), 2 to a
+// degree-5 minimax polynomial on the FMA pipe (worst relative error 2.3e-7,
+// fit_exp2_poly.py), so the two units share the work (measured: +3% over
+// MUFU only at 36 909 tokens; 3/8 and 4/8 are no better).
 //
 // One CTA per 128-row query tile of one head. Warps: 0 TMA producer (K_hi,
 // K_lo, V_hi, V_lo of 96 keys into a 4-slot ring), 1 MMA issuer, 2-3 idle,
@@ -55,6 +58,37 @@ constexpr uint32_t kColQHi = 0, kColQLo = 32, kColS = 64, kColPHi = 160, kColPLo
 static_assert(kColO + kOCols <= kTmemCols, "tensor memory columns");
 
 constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64)
+
+// 2^f ~ sum c_i f^i on [-1/2, 1/2], degree 5 (Remez, fit_exp2_poly.py);
+// evaluated after the Cody-Waite split x = j + f (j = round(x) by adding
+// 1.5 * 2^23), 2^j applied to the exponent field.
+constexpr float kE5C0 = 1.000000119e+00f;
+constexpr float kE5C1 = 6.931469440e-01f;
+constexpr float kE5C2 = 2.402212024e-01f;
+constexpr float kE5C3 = 5.550713092e-02f;
+constexpr float kE5C4 = 9.675540961e-03f;
+constexpr float kE5C5 = 1.327647245e-03f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kFmaPer8 = 2;                 // of every 8 score pairs, on the FMA pipe
+
+// 2^a, 2^b on the FMA pipe (|a|, |b| <= 125), packed f32x2 arithmetic.
+__device__ __forceinline__ void exp2_pair_fma(float a, float b, float& pa, float& pb) {
+    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+    const uint64_t x = f2_pack(a, b);
+    const uint64_t t = f2_add(x, magic2);                          // j in the low mantissa bits
+    const uint64_t nj = f2_fma(t, f2_pack(-1.0f, -1.0f), magic2);  // -j, exact
+    const uint64_t f = f2_add(x, nj);                              // x - j, exact, |f| <= 1/2
+    uint64_t y = f2_fma(f2_pack(kE5C5, kE5C5), f, f2_pack(kE5C4, kE5C4));
+    y = f2_fma(y, f, f2_pack(kE5C3, kE5C3));
+    y = f2_fma(y, f, f2_pack(kE5C2, kE5C2));
+    y = f2_fma(y, f, f2_pack(kE5C1, kE5C1));
+    y = f2_fma(y, f, f2_pack(kE5C0, kE5C0));
+    uint32_t q0, q1, t0, t1;
+    u2_unpack(y, q0, q1);
+    u2_unpack(t, t0, t1);
+    pa = __uint_as_float(q0 + (t0 << 23));
+    pb = __uint_as_float(q1 + (t1 << 23));
+}
 
 struct SharedStorage {
     uint8_t kv[kStages][4][kTileBytes];  // [slot][K_hi, K_lo, V_hi, V_lo], 128B-swizzled
@@ -306,9 +340,23 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
                     if (c >= valid) s[c] = -INFINITY;
             }
             uint32_t ph[kCols / 2], pl[kCols / 2];
+            if (j == nkb - 1) {  // masked columns are -inf: MUFU only (2^-inf = 0)
 #pragma unroll
-            for (int c = 0; c < kCols / 2; ++c)
-                split_pair(ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]), ph[c], pl[c]);
+                for (int c = 0; c < kCols / 2; ++c)
+                    split_pair(ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]), ph[c], pl[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < kCols / 2; ++c) {
+                    float pa, pb;
+                    if (c % 8 < kFmaPer8) {
+                        exp2_pair_fma(s[2 * c], s[2 * c + 1], pa, pb);
+                    } else {
+                        pa = ex2_approx(s[2 * c]);
+                        pb = ex2_approx(s[2 * c + 1]);
+                    }
+                    split_pair(pa, pb, ph[c], pl[c]);
+                }
+            }
             if (j > 0 && !uwait(bar_pfree, (j - 1) & 1)) {
                 ok = false;
                 break;

@@ -16,7 +16,9 @@ nearest), so |f| <= 1/2 and f = x - j has no rounding error; then
 
 Running this script prints the float32 coefficients and the worst relative
 error of the float32 Horner evaluation over a dense grid. The values it
-printed are written into attn_fwd.cu (kExp2C0..kExp2C3).
+printed are written into attn_fwd.cu (degree 3, kExp2C0..kExp2C3: P is
+rounded to bf16 there) and attn_fwd_f32.cu (degree 5, kE5C0..kE5C5: the fp32
+mode needs the MUFU instruction's own ~2^-22).
 """
 from __future__ import annotations
 
@@ -87,7 +89,7 @@ def check(coef, degree):
 
 
 if __name__ == "__main__":
-    for deg in (3,):
+    for deg in (3, 5):
         c = remez_exp2(deg)
         c32, worst = check(c, deg)
         print(f"degree {deg}: " + ", ".join(f"{v:.9e}f" for v in c32) + f"   max rel err {worst:.3e}")
