@@ -48,6 +48,12 @@
  *     returns a negative vggt_status and launches nothing.
  *   - No call traps on the device. Device-side waits are bounded; a wait that
  *     runs out sets a device status word that vggt_get_device_status() reads.
+ *   - The attention calls can be captured into a CUDA graph (stream capture on
+ *     `stream`); a replay repeats the call on the same buffers. The first call
+ *     on each device creates the library's scratch pool and sets kernel
+ *     attributes, which cannot happen during a capture: make one ordinary
+ *     call per device (and per variant: frame/global/descriptor, fp32 mode)
+ *     before capturing.
  */
 #ifndef VGGT_ATTN_H
 #define VGGT_ATTN_H

@@ -400,3 +400,29 @@ def test_frame_attention_at_the_token_limit(F):
     mx, rf = errors(got, ref)
     assert np.isfinite(got).all()
     assert mx <= MAX_ABS and rf <= REL_FRO, (mx, rf)
+
+
+@pytest.mark.parametrize("kind", ["global", "frame", "descriptor", "noalloc"])
+def test_calls_replay_from_a_cuda_graph(F, kind):
+    # every call is stream-ordered and allocates from a stream-ordered pool,
+    # so it can be captured into a CUDA graph; a replay repeats the call
+    S, g = 2, 16
+    T = 5 + g * g
+    q, k, v, pos = (t.cuda() for t in synth.make_qkv(S, g, seed=21))
+    fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame, "descriptor": F.vggt_attn_descriptor,
+          "noalloc": F.vggt_attn_global_noalloc}[kind]
+    kd = 3 if kind == "descriptor" else 0
+    ref = fn(q, k, v, pos, S=S, T=T, kv_down=kd)
+    torch.cuda.synchronize()
+    out = torch.empty_like(q)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        fn(q, k, v, pos, out, S=S, T=T, kv_down=kd, stream=side)
+    for _ in range(3):
+        out.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    assert torch.equal(out, ref)
