@@ -50,6 +50,8 @@ Options beyond the pages' default reading (both off by default):
   trained LayerNorm carries them; the pages give no values, so the default is
   the identity).
 
+* several scenes per call (``attn_scenes``): each scene attended on its own
+  (the vggt-jax README feeds ``[B, S, 3, H, W]`` image batches);
 * token subsets (``attn_subset``): frames whose last ``n_skip_back`` tokens
   take no part in a call, plus ``n_extra`` sequence tokens after the frames
   that take part in global attention only -- the VGGT-Omega page's register
@@ -423,6 +425,32 @@ def attn_descriptor_stream(q, k, v, pos, S: int, T: int, kd: int, chunk: int, ro
         n_keys = min(S, (int(c) + 1) * chunk) * tk
         q_hat = qk_prologue(np.asarray(q)[r], np.asarray(pos)[r], *_ln(ln, "q"))
         out[sel] = cross_attention(q_hat, k_hat[:n_keys], vp[:n_keys])
+    return out
+
+
+def attn_scenes(kind: str, q, k, v, pos, B: int, S: int, T: int, kd: int = 1, rows=None, layout=None,
+                ln=None) -> np.ndarray:
+    """``B`` independent scenes in one batch (the pages' inputs are
+    ``[B, S, 3, H, W]``): scene ``b`` is token rows ``[b*S*T, (b+1)*S*T)``, and
+    every scene is attended on its own -- ``kind`` "global" or "descriptor"
+    as ``attn_global`` / ``attn_descriptor`` of that scene's rows. Returns the
+    outputs of the selected rows (all by default), in that order."""
+    n_scene = S * T
+    rows = _rows(B * n_scene, rows)
+    q, k, v, pos = (np.asarray(x) for x in (q, k, v, pos))
+    out = np.empty((rows.size,) + q.shape[1:])
+    scene = rows // n_scene
+    for b in np.unique(scene):
+        sel = np.nonzero(scene == b)[0]
+        lo, hi = b * n_scene, (b + 1) * n_scene
+        local = rows[sel] - lo
+        if kind == "global":
+            out[sel] = attn_global(q[lo:hi], k[lo:hi], v[lo:hi], pos[lo:hi], S, T, rows=local, ln=ln)
+        elif kind == "descriptor":
+            out[sel] = attn_descriptor(q[lo:hi], k[lo:hi], v[lo:hi], pos[lo:hi], S, T, kd, rows=local,
+                                       layout=layout, ln=ln)
+        else:
+            raise ValueError("kind must be 'global' or 'descriptor'")
     return out
 
 

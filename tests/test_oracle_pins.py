@@ -707,3 +707,32 @@ def test_subset_brute_force_tiny():
     for r, i in enumerate(frame_rows):
         keys = [j for j in frame_rows if j // T == i // T]
         assert np.allclose(got[r, 0], attend(i, keys), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------- several scenes per call
+
+
+def test_scenes_are_attended_independently():
+    B, S, g = 3, 2, 3
+    T = 5 + g * g
+    rng = np.random.default_rng(81)
+    q, k, v = (rng.normal(size=(B * S * T, 2, 64)) for _ in range(3))
+    pos = np.tile(_scene(S, g)[3], (B, 1))
+    for kind, kd in (("global", 1), ("descriptor", 2)):
+        got = O.attn_scenes(kind, q, k, v, pos, B, S, T, kd)
+        for b in range(B):
+            r = slice(b * S * T, (b + 1) * S * T)
+            one = (O.attn_global(q[r], k[r], v[r], pos[r], S, T) if kind == "global"
+                   else O.attn_descriptor(q[r], k[r], v[r], pos[r], S, T, kd))
+            assert np.array_equal(got[r], one)
+        # a change in scene 1 leaves scene 0 alone, and B = 1 is the plain call
+        k2 = k.copy()
+        k2[S * T:2 * S * T] += 1.0
+        assert np.array_equal(O.attn_scenes(kind, q, k2, v, pos, B, S, T, kd)[:S * T], got[:S * T])
+    one = O.attn_scenes("global", q[:S * T], k[:S * T], v[:S * T], pos[:S * T], 1, S, T)
+    assert np.array_equal(one, O.attn_global(q[:S * T], k[:S * T], v[:S * T], pos[:S * T], S, T))
+    # brute force: one scene's output is the mean of that scene's values when q = 0
+    z = O.attn_scenes("global", np.zeros_like(q), k, v, pos, B, S, T)
+    for b in range(B):
+        r = slice(b * S * T, (b + 1) * S * T)
+        assert np.allclose(z[r], v[r].mean(axis=0), rtol=0, atol=1e-12)
