@@ -214,6 +214,9 @@ class OracleLeg:
             O.attn_descriptor_stream(self.q, self.k, self.v, self.pos, w.S, w.T, w.kv_down, w.chunk, rows=rows)
             chunk_of = rows // (w.T * w.chunk)
             keys = float((numpy.minimum(w.S, (chunk_of + 1) * w.chunk) * w.T_k).mean())
+        elif w.kind == "global_batch":
+            O.attn_scenes("global", self.q, self.k, self.v, self.pos, w.B, w.S, w.T, rows=rows)
+            keys = w.n_k
         elif w.kind.startswith("subset"):
             kind = w.kind[len("subset_"):]
             kept = O.subset_rows(w.S, w.T, w.skip, w.n_extra if kind == "global" else 0)
@@ -317,6 +320,9 @@ def run_gpu(args):
 
         def call(qq, kk, vv, pp, oo):
             fn32(qq, kk, vv, pp, oo, S=w.S, T=w.T)
+    elif w.kind == "global_batch":
+        def call(qq, kk, vv, pp, oo):
+            F.vggt_attn_global_batch(qq, kk, vv, pp, oo, B=w.B, S=w.S, T=w.T)
     elif w.kind.startswith("subset"):
         def call(qq, kk, vv, pp, oo):
             F.vggt_attn_subset(qq, kk, vv, pp, oo, S=w.S, T=w.T, n_skip_back=w.skip, n_extra=w.n_extra,
@@ -380,7 +386,8 @@ def run_gpu(args):
     kind_core = "descriptor" if w.kind == "stream" else w.kind
     f32 = w.kind.endswith("_f32")
     q_hat = torch.empty((H, w.n_q, 64), dtype=torch.bfloat16, device=dev)
-    k_hat = torch.empty((H, w.n_k, 64), dtype=torch.bfloat16, device=dev)
+    nk_rows = w.n_q if w.kind == "global_batch" else w.n_k  # key rows of all segments
+    k_hat = torch.empty((H, nk_rows, 64), dtype=torch.bfloat16, device=dev)
     # the bf16 kernels below time the same shapes (on bf16 copies in the fp32
     # mode, whose own attention kernel is timed as the whole step)
     qb, kb, vb = (t.to(torch.bfloat16) for t in (q, k, v)) if f32 else (q, k, v)
@@ -392,13 +399,15 @@ def run_gpu(args):
     else:
         # (subsets: the first n_k rows stand in for the kept ones -- the same
         # sizes, so the same kernel time)
-        F.vggt_qk_prologue(kb[:w.n_k], pos[:w.n_k], k_hat)
-        v_use = vb[:w.n_k]
+        F.vggt_qk_prologue(kb[:nk_rows], pos[:nk_rows], k_hat)
+        v_use = vb[:nk_rows]
     F.vggt_qk_prologue(qb[:w.n_q], pos[:w.n_q], q_hat)
     if w.kind in ("frame", "frame_f32"):
         n_seg, q_len, k_len = w.S, w.T, w.T
     elif w.kind == "subset_frame":
         n_seg, q_len, k_len = w.S, w.T_k, w.T_k
+    elif w.kind == "global_batch":
+        n_seg, q_len, k_len = w.B, w.S * w.T, w.S * w.T
     else:
         n_seg, q_len, k_len = 1, w.n_q, w.n_k
     reps = max(5, min(args.steps, 50))

@@ -50,6 +50,8 @@ __all__ = [
     "vggt_attn_subset",
     "vggt_attn_frame_f32",
     "vggt_attn_global_f32",
+    "vggt_attn_global_batch",
+    "vggt_attn_descriptor_batch",
     "FrameLayout",
     "QKNorm",
     "EXPORTED_SYMBOLS",
@@ -86,6 +88,8 @@ EXPORTED_SYMBOLS = (
     "vggt_attn_subset",
     "vggt_attn_frame_f32",
     "vggt_attn_global_f32",
+    "vggt_attn_global_batch",
+    "vggt_attn_descriptor_batch",
 )
 
 if not os.path.exists(LIB_PATH):
@@ -165,6 +169,10 @@ lib.vggt_descriptor_keys.restype = _i
 for _name in ("vggt_attn_frame_f32", "vggt_attn_global_f32"):
     getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _NP, _p]
     getattr(lib, _name).restype = _i
+lib.vggt_attn_global_batch.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _NP, _p]
+lib.vggt_attn_global_batch.restype = _i
+lib.vggt_attn_descriptor_batch.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _LP, _NP, _p]
+lib.vggt_attn_descriptor_batch.restype = _i
 lib.vggt_attn_subset.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _NP, _p]
 lib.vggt_attn_subset.restype = _i
 lib.vggt_desc_cache_create_ex.argtypes = [ctypes.POINTER(_p), _i, _i, _i, _i, _i, _LP, _NP]
@@ -375,6 +383,36 @@ def vggt_attn_subset(q, k, v, pos, out=None, S=None, T=None, n_skip_back=0, n_ex
                               int(H), int(D), {"frame": 0, "global": 1}[kind], norm, _stream(stream))
     del keep
     _check(rc, "vggt_attn_subset")
+    return out
+
+
+def vggt_attn_global_batch(q, k, v, pos, out=None, B=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
+    """B scenes of S frames of T tokens (q, k, v [B*S*T, H, D]); each scene's
+    global attention on its own. Returns ``out``."""
+    if out is None:
+        out = torch.empty_like(q)
+    norm, keep = _norm(ln)
+    rc = lib.vggt_attn_global_batch(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                    _ptr(v, torch.bfloat16, "v"), _ptr(pos, torch.float32, "pos"),
+                                    _ptr(out, torch.bfloat16, "out"), int(B), int(S), int(T), int(H), int(D), norm,
+                                    _stream(stream))
+    del keep
+    _check(rc, "vggt_attn_global_batch")
+    return out
+
+
+def vggt_attn_descriptor_batch(q, k, v, pos, out=None, B=None, S=None, T=None, H=16, D=64, kv_down=4, layout=None,
+                               ln=None, stream=None):
+    """B scenes; each scene's descriptor attention over its own pooled frames."""
+    if out is None:
+        out = torch.empty_like(q)
+    norm, keep = _norm(ln)
+    rc = lib.vggt_attn_descriptor_batch(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                        _ptr(v, torch.bfloat16, "v"), _ptr(pos, torch.float32, "pos"),
+                                        _ptr(out, torch.bfloat16, "out"), int(B), int(S), int(T), int(H), int(D),
+                                        int(kv_down), _layout(layout), norm, _stream(stream))
+    del keep
+    _check(rc, "vggt_attn_descriptor_batch")
     return out
 
 

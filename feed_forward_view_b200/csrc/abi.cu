@@ -194,8 +194,10 @@ enum class Kind { kFrame, kGlobal, kDescriptor };
 // plain == true: the original calls, whose frames are VGGT-1B's (T = 5 +
 // g*g). The _ex calls take any T for frame and global attention (they do not
 // look at the token order) and the caller's layout for the descriptor.
+// B scenes of S frames each (B = 1 for the single-scene calls): global and
+// descriptor attention stay within a scene.
 int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-              const float* pos, uint16_t* out, int S, int T, int H, int D, int kv_down,
+              const float* pos, uint16_t* out, int B, int S, int T, int H, int D, int kv_down,
               const vggt_frame_layout* layout, const vggt_qk_norm* norm, cudaStream_t stream);
 
 }  // namespace
@@ -248,9 +250,11 @@ int pool_and_prologue(const uint16_t* k, const uint16_t* v, const float* pos, in
 }
 
 int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-              const float* pos, uint16_t* out, int S, int T, int H, int D, int kv_down,
+              const float* pos, uint16_t* out, int B, int S, int T, int H, int D, int kv_down,
               const vggt_frame_layout* layout, const vggt_qk_norm* norm, cudaStream_t stream) {
-    int rc = check_common(q, k, v, pos, out, S, T, H, D);
+    if (B < 0 || S < 0) return VGGT_ERR_SHAPE;
+    if (B > 0 && S > VGGT_MAX_TOKENS / B) return VGGT_ERR_SHAPE;
+    int rc = check_common(q, k, v, pos, out, B * S, T, H, D);
     vggt::FrameLayout L{};
     if ((rc == VGGT_OK || rc == 1) && (plain || kind == Kind::kDescriptor)) {
         const int lrc = make_layout(layout, T, &L);
@@ -265,12 +269,12 @@ int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const
         if (nrc != VGGT_OK) rc = nrc;
     }
     if (rc != VGGT_OK) return rc == 1 ? VGGT_OK : rc;
-    if (kind == Kind::kFrame) return run_attention(q, k, v, pos, out, S, T, H, norms, stream);
-    if (kind == Kind::kGlobal) return run_attention(q, k, v, pos, out, 1, S * T, H, norms, stream);
+    if (kind == Kind::kFrame) return run_attention(q, k, v, pos, out, B * S, T, H, norms, stream);
+    if (kind == Kind::kGlobal) return run_attention(q, k, v, pos, out, B, S * T, H, norms, stream);
 
     const int Tk = L.pooled(kv_down);
-    const long long nq = static_cast<long long>(S) * T;
-    const long long nk = static_cast<long long>(S) * Tk;
+    const long long nq = static_cast<long long>(B) * S * T;
+    const long long nk = static_cast<long long>(B) * S * Tk;
     DeviceState* st = device_state();
     if (!st) return VGGT_ERR_CUDA;
     // scratch: q_hat [H, nq, 64] | k_hat [H, nk, 64] | pooled v [nk, H, 64] | pooled pos [nk, 2]
@@ -285,11 +289,12 @@ int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const
     uint16_t* k_hat = q_hat + q_bytes / sizeof(uint16_t);
     uint16_t* vp = k_hat + k_bytes / sizeof(uint16_t);
     float* pp = reinterpret_cast<float*>(vp + k_bytes / sizeof(uint16_t));
-    rc = pool_and_prologue(k, v, pos, S, T, L, kv_down, H, k_hat, nk, vp, pp, q, pos, nq, q_hat, norms,
+    rc = pool_and_prologue(k, v, pos, B * S, T, L, kv_down, H, k_hat, nk, vp, pp, q, pos, nq, q_hat, norms,
                            stream);
     if (rc == VGGT_OK) {
         // every query row attends to all S*Tk descriptors: one segment
-        AttnProblem p{q_hat, k_hat, vp, out, 1, static_cast<int>(nq), static_cast<int>(nk), H, nq, nk};
+        // scene b: its S*T query rows attend to its S*Tk descriptors
+        AttnProblem p{q_hat, k_hat, vp, out, B, S * T, S * Tk, H, nq, nk};
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -333,41 +338,53 @@ extern "C" {
 
 int vggt_attn_frame(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                     vggt_bf16* out, int S, int T, int H, int D, int kv_down, cudaStream_t stream) {
-    return attn_call(Kind::kFrame, true, q, k, v, pos, out, S, T, H, D, kv_down, nullptr, nullptr,
+    return attn_call(Kind::kFrame, true, q, k, v, pos, out, 1, S, T, H, D, kv_down, nullptr, nullptr,
                      stream);
 }
 
 int vggt_attn_global(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                      vggt_bf16* out, int S, int T, int H, int D, int kv_down, cudaStream_t stream) {
-    return attn_call(Kind::kGlobal, true, q, k, v, pos, out, S, T, H, D, kv_down, nullptr, nullptr,
+    return attn_call(Kind::kGlobal, true, q, k, v, pos, out, 1, S, T, H, D, kv_down, nullptr, nullptr,
                      stream);
 }
 
 int vggt_attn_descriptor(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
                          const float* pos, vggt_bf16* out, int S, int T, int H, int D, int kv_down,
                          cudaStream_t stream) {
-    return attn_call(Kind::kDescriptor, true, q, k, v, pos, out, S, T, H, D, kv_down, nullptr, nullptr,
+    return attn_call(Kind::kDescriptor, true, q, k, v, pos, out, 1, S, T, H, D, kv_down, nullptr, nullptr,
                      stream);
 }
 
 int vggt_attn_frame_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                        vggt_bf16* out, int S, int T, int H, int D, const vggt_qk_norm* norm,
                        cudaStream_t stream) {
-    return attn_call(Kind::kFrame, false, q, k, v, pos, out, S, T, H, D, 1, nullptr, norm, stream);
+    return attn_call(Kind::kFrame, false, q, k, v, pos, out, 1, S, T, H, D, 1, nullptr, norm, stream);
 }
 
 int vggt_attn_global_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                         vggt_bf16* out, int S, int T, int H, int D, const vggt_qk_norm* norm,
                         cudaStream_t stream) {
-    return attn_call(Kind::kGlobal, false, q, k, v, pos, out, S, T, H, D, 1, nullptr, norm, stream);
+    return attn_call(Kind::kGlobal, false, q, k, v, pos, out, 1, S, T, H, D, 1, nullptr, norm, stream);
 }
 
 int vggt_attn_descriptor_ex(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
                             const float* pos, vggt_bf16* out, int S, int T, int H, int D, int kv_down,
                             const vggt_frame_layout* layout, const vggt_qk_norm* norm,
                             cudaStream_t stream) {
-    return attn_call(Kind::kDescriptor, false, q, k, v, pos, out, S, T, H, D, kv_down, layout, norm,
+    return attn_call(Kind::kDescriptor, false, q, k, v, pos, out, 1, S, T, H, D, kv_down, layout, norm,
                      stream);
+}
+
+int vggt_attn_global_batch(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                           vggt_bf16* out, int B, int S, int T, int H, int D, const vggt_qk_norm* norm,
+                           cudaStream_t stream) {
+    return attn_call(Kind::kGlobal, false, q, k, v, pos, out, B, S, T, H, D, 1, nullptr, norm, stream);
+}
+
+int vggt_attn_descriptor_batch(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
+                               vggt_bf16* out, int B, int S, int T, int H, int D, int kv_down,
+                               const vggt_frame_layout* layout, const vggt_qk_norm* norm, cudaStream_t stream) {
+    return attn_call(Kind::kDescriptor, false, q, k, v, pos, out, B, S, T, H, D, kv_down, layout, norm, stream);
 }
 
 int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, int N, int H, int D,

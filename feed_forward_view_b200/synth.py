@@ -37,7 +37,8 @@ class Workload:
     # "global" | "frame" | "descriptor" | "stream" (descriptors, chunk by
     # chunk) | "subset_global" | "subset_frame" (a frame's last `skip` tokens
     # take no part; `n_extra` sequence tokens follow the frames) |
-    # "global_f32" | "frame_f32" (the fp32 mode)
+    # "global_f32" | "frame_f32" (the fp32 mode) | "global_batch" (B scenes,
+    # each on its own)
     kind: str
     S: int
     g: int
@@ -49,6 +50,7 @@ class Workload:
     n_back: int = 0           # tokens after the grid
     skip: int = 0             # trailing tokens per frame left out ("subset_*")
     n_extra: int = 0          # sequence tokens after the frames ("subset_*")
+    B: int = 1                # scenes per call ("global_batch")
 
     @property
     def T(self) -> int:
@@ -61,7 +63,7 @@ class Workload:
     @property
     def rows(self) -> int:
         """Token rows of the input tensors."""
-        return self.S * self.T + self.n_extra
+        return self.B * self.S * self.T + self.n_extra
 
     @property
     def n_q(self) -> int:
@@ -70,7 +72,7 @@ class Workload:
             return self.S * (self.T - self.skip) + self.n_extra
         if self.kind == "subset_frame":
             return self.S * (self.T - self.skip)
-        return self.S * self.T
+        return self.B * self.S * self.T
 
     @property
     def T_k(self) -> int:
@@ -85,6 +87,8 @@ class Workload:
     def n_k(self) -> int:
         if self.kind == "subset_global":
             return self.n_q
+        if self.kind == "global_batch":
+            return self.S * self.T  # keys per scene
         return self.S * self.T_k
 
     def flops(self) -> float:
@@ -93,6 +97,8 @@ class Workload:
             pairs = self.S * self.T * self.T
         elif self.kind == "subset_frame":
             pairs = self.S * self.T_k * self.T_k
+        elif self.kind == "global_batch":
+            pairs = self.B * (self.S * self.T) ** 2
         elif self.kind == "stream":
             # chunk c's queries see the descriptors of chunks 0..c
             pairs = sum(min(self.chunk, self.S - f0) * self.T * min(self.S, f0 + self.chunk) * self.T_k
@@ -144,7 +150,12 @@ F32_WORKLOADS = {w.name: w for w in (
     Workload("global_s9_g64_f32", "global_f32", S=9, g=64),
     Workload("frame_s8_g37_f32", "frame_f32", S=8, g=37),
 )}
-ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS, **SUBSET_WORKLOADS, **F32_WORKLOADS}
+# Small scenes batched: 32 scenes of the two-frame 224^2 workload in one call.
+BATCH_WORKLOADS = {w.name: w for w in (
+    Workload("global_b32_s2_g16", "global_batch", S=2, g=16, B=32),
+)}
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS, **SUBSET_WORKLOADS, **F32_WORKLOADS,
+                 **BATCH_WORKLOADS}
 
 
 def grid_side(T: int) -> int:
@@ -250,7 +261,7 @@ def make_workload(w: Workload, seed: int):
         return make_qkv_f32(w.S, w.layout, seed, w.H, w.D)
     if w.kind.startswith("subset"):
         return make_sequence_qkv(w.S, w.layout, w.n_extra, seed, w.H, w.D)
-    return make_qkv(w.S, w.g, seed, w.H, w.D)
+    return make_qkv(w.B * w.S, w.g, seed, w.H, w.D)
 
 
 def sample_rows(n: int, count: int, seed: int) -> torch.Tensor:

@@ -343,6 +343,25 @@ VGGT_API int vggt_attn_frame_f32(const float* q, const float* k, const float* v,
 VGGT_API int vggt_attn_global_f32(const float* q, const float* k, const float* v, const float* pos, float* out,
                                   int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream);
 
+/*
+ * Several scenes per call (the vggt-jax README feeds [B, S, 3, H, W] image
+ * batches): q, k, v, out [B, S, T, H, D] and pos [B, S, T, 2], scene b being
+ * token rows [b*S*T, (b+1)*S*T). Every scene is attended on its own: global
+ * attention over its S*T tokens, or descriptor attention over its S*T_k
+ * pooled descriptors (layout and affine as in the _ex calls; either may be
+ * NULL). B == 1 is vggt_attn_global_ex / vggt_attn_descriptor_ex; B == 0 is a
+ * no-op. Frame attention needs no batched form: B scenes of S frames are
+ * B*S frames. One launch per step for all scenes, so small scenes fill the
+ * GPU together. B*S*T <= VGGT_MAX_TOKENS.
+ */
+VGGT_API int vggt_attn_global_batch(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                                    const float* pos, vggt_bf16* out, int B, int S, int T, int H, int D,
+                                    const vggt_qk_norm* norm, cudaStream_t stream);
+VGGT_API int vggt_attn_descriptor_batch(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
+                                        const float* pos, vggt_bf16* out, int B, int S, int T, int H, int D,
+                                        int kv_down, const vggt_frame_layout* layout, const vggt_qk_norm* norm,
+                                        cudaStream_t stream);
+
 /* vggt_kv_pool and vggt_kv_pool_tokens with a frame layout (NULL: default). */
 VGGT_API int vggt_kv_pool_ex(const vggt_bf16* k, const vggt_bf16* v, const float* pos,
                              vggt_bf16* k_out, vggt_bf16* v_out, float* pos_out, int S, int T, int H,

@@ -251,3 +251,15 @@ def test_f32_mode_argument_checks():
         assert fn(FAKE, FAKE, FAKE + 8, FAKE, FAKE, 2, 10, 16, 64, None, None) == E_UNSUP
         norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
         assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 64, norm, None) == E_UNSUP
+
+
+def test_batch_argument_checks():
+    g, d = F.lib.vggt_attn_global_batch, F.lib.vggt_attn_descriptor_batch
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 261, 16, 64, None, None) == OK
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 3, 0, 261, 16, 64, None, None) == OK
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 261, 16, 64, None, None) == E_SHAPE
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 12, 1 << 10, 261, 16, 64, None, None) == E_SHAPE  # too many tokens
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 2, 261, 16, 32, None, None) == E_UNSUP
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 261, 16, 64, 4, None, None, None) == OK
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 260, 16, 64, 4, None, None, None) == E_SHAPE  # not 5 + g*g
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 261, 16, 64, 0, None, None, None) == E_SHAPE

@@ -242,3 +242,33 @@ def test_subset_without_skips_equals_the_ex_calls(F):
         b = ex(q, k, v, pos, S=S, T=T)
         status_ok(F)
         assert torch.equal(a, b), kind
+
+
+# ----------------------------------------------------------------- several scenes per call
+
+
+@pytest.mark.parametrize("kind,B,S,layout,kd", [
+    ("global", 4, 2, (5, 16, 16, 0), 1),
+    ("global", 3, 3, (0, 9, 11, 2), 1),
+    ("descriptor", 3, 4, (5, 12, 12, 0), 4),
+    ("descriptor", 2, 3, (0, 10, 14, 4), 3),
+])
+def test_scene_batches_match_oracle(F, kind, B, S, layout, kd):
+    q, k, v, pos = synth.make_layout_qkv(B * S, layout, seed=91)
+    T = q.shape[0] // (B * S)
+    ln = synth.ln_affine(14) if B == 3 else None
+    d = [t.cuda() for t in (q, k, v, pos)]
+    if kind == "global":
+        out = F.vggt_attn_global_batch(*d, B=B, S=S, T=T, ln=ln)
+    else:
+        out = F.vggt_attn_descriptor_batch(*d, B=B, S=S, T=T, kv_down=kd, layout=layout, ln=ln)
+    status_ok(F)
+    ref = O.attn_scenes(kind, f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), B, S, T, kd, layout=layout,
+                        ln=ln64(ln))
+    check(out, ref, (kind, B, S, layout, kd))
+    # scene by scene with the single-scene calls: identical bits
+    for b in range(B):
+        r = slice(b * S * T, (b + 1) * S * T)
+        one = (F.vggt_attn_global_ex(*(t[r] for t in d), S=S, T=T, ln=ln) if kind == "global" else
+               F.vggt_attn_descriptor_ex(*(t[r] for t in d), S=S, T=T, kv_down=kd, layout=layout, ln=ln))
+        assert torch.equal(one, out[r])
