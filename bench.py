@@ -319,7 +319,7 @@ def run_gpu(args):
         fn32 = F.vggt_attn_global_f32 if w.kind == "global_f32" else F.vggt_attn_frame_f32
 
         def call(qq, kk, vv, pp, oo):
-            fn32(qq, kk, vv, pp, oo, S=w.S, T=w.T)
+            fn32(qq, kk, vv, pp, oo, S=w.S, T=w.T, terms=w.terms)
     elif w.kind == "global_batch":
         def call(qq, kk, vv, pp, oo):
             F.vggt_attn_global_batch(qq, kk, vv, pp, oo, B=w.B, S=w.S, T=w.T)
@@ -559,7 +559,8 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": warmed, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32 (bf16x3 tensor-core products)" if f32 else "bf16",
+            "dtype": (f"f32 ({w.terms} bf16 terms, {w.terms * (w.terms + 1) // 2} tensor-core products)"
+                      if f32 else "bf16"),
             "data": "synthetic",
             "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
                        "keys": w.T if w.kind == "frame" else (w.T_k if w.kind == "subset_frame" else w.n_k), "H": w.H, "D": w.D,
@@ -571,7 +572,8 @@ def run_gpu(args):
                          "kernel": ("stream step: per chunk pool + prologue + attn_fwd_kernel"
                                     if w.kind == "stream" else
                                     "fp32-mode step: prologue, operand split, attn_fwd_f32_kernel (flops counted "
-                                    "once per pair; the tensor cores run 3 products)" if f32 else "attn_fwd_kernel"),
+                                    f"once per pair; the tensor cores run {w.terms * (w.terms + 1) // 2} products)"
+                                    if f32 else "attn_fwd_kernel"),
                          "achieved": attn_tf,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
                          "peak_source": f"{peak_src} bf16 burst",

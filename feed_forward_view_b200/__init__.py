@@ -167,7 +167,7 @@ lib.vggt_qk_prologue_ex.restype = _i
 lib.vggt_descriptor_keys.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _LP, _f32p, _f32p, _p]
 lib.vggt_descriptor_keys.restype = _i
 for _name in ("vggt_attn_frame_f32", "vggt_attn_global_f32"):
-    getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _NP, _p]
+    getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _NP, _i, _p]
     getattr(lib, _name).restype = _i
 lib.vggt_attn_global_batch.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _NP, _p]
 lib.vggt_attn_global_batch.restype = _i
@@ -416,26 +416,28 @@ def vggt_attn_descriptor_batch(q, k, v, pos, out=None, B=None, S=None, T=None, H
     return out
 
 
-def _attn_f32(fn, q, k, v, pos, out, S, T, H, D, ln, stream):
+def _attn_f32(fn, q, k, v, pos, out, S, T, H, D, ln, terms, stream):
     if out is None:
         out = torch.empty_like(q)
     norm, keep = _norm(ln)
     rc = fn(_ptr(q, torch.float32, "q"), _ptr(k, torch.float32, "k"), _ptr(v, torch.float32, "v"),
             _ptr(pos, torch.float32, "pos"), _ptr(out, torch.float32, "out"),
-            int(S), int(T), int(H), int(D), norm, _stream(stream))
+            int(S), int(T), int(H), int(D), norm, int(terms), _stream(stream))
     del keep
     _check(rc, fn.__name__)
     return out
 
 
-def vggt_attn_frame_f32(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
-    """Frame attention in the fp32 mode: fp32 q, k, v [S*T, H, D] in, fp32 out."""
-    return _attn_f32(lib.vggt_attn_frame_f32, q, k, v, pos, out, S, T, H, D, ln, stream)
+def vggt_attn_frame_f32(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, terms=2, stream=None):
+    """Frame attention in the fp32 mode: fp32 q, k, v [S*T, H, D] in, fp32 out;
+    operands carried as `terms` (2 or 3) bf16 terms."""
+    return _attn_f32(lib.vggt_attn_frame_f32, q, k, v, pos, out, S, T, H, D, ln, terms, stream)
 
 
-def vggt_attn_global_f32(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, stream=None):
-    """Global attention in the fp32 mode: fp32 q, k, v [S*T, H, D] in, fp32 out."""
-    return _attn_f32(lib.vggt_attn_global_f32, q, k, v, pos, out, S, T, H, D, ln, stream)
+def vggt_attn_global_f32(q, k, v, pos, out=None, S=None, T=None, H=16, D=64, ln=None, terms=2, stream=None):
+    """Global attention in the fp32 mode: fp32 q, k, v [S*T, H, D] in, fp32 out;
+    operands carried as `terms` (2 or 3) bf16 terms."""
+    return _attn_f32(lib.vggt_attn_global_f32, q, k, v, pos, out, S, T, H, D, ln, terms, stream)
 
 
 def vggt_kv_pool_tokens_ex(T: int, kv_down: int, layout=None) -> int:

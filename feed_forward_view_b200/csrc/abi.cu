@@ -490,9 +490,11 @@ int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
 
 namespace {
 
-// The fp32 mode: prologue (q fp32, k split into hi/lo), split v, attention.
+// The fp32 mode: prologue (q fp32, k split into its bf16 terms), split v,
+// attention.
 int attn_f32_call(bool global, const float* q, const float* k, const float* v, const float* pos, float* out,
-                  int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream) {
+                  int S, int T, int H, int D, const vggt_qk_norm* norm, int terms, cudaStream_t stream) {
+    if (terms != 2 && terms != 3) return VGGT_ERR_UNSUPPORTED;
     int rc = check_common(q, k, v, pos, out, S, T, H, D);
     Norms norms;
     if (rc == VGGT_OK || rc == 1) {
@@ -504,23 +506,25 @@ int attn_f32_call(bool global, const float* q, const float* k, const float* v, c
     if (!st) return VGGT_ERR_CUDA;
     const long long n = static_cast<long long>(S) * T;
     const size_t plane2 = head_plane_bytes(n, H);  // one bf16 [H, n, 64] plane
-    // scratch: q_hat fp32 | k_hi | k_lo | v_hi | v_lo
+    // scratch: q_hat fp32 | the k_hat terms | the v terms
     void* scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, 6 * plane2, st->pool, stream) != cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&scratch, (2 + 2 * static_cast<size_t>(terms)) * plane2, st->pool, stream) !=
+        cudaSuccess) {
         cudaGetLastError();
         return VGGT_ERR_ALLOC;
     }
     float* q_hat = static_cast<float*>(scratch);
-    uint16_t* k_hi = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(scratch) + 2 * plane2);
-    uint16_t* k_lo = k_hi + plane2 / 2;
-    uint16_t* v_hi = k_lo + plane2 / 2;
-    uint16_t* v_lo = v_hi + plane2 / 2;
-    vggt::PrologueJobF32 jq{q, pos, q_hat, nullptr, static_cast<int>(n), n, norms.q, 0};
-    vggt::PrologueJobF32 jk{k, pos, k_hi, k_lo, static_cast<int>(n), n, norms.k, 1};
+    uint16_t* kt[3] = {nullptr, nullptr, nullptr};
+    uint16_t* vt[3] = {nullptr, nullptr, nullptr};
+    uint16_t* next = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(scratch) + 2 * plane2);
+    for (int t = 0; t < terms; ++t, next += plane2 / 2) kt[t] = next;
+    for (int t = 0; t < terms; ++t, next += plane2 / 2) vt[t] = next;
+    vggt::PrologueJobF32 jq{q, pos, {q_hat, nullptr, nullptr}, static_cast<int>(n), n, norms.q, 0};
+    vggt::PrologueJobF32 jk{k, pos, {kt[0], kt[1], kt[2]}, static_cast<int>(n), n, norms.k, terms};
     rc = to_status(vggt::launch_qk_prologue_f32(jq, jk, H, stream));
-    if (rc == VGGT_OK) rc = to_status(vggt::launch_split_bf16(v, v_hi, v_lo, n * H * VGGT_HEAD_DIM, stream));
+    if (rc == VGGT_OK) rc = to_status(vggt::launch_split_bf16(v, vt, terms, n * H * VGGT_HEAD_DIM, stream));
     if (rc == VGGT_OK) {
-        vggt::AttnProblemF32 p{q_hat, k_hi, k_lo, v_hi, v_lo, out, global ? 1 : S,
+        vggt::AttnProblemF32 p{q_hat, {kt[0], kt[1], kt[2]}, {vt[0], vt[1], vt[2]}, terms, out, global ? 1 : S,
                                global ? static_cast<int>(n) : T, global ? static_cast<int>(n) : T, H, n, n};
         rc = to_status(vggt::launch_attention_f32(p, st->status, st->wait_limit, stream));
     }
@@ -533,13 +537,13 @@ int attn_f32_call(bool global, const float* q, const float* k, const float* v, c
 extern "C" {
 
 int vggt_attn_frame_f32(const float* q, const float* k, const float* v, const float* pos, float* out, int S, int T,
-                        int H, int D, const vggt_qk_norm* norm, cudaStream_t stream) {
-    return attn_f32_call(false, q, k, v, pos, out, S, T, H, D, norm, stream);
+                        int H, int D, const vggt_qk_norm* norm, int terms, cudaStream_t stream) {
+    return attn_f32_call(false, q, k, v, pos, out, S, T, H, D, norm, terms, stream);
 }
 
 int vggt_attn_global_f32(const float* q, const float* k, const float* v, const float* pos, float* out, int S, int T,
-                         int H, int D, const vggt_qk_norm* norm, cudaStream_t stream) {
-    return attn_f32_call(true, q, k, v, pos, out, S, T, H, D, norm, stream);
+                         int H, int D, const vggt_qk_norm* norm, int terms, cudaStream_t stream) {
+    return attn_f32_call(true, q, k, v, pos, out, S, T, H, D, norm, terms, stream);
 }
 
 int vggt_kv_pool_tokens(int T, int kv_down) { return vggt_kv_pool_tokens_ex(T, kv_down, nullptr); }

@@ -7,25 +7,29 @@
 //  precision study: its attention runs in FP32 -- TF32x3 Triton kernels -- for
 //  parity with the FP32 reference.)
 //
-// Every fp32 operand x is carried as two bf16 terms, x_hi = bf16(x) and
-// x_lo = bf16(x - x_hi), which represent x to about 2^-17 relative. A product
-// a b is then a_hi b_hi + a_hi b_lo + a_lo b_hi (the dropped a_lo b_lo is about
-// 2^-18 a b), each term a bf16 MMA with fp32 accumulation:
-//   S    = Q_hi K_hi^T + Q_hi K_lo^T + Q_lo K_hi^T          (3 x 4 K-steps, N = 96)
-//   [O|l] += P_hi [V_hi|1] + P_lo [V_hi|1] + P_hi [V_lo]    (3 x 6 K-steps, N = 80/80/64)
-// The row sum l comes from the ones column of the first two products (l =
-// sum of P_hi + P_lo, the P that multiplies V). The exponentials must be good
-// to ~2^-22: 6 of every 8 score pairs go to MUFU ex2 (that accuracy), 2 to a
-// degree-5 minimax polynomial on the FMA pipe (worst relative error 2.3e-7,
-// fit_exp2_poly.py), so the two units share the work (measured: +3% over
-// MUFU only at 36 909 tokens; 3/8 and 4/8 are no better).
+// Every fp32 operand x is carried as kTerms bf16 terms x_0 = bf16(x),
+// x_1 = bf16(x - x_0) (and x_2 = bf16(x - x_0 - x_1)). A product a b is the
+// sum of the term products a_i b_j with i + j < kTerms -- each a bf16 MMA with
+// fp32 accumulation; the dropped ones are ~2^-18 (two terms) or ~2^-27 (three
+// terms) of a b:
+//   two terms:   3 products (0,0) (0,1) (1,0)                    ~2^-17
+//   three terms: 6 products (0,0) (0,1) (1,0) (0,2) (1,1) (2,0)   ~fp32
+//   S     = sum Q_i K_j^T                  (4 K-steps each, N = 96)
+//   [O|l] += sum P_i [V_j | 1 if j == 0]   (6 K-steps each, N = 80 or 64)
+// The row sum l comes from the ones column of the products with V_0 (their P
+// terms are all of P's terms, so l = sum of P, the P that multiplies V). The
+// exponentials must be good to ~2^-22: 6 of every 8 score pairs go to MUFU
+// ex2 (that accuracy), 2 to a degree-5 minimax polynomial on the FMA pipe
+// (worst relative error 2.3e-7, fit_exp2_poly.py), so the two units share
+// the work (measured: +3% over MUFU only at 36 909 tokens; 3/8 and 4/8 are no
+// better).
 //
-// One CTA per 128-row query tile of one head. Warps: 0 TMA producer (K_hi,
-// K_lo, V_hi, V_lo of 96 keys into a 4-slot ring), 1 MMA issuer, 2-3 idle,
-// 4-11 softmax (2 per TMEM lane quarter, 48 score columns each). Tensor
-// memory: Q_hi [0, 32), Q_lo [32, 64), S [64, 160), P_hi [160, 208),
-// P_lo [208, 256), [O | l] [256, 336). The softmax warps and the issuer meet
-// once per key block exactly as in the bf16 kernel (attn_fwd.cu): right after
+// One CTA per 128-row query tile of one head. Warps: 0 TMA producer (the K
+// and V terms of 96 keys into a ring of 4 slots for two terms, 2 for three),
+// 1 MMA issuer, 2-3 idle, 4-11 softmax (2 per TMEM lane quarter, 48 score
+// columns each). Tensor memory: the Q terms (32 columns each), S (96), the P
+// terms (48 each), [O | l] (80). The softmax warps and the issuer meet once
+// per key block exactly as in the bf16 kernel (attn_fwd.cu): right after
 // loading S_j the softmax warps arrive on bar_c (P_{j-1} written, S free; the
 // first warp has checked that K_{j+1} landed), and on that signal the issuer
 // issues PV_{j-1} and S_{j+1}. No row maximum either: the prologue bounds
@@ -47,17 +51,52 @@ using attn::Waiter;
 
 constexpr int kBM = 128;                          // query rows per CTA
 constexpr int kBN = 96;                           // keys per block
-constexpr int kStages = 4;                        // K/V ring depth
 constexpr int kTileBytes = kBN * kHeadDim * 2;    // one 96 x 64 bf16 tile, 12 KB
 constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum block
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 128 + 32 * kSoftmaxWarps;  // 384
 constexpr int kCols = 48;                           // score columns per softmax thread
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQHi = 0, kColQLo = 32, kColS = 64, kColPHi = 160, kColPLo = 208, kColO = 256;
-static_assert(kColO + kOCols <= kTmemCols, "tensor memory columns");
+
+// Per term count: the K and V ring depths (separate rings, each with its own
+// producer warp, so that a slot of either frees on its own MMA) and the tensor
+// memory columns. Two terms: 4 + 4 slots of 2 tiles; three terms: 3 + 2 slots
+// of 3 tiles (a third V slot does not fit beside them in 227 KB).
+template <int kTerms>
+struct Cfg {
+    static_assert(kTerms == 2 || kTerms == 3, "two or three bf16 terms");
+    static constexpr int kStagesK = kTerms == 2 ? 4 : 3;
+    static constexpr int kStagesV = kTerms == 2 ? 4 : 2;
+    static constexpr int kPairs = kTerms * (kTerms + 1) / 2;  // term products kept
+    static constexpr uint32_t kColQ = 0;                      // 32 per term
+    static constexpr uint32_t kColS = 32 * kTerms;
+    static constexpr uint32_t kColP = kColS + kBN;            // 48 per term
+    static constexpr uint32_t kColO = kColP + (kBN / 2) * kTerms;
+    static constexpr uint32_t kColA = kColO + kOCols;         // the folded partial sums
+    static_assert(kColA + kOCols <= kTmemCols, "tensor memory columns");
+};
+
+// The kept term products in order of size: (0,0), then (0,1) (1,0), then
+// (0,2) (1,1) (2,0). Product i multiplies term pair_a(i) of the left operand
+// with term pair_b(i) of the right one.
+__host__ __device__ constexpr int pair_level(int i) { return i == 0 ? 0 : (i < 3 ? 1 : 2); }
+__host__ __device__ constexpr int pair_a(int i) { return i - pair_level(i) * (pair_level(i) + 1) / 2; }
+__host__ __device__ constexpr int pair_b(int i) { return pair_level(i) - pair_a(i); }
+static_assert(pair_a(2) == 1 && pair_b(2) == 0 && pair_a(3) == 0 && pair_b(3) == 2 && pair_a(5) == 2 &&
+                  pair_b(5) == 0,
+              "term pairs");
 
 constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64)
+
+// [O | l] accumulates in tensor memory over kFold key blocks at a time; the
+// softmax warps then fold that partial into a second tensor-memory sum with
+// round-to-nearest fp32 adds, and the next block's products start afresh.
+// Accumulating all 385 blocks of a 36 909-key row in place lost ~1e-4
+// relative (measured: the tensor core's accumulator adds do not round to
+// nearest, and their error grows with the number of updates, so three terms
+// came out worse than two); folding every 8 blocks caps each run of in-place
+// updates.
+constexpr int kFold = 8;
 
 // 2^f ~ sum c_i f^i on [-1/2, 1/2], degree 5 (Remez, fit_exp2_poly.py);
 // evaluated after the Cody-Waite split x = j + f (j = round(x) by adding
@@ -90,12 +129,38 @@ __device__ __forceinline__ void exp2_pair_fma(float a, float b, float& pa, float
     pb = __uint_as_float(q1 + (t1 << 23));
 }
 
+// 8 consecutive columns at each of two addresses, waited for.
+__device__ __forceinline__ void tmem_ld8x2(uint32_t taddr0, uint32_t taddr1, uint32_t (&r0)[8], uint32_t (&r1)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%16];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%17];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]), "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]),
+          "=r"(r1[0]), "=r"(r1[1]), "=r"(r1[2]), "=r"(r1[3]), "=r"(r1[4]), "=r"(r1[5]), "=r"(r1[6]), "=r"(r1[7])
+        : "r"(taddr0), "r"(taddr1)
+        : "memory");
+}
+// 8 consecutive columns, waited for.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+        "tcgen05.wait::st.sync.aligned;"
+        :
+        : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+template <int kTerms>
 struct SharedStorage {
-    uint8_t kv[kStages][4][kTileBytes];  // [slot][K_hi, K_lo, V_hi, V_lo], 128B-swizzled
-    uint8_t ones[kTileBytes];            // [1, 0, ..., 0] per key row, 128B-swizzled
-    uint64_t bar_kvfull[kStages];
-    uint64_t bar_kvempty[kStages];
-    uint64_t bar_q;      // Q_hi / Q_lo in tensor memory
+    using C = Cfg<kTerms>;
+    uint8_t k[C::kStagesK][kTerms][kTileBytes];  // K terms, 128B-swizzled
+    uint8_t v[C::kStagesV][kTerms][kTileBytes];  // V terms, 128B-swizzled
+    uint8_t ones[kTileBytes];                    // [1, 0, ..., 0] per key row, 128B-swizzled
+    uint64_t bar_kfull[C::kStagesK];
+    uint64_t bar_kempty[C::kStagesK];
+    uint64_t bar_vfull[C::kStagesV];
+    uint64_t bar_vempty[C::kStagesV];
+    uint64_t bar_q;      // the Q terms in tensor memory
     uint64_t bar_s;      // S_j computed
     uint64_t bar_c;      // P_{j-1} written and S_j read
     uint64_t bar_pfree;  // PV_j finished
@@ -103,8 +168,19 @@ struct SharedStorage {
     uint32_t tmem_base;
     int abort;
 };
-constexpr size_t kSmemBytes = sizeof(SharedStorage) + 1024;  // + alignment slack
-static_assert(kSmemBytes <= 227 * 1024, "shared memory beyond the per-CTA limit");
+template <int kTerms>
+constexpr size_t smem_bytes() {
+    return sizeof(SharedStorage<kTerms>) + 1024;  // + alignment slack
+}
+static_assert(smem_bytes<2>() <= 227 * 1024 && smem_bytes<3>() <= 227 * 1024,
+              "shared memory beyond the per-CTA limit");
+
+// The TMA maps of the K terms (head-major planes) and the V terms
+// (token-major), unused entries zero.
+struct Maps {
+    CUtensorMap k[3];
+    CUtensorMap v[3];
+};
 
 struct Params {
     const float* q_hat;  // fp32, head planes q_stride rows apart
@@ -116,20 +192,28 @@ struct Params {
     int tiles_per_seg;
 };
 
-// hi/lo bf16 terms of two fp32 values, packed low half first.
-__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const float ah = __bfloat162float(__float2bfloat16_rn(a));
-    const float bh = __bfloat162float(__float2bfloat16_rn(b));
-    hi = pack_bf16x2(ah, bh);
-    lo = pack_bf16x2(a - ah, b - bh);
+// The kTerms bf16 terms of two fp32 values, each packed low half first: one
+// paired round-to-nearest conversion per term, the rounded values read back
+// from the packed word by bit operations, the remainders exact in fp32.
+template <int kTerms>
+__device__ __forceinline__ void split_terms(float a, float b, uint32_t (&w)[kTerms]) {
+#pragma unroll
+    for (int i = 0; i < kTerms; ++i) {
+        w[i] = pack_bf16x2(a, b);
+        if (i + 1 < kTerms) {
+            a -= __uint_as_float(w[i] << 16);
+            b -= __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
 }
 
+template <int kTerms>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_klo,
-                    const __grid_constant__ CUtensorMap tm_vhi, const __grid_constant__ CUtensorMap tm_vlo,
-                    const Params prm) {
+attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
+    using C = Cfg<kTerms>;
+    constexpr int kSK = C::kStagesK, kSV = C::kStagesV;
     extern __shared__ uint8_t smem_raw[];
-    SharedStorage& sm = *reinterpret_cast<SharedStorage*>(
+    SharedStorage<kTerms>& sm = *reinterpret_cast<SharedStorage<kTerms>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
     const int warp = __shfl_sync(0xFFFFFFFFu, static_cast<int>(threadIdx.x >> 5), 0);
@@ -141,27 +225,36 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
     const int nkb = (prm.k_len + kBN - 1) / kBN;
     const int last_valid = prm.k_len - (nkb - 1) * kBN;
 
-    const uint32_t bar_kvfull0 = smem_u32(&sm.bar_kvfull[0]);
-    const uint32_t bar_kvempty0 = smem_u32(&sm.bar_kvempty[0]);
+    const uint32_t bar_kfull0 = smem_u32(&sm.bar_kfull[0]);
+    const uint32_t bar_kempty0 = smem_u32(&sm.bar_kempty[0]);
+    const uint32_t bar_vfull0 = smem_u32(&sm.bar_vfull[0]);
+    const uint32_t bar_vempty0 = smem_u32(&sm.bar_vempty[0]);
     const uint32_t bar_q = smem_u32(&sm.bar_q);
     const uint32_t bar_s = smem_u32(&sm.bar_s);
     const uint32_t bar_c = smem_u32(&sm.bar_c);
     const uint32_t bar_pfree = smem_u32(&sm.bar_pfree);
     const uint32_t bar_o = smem_u32(&sm.bar_o);
-    const uint32_t kv_smem0 = smem_u32(sm.kv[0][0]);
+    const uint32_t k_smem0 = smem_u32(sm.k[0][0]);
+    const uint32_t v_smem0 = smem_u32(sm.v[0][0]);
     const uint32_t ones_smem = smem_u32(sm.ones);
-    auto bar_kvfull = [&](int s) { return bar_kvfull0 + 8u * s; };
-    auto bar_kvempty = [&](int s) { return bar_kvempty0 + 8u * s; };
-    // tile i (0 K_hi, 1 K_lo, 2 V_hi, 3 V_lo) of slot s
-    auto tile_smem = [&](int s, int i) { return kv_smem0 + static_cast<uint32_t>(kTileBytes) * (4 * s + i); };
+    auto bar_kfull = [&](int s) { return bar_kfull0 + 8u * s; };
+    auto bar_kempty = [&](int s) { return bar_kempty0 + 8u * s; };
+    auto bar_vfull = [&](int s) { return bar_vfull0 + 8u * s; };
+    auto bar_vempty = [&](int s) { return bar_vempty0 + 8u * s; };
+    auto k_tile = [&](int s, int t) { return k_smem0 + static_cast<uint32_t>(kTileBytes) * (kTerms * s + t); };
+    auto v_tile = [&](int s, int t) { return v_smem0 + static_cast<uint32_t>(kTileBytes) * (kTerms * s + t); };
 
     attn::fill_ones_tile(sm.ones, kTileBytes, kThreads);
     fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_kvfull(s), 1);
-            mbar_init(bar_kvempty(s), 1);
+        for (int s = 0; s < kSK; ++s) {
+            mbar_init(bar_kfull(s), 1);
+            mbar_init(bar_kempty(s), 1);
+        }
+        for (int s = 0; s < kSV; ++s) {
+            mbar_init(bar_vfull(s), 1);
+            mbar_init(bar_vempty(s), 1);
         }
         mbar_init(bar_q, kSoftmaxWarps);
         mbar_init(bar_s, 1);
@@ -172,11 +265,9 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_khi);
-        tma_prefetch_desc(&tm_klo);
-        tma_prefetch_desc(&tm_vhi);
-        tma_prefetch_desc(&tm_vlo);
+    if ((warp == 0 || warp == 2) && lane == 0) {
+#pragma unroll
+        for (int t = 0; t < kTerms; ++t) tma_prefetch_desc(warp == 0 ? &maps.k[t] : &maps.v[t]);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
@@ -188,24 +279,30 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, sm.tmem_base, 0);
     const Waiter wait{prm.wait_limit, &sm.abort, prm.status};
 
-    if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------ TMA producers: 0 K, 2 V
         if (lane == 0) {
+            const bool is_k = warp == 0;
+            const int n_st = is_k ? kSK : kSV;
             int n_issued = 0;
             for (int j = 0; j < nkb; ++j) {
-                const int s = j % kStages;
-                const uint32_t use = j / kStages;
-                if (use > 0 && !wait(bar_kvempty(s), (use - 1) & 1)) break;
-                mbar_arrive_expect_tx(bar_kvfull(s), 4 * kTileBytes);
+                const int s = j % n_st;
+                const uint32_t use = j / n_st;
+                const uint32_t full = is_k ? bar_kfull(s) : bar_vfull(s);
+                if (use > 0 && !wait(is_k ? bar_kempty(s) : bar_vempty(s), (use - 1) & 1)) break;
+                mbar_arrive_expect_tx(full, kTerms * kTileBytes);
                 const int row = k_row0 + j * kBN;
-                tma_load_3d(tile_smem(s, 0), &tm_khi, bar_kvfull(s), 0, row, h);
-                tma_load_3d(tile_smem(s, 1), &tm_klo, bar_kvfull(s), 0, row, h);
-                tma_load_3d(tile_smem(s, 2), &tm_vhi, bar_kvfull(s), 0, h, row);
-                tma_load_3d(tile_smem(s, 3), &tm_vlo, bar_kvfull(s), 0, h, row);
+#pragma unroll
+                for (int t = 0; t < kTerms; ++t) {
+                    if (is_k)
+                        tma_load_3d(k_tile(s, t), &maps.k[t], full, 0, row, h);
+                    else
+                        tma_load_3d(v_tile(s, t), &maps.v[t], full, 0, h, row);
+                }
                 ++n_issued;
             }
-            for (int j = max(0, n_issued - kStages); j < n_issued; ++j)
-                drain_wait(bar_kvfull(j % kStages), (j / kStages) & 1, prm.wait_limit);
+            for (int j = max(0, n_issued - n_st); j < n_issued; ++j)
+                drain_wait(is_k ? bar_kfull(j % n_st) : bar_vfull(j % n_st), (j / n_st) & 1, prm.wait_limit);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
@@ -215,61 +312,58 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
         auto uwait = [&](uint32_t bar, uint32_t parity) {
             return __all_sync(0xFFFFFFFFu, wait(bar, parity)) != 0;
         };
-        const uint32_t s_tm = tmem + kColS, o_tm = tmem + kColO;
-        const uint32_t qh_tm = tmem + kColQHi, ql_tm = tmem + kColQLo;
-        const uint32_t ph_tm = tmem + kColPHi, pl_tm = tmem + kColPLo;
-        // S_j: 3 products x 4 steps of 16 head dims (8 TMEM columns of Q, 32
-        // bytes of each 128-byte K row)
+        const uint32_t s_tm = tmem + C::kColS, o_tm = tmem + C::kColO;
+        const uint32_t q_tm = tmem + C::kColQ, p_tm = tmem + C::kColP;
+        // S_j: the kept products Q_a K_b^T, 4 steps of 16 head dims each (8
+        // TMEM columns of Q, 32 bytes of each 128-byte K row)
         auto issue_s = [&](int j) {
-            const int s = j % kStages;
-            const uint64_t kh = smem_desc_sw128(tile_smem(s, 0), 16, 1024);
-            const uint64_t kl = smem_desc_sw128(tile_smem(s, 1), 16, 1024);
+            const int s = j % kSK;
             if (elect_one()) {
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(s_tm, qh_tm + 8 * kk, kh + static_cast<uint64_t>((kk * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
+                for (int i = 0; i < C::kPairs; ++i) {
+                    const uint64_t kd = smem_desc_sw128(k_tile(s, pair_b(i)), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(s_tm, qh_tm + 8 * kk, kl + static_cast<uint64_t>((kk * 32) >> 4), idesc_s, 1u);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(s_tm, ql_tm + 8 * kk, kh + static_cast<uint64_t>((kk * 32) >> 4), idesc_s, 1u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(s_tm, q_tm + 32 * pair_a(i) + 8 * kk, kd + static_cast<uint64_t>((kk * 32) >> 4),
+                               idesc_s, (i > 0 || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(bar_s);
+                mma_commit(bar_kempty(s));
             }
             __syncwarp();
         };
-        // PV_j: 3 products x 6 steps of 16 keys; the first two carry the ones
-        // column (the B operand's second 64-column block, a leading byte
-        // offset away from the V_hi tile)
+        // PV_j: the kept products P_a [V_b | 1], 6 steps of 16 keys each; the
+        // products with V_0 carry the ones column (the B operand's second
+        // 64-column block, a leading byte offset away from the V_0 tile), so
+        // the row sum collects every term of P
         auto issue_pv = [&](int j) {
-            const int s = j % kStages;
-            const uint32_t vh_addr = tile_smem(s, 2);
-            const uint64_t vh = smem_desc_sw128(vh_addr, ones_smem - vh_addr, 1024);
-            const uint64_t vl = smem_desc_sw128(tile_smem(s, 3), 16, 1024);
+            const int s = j % kSV;
+            const uint32_t v0_addr = v_tile(s, 0);
             if (elect_one()) {
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 6; ++kk)
-                    mma_ts(o_tm, ph_tm + 8 * kk, vh + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_o,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                for (int i = 0; i < C::kPairs; ++i) {
+                    const int b = pair_b(i);
+                    const uint64_t vd = b == 0 ? smem_desc_sw128(v0_addr, ones_smem - v0_addr, 1024)
+                                               : smem_desc_sw128(v_tile(s, b), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < 6; ++kk)
-                    mma_ts(o_tm, pl_tm + 8 * kk, vh + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_o, 1u);
-#pragma unroll
-                for (int kk = 0; kk < 6; ++kk)
-                    mma_ts(o_tm, ph_tm + 8 * kk, vl + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_o64, 1u);
+                    for (int kk = 0; kk < 6; ++kk)
+                        mma_ts(o_tm, p_tm + 48 * pair_a(i) + 8 * kk, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4),
+                               b == 0 ? idesc_o : idesc_o64, (j % kFold != 0 || i > 0 || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(bar_pfree);
-                mma_commit(bar_kvempty(s));
+                mma_commit(bar_vempty(s));
             }
             __syncwarp();
         };
-        bool ok = uwait(bar_q, 0) && uwait(bar_kvfull(0), 0);
+        bool ok = uwait(bar_q, 0) && uwait(bar_kfull(0), 0);
         if (ok) issue_s(0);
         ok = ok && uwait(bar_c, 0);  // S_0 read (and K_1 landed)
         if (ok && nkb > 1) issue_s(1);
         for (int j = 0; ok && j < nkb; ++j) {
             if (!uwait(bar_c, (j + 1) & 1)) break;  // P_j written, S_{j+1} read, K_{j+2} landed
+            if (!uwait(bar_vfull(j % kSV), (j / kSV) & 1)) break;
             issue_pv(j);
             if (j + 2 < nkb) issue_s(j + 2);
         }
@@ -289,24 +383,32 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
         const bool row_live = row_in_seg < prm.q_len;
         const long long grow = static_cast<long long>(seg) * prm.q_len + row_in_seg;
         // Q into tensor memory: this thread's 32 dims of its row, scaled by
-        // log2(e)/8 in fp32, as hi and lo bf16 terms (16 columns each).
+        // log2(e)/8 in fp32, as kTerms bf16 terms (16 columns each).
         {
-            uint32_t qh[16], ql[16];
+            uint32_t qt[kTerms][16];
             if (row_live) {
                 const float4* src = reinterpret_cast<const float4*>(
                     prm.q_hat + (static_cast<long long>(h) * prm.q_stride + grow) * kHeadDim + 32 * half);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 w = __ldg(src + i);
-                    split_pair(w.x * kScaleLog2, w.y * kScaleLog2, qh[2 * i], ql[2 * i]);
-                    split_pair(w.z * kScaleLog2, w.w * kScaleLog2, qh[2 * i + 1], ql[2 * i + 1]);
+                    uint32_t a[kTerms], b[kTerms];
+                    split_terms<kTerms>(w.x * kScaleLog2, w.y * kScaleLog2, a);
+                    split_terms<kTerms>(w.z * kScaleLog2, w.w * kScaleLog2, b);
+#pragma unroll
+                    for (int t = 0; t < kTerms; ++t) {
+                        qt[t][2 * i] = a[t];
+                        qt[t][2 * i + 1] = b[t];
+                    }
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) qh[i] = ql[i] = 0u;
+                for (int t = 0; t < kTerms; ++t)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) qt[t][i] = 0u;
             }
-            tmem_st16(lane_base + kColQHi + 16 * half, qh);
-            tmem_st16(lane_base + kColQLo + 16 * half, ql);
+#pragma unroll
+            for (int t = 0; t < kTerms; ++t) tmem_st16(lane_base + C::kColQ + 32 * t + 16 * half, qt[t]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_q);
@@ -321,12 +423,12 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
             float s[kCols];
             {
                 uint32_t r[kCols];
-                tmem_ld48(lane_base + kColS + kCols * half, r);
+                tmem_ld48(lane_base + C::kColS + kCols * half, r);
 #pragma unroll
                 for (int i = 0; i < kCols; ++i) s[i] = __uint_as_float(r[i]);
             }
             if (quarter == 0 && half == 0 && j + 1 < nkb &&
-                !uwait(bar_kvfull((j + 1) % kStages), ((j + 1) / kStages) & 1)) {
+                !uwait(bar_kfull((j + 1) % kSK), ((j + 1) / kSK) & 1)) {
                 ok = false;
                 break;
             }
@@ -339,11 +441,16 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
                 for (int c = 0; c < kCols; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
-            uint32_t ph[kCols / 2], pl[kCols / 2];
+            uint32_t pt[kTerms][kCols / 2];
+            auto put = [&](int c, float pa, float pb) {
+                uint32_t w[kTerms];
+                split_terms<kTerms>(pa, pb, w);
+#pragma unroll
+                for (int t = 0; t < kTerms; ++t) pt[t][c] = w[t];
+            };
             if (j == nkb - 1) {  // masked columns are -inf: MUFU only (2^-inf = 0)
 #pragma unroll
-                for (int c = 0; c < kCols / 2; ++c)
-                    split_pair(ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]), ph[c], pl[c]);
+                for (int c = 0; c < kCols / 2; ++c) put(c, ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]));
             } else {
 #pragma unroll
                 for (int c = 0; c < kCols / 2; ++c) {
@@ -354,7 +461,7 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
                         pa = ex2_approx(s[2 * c]);
                         pb = ex2_approx(s[2 * c + 1]);
                     }
-                    split_pair(pa, pb, ph[c], pl[c]);
+                    put(c, pa, pb);
                 }
             }
             if (j > 0 && !uwait(bar_pfree, (j - 1) & 1)) {
@@ -362,8 +469,26 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
                 break;
             }
             tc_fence_after();
-            tmem_st24(lane_base + kColPHi + (kCols / 2) * half, ph);
-            tmem_st24(lane_base + kColPLo + (kCols / 2) * half, pl);
+            if (j > 0 && j % kFold == 0) {
+                // PV_{j-1} closed a run of kFold blocks: fold [O | l] into the
+                // sum (the first fold copies); PV_j then starts afresh. The l
+                // column (64) is the same for both halves: half 0 folds it.
+                const bool first = j == kFold;
+#pragma unroll
+                for (int piece = 0; piece < 5; ++piece) {
+                    if (piece == 4 && half != 0) break;
+                    const uint32_t col = piece < 4 ? 32 * half + 8 * piece : kHeadDim;
+                    uint32_t ov[8], av[8];
+                    tmem_ld8x2(lane_base + C::kColO + col, lane_base + C::kColA + col, ov, av);
+                    if (!first) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) + __uint_as_float(av[i]));
+                    }
+                    tmem_st8(lane_base + C::kColA + col, ov);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < kTerms; ++t) tmem_st24(lane_base + C::kColP + 48 * t + (kCols / 2) * half, pt[t]);
         }
         if (ok) {
             tc_fence_before();
@@ -373,7 +498,13 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
         if (ok && uwait(bar_o, 0)) {
             tc_fence_after();
             uint32_t o[33];  // this thread's 32 output dims and l (column 64)
-            tmem_ld32_1(lane_base + kColO + 32 * half, lane_base + kColO + kHeadDim, o);
+            tmem_ld32_1(lane_base + C::kColO + 32 * half, lane_base + C::kColO + kHeadDim, o);
+            if (nkb > kFold) {  // plus the folded sum
+                uint32_t a[33];
+                tmem_ld32_1(lane_base + C::kColA + 32 * half, lane_base + C::kColA + kHeadDim, a);
+#pragma unroll
+                for (int i = 0; i < 33; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) + __uint_as_float(a[i]));
+            }
             const float l = __uint_as_float(o[32]);
             if (row_live) {
                 if (!(l > 0.0f && l <= 3.0e38f)) atomicOr(prm.status, kStatusRange);
@@ -396,30 +527,37 @@ attn_fwd_f32_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_con
 
 // ---------------------------------------------------------------- host
 
-}  // namespace
-
-cudaError_t launch_attention_f32(const AttnProblemF32& p, int* status, long long wait_limit, cudaStream_t stream) {
-    if (p.n_seg <= 0 || p.H <= 0 || p.q_len <= 0 || p.k_len <= 0) return cudaSuccess;
+template <int kTerms>
+cudaError_t launch_terms(const AttnProblemF32& p, const Params& prm, cudaStream_t stream) {
     const uint64_t nk = static_cast<uint64_t>(p.n_seg) * p.k_len;
     const uint64_t row_bytes = kHeadDim * 2;
     const uint64_t ks = static_cast<uint64_t>(p.k_stride);
-    CUtensorMap tm_khi, tm_klo, tm_vhi, tm_vlo;
-    if (!make_map(&tm_khi, p.k_hi, ks, p.H, row_bytes, ks * row_bytes, kBN, 1) ||
-        !make_map(&tm_klo, p.k_lo, ks, p.H, row_bytes, ks * row_bytes, kBN, 1) ||
-        !make_map(&tm_vhi, p.v_hi, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN) ||
-        !make_map(&tm_vlo, p.v_lo, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
-        return cudaErrorInvalidValue;
+    Maps maps{};
+    for (int t = 0; t < kTerms; ++t)
+        if (!make_map(&maps.k[t], p.k[t], ks, p.H, row_bytes, ks * row_bytes, kBN, 1) ||
+            !make_map(&maps.v[t], p.v[t], p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
+            return cudaErrorInvalidValue;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_set[dev]) {
-        e = cudaFuncSetAttribute(attn_fwd_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kSmemBytes));
+        e = cudaFuncSetAttribute(attn_fwd_f32_kernel<kTerms>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_bytes<kTerms>()));
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    dim3 grid(p.n_seg * prm.tiles_per_seg, p.H);
+    attn_fwd_f32_kernel<kTerms><<<grid, kThreads, smem_bytes<kTerms>(), stream>>>(maps, prm);
+    return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention_f32(const AttnProblemF32& p, int* status, long long wait_limit, cudaStream_t stream) {
+    if (p.terms != 2 && p.terms != 3) return cudaErrorInvalidValue;
+    if (p.n_seg <= 0 || p.H <= 0 || p.q_len <= 0 || p.k_len <= 0) return cudaSuccess;
     Params prm;
     prm.q_hat = p.q_hat;
     prm.out = p.out;
@@ -430,9 +568,7 @@ cudaError_t launch_attention_f32(const AttnProblemF32& p, int* status, long long
     prm.k_len = p.k_len;
     prm.H = p.H;
     prm.tiles_per_seg = (p.q_len + kBM - 1) / kBM;
-    dim3 grid(p.n_seg * prm.tiles_per_seg, p.H);
-    attn_fwd_f32_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_khi, tm_klo, tm_vhi, tm_vlo, prm);
-    return cudaPeekAtLastError();
+    return p.terms == 3 ? launch_terms<3>(p, prm, stream) : launch_terms<2>(p, prm, stream);
 }
 
 }  // namespace vggt

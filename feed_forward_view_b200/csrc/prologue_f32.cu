@@ -1,14 +1,17 @@
 // prologue_f32.cu -- the QK prologue and the operand split of the fp32 mode.
 //
 // The fp32 mode takes fp32 q, k, v and evaluates both attention products on
-// the bf16 tensor cores with every fp32 operand x carried as two bf16 terms,
-// x_hi = bf16(x) and x_lo = bf16(x - x_hi) (x - x_hi is exact in fp32), which
-// represent x to about 2^-17 relative. This file writes those operands:
+// the bf16 tensor cores with every fp32 operand x carried as bf16 terms:
+// x_0 = bf16(x), x_1 = bf16(x - x_0), and with three terms x_2 = bf16(x - x_0
+// - x_1) (each difference is exact in fp32). Two terms represent x to about
+// 2^-17 relative; three carry all 24 significant bits of an fp32 value
+// (8 + 8 + 8). This file writes those operands:
 //   q_hat: LayerNorm (+ affine) + 2D RoPE of q in fp32, stored fp32
 //          head-major [H, n, 64] (the attention kernel scales and splits it
 //          when it copies it into tensor memory);
-//   k_hat: the same prologue, stored split: k_hi and k_lo bf16 head-major;
-//   v:     split: v_hi and v_lo bf16 token-major [n, H, 64].
+//   k_hat: the same prologue, stored as its bf16 terms, one head-major plane
+//          per term;
+//   v:     its bf16 terms, one token-major [n, H, 64] array per term.
 // The prologue arithmetic (prologue.cuh) is the bf16 path's, fed with fp32
 // inputs. (LayerNorm: "Norm: Layer Normalization" slide; RoPE base 100 and
 // eps 1e-5: the VGGT-Omega config.json table; frequency schedule:
@@ -23,11 +26,34 @@ namespace {
 
 constexpr int kWarpsPerBlock = 8;
 
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const float ah = __bfloat162float(__float2bfloat16_rn(a));
-    const float bh = __bfloat162float(__float2bfloat16_rn(b));
-    hi = prologue::pack2(ah, bh);
-    lo = prologue::pack2(a - ah, b - bh);
+// The bf16 terms of two fp32 values (low half first), kTerms of them: each
+// term rounds to nearest, the remainders are exact in fp32.
+template <int kTerms>
+__device__ __forceinline__ void split_terms(float a, float b, uint32_t (&w)[kTerms]) {
+#pragma unroll
+    for (int i = 0; i < kTerms; ++i) {
+        w[i] = prologue::pack2(a, b);
+        if (i + 1 < kTerms) {
+            a -= __uint_as_float(w[i] << 16);
+            b -= __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+}
+
+template <int kTerms>
+__device__ __forceinline__ void store_terms(const PrologueJobF32& job, size_t row, int d1, const float (&o1)[4],
+                                            const float (&o2)[4]) {
+    uint32_t w[4][kTerms];
+    split_terms<kTerms>(o1[0], o1[1], w[0]);
+    split_terms<kTerms>(o1[2], o1[3], w[1]);
+    split_terms<kTerms>(o2[0], o2[1], w[2]);
+    split_terms<kTerms>(o2[2], o2[3], w[3]);
+#pragma unroll
+    for (int i = 0; i < kTerms; ++i) {
+        uint16_t* plane = static_cast<uint16_t*>(job.out[i]) + row;
+        *reinterpret_cast<uint2*>(plane + d1) = make_uint2(w[0][i], w[1][i]);
+        *reinterpret_cast<uint2*>(plane + d1 + 16) = make_uint2(w[2][i], w[3][i]);
+    }
 }
 
 template <bool kAffine>
@@ -51,20 +77,12 @@ __device__ __forceinline__ void process_token_f32(const PrologueJobF32& job, con
         prologue::norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, o1, o2);
         if (!live) continue;
         const size_t row = (static_cast<size_t>(h) * job.out_stride + t) * kHeadDim;
-        if (job.split) {
-            uint32_t h1[2], l1[2], h2[2], l2[2];
-            split2(o1[0], o1[1], h1[0], l1[0]);
-            split2(o1[2], o1[3], h1[1], l1[1]);
-            split2(o2[0], o2[1], h2[0], l2[0]);
-            split2(o2[2], o2[3], h2[1], l2[1]);
-            uint16_t* hi = static_cast<uint16_t*>(job.out_hi) + row;
-            uint16_t* lo = static_cast<uint16_t*>(job.out_lo) + row;
-            *reinterpret_cast<uint2*>(hi + d1) = make_uint2(h1[0], h1[1]);
-            *reinterpret_cast<uint2*>(hi + d1 + 16) = make_uint2(h2[0], h2[1]);
-            *reinterpret_cast<uint2*>(lo + d1) = make_uint2(l1[0], l1[1]);
-            *reinterpret_cast<uint2*>(lo + d1 + 16) = make_uint2(l2[0], l2[1]);
+        if (job.terms == 2) {
+            store_terms<2>(job, row, d1, o1, o2);
+        } else if (job.terms == 3) {
+            store_terms<3>(job, row, d1, o1, o2);
         } else {
-            float* o = static_cast<float*>(job.out_hi) + row;
+            float* o = static_cast<float*>(job.out[0]) + row;
             *reinterpret_cast<float4*>(o + d1) = make_float4(o1[0], o1[1], o1[2], o1[3]);
             *reinterpret_cast<float4*>(o + d1 + 16) = make_float4(o2[0], o2[1], o2[2], o2[3]);
         }
@@ -92,16 +110,19 @@ qk_prologue_f32_kernel(const __grid_constant__ PrologueJobF32 a, const __grid_co
     }
 }
 
-// hi = bf16(x), lo = bf16(x - hi), 4 values per thread per step.
+// The kTerms bf16 terms of x, 4 values per thread per step.
+template <int kTerms>
 __global__ void __launch_bounds__(256)
-split_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__ hi, uint2* __restrict__ lo, long long n4) {
+split_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__ t0, uint2* __restrict__ t1,
+                  uint2* __restrict__ t2, long long n4) {
     for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n4; i += static_cast<long long>(gridDim.x) * 256) {
         const float4 v = __ldg(x + i);
-        uint2 h, l;
-        split2(v.x, v.y, h.x, l.x);
-        split2(v.z, v.w, h.y, l.y);
-        hi[i] = h;
-        lo[i] = l;
+        uint32_t a[kTerms], b[kTerms];
+        split_terms<kTerms>(v.x, v.y, a);
+        split_terms<kTerms>(v.z, v.w, b);
+        t0[i] = make_uint2(a[0], b[0]);
+        t1[i] = make_uint2(a[1], b[1]);
+        if (kTerms == 3) t2[i] = make_uint2(a[kTerms - 1], b[kTerms - 1]);
     }
 }
 
@@ -125,14 +146,17 @@ cudaError_t launch_qk_prologue_f32(const PrologueJobF32& a, const PrologueJobF32
     return cudaPeekAtLastError();
 }
 
-cudaError_t launch_split_bf16(const float* x, uint16_t* hi, uint16_t* lo, long long n, cudaStream_t stream) {
+cudaError_t launch_split_bf16(const float* x, uint16_t* const (&out)[3], int terms, long long n,
+                              cudaStream_t stream) {
     const long long n4 = n / 4;  // n is a multiple of 64
     if (n4 <= 0) return cudaSuccess;
     long long blocks = (n4 + 255) / 256;
     const long long cap = static_cast<long long>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    split_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<const float4*>(x), reinterpret_cast<uint2*>(hi), reinterpret_cast<uint2*>(lo), n4);
+    auto kernel = terms == 3 ? split_bf16_kernel<3> : split_bf16_kernel<2>;
+    kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(x), reinterpret_cast<uint2*>(out[0]), reinterpret_cast<uint2*>(out[1]),
+        reinterpret_cast<uint2*>(out[2]), n4);
     return cudaPeekAtLastError();
 }
 

@@ -85,33 +85,32 @@ struct FrameLayout {
 
 // fp32 mode. One fp32 tensor x [n, H, 64] (positions pos [n, 2]) through the
 // prologue; out head-major at row t of head h: (h * out_stride + t) * 64.
-// split == 0: fp32 results to out_hi; split == 1: bf16 hi / lo terms to
-// out_hi / out_lo (hi = bf16(y), lo = bf16(y - hi)).
+// terms == 0: fp32 results to out[0]; terms == 2 or 3: that many bf16 terms
+// (y_0 = bf16(y), y_1 = bf16(y - y_0), y_2 = bf16(y - y_0 - y_1)) to out[0..].
 struct PrologueJobF32 {
     const float* x;
     const float* pos;
-    void* out_hi;
-    void* out_lo;
+    void* out[3];
     int n;
     long long out_stride;
     LnAffine ln;
-    int split;
+    int terms;
 };
 cudaError_t launch_qk_prologue_f32(const PrologueJobF32& a, const PrologueJobF32& b, int H,
                                    cudaStream_t stream);
-// hi/lo bf16 terms of n fp32 values (n a multiple of 4), same layout.
-cudaError_t launch_split_bf16(const float* x, uint16_t* hi, uint16_t* lo, long long n, cudaStream_t stream);
+// The bf16 terms (2 or 3) of n fp32 values (n a multiple of 4), same layout.
+cudaError_t launch_split_bf16(const float* x, uint16_t* const (&out)[3], int terms, long long n,
+                              cudaStream_t stream);
 
 // fp32-mode attention: segments as in AttnProblem; q_hat fp32 head-major
-// (plane stride q_stride), k_hi / k_lo bf16 head-major (plane stride
-// k_stride), v_hi / v_lo bf16 [n_seg*k_len, H, 64], out fp32
-// [n_seg*q_len, H, 64].
+// (plane stride q_stride), the bf16 terms of k_hat head-major (plane stride
+// k_stride) and of v [n_seg*k_len, H, 64], out fp32 [n_seg*q_len, H, 64];
+// terms 2 or 3.
 struct AttnProblemF32 {
     const float* q_hat;
-    const uint16_t* k_hi;
-    const uint16_t* k_lo;
-    const uint16_t* v_hi;
-    const uint16_t* v_lo;
+    const uint16_t* k[3];
+    const uint16_t* v[3];
+    int terms;
     float* out;
     int n_seg;
     int q_len;

@@ -51,6 +51,7 @@ class Workload:
     skip: int = 0             # trailing tokens per frame left out ("subset_*")
     n_extra: int = 0          # sequence tokens after the frames ("subset_*")
     B: int = 1                # scenes per call ("global_batch")
+    terms: int = 2            # bf16 terms per fp32 operand ("*_f32")
 
     @property
     def T(self) -> int:
@@ -145,10 +146,11 @@ SUBSET_WORKLOADS = {w.name: w for w in (
     Workload("omega_frame_s32_g32", "subset_frame", S=32, g=32, n_front=0, n_back=16, skip=16, n_extra=5),
 )}
 # The fp32 mode on the dense global workload (9 frames of 1024^2 at patch 16)
-# and on eight 518^2 frames.
+# and on eight 518^2 frames, with two bf16 terms per operand, and with three.
 F32_WORKLOADS = {w.name: w for w in (
     Workload("global_s9_g64_f32", "global_f32", S=9, g=64),
     Workload("frame_s8_g37_f32", "frame_f32", S=8, g=37),
+    Workload("global_s9_g64_f32x3", "global_f32", S=9, g=64, terms=3),
 )}
 # Small scenes batched: 32 scenes of the two-frame 224^2 workload in one call.
 BATCH_WORKLOADS = {w.name: w for w in (

@@ -328,20 +328,28 @@ VGGT_API int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt
 /*
  * The fp32 mode: frame / global attention (as vggt_attn_frame_ex /
  * vggt_attn_global_ex, any T >= 1, optional QK LayerNorm affine) on fp32
- * q, k, v [S*T, H, D] with fp32 out, to about fp32 accuracy -- the precision
- * the vggt-jax README's FP32 parity runs use (its attention: TF32x3 Triton
- * kernels). The prologue runs in fp32; both attention products run on the
- * bf16 tensor cores with every fp32 operand x carried as x_hi = bf16(x) plus
- * x_lo = bf16(x - x_hi): a b = a_hi b_hi + a_hi b_lo + a_lo b_hi (three MMAs,
- * the dropped term is ~2^-18 a b), fp32 accumulation, exponentials to ~2^-22.
+ * q, k, v [S*T, H, D] with fp32 out -- the precision the vggt-jax README's
+ * FP32 parity runs use (its attention: TF32x3 Triton kernels). The prologue
+ * runs in fp32; both attention products run on the bf16 tensor cores with
+ * every fp32 operand x carried as `terms` bf16 terms x_0 = bf16(x),
+ * x_1 = bf16(x - x_0), x_2 = bf16(x - x_0 - x_1); a b is the sum of the term
+ * products a_i b_j with i + j < terms, accumulated in fp32, exponentials to
+ * ~2^-22:
+ *   terms == 2: 3 products, the dropped ones ~2^-18 a b (outputs to ~1e-5 of
+ *               max|v|), about 3x the tensor-core work of the bf16 path;
+ *   terms == 3: 6 products, the dropped ones ~2^-27 a b (outputs to about
+ *               fp32 rounding, ~1e-6 of max|v|), about 6x.
+ * Other values of terms: VGGT_ERR_UNSUPPORTED.
  * Pointers: q, k, v, out 16-byte aligned (fp32 arrays), pos 8-byte aligned.
- * Scratch: 12 bytes per (token, head, dim) -- fp32 q_hat and the bf16 hi/lo
- * terms of k_hat and v. About 3x the tensor-core work of the bf16 path.
+ * Scratch: 4 + 4*terms bytes per (token, head, dim) -- fp32 q_hat and the
+ * bf16 terms of k_hat and v.
  */
 VGGT_API int vggt_attn_frame_f32(const float* q, const float* k, const float* v, const float* pos, float* out,
-                                 int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream);
+                                 int S, int T, int H, int D, const vggt_qk_norm* norm, int terms,
+                                 cudaStream_t stream);
 VGGT_API int vggt_attn_global_f32(const float* q, const float* k, const float* v, const float* pos, float* out,
-                                  int S, int T, int H, int D, const vggt_qk_norm* norm, cudaStream_t stream);
+                                  int S, int T, int H, int D, const vggt_qk_norm* norm, int terms,
+                                  cudaStream_t stream);
 
 /*
  * Several scenes per call (the vggt-jax README feeds [B, S, 3, H, W] image

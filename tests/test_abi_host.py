@@ -244,13 +244,17 @@ def test_subset_argument_checks():
 def test_f32_mode_argument_checks():
     for name in ("vggt_attn_frame_f32", "vggt_attn_global_f32"):
         fn = getattr(F.lib, name)
-        assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 100, 16, 64, None, None) == OK
-        assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 16, 64, None, None) == E_SHAPE
-        assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 32, None, None) == E_UNSUP
-        assert fn(FAKE, None, FAKE, FAKE, FAKE, 2, 10, 16, 64, None, None) == E_NULL
-        assert fn(FAKE, FAKE, FAKE + 8, FAKE, FAKE, 2, 10, 16, 64, None, None) == E_UNSUP
-        norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
-        assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 64, norm, None) == E_UNSUP
+        for terms in (2, 3):
+            assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 100, 16, 64, None, terms, None) == OK
+            assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 16, 64, None, terms, None) == E_SHAPE
+            assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 32, None, terms, None) == E_UNSUP
+            assert fn(FAKE, None, FAKE, FAKE, FAKE, 2, 10, 16, 64, None, terms, None) == E_NULL
+            assert fn(FAKE, FAKE, FAKE + 8, FAKE, FAKE, 2, 10, 16, 64, None, terms, None) == E_UNSUP
+            norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
+            assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 64, norm, terms, None) == E_UNSUP
+        for terms in (0, 1, 4, -1):  # only two or three bf16 terms
+            assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 64, None, terms, None) == E_UNSUP
+            assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 10, 16, 64, None, terms, None) == E_UNSUP
 
 
 def test_batch_argument_checks():
