@@ -130,6 +130,7 @@ PROFILE_WORKLOADS = {w.name: w for w in (
     Workload("global_s6_g64", "global", S=6, g=64),
     Workload("descriptor_s40_g37_kd4", "descriptor", S=40, g=37, kv_down=4),
     Workload("global_s6_g64_f32", "global_f32", S=6, g=64),
+    Workload("global_s6_g64_f32x3", "global_f32", S=6, g=64, terms=3),
 )}
 
 # The descriptor workload streamed in chunks of 10 frames (FlashVGGTStream's
