@@ -32,6 +32,10 @@ METRIC = "global-attention fwd TFLOP/s and tokens/s on 1 B200; % of dense bf16 p
 DEFAULT_WORKLOAD = "global_s9_g64"
 L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures, reported beside the measured ones for context: dense
+# bf16 tensor throughput (the sparse figure halved) and HBM3e bandwidth.
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_kernel_global_s6_g64.txt")
 KERNEL_SOURCES = ("feed_forward_view_b200/csrc/attn_fwd.cu", "feed_forward_view_b200/csrc/attn_common.cuh",
                   "feed_forward_view_b200/csrc/sm100.cuh")
@@ -449,7 +453,8 @@ def run_gpu(args):
         pool_ms = k0.elapsed_time(k1) / reps
         pool_bytes = 2 * (w.n_q + w.n_k) * H * 64 * 2 + (w.n_q + w.n_k) * 8
         pool = {"ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
-                "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"])}
+                "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]),
+                "frac_of_datasheet": pool_bytes / (pool_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS}
         # the pooling fused with the key prologue (what the call runs): the
         # same bytes, with normalised keys written instead of pooled ones
         for _ in range(3):
@@ -462,7 +467,8 @@ def run_gpu(args):
         torch.cuda.synchronize(dev)
         fk_ms = k0.elapsed_time(k1) / reps
         fused_keys = {"ms": fk_ms, "gbs": pool_bytes / (fk_ms * 1e-3) / 1e9,
-                      "frac_hbm": pool_bytes / (fk_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"])}
+                      "frac_hbm": pool_bytes / (fk_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]),
+                      "frac_of_datasheet": pool_bytes / (fk_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS}
 
     # ---- end to end through the public call with host buffers: every step
     # uploads its inputs from pinned host memory and reads its output back.
@@ -578,10 +584,12 @@ def run_gpu(args):
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
                          "peak_source": f"{peak_src} bf16 burst",
                          "frac_of_sustained": attn_tf / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "frac_of_datasheet": attn_tf / DATASHEET_BF16_TFLOPS,
                          "traffic": traffic, "kernel_ms": attn_ms,
                          "share_of_step": attn_ms / ms_step},
             "kernels": {"qk_prologue": {"ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
-                                        "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+                                        "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                                        "frac_of_datasheet": pro_bytes / (pro_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS},
                         **({"kv_pool": pool} if pool else {}),
                         **({"descriptor_keys": fused_keys} if fused_keys else {})},
             # every score costs one exponential: exponentials per second in
