@@ -18,17 +18,17 @@
 //   [O|l] += sum P_i [V_j | 1 if j == 0]   (6 K-steps each, N = 80 or 64)
 // The row sum l comes from the ones column of the products with V_0 (their P
 // terms are all of P's terms, so l = sum of P, the P that multiplies V). The
-// exponentials must be good to ~2^-22: 6 of every 8 score pairs go to MUFU
-// ex2 (that accuracy), 2 to a degree-5 minimax polynomial on the FMA pipe
-// (worst relative error 2.3e-7, fit_exp2_poly.py), so the two units share
-// the work (measured: +3% over MUFU only at 36 909 tokens; 3/8 and 4/8 are no
-// better).
+// exponentials must be good to ~2^-22: every one is MUFU ex2. (Sending 2 of
+// every 8 score pairs to a degree-5 polynomial on the FMA pipe, as the bf16
+// kernel does with degree 3, measured 1.4% slower here: with three or six
+// products per useful one the tensor pipe, not MUFU, is the busiest unit.)
 //
-// One CTA per 128-row query tile of one head. Warps: 0 TMA producer (the K
-// and V terms of 96 keys into a ring of 4 slots for two terms, 2 for three),
-// 1 MMA issuer, 2-3 idle, 4-11 softmax (2 per TMEM lane quarter, 48 score
-// columns each). Tensor memory: the Q terms (32 columns each), S (96), the P
-// terms (48 each), [O | l] (80). The softmax warps and the issuer meet once
+// One CTA per 128-row query tile of one head. Warps: 0 TMA producer for the
+// K terms of 96 keys, 2 for the V terms (separate rings: 4 + 4 slots for two
+// terms, 3 + 2 for three), 1 MMA issuer, 3 idle, 4-11 softmax (2 per TMEM
+// lane quarter, 48 score columns each). Tensor memory: the Q terms (32
+// columns each), S (96), the P terms (48 each), [O | l] (80) and its folded
+// sum (80, see kFold). The softmax warps and the issuer meet once
 // per key block exactly as in the bf16 kernel (attn_fwd.cu): right after
 // loading S_j the softmax warps arrive on bar_c (P_{j-1} written, S free; the
 // first warp has checked that K_{j+1} landed), and on that signal the issuer
@@ -97,37 +97,6 @@ constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64
 // came out worse than two); folding every 8 blocks caps each run of in-place
 // updates.
 constexpr int kFold = 8;
-
-// 2^f ~ sum c_i f^i on [-1/2, 1/2], degree 5 (Remez, fit_exp2_poly.py);
-// evaluated after the Cody-Waite split x = j + f (j = round(x) by adding
-// 1.5 * 2^23), 2^j applied to the exponent field.
-constexpr float kE5C0 = 1.000000119e+00f;
-constexpr float kE5C1 = 6.931469440e-01f;
-constexpr float kE5C2 = 2.402212024e-01f;
-constexpr float kE5C3 = 5.550713092e-02f;
-constexpr float kE5C4 = 9.675540961e-03f;
-constexpr float kE5C5 = 1.327647245e-03f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-constexpr int kFmaPer8 = 2;                 // of every 8 score pairs, on the FMA pipe
-
-// 2^a, 2^b on the FMA pipe (|a|, |b| <= 125), packed f32x2 arithmetic.
-__device__ __forceinline__ void exp2_pair_fma(float a, float b, float& pa, float& pb) {
-    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
-    const uint64_t x = f2_pack(a, b);
-    const uint64_t t = f2_add(x, magic2);                          // j in the low mantissa bits
-    const uint64_t nj = f2_fma(t, f2_pack(-1.0f, -1.0f), magic2);  // -j, exact
-    const uint64_t f = f2_add(x, nj);                              // x - j, exact, |f| <= 1/2
-    uint64_t y = f2_fma(f2_pack(kE5C5, kE5C5), f, f2_pack(kE5C4, kE5C4));
-    y = f2_fma(y, f, f2_pack(kE5C3, kE5C3));
-    y = f2_fma(y, f, f2_pack(kE5C2, kE5C2));
-    y = f2_fma(y, f, f2_pack(kE5C1, kE5C1));
-    y = f2_fma(y, f, f2_pack(kE5C0, kE5C0));
-    uint32_t q0, q1, t0, t1;
-    u2_unpack(y, q0, q1);
-    u2_unpack(t, t0, t1);
-    pa = __uint_as_float(q0 + (t0 << 23));
-    pb = __uint_as_float(q1 + (t1 << 23));
-}
 
 // 8 consecutive columns at each of two addresses, waited for.
 __device__ __forceinline__ void tmem_ld8x2(uint32_t taddr0, uint32_t taddr1, uint32_t (&r0)[8], uint32_t (&r1)[8]) {
@@ -448,22 +417,8 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
 #pragma unroll
                 for (int t = 0; t < kTerms; ++t) pt[t][c] = w[t];
             };
-            if (j == nkb - 1) {  // masked columns are -inf: MUFU only (2^-inf = 0)
 #pragma unroll
-                for (int c = 0; c < kCols / 2; ++c) put(c, ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < kCols / 2; ++c) {
-                    float pa, pb;
-                    if (c % 8 < kFmaPer8) {
-                        exp2_pair_fma(s[2 * c], s[2 * c + 1], pa, pb);
-                    } else {
-                        pa = ex2_approx(s[2 * c]);
-                        pb = ex2_approx(s[2 * c + 1]);
-                    }
-                    put(c, pa, pb);
-                }
-            }
+            for (int c = 0; c < kCols / 2; ++c) put(c, ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]));  // 2^-inf = 0
             if (j > 0 && !uwait(bar_pfree, (j - 1) & 1)) {
                 ok = false;
                 break;

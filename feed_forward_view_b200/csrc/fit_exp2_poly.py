@@ -15,10 +15,11 @@ nearest), so |f| <= 1/2 and f = x - j has no rounding error; then
 2^x = 2^j * p(f), with 2^j applied by adding j to the float32 exponent field.
 
 Running this script prints the float32 coefficients and the worst relative
-error of the float32 Horner evaluation over a dense grid. The values it
-printed are written into attn_fwd.cu (degree 3, kExp2C0..kExp2C3: P is
-rounded to bf16 there) and attn_fwd_f32.cu (degree 5, kE5C0..kE5C5: the fp32
-mode needs the MUFU instruction's own ~2^-22).
+error of the float32 Horner evaluation over a dense grid. The degree-3
+values it printed are written into attn_fwd.cu (kExp2C0..kExp2C3: P is
+rounded to bf16 there). The fp32-mode kernel takes every exponential from
+MUFU; a degree-5 fit (`--degree 5`) would match MUFU's ~2^-22 if it needed
+one.
 """
 from __future__ import annotations
 
@@ -89,7 +90,10 @@ def check(coef, degree):
 
 
 if __name__ == "__main__":
-    for deg in (3, 5):
+    import sys
+
+    degrees = [int(sys.argv[sys.argv.index("--degree") + 1])] if "--degree" in sys.argv else [3]
+    for deg in degrees:
         c = remez_exp2(deg)
         c32, worst = check(c, deg)
         print(f"degree {deg}: " + ", ".join(f"{v:.9e}f" for v in c32) + f"   max rel err {worst:.3e}")

@@ -76,6 +76,26 @@ def test_f32_mode_matches_oracle(F, kind, S, layout, affine, terms):
     assert mx <= bar_abs * float(v.abs().max()) and rf <= bar_fro, (kind, S, layout, terms, mx, rf)
 
 
+@pytest.mark.parametrize("terms", [2, 3])
+@pytest.mark.parametrize("layout", [
+    (0, 32, 24, 0),   # 768 keys: 8 blocks, no fold
+    (1, 32, 24, 0),   # 769 keys: 9 blocks, the fold lands on the last block
+    (1, 32, 48, 0),   # 1537 keys: 17 blocks, a copy fold and an add fold
+])
+def test_f32_mode_fold_boundaries(F, layout, terms):
+    # [O | l] is folded into a second sum every 8 key blocks of 96 keys; key
+    # counts around those boundaries, one frame attended globally
+    q, k, v, pos = synth.make_qkv_f32(1, layout, seed=75)
+    T = q.shape[0]
+    out = F.vggt_attn_global_f32(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), S=1, T=T, terms=terms)
+    torch.cuda.synchronize()
+    assert F.vggt_get_device_status() == 0
+    ref = O.attn_global(f64(q), f64(k), f64(v), pos.numpy().astype(np.float64), 1, T)
+    mx, rf = errs(f64(out), ref)
+    bar_abs, bar_fro = BARS[terms]
+    assert mx <= bar_abs * float(v.abs().max()) and rf <= bar_fro, (layout, terms, mx, rf)
+
+
 def test_f32_mode_is_far_more_accurate_than_bf16(F):
     S, layout = 2, (5, 16, 16, 0)
     q, k, v, pos = synth.make_qkv_f32(S, layout, seed=72)
