@@ -10,8 +10,8 @@
 // Every fp32 operand x is carried as kTerms bf16 terms x_0 = bf16(x),
 // x_1 = bf16(x - x_0) (and x_2 = bf16(x - x_0 - x_1)). A product a b is the
 // sum of the term products a_i b_j with i + j < kTerms -- each a bf16 MMA with
-// fp32 accumulation; the dropped ones are ~2^-18 (two terms) or ~2^-27 (three
-// terms) of a b:
+// fp32 accumulation; the dropped ones are typically ~2^-18 (two terms) or
+// ~2^-27 (three terms) of a b, at most 2^-16 and 2^-23:
 //   two terms:   3 products (0,0) (0,1) (1,0)                    ~2^-17
 //   three terms: 6 products (0,0) (0,1) (1,0) (0,2) (1,1) (2,0)   ~fp32
 //   S     = sum Q_i K_j^T                  (4 K-steps each, N = 96)

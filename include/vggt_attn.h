@@ -335,10 +335,11 @@ VGGT_API int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt
  * x_1 = bf16(x - x_0), x_2 = bf16(x - x_0 - x_1); a b is the sum of the term
  * products a_i b_j with i + j < terms, accumulated in fp32, exponentials to
  * ~2^-22:
- *   terms == 2: 3 products, the dropped ones ~2^-18 a b (outputs to ~1e-5 of
- *               max|v|), about 3x the tensor-core work of the bf16 path;
- *   terms == 3: 6 products, the dropped ones ~2^-27 a b (outputs to about
- *               fp32 rounding, ~1e-6 of max|v|), about 6x.
+ *   terms == 2: 3 products, the dropped ones ~2^-18 a b (at most 2^-16);
+ *               outputs to ~1e-5 of max|v|; about 3x the tensor-core work
+ *               of the bf16 path;
+ *   terms == 3: 6 products, the dropped ones ~2^-27 a b (at most 2^-23);
+ *               outputs to about fp32 rounding, ~1e-6 of max|v|; about 6x.
  * Other values of terms: VGGT_ERR_UNSUPPORTED.
  * Pointers: q, k, v, out 16-byte aligned (fp32 arrays), pos 8-byte aligned.
  * Scratch: 4 + 4*terms bytes per (token, head, dim) -- fp32 q_hat and the
