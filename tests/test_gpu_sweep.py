@@ -57,7 +57,7 @@ def cases(n, seed):
     return out
 
 
-@pytest.mark.parametrize("i,H,S,layout,kd", cases(40, 2024))
+@pytest.mark.parametrize("i,H,S,layout,kd", cases(80, 2024))
 def test_sweep_bf16_entry_points(F, i, H, S, layout, kd):
     q, k, v, pos = (t.cuda() for t in synth.make_layout_qkv(S, layout, seed=100 + i, H=H))
     T = q.shape[0] // S
@@ -93,7 +93,7 @@ def test_sweep_bf16_entry_points(F, i, H, S, layout, kd):
     assert F.vggt_get_device_status() == 0
 
 
-@pytest.mark.parametrize("i,H,S,layout,kd", cases(16, 77))
+@pytest.mark.parametrize("i,H,S,layout,kd", cases(32, 77))
 def test_sweep_stream_and_fp32(F, i, H, S, layout, kd):
     T = sum(layout[::3]) + layout[1] * layout[2]
     if layout[1] * layout[2] > 0:
