@@ -587,7 +587,10 @@ def run_gpu(args):
                          "frac_of_datasheet": attn_tf / DATASHEET_BF16_TFLOPS,
                          "traffic": traffic, "kernel_ms": attn_ms,
                          "share_of_step": attn_ms / ms_step},
-            "kernels": {"qk_prologue": {"ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
+            # (the fp32 mode's own prologue runs inside its step; the bf16
+            # prologue on the same shape is reported for comparison)
+            "kernels": {("qk_prologue_bf16_same_shape" if f32 else "qk_prologue"): {
+                                        "ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
                                         "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
                                         "frac_of_datasheet": pro_bytes / (pro_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS},
                         **({"kv_pool": pool} if pool else {}),
