@@ -8,7 +8,9 @@
 // pool returns it to the system at every synchronisation, and taking a
 // gigabyte back costs milliseconds of host time per call, during which the
 // GPU idles); vggt_release_scratch hands it back on request.
+#include <atomic>
 #include <cmath>
+#include <mutex>
 #include <new>
 #include <cstdint>
 #include <cstdio>
@@ -29,11 +31,13 @@ constexpr int kMaxDevices = 64;
 __device__ int g_device_status;  // kStatusTimeout / kStatusRange bits, 0 when clear
 
 struct DeviceState {
-    int* status = nullptr;  // device address of g_device_status
+    std::atomic<bool> ready{false};  // status and pool set up
+    int* status = nullptr;           // device address of g_device_status
     long long wait_limit = kDefaultWaitLimit;
     cudaMemPool_t pool = nullptr;  // scratch pool, release threshold at its maximum
 };
 DeviceState g_dev[kMaxDevices];
+std::mutex g_init_mutex;  // serialises the one-time set-up of a device's state
 
 // State of the current device, with the status word's device address looked
 // up once per device (with that device current).
@@ -41,6 +45,10 @@ DeviceState* device_state() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     DeviceState& st = g_dev[dev];
+    if (st.ready.load(std::memory_order_acquire)) return &st;
+    // first call on this device (host threads may race to it): set up once
+    std::lock_guard<std::mutex> lock(g_init_mutex);
+    if (st.ready.load(std::memory_order_relaxed)) return &st;
     if (!st.status) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
@@ -64,6 +72,7 @@ DeviceState* device_state() {
         }
         st.pool = pool;
     }
+    st.ready.store(true, std::memory_order_release);
     return &st;
 }
 

@@ -54,6 +54,10 @@
  *     attributes, which cannot happen during a capture: make one ordinary
  *     call per device (and per variant: frame/global/descriptor, fp32 mode)
  *     before capturing.
+ *   - Host threads may call the library concurrently (each on its own
+ *     stream); a device's one-time set-up is serialised inside. A descriptor
+ *     cache handle is not: one thread (or one stream order) at a time.
+ *     vggt_set_wait_limit is meant for set-up, not for concurrent use.
  */
 #ifndef VGGT_ATTN_H
 #define VGGT_ATTN_H
