@@ -31,6 +31,7 @@ __all__ = [
     "vggt_attn_global_noalloc",
     "vggt_get_device_status",
     "vggt_release_scratch",
+    "vggt_scratch_pool_info",
     "vggt_desc_cache_create",
     "vggt_desc_cache_destroy",
     "vggt_desc_cache_frames",
@@ -69,6 +70,7 @@ EXPORTED_SYMBOLS = (
     "vggt_kv_pool_tokens",
     "vggt_get_device_status",
     "vggt_release_scratch",
+    "vggt_scratch_pool_info",
     "vggt_desc_cache_create",
     "vggt_desc_cache_destroy",
     "vggt_desc_cache_frames",
@@ -126,6 +128,8 @@ lib.vggt_attn_descriptor_chunk.argtypes = [_p, _p, _p, _p, _p, _p, _i, _p]
 lib.vggt_attn_descriptor_chunk.restype = _i
 lib.vggt_release_scratch.argtypes = []
 lib.vggt_release_scratch.restype = _i
+lib.vggt_scratch_pool_info.argtypes = [ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_ulonglong)]
+lib.vggt_scratch_pool_info.restype = _i
 lib.vggt_get_device_status.argtypes = [_p]
 lib.vggt_get_device_status.restype = _i
 lib.vggt_status_string.argtypes = [_i]
@@ -602,6 +606,15 @@ def vggt_attn_descriptor_chunk(h, q, k, v, pos, out, C, stream=None):
 def vggt_release_scratch() -> None:
     """Return the library's unused scratch memory on the current device."""
     _check(lib.vggt_release_scratch(), "vggt_release_scratch")
+
+
+def vggt_scratch_pool_info() -> tuple[bool, int]:
+    """(exists, reserved bytes) of the library's scratch pool on the current
+    device."""
+    exists = ctypes.c_int(0)
+    reserved = ctypes.c_ulonglong(0)
+    _check(lib.vggt_scratch_pool_info(ctypes.byref(exists), ctypes.byref(reserved)), "vggt_scratch_pool_info")
+    return bool(exists.value), int(reserved.value)
 
 
 def vggt_set_wait_limit(cycles: int) -> int:

@@ -14,6 +14,7 @@
 #include <new>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 
 #include <cuda_runtime.h>
 
@@ -31,47 +32,79 @@ constexpr int kMaxDevices = 64;
 __device__ int g_device_status;  // kStatusTimeout / kStatusRange bits, 0 when clear
 
 struct DeviceState {
-    std::atomic<bool> ready{false};  // status and pool set up
-    int* status = nullptr;           // device address of g_device_status
-    long long wait_limit = kDefaultWaitLimit;
+    std::atomic<bool> status_ready{false};  // status word address looked up
+    std::atomic<bool> ready{false};         // and the scratch pool created
+    int* status = nullptr;                  // device address of g_device_status
+    std::atomic<long long> wait_limit{kDefaultWaitLimit};
     cudaMemPool_t pool = nullptr;  // scratch pool, release threshold at its maximum
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_init_mutex;  // serialises the one-time set-up of a device's state
 
-// State of the current device, with the status word's device address looked
-// up once per device (with that device current).
-DeviceState* device_state() {
+// The current device's state with the status word's device address looked
+// up (once per device, with that device current). Creates no memory pool:
+// calls that allocate nothing (the core, the no-alloc call, the status and
+// wait-limit calls) use this alone.
+DeviceState* status_state() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     DeviceState& st = g_dev[dev];
-    if (st.ready.load(std::memory_order_acquire)) return &st;
+    if (st.status_ready.load(std::memory_order_acquire)) return &st;
     // first call on this device (host threads may race to it): set up once
     std::lock_guard<std::mutex> lock(g_init_mutex);
+    if (st.status_ready.load(std::memory_order_relaxed)) return &st;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    st.status = static_cast<int*>(p);
+    st.status_ready.store(true, std::memory_order_release);
+    return &st;
+}
+
+// Cap on a scratch pool's size from VGGT_SCRATCH_POOL_MAX_BYTES (a positive
+// decimal byte count), read when the pool is created; 0 (the driver's
+// default, no cap of its own) when unset or not a positive number. A call
+// whose scratch does not fit under the cap returns VGGT_ERR_ALLOC and
+// launches nothing.
+size_t scratch_pool_cap() {
+    const char* text = std::getenv("VGGT_SCRATCH_POOL_MAX_BYTES");
+    if (!text || !*text) return 0;
+    char* end = nullptr;
+    const unsigned long long v = std::strtoull(text, &end, 10);
+    if (*end != '\0' || text[0] == '-') return 0;
+    return static_cast<size_t>(v);
+}
+
+// The current device's state with the scratch pool created as well (once per
+// device), for the calls that take scratch from it.
+DeviceState* device_state() {
+    DeviceState* s = status_state();
+    if (!s) return nullptr;
+    DeviceState& st = *s;
+    if (st.ready.load(std::memory_order_acquire)) return &st;
+    std::lock_guard<std::mutex> lock(g_init_mutex);
     if (st.ready.load(std::memory_order_relaxed)) return &st;
-    if (!st.status) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-        st.status = static_cast<int*>(p);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    props.maxSize = scratch_pool_cap();
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
     }
-    if (!st.pool) {
-        cudaMemPoolProps props = {};
-        props.allocType = cudaMemAllocationTypePinned;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = dev;
-        cudaMemPool_t pool = nullptr;
-        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
-            cudaGetLastError();
-            return nullptr;
-        }
-        uint64_t keep = UINT64_MAX;
-        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
-            cudaGetLastError();
-            cudaMemPoolDestroy(pool);
-            return nullptr;
-        }
-        st.pool = pool;
+    uint64_t keep = UINT64_MAX;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+        cudaGetLastError();
+        cudaMemPoolDestroy(pool);
+        return nullptr;
     }
+    st.pool = pool;
     st.ready.store(true, std::memory_order_release);
     return &st;
 }
@@ -214,7 +247,7 @@ int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const
 namespace vggt {
 
 bool device_status_word(int** status, long long* wait_limit) {
-    DeviceState* st = device_state();
+    DeviceState* st = status_state();
     if (!st) return false;
     *status = st->status;
     *wait_limit = st->wait_limit;
@@ -429,7 +462,7 @@ int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf
     if (!q_hat || !k_hat || !v || !out) return VGGT_ERR_NULL;
     if (!aligned16(q_hat) || !aligned16(k_hat) || !aligned16(v) || !aligned16(out))
         return VGGT_ERR_UNSUPPORTED;
-    DeviceState* st = device_state();
+    DeviceState* st = status_state();
     if (!st) return VGGT_ERR_CUDA;
     AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H,
                   static_cast<long long>(n_seg) * q_len, static_cast<long long>(n_seg) * k_len};
@@ -740,8 +773,26 @@ int vggt_release_scratch(void) {
     return VGGT_OK;
 }
 
+int vggt_scratch_pool_info(int* exists, unsigned long long* reserved) {
+    if (!exists || !reserved) return VGGT_ERR_NULL;
+    *exists = 0;
+    *reserved = 0;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VGGT_ERR_CUDA;
+    DeviceState& st = g_dev[dev];
+    if (!st.ready.load(std::memory_order_acquire)) return VGGT_OK;
+    uint64_t bytes = 0;
+    if (cudaMemPoolGetAttribute(st.pool, cudaMemPoolAttrReservedMemCurrent, &bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return VGGT_ERR_CUDA;
+    }
+    *exists = 1;
+    *reserved = static_cast<unsigned long long>(bytes);
+    return VGGT_OK;
+}
+
 int vggt_get_device_status(cudaStream_t stream) {
-    DeviceState* st = device_state();
+    DeviceState* st = status_state();
     if (!st) return VGGT_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return VGGT_ERR_CUDA;
     int h = 0;
@@ -776,15 +827,13 @@ const char* vggt_status_string(int status) {
 }
 
 long long vggt_set_wait_limit(long long cycles) {
-    DeviceState* st = device_state();
+    DeviceState* st = status_state();
     if (!st) return -1;
-    const long long prev = st->wait_limit;
-    st->wait_limit = cycles < 1 ? kDefaultWaitLimit : cycles;
-    return prev;
+    return st->wait_limit.exchange(cycles < 1 ? kDefaultWaitLimit : cycles);
 }
 
 int vggt_debug_wait_timeout(cudaStream_t stream) {
-    DeviceState* st = device_state();
+    DeviceState* st = status_state();
     if (!st) return VGGT_ERR_CUDA;
     return to_status(vggt::launch_wait_probe(st->status, st->wait_limit, stream));
 }

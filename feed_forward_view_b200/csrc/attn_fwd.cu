@@ -91,6 +91,8 @@
 // Every wait is bounded; on timeout the CTA records the timeout in the device
 // status word, stops issuing work, drains what it has in flight and frees its
 // tensor memory before exiting.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -664,12 +666,14 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
         !make_map(&tm_v, p.v, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
         return cudaErrorInvalidValue;
 
-    static bool attr_set[64] = {};
+    // Set once per device; host threads that race here both set the same
+    // attribute, and the flag is published atomically.
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         // The register split (setmaxnreg) needs the full launch allocation
         // (kLaunchRegs per thread); with fewer registers the softmax
         // warpgroups' increase could never be granted. Refuse to launch such
@@ -682,7 +686,7 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
         e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes));
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     Params prm;
     prm.q_hat = p.q_hat;

@@ -38,6 +38,8 @@
 // Every wait is bounded; on timeout the CTA records it in the device status
 // word, stops issuing, drains what it has in flight and frees its tensor
 // memory.
+#include <atomic>
+
 #include <cuda_bf16.h>
 
 #include "attn_common.cuh"
@@ -492,16 +494,18 @@ cudaError_t launch_terms(const AttnProblemF32& p, const Params& prm, cudaStream_
         if (!make_map(&maps.k[t], p.k[t], ks, p.H, row_bytes, ks * row_bytes, kBN, 1) ||
             !make_map(&maps.v[t], p.v[t], p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
             return cudaErrorInvalidValue;
-    static bool attr_set[64] = {};
+    // Set once per device; host threads that race here both set the same
+    // attribute, and the flag is published atomically.
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(attn_fwd_f32_kernel<kTerms>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem_bytes<kTerms>()));
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     dim3 grid(p.n_seg * prm.tiles_per_seg, p.H);
     attn_fwd_f32_kernel<kTerms><<<grid, kThreads, smem_bytes<kTerms>(), stream>>>(maps, prm);

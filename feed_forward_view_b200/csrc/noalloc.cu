@@ -17,6 +17,7 @@
 // example on two streams without ordering between them) race on it. Nothing in
 // it needs to start at zero: the prologue overwrites every byte the attention
 // kernel then reads, and rows past the end are never read from it.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -30,22 +31,24 @@ namespace {
 __device__ __align__(256) unsigned char g_noalloc_scratch[VGGT_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
+// Host threads may make their first call on a device at the same time: the
+// cached address is published atomically (both would store the same value).
+std::atomic<void*> g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device, looked up once
 // per device; nullptr if the lookup fails.
 void* scratch_on_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+    void* addr = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!addr) {
+        if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) {
             cudaGetLastError();
             return nullptr;
         }
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(addr, std::memory_order_release);
     }
-    return g_scratch_addr[dev];
+    return addr;
 }
 
 int square_grid_side(int T) {
@@ -70,6 +73,8 @@ extern "C" int vggt_attn_global_noalloc(const vggt_bf16* q, const vggt_bf16* k,
     if (square_grid_side(T) < 0) return VGGT_ERR_SHAPE;
     if (kv_down != 0 && kv_down != 1) return VGGT_ERR_SHAPE;
     if (H > 65535) return VGGT_ERR_SHAPE;
+    // the token count first, so that the byte count below cannot wrap
+    if (static_cast<long long>(S) * T > VGGT_MAX_TOKENS) return VGGT_ERR_SHAPE;
     // normalised q and k, head-major bf16: 2 * N * H * D * 2 bytes
     const unsigned long long n = static_cast<unsigned long long>(S) * static_cast<unsigned>(T);
     const unsigned long long plane = n * static_cast<unsigned>(H) * VGGT_HEAD_DIM * sizeof(uint16_t);

@@ -43,6 +43,12 @@
  *     would cost milliseconds of host time per call to take it back), so
  *     after a call the library holds up to the largest scratch any call
  *     needed -- about 4 * S*T * H * D bytes; vggt_release_scratch returns it.
+ *     The environment variable VGGT_SCRATCH_POOL_MAX_BYTES (a positive decimal
+ *     byte count), read when a device's pool is created, caps that pool: a
+ *     call whose scratch does not fit returns VGGT_ERR_ALLOC and launches
+ *     nothing. Calls that need no scratch (vggt_attn_core,
+ *     vggt_attn_global_noalloc, the status and wait-limit calls) never create
+ *     the pool.
  *   - Outputs must not overlap inputs.
  *   - Every argument is checked on the host before any launch; an invalid call
  *     returns a negative vggt_status and launches nothing.
@@ -87,7 +93,9 @@ typedef enum vggt_status {
     VGGT_ERR_SHAPE = -3,       /* negative sizes, T != 5 + g*g (plain calls) or a
                                   layout that does not add up to T, bad kv_down, or
                                   a size beyond the library's limits              */
-    VGGT_ERR_ALLOC = -4,       /* scratch allocation failed                        */
+    VGGT_ERR_ALLOC = -4,       /* scratch allocation failed (device memory, or the
+                                  VGGT_SCRATCH_POOL_MAX_BYTES cap); nothing was
+                                  launched and no output written                  */
     VGGT_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed             */
     VGGT_ERR_TIMEOUT = -6,     /* a bounded device-side wait ran out (reported by
                                   vggt_get_device_status)                          */
@@ -453,6 +461,13 @@ VGGT_API int vggt_get_device_status(cudaStream_t stream);
    they need it. VGGT_OK, or VGGT_ERR_CUDA. Host only. (No counterpart on the
    pages: memory management of this library.) */
 VGGT_API int vggt_release_scratch(void);
+
+/* Whether the library's scratch pool exists on the current device (*exists
+   = 0 or 1: the first call that needs scratch creates it) and how many bytes
+   it currently holds from the system (*reserved, 0 when it does not exist).
+   VGGT_OK, VGGT_ERR_NULL or VGGT_ERR_CUDA. Host only. (No counterpart on the
+   pages: memory management of this library.) */
+VGGT_API int vggt_scratch_pool_info(int* exists, unsigned long long* reserved);
 
 /* Human-readable name of a vggt_status value (static storage). */
 VGGT_API const char* vggt_status_string(int status);

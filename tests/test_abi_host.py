@@ -267,3 +267,25 @@ def test_batch_argument_checks():
     assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 261, 16, 64, 4, None, None, None) == OK
     assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 260, 16, 64, 4, None, None, None) == E_SHAPE  # not 5 + g*g
     assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 261, 16, 64, 0, None, None, None) == E_SHAPE
+
+
+def test_noalloc_argument_checks():
+    na = F.lib.vggt_attn_global_noalloc
+    p = [FAKE] * 5
+    assert na(*p, 1, 4101, 16, 64, 0, None) == E_SHAPE       # 16.8 MB of scratch > the 16 MiB array
+    assert na(*p, 2, 261, 16, 32, 0, None) == E_UNSUP
+    assert na(*p, 2, 262, 16, 64, 0, None) == E_SHAPE        # T - 5 not a square
+    assert na(*p, 2, 261, 16, 64, 2, None) == E_SHAPE        # kv_down
+    assert na(None, None, None, None, None, 0, 261, 16, 64, 0, None) == OK
+    # token counts beyond the library's limit are rejected before the byte
+    # count is formed (which could wrap for sizes near 2^31)
+    big = 2 ** 31 - 1
+    assert na(*p, big, 5 + 215 * 215, 1, 64, 0, None) == E_SHAPE
+    assert na(*p, big, 5 + 46340 * 46340, 65535, 64, 0, None) == E_SHAPE
+
+
+def test_scratch_pool_info_needs_its_pointers():
+    import ctypes
+    e, r = ctypes.c_int(7), ctypes.c_ulonglong(7)
+    assert F.lib.vggt_scratch_pool_info(None, ctypes.byref(r)) == E_NULL
+    assert F.lib.vggt_scratch_pool_info(ctypes.byref(e), None) == E_NULL
