@@ -186,7 +186,7 @@ class OracleLeg:
         import numpy as np
         import torch
 
-        from feed_forward_view_b200 import synth
+        import synth
         from oracle import vggt_oracle as O
 
         self.w, self.O, self.synth = w, O, synth
@@ -247,7 +247,7 @@ def blas_threads() -> int:
 
 def run_reference(args):
     """--impl reference: the oracle on the host cores, bounded sample per step."""
-    from feed_forward_view_b200 import synth
+    import synth
 
     rank, _, world = int(os.environ.get("RANK", "0")), 0, int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
@@ -296,7 +296,7 @@ def run_gpu(args):
     import torch
 
     import feed_forward_view_b200 as F
-    from feed_forward_view_b200 import synth
+    import synth
 
     rank, local, world = dist_setup(args.gpus)
     torch.cuda.set_device(local)

@@ -505,15 +505,3 @@ def attn_subset(q, k, v, pos, S: int, T: int, n_skip_back: int, n_extra: int, ki
         k_hat = qk_prologue(k[kr], pos[kr], *_ln(ln, "k"))
         out[sel] = cross_attention(q_hat, k_hat, v[kr])
     return out
-
-
-def flops(kind: str, S: int, T: int, Tk: int, H: int, D: int, n_rows=None) -> float:
-    """Algorithmic attention FLOPs, ``4*H*D`` per (query, key) pair."""
-    if kind == "frame":
-        keys = T
-    elif kind == "descriptor":
-        keys = S * Tk
-    else:
-        keys = S * T
-    n = S * T if n_rows is None else n_rows
-    return 4.0 * H * D * n * keys

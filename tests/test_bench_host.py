@@ -65,7 +65,7 @@ def test_clock_summary_parsing():
 
 
 def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
-    from feed_forward_view_b200 import synth
+    import synth
 
     w = synth.WORKLOADS["global_s9_g64"]
     f = tmp_path / "summary.txt"
@@ -81,7 +81,7 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
 @pytest.mark.parametrize("name", ["global_s2_g16", "frame_s8_g37", "descriptor_s200_g37_kd4",
                                   "omega_frame_s32_g32", "omega_global_s32_g32", "frame_s8_g37_f32"])
 def test_oracle_leg_runs_on_a_small_sample(name):
-    from feed_forward_view_b200 import synth
+    import synth
 
     w = synth.ALL_WORKLOADS[name]
     if w.n_q > 50000:

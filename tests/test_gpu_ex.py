@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from oracle import vggt_oracle as O
-from feed_forward_view_b200 import synth
+import synth
 
 pytestmark = pytest.mark.gpu
 

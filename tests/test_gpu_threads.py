@@ -15,7 +15,7 @@ SCRIPT = r"""
 import threading
 import torch
 import feed_forward_view_b200 as F
-from feed_forward_view_b200 import synth
+import synth
 
 n = 4
 q, k, v, pos = (t.cuda() for t in synth.make_qkv(S=2, g=16, seed=0))
