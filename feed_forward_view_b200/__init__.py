@@ -28,6 +28,7 @@ __all__ = [
     "vggt_kv_pool_tokens",
     "vggt_qk_prologue",
     "vggt_attn_core",
+    "vggt_attn_core_online",
     "vggt_attn_global_noalloc",
     "vggt_get_device_status",
     "vggt_release_scratch",
@@ -62,6 +63,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "vggt_qk_prologue",
     "vggt_attn_core",
+    "vggt_attn_core_online",
     "vggt_attn_global_noalloc",
     "vggt_attn_frame",
     "vggt_attn_global",
@@ -112,8 +114,9 @@ lib.vggt_kv_pool.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.vggt_kv_pool.restype = _i
 lib.vggt_qk_prologue.argtypes = [_p, _p, _p, _i, _i, _i, _p]
 lib.vggt_qk_prologue.restype = _i
-lib.vggt_attn_core.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
-lib.vggt_attn_core.restype = _i
+for _name in ("vggt_attn_core", "vggt_attn_core_online"):
+    getattr(lib, _name).argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+    getattr(lib, _name).restype = _i
 lib.vggt_kv_pool_tokens.argtypes = [_i, _i]
 lib.vggt_kv_pool_tokens.restype = _i
 lib.vggt_desc_cache_create.argtypes = [ctypes.POINTER(_p), _i, _i, _i, _i, _i]
@@ -272,6 +275,16 @@ def vggt_attn_core(q_hat, k_hat, v, out, n_seg, q_len, k_len, H=16, D=64, stream
                             _ptr(v, torch.bfloat16, "v"), _ptr(out, torch.bfloat16, "out"),
                             int(n_seg), int(q_len), int(k_len), int(H), int(D), _stream(stream))
     _check(rc, "vggt_attn_core")
+    return out
+
+
+def vggt_attn_core_online(q_hat, k_hat, v, out, n_seg, q_len, k_len, H=16, D=64, stream=None):
+    """vggt_attn_core for any finite q_hat / k_hat (running row maximum).
+    Returns ``out``."""
+    rc = lib.vggt_attn_core_online(_ptr(q_hat, torch.bfloat16, "q_hat"), _ptr(k_hat, torch.bfloat16, "k_hat"),
+                                   _ptr(v, torch.bfloat16, "v"), _ptr(out, torch.bfloat16, "out"),
+                                   int(n_seg), int(q_len), int(k_len), int(H), int(D), _stream(stream))
+    _check(rc, "vggt_attn_core_online")
     return out
 
 

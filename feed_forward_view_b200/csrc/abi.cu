@@ -178,23 +178,36 @@ bool make_affine(const float* w, const float* b, vggt::LnAffine* a, double* boun
     return true;
 }
 
-// The query and key affines of a call. The attention kernel evaluates
-// exp(score) without subtracting a row maximum (exact up to rounding, as
-// softmax ignores a common factor), which needs every score bounded: with
-// |q_hat| <= Bq and |k_hat| <= Bk the score in log2 units is at most
-// Bq * Bk / 8 * log2(e) (+1% for the bf16 roundings), and this stays below
-// kMaxLog2Score so that exponentials, their sums over up to 2^21 keys and the
-// weighted value sums keep far from the fp32 limits. Beyond it: UNSUPPORTED.
-constexpr double kMaxLog2Score = 64.0;
+// The query and key affines of a call, and which attention path runs them.
+//
+// With Bq = 8 * max|q_weight| + ||q_bias||_2 (a bound on the norm of a
+// normalised query, the plain LayerNorm's being below 8) and Bk likewise,
+// every score is at most Bq * Bk / 8 in magnitude, and q_hat / k_hat stored
+// in bf16 (2^-9 relative rounding per element) move a score by about
+// 2^-9 |q_hat| |k_hat| / 8. The plain LayerNorm keeps both small: the bf16
+// kernel then evaluates exp(score) with no row maximum (exact up to rounding:
+// softmax ignores a common factor) and its outputs stay within the bf16
+// path's error. An affine that enlarges Bq * Bk beyond kPreciseRatio times
+// the plain 8 * 8 enlarges that error in proportion (measured on N(0, 1)
+// inputs: relative Frobenius error 2.9e-3 at weight 1, 4.3e-3 at 1.25, 5e-3
+// at 1.41), and the score range without bound. Such calls run in precise
+// mode: q_hat in fp32, k_hat as two bf16 terms (16 significant bits), the
+// online softmax (running row maximum), on the term-split attention kernel;
+// any finite affine is accepted. Only a weight or bias that is not finite is
+// refused.
+constexpr double kPreciseRatio = 1.21;  // 1.1^2: weights up to 1.1 on both sides, no bias
 struct Norms {
     vggt::LnAffine q, k;
+    bool online = false;   // running row maximum (set with precise)
+    bool precise = false;  // q_hat fp32, k_hat in two bf16 terms
 };
 int make_norms(const vggt_qk_norm* n, Norms* out) {
     double bq = 8.0, bk = 8.0;
     if (!make_affine(n ? n->q_weight : nullptr, n ? n->q_bias : nullptr, &out->q, &bq) ||
         !make_affine(n ? n->k_weight : nullptr, n ? n->k_bias : nullptr, &out->k, &bk))
         return VGGT_ERR_UNSUPPORTED;
-    if (bq * bk / 8.0 * 1.4426950408889634 * 1.01 > kMaxLog2Score) return VGGT_ERR_UNSUPPORTED;
+    out->precise = bq * bk > kPreciseRatio * 64.0;
+    out->online = out->precise;
     return VGGT_OK;
 }
 
@@ -204,6 +217,106 @@ size_t head_plane_bytes(long long n_tokens, int H) {
 
 int to_status(cudaError_t e) { return e == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA; }
 
+// Precise mode's operands in scratch: q_hat fp32 [H, nq, 64], then the two
+// bf16 terms of k_hat, each a head-major plane (k_stride rows per head).
+struct PreciseOperands {
+    float* q_hat;
+    uint16_t* k_hat[2];
+};
+// Carves them from the start of `scratch` (4 * head_plane_bytes(nq, H) bytes
+// for q_hat and the k planes when nk == nq; in general 2 * plane(nq) + 2 *
+// plane(nk)); the k planes hold nk rows per head.
+PreciseOperands precise_operands(void* scratch, long long nq, int H, long long nk = -1) {
+    if (nk < 0) nk = nq;
+    PreciseOperands po;
+    po.q_hat = static_cast<float*>(scratch);
+    po.k_hat[0] = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(scratch) + 2 * head_plane_bytes(nq, H));
+    po.k_hat[1] = po.k_hat[0] + head_plane_bytes(nk, H) / sizeof(uint16_t);
+    return po;
+}
+size_t precise_bytes(long long nq, long long nk, int H) { return 2 * head_plane_bytes(nq, H) + 2 * head_plane_bytes(nk, H); }
+
+// Precise-mode prologue: nq query rows (token q_map(r) of q / q_pos) to
+// po.q_hat in fp32, nk key rows (token k_map(r) of k / k_pos) as two bf16
+// terms into po.k_hat (k_stride rows per head plane); one launch. nq may be 0.
+int precise_prologue(const uint16_t* q, const float* q_pos, long long nq, const vggt::RowMap& q_map,
+                     const uint16_t* k, const float* k_pos, long long nk, const vggt::RowMap& k_map,
+                     const PreciseOperands& po, long long k_stride, const Norms& norms, int H, cudaStream_t stream) {
+    vggt::PrologueJobF32 jq{};
+    jq.x = q;
+    jq.pos = q_pos;
+    jq.out[0] = po.q_hat;
+    jq.n = static_cast<int>(nq);
+    jq.out_stride = nq;
+    jq.ln = norms.q;
+    jq.terms = 0;
+    jq.x_bf16 = true;
+    jq.in_map = q_map;
+    vggt::PrologueJobF32 jk{};
+    jk.x = k;
+    jk.pos = k_pos;
+    jk.out[0] = po.k_hat[0];
+    jk.out[1] = po.k_hat[1];
+    jk.n = static_cast<int>(nk);
+    jk.out_stride = k_stride;
+    jk.ln = norms.k;
+    jk.terms = 2;
+    jk.x_bf16 = true;
+    jk.in_map = k_map;
+    if (nq == 0) return to_status(vggt::launch_qk_prologue_f32(jk, vggt::PrologueJobF32{}, H, stream));
+    return to_status(vggt::launch_qk_prologue_f32(jq, jk, H, stream));
+}
+
+// Precise-mode attention of po's operands (q_stride / k_stride rows per head
+// plane) with the bf16 values v [n_seg*k_len, H, 64] into the bf16 out.
+int precise_attention(const PreciseOperands& po, long long k_stride, const uint16_t* v, uint16_t* out, int n_seg,
+                      int q_len, int k_len, int H, long long q_stride, const vggt::RowMap& out_map,
+                      DeviceState* st, cudaStream_t stream) {
+    vggt::AttnProblemF32 p{};
+    p.q_hat = po.q_hat;
+    p.k[0] = po.k_hat[0];
+    p.k[1] = po.k_hat[1];
+    p.v[0] = v;
+    p.terms = 2;
+    p.terms_pv = 1;
+    p.online = true;
+    p.out = out;
+    p.n_seg = n_seg;
+    p.q_len = q_len;
+    p.k_len = k_len;
+    p.H = H;
+    p.q_stride = q_stride;
+    p.k_stride = k_stride;
+    p.out_map = out_map;
+    return to_status(vggt::launch_attention_f32(p, st->status, st->wait_limit, stream));
+}
+
+// Precise-mode descriptors: pools the S frames of k / v / pos into v_out /
+// pos_out and writes the normalised pooled keys (fp32 means, no bf16
+// rounding) as two bf16 terms head-major into k_hi / k_lo (k_stride rows per
+// head plane).
+int precise_pool_keys(const uint16_t* k, const uint16_t* v, const float* pos, int S, int T,
+                      const vggt::FrameLayout& L, int kd, int H, uint16_t* k_hi, uint16_t* k_lo, long long k_stride,
+                      uint16_t* v_out, float* pos_out, const Norms& norms, cudaStream_t stream) {
+    vggt::PoolJob job{};
+    job.k = k;
+    job.v = v;
+    job.pos = pos;
+    job.k_out = nullptr;
+    job.k_hat = k_hi;
+    job.k_hat_lo = k_lo;
+    job.k_hat_stride = k_stride;
+    job.v_out = v_out;
+    job.pos_out = pos_out;
+    job.S = S;
+    job.T = T;
+    job.layout = L;
+    job.kd = kd;
+    job.H = H;
+    job.k_ln = norms.k;
+    return to_status(vggt::launch_kv_pool(job, stream));
+}
+
 // Frame (n_seg = S, q_len = k_len = T) or global (n_seg = 1, q_len = k_len
 // = S*T) attention: prologue on q and k (one launch), then attention; the
 // scratch q_hat | k_hat is freed on the stream.
@@ -212,6 +325,20 @@ int run_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const
     DeviceState* st = device_state();
     if (!st) return VGGT_ERR_CUDA;
     const long long n = static_cast<long long>(n_seg) * len;
+    if (norms.precise) {
+        // scratch: q_hat fp32 [H, n, 64] | k_hat terms 0 and 1 [H, n, 64]
+        void* scratch = nullptr;
+        if (cudaMallocFromPoolAsync(&scratch, 4 * head_plane_bytes(n, H), st->pool, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return VGGT_ERR_ALLOC;
+        }
+        PreciseOperands po = precise_operands(scratch, n, H);
+        int rc = precise_prologue(q, pos, n, vggt::RowMap{}, k, pos, n, vggt::RowMap{}, po, n, norms, H, stream);
+        if (rc == VGGT_OK)
+            rc = precise_attention(po, n, v, out, n_seg, len, len, H, n, vggt::RowMap{}, st, stream);
+        cudaFreeAsync(scratch, stream);
+        return rc;
+    }
     void* scratch = nullptr;
     if (cudaMallocFromPoolAsync(&scratch, 2 * head_plane_bytes(n, H), st->pool, stream) != cudaSuccess) {
         cudaGetLastError();
@@ -224,6 +351,7 @@ int run_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const
     int rc = to_status(vggt::launch_qk_prologue(jq, jk, H, stream));
     if (rc == VGGT_OK) {
         AttnProblem p{q_hat, k_hat, v, out, n_seg, len, len, H, n, n};
+        p.online = norms.online;
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -319,6 +447,30 @@ int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const
     const long long nk = static_cast<long long>(B) * S * Tk;
     DeviceState* st = device_state();
     if (!st) return VGGT_ERR_CUDA;
+    if (norms.precise) {
+        // scratch: q_hat fp32 | k_hat terms [H, nk, 64] x 2 | pooled v
+        // [nk, H, 64] | pooled pos [nk, 2]. The keys are pooled as fp32 means
+        // and normalised into the two term planes in the same pass.
+        const size_t ops = precise_bytes(nq, nk, H), kb = head_plane_bytes(nk, H);
+        void* scratch = nullptr;
+        if (cudaMallocFromPoolAsync(&scratch, ops + kb + static_cast<size_t>(nk) * 2 * sizeof(float), st->pool,
+                                    stream) != cudaSuccess) {
+            cudaGetLastError();
+            return VGGT_ERR_ALLOC;
+        }
+        const PreciseOperands po = precise_operands(scratch, nq, H, nk);
+        uint16_t* vp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(scratch) + ops);
+        float* pp = reinterpret_cast<float*>(vp + kb / sizeof(uint16_t));
+        rc = precise_prologue(q, pos, nq, vggt::RowMap{}, nullptr, nullptr, 0, vggt::RowMap{}, po, nk, norms, H,
+                              stream);
+        if (rc == VGGT_OK)
+            rc = precise_pool_keys(k, v, pos, B * S, T, L, kv_down, H, po.k_hat[0], po.k_hat[1], nk, vp, pp, norms,
+                                   stream);
+        if (rc == VGGT_OK)
+            rc = precise_attention(po, nk, vp, out, B, S * T, S * Tk, H, nq, vggt::RowMap{}, st, stream);
+        cudaFreeAsync(scratch, stream);
+        return rc;
+    }
     // scratch: q_hat [H, nq, 64] | k_hat [H, nk, 64] | pooled v [nk, H, 64] | pooled pos [nk, 2]
     const size_t q_bytes = head_plane_bytes(nq, H), k_bytes = head_plane_bytes(nk, H);
     void* scratch = nullptr;
@@ -337,6 +489,7 @@ int attn_call(Kind kind, bool plain, const uint16_t* q, const uint16_t* k, const
         // every query row attends to all S*Tk descriptors: one segment
         // scene b: its S*T query rows attend to its S*Tk descriptors
         AttnProblem p{q_hat, k_hat, vp, out, B, S * T, S * Tk, H, nq, nk};
+        p.online = norms.online;
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -450,9 +603,12 @@ int vggt_qk_prologue_ex(const vggt_bf16* x, const float* pos, vggt_bf16* x_hat, 
     return to_status(vggt::launch_qk_prologue(j, none, H, stream));
 }
 
-int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
-                   vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
-                   cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int attn_core_call(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v, vggt_bf16* out, int n_seg,
+                   int q_len, int k_len, int H, int D, bool online, cudaStream_t stream) {
     if (n_seg < 0 || q_len < 0 || k_len < 0 || H < 0 || D < 0) return VGGT_ERR_SHAPE;
     if (D != VGGT_HEAD_DIM) return VGGT_ERR_UNSUPPORTED;
     if (static_cast<long long>(n_seg) * q_len > VGGT_MAX_TOKENS ||
@@ -466,7 +622,24 @@ int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf
     if (!st) return VGGT_ERR_CUDA;
     AttnProblem p{q_hat, k_hat, v, out, n_seg, q_len, k_len, H,
                   static_cast<long long>(n_seg) * q_len, static_cast<long long>(n_seg) * k_len};
+    p.online = online;
     return to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
+                   vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
+                   cudaStream_t stream) {
+    return attn_core_call(q_hat, k_hat, v, out, n_seg, q_len, k_len, H, D, false, stream);
+}
+
+int vggt_attn_core_online(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
+                          vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
+                          cudaStream_t stream) {
+    return attn_core_call(q_hat, k_hat, v, out, n_seg, q_len, k_len, H, D, true, stream);
 }
 
 int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v, const float* pos,
@@ -497,9 +670,33 @@ int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
         map.stride = T;
         map.n_grouped = n_frames_rows;
     }
+    const size_t plane = head_plane_bytes(n, H);
+    if (norms.precise) {
+        // scratch: q_hat fp32 | k_hat terms [H, n, 64] x 2 and, when rows are
+        // left out, the gathered values [n, H, 64]
+        const size_t ops = precise_bytes(n, n, H);
+        void* scratch = nullptr;
+        if (cudaMallocFromPoolAsync(&scratch, ops + (n_skip_back > 0 ? plane : 0), st->pool, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return VGGT_ERR_ALLOC;
+        }
+        const PreciseOperands po = precise_operands(scratch, n, H);
+        const uint16_t* v_use = v;
+        int rc = VGGT_OK;
+        if (n_skip_back > 0) {
+            uint16_t* v_c = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(scratch) + ops);
+            rc = to_status(vggt::launch_gather_rows(v, v_c, n, H * VGGT_HEAD_DIM, map, stream));
+            v_use = v_c;
+        }
+        if (rc == VGGT_OK) rc = precise_prologue(q, pos, n, map, k, pos, n, map, po, n, norms, H, stream);
+        if (rc == VGGT_OK)
+            rc = precise_attention(po, n, v_use, out, global ? 1 : S, global ? static_cast<int>(n) : keep,
+                                   global ? static_cast<int>(n) : keep, H, n, map, st, stream);
+        cudaFreeAsync(scratch, stream);
+        return rc;
+    }
     // scratch: q_hat | k_hat [H, n, 64] and, when rows are left out, the
     // gathered values [n, H, 64]
-    const size_t plane = head_plane_bytes(n, H);
     void* scratch = nullptr;
     if (cudaMallocFromPoolAsync(&scratch, (n_skip_back > 0 ? 3 : 2) * plane, st->pool, stream) != cudaSuccess) {
         cudaGetLastError();
@@ -522,6 +719,7 @@ int vggt_attn_subset(const vggt_bf16* q, const vggt_bf16* k, const vggt_bf16* v,
     if (rc == VGGT_OK) {
         AttnProblem p{q_hat, k_hat, v_use, out, global ? 1 : S, global ? static_cast<int>(n) : keep,
                       global ? static_cast<int>(n) : keep, H, n, n, map};
+        p.online = norms.online;
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -568,6 +766,7 @@ int attn_f32_call(bool global, const float* q, const float* k, const float* v, c
     if (rc == VGGT_OK) {
         vggt::AttnProblemF32 p{q_hat, {kt[0], kt[1], kt[2]}, {vt[0], vt[1], vt[2]}, terms, out, global ? 1 : S,
                                global ? static_cast<int>(n) : T, global ? static_cast<int>(n) : T, H, n, n};
+        p.online = norms.online;
         rc = to_status(vggt::launch_attention_f32(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -644,6 +843,7 @@ struct vggt_desc_cache {
     long long capacity;  // max_frames * Tk descriptor rows
     int frames;          // frames appended so far
     uint16_t* k_hat;     // [H][capacity][64] normalised pooled keys, head-major
+    uint16_t* k_lo;      // precise mode: their second bf16 terms, same layout (else null)
     uint16_t* v;         // [capacity][H][64] pooled values, token-major
     float* pos;          // [capacity][2] cell-mean positions
 };
@@ -687,14 +887,16 @@ int vggt_desc_cache_create_ex(vggt_desc_cache** cache, int max_frames, int T, in
     c->capacity = capacity;
     c->frames = 0;
     const size_t plane = head_plane_bytes(capacity, H);
+    const int k_planes = norms.precise ? 2 : 1;
     void* mem = nullptr;
-    if (cudaMalloc(&mem, 2 * plane + static_cast<size_t>(capacity) * 2 * sizeof(float)) != cudaSuccess) {
+    if (cudaMalloc(&mem, (k_planes + 1) * plane + static_cast<size_t>(capacity) * 2 * sizeof(float)) != cudaSuccess) {
         cudaGetLastError();
         delete c;
         return VGGT_ERR_ALLOC;
     }
     c->k_hat = static_cast<uint16_t*>(mem);
-    c->v = c->k_hat + plane / sizeof(uint16_t);
+    c->k_lo = norms.precise ? c->k_hat + plane / sizeof(uint16_t) : nullptr;
+    c->v = c->k_hat + k_planes * plane / sizeof(uint16_t);
     c->pos = reinterpret_cast<float*>(c->v + plane / sizeof(uint16_t));
     *cache = c;
     return VGGT_OK;
@@ -738,6 +940,30 @@ int vggt_attn_descriptor_chunk(vggt_desc_cache* cache, const vggt_bf16* q, const
     const long long n_q = static_cast<long long>(C) * T;
     const long long row0 = static_cast<long long>(cache->frames) * Tk;  // first new descriptor
     const long long n_new = static_cast<long long>(C) * Tk;
+    if (cache->norms.precise) {
+        // scratch: the chunk's q_hat fp32 [H, C*T, 64]; its descriptors go
+        // straight into the cache (keys as two term planes, fp32 means
+        // normalised in the pooling pass).
+        void* scratch = nullptr;
+        if (cudaMallocFromPoolAsync(&scratch, 2 * head_plane_bytes(n_q, H), st->pool, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return VGGT_ERR_ALLOC;
+        }
+        const PreciseOperands all{static_cast<float*>(scratch), {cache->k_hat, cache->k_lo}};
+        rc = precise_prologue(q, pos, n_q, vggt::RowMap{}, nullptr, nullptr, 0, vggt::RowMap{}, all,
+                              cache->capacity, cache->norms, H, stream);
+        if (rc == VGGT_OK)
+            rc = precise_pool_keys(k, v, pos, C, T, cache->layout, cache->kv_down, H,
+                                   cache->k_hat + row0 * VGGT_HEAD_DIM, cache->k_lo + row0 * VGGT_HEAD_DIM,
+                                   cache->capacity, cache->v + row0 * H * VGGT_HEAD_DIM, cache->pos + row0 * 2,
+                                   cache->norms, stream);
+        if (rc == VGGT_OK)
+            rc = precise_attention(all, cache->capacity, cache->v, out, 1, static_cast<int>(n_q),
+                                   static_cast<int>(row0 + n_new), H, n_q, vggt::RowMap{}, st, stream);
+        cudaFreeAsync(scratch, stream);
+        if (rc == VGGT_OK) cache->frames += C;
+        return rc;
+    }
     // Scratch: the chunk's q_hat [H, C*T, 64].
     void* scratch = nullptr;
     if (cudaMallocFromPoolAsync(&scratch, head_plane_bytes(n_q, H), st->pool, stream) != cudaSuccess) {
@@ -756,6 +982,7 @@ int vggt_attn_descriptor_chunk(vggt_desc_cache* cache, const vggt_bf16* q, const
     if (rc == VGGT_OK) {
         AttnProblem p{q_hat, cache->k_hat, cache->v, out, 1, static_cast<int>(n_q),
                       static_cast<int>(row0 + n_new), H, n_q, cache->capacity};
+        p.online = cache->norms.online;
         rc = to_status(vggt::launch_attention(p, st->status, st->wait_limit, stream));
     }
     cudaFreeAsync(scratch, stream);
@@ -813,15 +1040,14 @@ const char* vggt_status_string(int status) {
         case VGGT_ERR_NULL: return "VGGT_ERR_NULL: a required pointer is NULL";
         case VGGT_ERR_UNSUPPORTED:
             return "VGGT_ERR_UNSUPPORTED: head dimension must be 64, pointers aligned (16 bytes; "
-                   "positions 8), the current device the cache's, and a QK LayerNorm affine finite "
-                   "and within the score bound";
+                   "positions 8), the current device the cache's, and a QK LayerNorm affine finite";
         case VGGT_ERR_SHAPE: return "VGGT_ERR_SHAPE: invalid sizes";
         case VGGT_ERR_ALLOC: return "VGGT_ERR_ALLOC: scratch allocation failed";
         case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA: CUDA call or launch failed";
         case VGGT_ERR_TIMEOUT: return "VGGT_ERR_TIMEOUT: a bounded device wait ran out";
         case VGGT_ERR_RANGE:
             return "VGGT_ERR_RANGE: an attention row sum was not a positive finite number "
-                   "(q_hat/k_hat outside the core's norm bound)";
+                   "(q_hat/k_hat outside vggt_attn_core's norm bound; vggt_attn_core_online takes any)";
         default: return "unknown vggt_status";
     }
 }

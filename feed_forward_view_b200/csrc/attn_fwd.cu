@@ -41,6 +41,23 @@
 // kernel reports a row sum that is not a positive finite number in the
 // status word, for callers that feed the core other vectors.)
 //
+// Online softmax (the kOnline instance), for inputs without that bound -- a
+// QK LayerNorm with a large learned scale or shift, or any vectors given to
+// the core directly. Each row keeps a reference maximum m (log2 units) and
+// evaluates p = 2^(score * log2(e) / 8 - m) (FlashAttention's running
+// maximum, VGGT slides section V). The reference moves lazily: only when a
+// block's maximum exceeds it by more than kRescaleLog2, so that p <= 2^8 in
+// between and most blocks need no rescaling at all. When it moves, the
+// thread rescales its part of [O | l] in TMEM by 2^(m_old - m_new) after the
+// previous PV MMA has finished and before it releases the next one. The two
+// softmax warps of a lane quarter hold the two halves of the same rows, and a
+// row's two threads must use the same m: per block each writes its half's
+// maximum to shared memory and arrives on the quarter's pair barrier, then
+// reads the other's after the barrier completes; both then take the same
+// decisions from the same values. Q stays unscaled in TMEM (no bf16
+// re-rounding of large scores); the scale by log2(e)/8 is part of the
+// packed FMA that subtracts m.
+//
 // Row sums on the tensor core: the PV MMA's B operand is 80 columns wide --
 // V_j (64 columns) followed by a constant shared-memory tile whose first
 // column is 1 and the rest 0 (the descriptor's leading byte offset points
@@ -144,6 +161,14 @@ static_assert(kBN / 16 == 6 && kHeadDim / 16 == 4,
 
 constexpr float kScaleLog2 = 0.125f * 1.4426950408889634f;  // log2(e) / sqrt(64)
 
+// Online instance: the reference maximum moves only when a block's maximum
+// exceeds it by more than this (log2 units), so every p stays <= 2^8 and the
+// fp32 sums of up to 2^21 such terms far from overflow. Exponents on the FMA
+// pipe are floored at kFmaFloor (the polynomial's exponent arithmetic holds
+// for x >= -125; 2^-120 is nothing beside the row's largest term, >= 1).
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kFmaFloor = -120.0f;
+
 // Exponentials per key block: of every 8 consecutive score pairs,
 // kExp2OnFma pairs are evaluated on the FMA pipe (polynomial below) and the
 // rest with the MUFU ex2 instruction, so that the two units share the work.
@@ -176,8 +201,19 @@ struct SharedStorage {
     int abort;
 };
 
-constexpr size_t kSmemBytes = sizeof(SharedStorage) + 1024;  // + alignment slack
-static_assert(kSmemBytes <= 227 * 1024, "shared memory beyond the per-CTA limit");
+// Online instance only, placed after SharedStorage: per (tile, lane quarter)
+// the pair barrier of its two softmax warps and their block maxima, double
+// buffered by block parity ([tile][quarter][parity][half][lane]).
+struct OnlineShared {
+    uint64_t bar_pair[2][4];
+    float xchg[2][4][2][2][32];
+};
+
+template <bool kOnline>
+constexpr size_t smem_bytes() {
+    return sizeof(SharedStorage) + (kOnline ? sizeof(OnlineShared) : 0) + 1024;  // + alignment slack
+}
+static_assert(smem_bytes<true>() <= 227 * 1024, "shared memory beyond the per-CTA limit");
 
 struct Params {
     const uint16_t* q_hat;  // head-major, head planes q_stride rows apart
@@ -306,12 +342,43 @@ __device__ __forceinline__ void exp_pack_row_mufu(const float (&s)[kCols], uint3
     for (int c = 0; c < kPairs; ++c) pk[c] = pack_bf16x2(ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]));
 }
 
+// Online instance: the largest of the thread's scores (masked ones -inf).
+__device__ __forceinline__ float row_max(const float (&s)[kCols]) {
+    float m = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+    for (int c = 3; c + 1 < kCols; c += 2) m = fmax3(m, s[c], s[c + 1]);
+    if constexpr (kCols % 2 == 0) m = fmaxf(m, s[kCols - 1]);
+    return m;
+}
+
+// Online instance: x = score * log2(e)/8 - m in place, one packed FMA per
+// pair; kFloor: the pairs the FMA-pipe polynomial takes are floored at
+// kFmaFloor (not for the masked last block, which uses MUFU alone and whose
+// -inf must stay -inf).
+template <bool kFloor>
+__device__ __forceinline__ void shift_scores(float (&s)[kCols], float m) {
+    const uint64_t c2 = f2_pack(kScaleLog2, kScaleLog2);
+    const uint64_t nm2 = f2_pack(-m, -m);
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c) f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), c2, nm2), s[2 * c], s[2 * c + 1]);
+    if constexpr (kFloor) {
+#pragma unroll
+        for (int k = 0; k < kFmaPairs; ++k) {
+            const int c = fma_pair(k);
+            s[2 * c] = fmaxf(s[2 * c], kFmaFloor);
+            s[2 * c + 1] = fmaxf(s[2 * c + 1], kFmaFloor);
+        }
+    }
+}
+
+template <bool kOnline>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const Params prm) {
     extern __shared__ uint8_t smem_raw[];
     SharedStorage& sm = *reinterpret_cast<SharedStorage*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    OnlineShared& on = *reinterpret_cast<OnlineShared*>(&sm + 1);  // online instance only
 
     // The warp index and the TMEM base go through a lane-0 shuffle so that the
     // compiler knows them to be warp-uniform: everything derived from them
@@ -369,6 +436,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_init(bar_pfree(t), 1);
             mbar_init(bar_o(t), 1);
             mbar_init(bar_tok(t), 1);
+        }
+        if constexpr (kOnline) {
+            for (int t = 0; t < 2; ++t)
+                for (int qr = 0; qr < 4; ++qr) mbar_init(smem_u32(&on.bar_pair[t][qr]), kColSplit);
         }
         sm.abort = 0;
         fence_barrier_init();
@@ -528,10 +599,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                     for (int i = 0; i < kQWords / 4; ++i) {
                         const uint4 w = __ldg(src + i);
-                        qr[4 * i] = scale_bf16x2(w.x);
-                        qr[4 * i + 1] = scale_bf16x2(w.y);
-                        qr[4 * i + 2] = scale_bf16x2(w.z);
-                        qr[4 * i + 3] = scale_bf16x2(w.w);
+                        if constexpr (kOnline) {  // unscaled: the shift applies log2(e)/8 in fp32
+                            qr[4 * i] = w.x;
+                            qr[4 * i + 1] = w.y;
+                            qr[4 * i + 2] = w.z;
+                            qr[4 * i + 3] = w.w;
+                        } else {
+                            qr[4 * i] = scale_bf16x2(w.x);
+                            qr[4 * i + 1] = scale_bf16x2(w.y);
+                            qr[4 * i + 2] = scale_bf16x2(w.z);
+                            qr[4 * i + 3] = scale_bf16x2(w.w);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -542,6 +620,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_q(t));
             }
+            // Online instance: the row's reference maximum (log2 units), its
+            // pair barrier and the shared-memory slots of its two halves.
+            float m_ref = -INFINITY;
+            const uint32_t bar_pair = kOnline ? smem_u32(&on.bar_pair[t][quarter]) : 0u;
+            float* const x_mine = &on.xchg[t][quarter][0][half][lane];  // + 64 per block parity
+            const int x_other = 32 - 64 * half;                         // the other half's slot
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
                 if (!uwait(bar_s(t), j & 1)) {
@@ -555,6 +639,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     tmem_load(lane_base + col_s(t) + kCols * half, r);
 #pragma unroll
                     for (int i = 0; i < kCols; ++i) s[i] = __uint_as_float(r[i]);
+                }
+                const bool masked = j == nkb - 1 && last_valid < kBN;
+                float mx = 0.0f;
+                if constexpr (kOnline) {
+                    // this half's block maximum, over the keys that exist
+                    if (masked) {
+                        const int valid = last_valid - kCols * half;
+#pragma unroll
+                        for (int c = 0; c < kCols; ++c)
+                            if (c >= valid) s[c] = -INFINITY;
+                    }
+                    mx = row_max(s);
+                    if constexpr (kColSplit == 2) {
+                        x_mine[64 * (j & 1)] = mx;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_pair);
+                    }
                 }
                 // The scores are in registers and P_{t,j-1} is in TMEM: S_t may
                 // take S_{t,j+1} and PV_{t,j-1} may run. S_{t,j+1} reads K_{j+1}:
@@ -573,11 +674,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_c(t));
                 uint32_t pk[kPairs];
-                if (j == nkb - 1 && last_valid < kBN) {
-                    const int valid = last_valid - kCols * half;  // of this thread's columns
+                // online: the factor that brings [O | l] to a moved reference
+                // (< 2^-8 when it moved, else exactly 1)
+                float alpha = 1.0f;
+                if constexpr (kOnline) {
+                    if constexpr (kColSplit == 2) {
+                        // the other half's maximum of the same rows
+                        if (!uwait(bar_pair, j & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        mx = fmaxf(mx, x_mine[64 * (j & 1) + x_other]);
+                    }
+                    const float mx2 = mx * kScaleLog2;
+                    if (mx2 > m_ref + kRescaleLog2) {  // always at j == 0 (m_ref = -inf)
+                        if (j > 0) alpha = ex2_approx(m_ref - mx2);
+                        m_ref = mx2;
+                    }
+                    if (masked)
+                        shift_scores<false>(s, m_ref);
+                    else
+                        shift_scores<true>(s, m_ref);
+                }
+                if (masked) {
+                    if constexpr (!kOnline) {
+                        const int valid = last_valid - kCols * half;  // of this thread's columns
 #pragma unroll
-                    for (int c = 0; c < kCols; ++c)
-                        if (c >= valid) s[c] = -INFINITY;
+                        for (int c = 0; c < kCols; ++c)
+                            if (c >= valid) s[c] = -INFINITY;
+                    }
                     exp_pack_row_mufu(s, pk);
                 } else {
                     exp_pack_row_mixed(s, pk);
@@ -589,6 +714,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
                 tc_fence_after();
                 tmem_store(lane_base + col_p(t) + kPairs * half, pk);
+                if constexpr (kOnline) {
+                    // [O | l] holds blocks 0..j-1 against the old reference (P is
+                    // stored, so its registers are free):
+                    // bring this thread's part of it to the new one before
+                    // PV_{t,j} adds block j (released by the next bar_c arrival).
+                    if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+                        const float a = alpha;
+                        if constexpr (kColSplit == 2) {
+                            // dims [32*half, +32) and column 64 + half (l, or a zero column)
+                            const uint32_t o0 = lane_base + col_o(t) + 32u * half;
+                            const uint32_t o1 = lane_base + col_o(t) + kHeadDim + half;
+                            uint32_t o[33];
+                            tmem_ld32_1(o0, o1, o);
+#pragma unroll
+                            for (int i = 0; i < 33; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+                            tmem_st32_1(o0, o1, o);
+                        } else {
+                            uint32_t o[kOCols];
+                            tmem_ld80(lane_base + col_o(t), o);
+#pragma unroll
+                            for (int i = 0; i < kOCols; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+                            tmem_st80(lane_base + col_o(t), o);
+                        }
+                    }
+                }
             }
             if (ok) {
                 // P of the last block is in TMEM (there is no next S to read).
@@ -666,27 +816,29 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
         !make_map(&tm_v, p.v, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
         return cudaErrorInvalidValue;
 
-    // Set once per device; host threads that race here both set the same
-    // attribute, and the flag is published atomically.
-    static std::atomic<bool> attr_set[64];
+    // Set once per device and instance; host threads that race here both set
+    // the same attribute, and the flag is published atomically.
+    static std::atomic<bool> attr_set[2][64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev].load(std::memory_order_acquire)) {
+    const void* kernel = p.online ? reinterpret_cast<const void*>(attn_fwd_kernel<true>)
+                                  : reinterpret_cast<const void*>(attn_fwd_kernel<false>);
+    const size_t smem = p.online ? smem_bytes<true>() : smem_bytes<false>();
+    if (!attr_set[p.online][dev].load(std::memory_order_acquire)) {
         // The register split (setmaxnreg) needs the full launch allocation
         // (kLaunchRegs per thread); with fewer registers the softmax
         // warpgroups' increase could never be granted. Refuse to launch such
         // a build.
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
+        e = cudaFuncGetAttributes(&fa, kernel);
         if (e != cudaSuccess) return e;
         if (static_cast<uint32_t>(fa.numRegs) * kThreads < 128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax)
             return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kSmemBytes));
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        attr_set[dev].store(true, std::memory_order_release);
+        attr_set[p.online][dev].store(true, std::memory_order_release);
     }
     Params prm;
     prm.q_hat = p.q_hat;
@@ -712,7 +864,10 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
 #endif
     prm.pairs_per_seg = (n_qtiles + prm.tiles_per_cta - 1) / prm.tiles_per_cta;
     dim3 grid(p.n_seg * prm.pairs_per_seg, p.H);
-    attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_v, prm);
+    if (p.online)
+        attn_fwd_kernel<true><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, prm);
+    else
+        attn_fwd_kernel<false><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, prm);
     return cudaPeekAtLastError();
 }
 

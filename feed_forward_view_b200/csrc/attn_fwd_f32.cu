@@ -23,6 +23,13 @@
 // kernel does with degree 3, measured 1.4% slower here: with three or six
 // products per useful one the tensor pipe, not MUFU, is the busiest unit.)
 //
+// The same kernel serves bf16 calls whose QK LayerNorm affine makes the
+// scores too large for a bf16 q_hat / k_hat to resolve (an element's
+// rounding, 2^-9 of it, moves a score by about 2^-9 |q_hat| |k_hat| / 8; with
+// weights of 8 that is several units): Q and K in two terms, as above, but P
+// and V in one (the bf16 v itself), the bf16 output of O / l, and the online
+// softmax (kTQ = 2, kTP = 1).
+//
 // One CTA per 128-row query tile of one head. Warps: 0 TMA producer for the
 // K terms of 96 keys, 2 for the V terms (separate rings: 4 + 4 slots for two
 // terms, 3 + 2 for three), 1 MMA issuer, 3 idle, 4-11 softmax (2 per TMEM
@@ -33,7 +40,12 @@
 // loading S_j the softmax warps arrive on bar_c (P_{j-1} written, S free; the
 // first warp has checked that K_{j+1} landed), and on that signal the issuer
 // issues PV_{j-1} and S_{j+1}. No row maximum either: the prologue bounds
-// every score to [-8, 8] (see attn_fwd.cu).
+// every score to [-8, 8] (see attn_fwd.cu). The kOnline instance, for a QK
+// LayerNorm affine without that bound, keeps a running row maximum exactly as
+// the bf16 kernel's online instance does (the two warps of a row swap their
+// block maxima through shared memory; the reference moves only when a block's
+// maximum exceeds it by more than 8 in log2 units); a move rescales the
+// current [O | l] run and, once it holds something, the folded sum.
 //
 // Every wait is bounded; on timeout the CTA records it in the device status
 // word, stops issuing, drains what it has in flight and frees its tensor
@@ -60,21 +72,30 @@ constexpr int kThreads = 128 + 32 * kSoftmaxWarps;  // 384
 constexpr int kCols = 48;                           // score columns per softmax thread
 constexpr uint32_t kTmemCols = 512;
 
-// Per term count: the K and V ring depths (separate rings, each with its own
-// producer warp, so that a slot of either frees on its own MMA) and the tensor
-// memory columns. Two terms: 4 + 4 slots of 2 tiles; three terms: 3 + 2 slots
-// of 3 tiles (a third V slot does not fit beside them in 227 KB).
-template <int kTerms>
+// Per term counts -- kTQ for Q and K (the score product), kTP for P and V
+// (the value product): the K and V ring depths (separate rings, each with its
+// own producer warp, so that a slot of either frees on its own MMA) and the
+// tensor memory columns.
+//   fp32 mode, two terms (kTQ = kTP = 2): 4 + 4 slots of 2 tiles;
+//   three terms (3, 3): 3 + 2 slots of 3 tiles (a third V slot does not fit
+//   beside them in 227 KB);
+//   precise scores for bf16 calls (2, 1): 4 K slots of 2 tiles, 6 V slots of
+//   one tile (the bf16 v itself); P in one bf16 term and a bf16 output, so the
+//   value product needs no fold.
+template <int kTQ, int kTP>
 struct Cfg {
-    static_assert(kTerms == 2 || kTerms == 3, "two or three bf16 terms");
-    static constexpr int kStagesK = kTerms == 2 ? 4 : 3;
-    static constexpr int kStagesV = kTerms == 2 ? 4 : 2;
-    static constexpr int kPairs = kTerms * (kTerms + 1) / 2;  // term products kept
-    static constexpr uint32_t kColQ = 0;                      // 32 per term
-    static constexpr uint32_t kColS = 32 * kTerms;
-    static constexpr uint32_t kColP = kColS + kBN;            // 48 per term
-    static constexpr uint32_t kColO = kColP + (kBN / 2) * kTerms;
-    static constexpr uint32_t kColA = kColO + kOCols;         // the folded partial sums
+    static_assert((kTQ == 2 || kTQ == 3) && (kTP == kTQ || (kTQ == 2 && kTP == 1)), "term counts");
+    static constexpr int kStagesK = kTQ == 2 ? 4 : 3;
+    static constexpr int kStagesV = kTP == 1 ? 6 : (kTP == 2 ? 4 : 2);
+    static constexpr int kPairsS = kTQ * (kTQ + 1) / 2;   // term products kept in S
+    static constexpr int kPairsPV = kTP * (kTP + 1) / 2;  // and in [O | l]
+    static constexpr bool kFoldOn = kTP > 1;              // fp32 outputs: fold every kFold blocks
+    static constexpr bool kBf16Out = kTP == 1;
+    static constexpr uint32_t kColQ = 0;                  // 32 per term
+    static constexpr uint32_t kColS = 32 * kTQ;
+    static constexpr uint32_t kColP = kColS + kBN;        // 48 per term
+    static constexpr uint32_t kColO = kColP + (kBN / 2) * kTP;
+    static constexpr uint32_t kColA = kColO + kOCols;     // the folded partial sums
     static_assert(kColA + kOCols <= kTmemCols, "tensor memory columns");
 };
 
@@ -121,11 +142,11 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
         : "memory");
 }
 
-template <int kTerms>
+template <int kTQ, int kTP>
 struct SharedStorage {
-    using C = Cfg<kTerms>;
-    uint8_t k[C::kStagesK][kTerms][kTileBytes];  // K terms, 128B-swizzled
-    uint8_t v[C::kStagesV][kTerms][kTileBytes];  // V terms, 128B-swizzled
+    using C = Cfg<kTQ, kTP>;
+    uint8_t k[C::kStagesK][kTQ][kTileBytes];  // K terms, 128B-swizzled
+    uint8_t v[C::kStagesV][kTP][kTileBytes];  // V terms, 128B-swizzled
     uint8_t ones[kTileBytes];                    // [1, 0, ..., 0] per key row, 128B-swizzled
     uint64_t bar_kfull[C::kStagesK];
     uint64_t bar_kempty[C::kStagesK];
@@ -139,11 +160,21 @@ struct SharedStorage {
     uint32_t tmem_base;
     int abort;
 };
-template <int kTerms>
+// Online instance only, placed after SharedStorage: per lane quarter the pair
+// barrier of its two softmax warps and their block maxima, double buffered by
+// block parity ([quarter][parity][half][lane]).
+struct OnlineShared {
+    uint64_t bar_pair[4];
+    float xchg[4][2][2][32];
+};
+constexpr float kRescaleLog2 = 8.0f;  // see attn_fwd.cu
+
+template <int kTQ, int kTP, bool kOnline>
 constexpr size_t smem_bytes() {
-    return sizeof(SharedStorage<kTerms>) + 1024;  // + alignment slack
+    return sizeof(SharedStorage<kTQ, kTP>) + (kOnline ? sizeof(OnlineShared) : 0) + 1024;  // + alignment slack
 }
-static_assert(smem_bytes<2>() <= 227 * 1024 && smem_bytes<3>() <= 227 * 1024,
+static_assert(smem_bytes<2, 2, true>() <= 227 * 1024 && smem_bytes<3, 3, true>() <= 227 * 1024 &&
+                  smem_bytes<2, 1, true>() <= 227 * 1024,
               "shared memory beyond the per-CTA limit");
 
 // The TMA maps of the K terms (head-major planes) and the V terms
@@ -155,12 +186,13 @@ struct Maps {
 
 struct Params {
     const float* q_hat;  // fp32, head planes q_stride rows apart
-    float* out;          // [n_seg*q_len, H, 64]
+    void* out;           // [n_seg*q_len, H, 64], fp32 (or bf16 when kTP == 1)
     int* status;
     long long wait_limit;
     long long q_stride;
     int q_len, k_len, H;
     int tiles_per_seg;
+    RowMap out_map;      // query row r is stored at output row map_row(out_map, r)
 };
 
 // The kTerms bf16 terms of two fp32 values, each packed low half first: one
@@ -178,14 +210,15 @@ __device__ __forceinline__ void split_terms(float a, float b, uint32_t (&w)[kTer
     }
 }
 
-template <int kTerms>
+template <int kTQ, int kTP, bool kOnline>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
-    using C = Cfg<kTerms>;
+    using C = Cfg<kTQ, kTP>;
     constexpr int kSK = C::kStagesK, kSV = C::kStagesV;
     extern __shared__ uint8_t smem_raw[];
-    SharedStorage<kTerms>& sm = *reinterpret_cast<SharedStorage<kTerms>*>(
+    SharedStorage<kTQ, kTP>& sm = *reinterpret_cast<SharedStorage<kTQ, kTP>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    OnlineShared& on = *reinterpret_cast<OnlineShared*>(&sm + 1);  // online instance only
 
     const int warp = __shfl_sync(0xFFFFFFFFu, static_cast<int>(threadIdx.x >> 5), 0);
     const int lane = threadIdx.x & 31;
@@ -212,8 +245,8 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
     auto bar_kempty = [&](int s) { return bar_kempty0 + 8u * s; };
     auto bar_vfull = [&](int s) { return bar_vfull0 + 8u * s; };
     auto bar_vempty = [&](int s) { return bar_vempty0 + 8u * s; };
-    auto k_tile = [&](int s, int t) { return k_smem0 + static_cast<uint32_t>(kTileBytes) * (kTerms * s + t); };
-    auto v_tile = [&](int s, int t) { return v_smem0 + static_cast<uint32_t>(kTileBytes) * (kTerms * s + t); };
+    auto k_tile = [&](int s, int t) { return k_smem0 + static_cast<uint32_t>(kTileBytes) * (kTQ * s + t); };
+    auto v_tile = [&](int s, int t) { return v_smem0 + static_cast<uint32_t>(kTileBytes) * (kTP * s + t); };
 
     attn::fill_ones_tile(sm.ones, kTileBytes, kThreads);
     fence_proxy_async_smem();
@@ -232,13 +265,15 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
         mbar_init(bar_c, kSoftmaxWarps);
         mbar_init(bar_pfree, 1);
         mbar_init(bar_o, 1);
+        if constexpr (kOnline) {
+            for (int qr = 0; qr < 4; ++qr) mbar_init(smem_u32(&on.bar_pair[qr]), 2);
+        }
         sm.abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     if ((warp == 0 || warp == 2) && lane == 0) {
-#pragma unroll
-        for (int t = 0; t < kTerms; ++t) tma_prefetch_desc(warp == 0 ? &maps.k[t] : &maps.v[t]);
+        for (int t = 0; t < (warp == 0 ? kTQ : kTP); ++t) tma_prefetch_desc(warp == 0 ? &maps.k[t] : &maps.v[t]);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
@@ -261,14 +296,14 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
                 const uint32_t use = j / n_st;
                 const uint32_t full = is_k ? bar_kfull(s) : bar_vfull(s);
                 if (use > 0 && !wait(is_k ? bar_kempty(s) : bar_vempty(s), (use - 1) & 1)) break;
-                mbar_arrive_expect_tx(full, kTerms * kTileBytes);
+                mbar_arrive_expect_tx(full, (is_k ? kTQ : kTP) * kTileBytes);
                 const int row = k_row0 + j * kBN;
+                if (is_k) {
 #pragma unroll
-                for (int t = 0; t < kTerms; ++t) {
-                    if (is_k)
-                        tma_load_3d(k_tile(s, t), &maps.k[t], full, 0, row, h);
-                    else
-                        tma_load_3d(v_tile(s, t), &maps.v[t], full, 0, h, row);
+                    for (int t = 0; t < kTQ; ++t) tma_load_3d(k_tile(s, t), &maps.k[t], full, 0, row, h);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < kTP; ++t) tma_load_3d(v_tile(s, t), &maps.v[t], full, 0, h, row);
                 }
                 ++n_issued;
             }
@@ -292,7 +327,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             if (elect_one()) {
                 tc_fence_after();
 #pragma unroll
-                for (int i = 0; i < C::kPairs; ++i) {
+                for (int i = 0; i < C::kPairsS; ++i) {
                     const uint64_t kd = smem_desc_sw128(k_tile(s, pair_b(i)), 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -314,14 +349,15 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             if (elect_one()) {
                 tc_fence_after();
 #pragma unroll
-                for (int i = 0; i < C::kPairs; ++i) {
+                for (int i = 0; i < C::kPairsPV; ++i) {
                     const int b = pair_b(i);
                     const uint64_t vd = b == 0 ? smem_desc_sw128(v0_addr, ones_smem - v0_addr, 1024)
                                                : smem_desc_sw128(v_tile(s, b), 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 6; ++kk)
                         mma_ts(o_tm, p_tm + 48 * pair_a(i) + 8 * kk, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4),
-                               b == 0 ? idesc_o : idesc_o64, (j % kFold != 0 || i > 0 || kk > 0) ? 1u : 0u);
+                               b == 0 ? idesc_o : idesc_o64,
+                               ((C::kFoldOn ? j % kFold != 0 : j > 0) || i > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar_pfree);
                 mma_commit(bar_vempty(s));
@@ -354,36 +390,42 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
         const bool row_live = row_in_seg < prm.q_len;
         const long long grow = static_cast<long long>(seg) * prm.q_len + row_in_seg;
         // Q into tensor memory: this thread's 32 dims of its row, scaled by
-        // log2(e)/8 in fp32, as kTerms bf16 terms (16 columns each).
+        // log2(e)/8 in fp32, as kTQ bf16 terms (16 columns each).
         {
-            uint32_t qt[kTerms][16];
+            uint32_t qt[kTQ][16];
             if (row_live) {
                 const float4* src = reinterpret_cast<const float4*>(
                     prm.q_hat + (static_cast<long long>(h) * prm.q_stride + grow) * kHeadDim + 32 * half);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 w = __ldg(src + i);
-                    uint32_t a[kTerms], b[kTerms];
-                    split_terms<kTerms>(w.x * kScaleLog2, w.y * kScaleLog2, a);
-                    split_terms<kTerms>(w.z * kScaleLog2, w.w * kScaleLog2, b);
+                    uint32_t a[kTQ], b[kTQ];
+                    split_terms<kTQ>(w.x * kScaleLog2, w.y * kScaleLog2, a);
+                    split_terms<kTQ>(w.z * kScaleLog2, w.w * kScaleLog2, b);
 #pragma unroll
-                    for (int t = 0; t < kTerms; ++t) {
+                    for (int t = 0; t < kTQ; ++t) {
                         qt[t][2 * i] = a[t];
                         qt[t][2 * i + 1] = b[t];
                     }
                 }
             } else {
 #pragma unroll
-                for (int t = 0; t < kTerms; ++t)
+                for (int t = 0; t < kTQ; ++t)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) qt[t][i] = 0u;
             }
 #pragma unroll
-            for (int t = 0; t < kTerms; ++t) tmem_st16(lane_base + C::kColQ + 32 * t + 16 * half, qt[t]);
+            for (int t = 0; t < kTQ; ++t) tmem_st16(lane_base + C::kColQ + 32 * t + 16 * half, qt[t]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_q);
         }
+        // online instance: the row's reference maximum (log2 units), the
+        // quarter's pair barrier and this half's exchange slot
+        float m_ref = -INFINITY;
+        const uint32_t bar_pair = kOnline ? smem_u32(&on.bar_pair[quarter]) : 0u;
+        float* const x_mine = &on.xchg[quarter][0][half][lane];  // + 64 per block parity
+        const int x_other = 32 - 64 * half;                      // the other half's slot
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
             if (!uwait(bar_s, j & 1)) {
@@ -398,6 +440,23 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
 #pragma unroll
                 for (int i = 0; i < kCols; ++i) s[i] = __uint_as_float(r[i]);
             }
+            float mx = 0.0f;
+            if constexpr (kOnline) {
+                // this half's block maximum over the keys that exist
+                if (j == nkb - 1 && last_valid < kBN) {
+                    const int valid = last_valid - kCols * half;
+#pragma unroll
+                    for (int c = 0; c < kCols; ++c)
+                        if (c >= valid) s[c] = -INFINITY;
+                }
+                mx = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+                for (int c = 3; c + 1 < kCols; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+                mx = fmaxf(mx, s[kCols - 1]);
+                x_mine[64 * (j & 1)] = mx;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_pair);
+            }
             if (quarter == 0 && half == 0 && j + 1 < nkb &&
                 !uwait(bar_kfull((j + 1) % kSK), ((j + 1) / kSK) & 1)) {
                 ok = false;
@@ -406,18 +465,36 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_c);
-            if (j == nkb - 1 && last_valid < kBN) {
+            if (!kOnline && j == nkb - 1 && last_valid < kBN) {
                 const int valid = last_valid - kCols * half;
 #pragma unroll
                 for (int c = 0; c < kCols; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
-            uint32_t pt[kTerms][kCols / 2];
-            auto put = [&](int c, float pa, float pb) {
-                uint32_t w[kTerms];
-                split_terms<kTerms>(pa, pb, w);
+            // online: the factor that brings the sums to a moved reference
+            // (< 2^-8 when it moved, else exactly 1)
+            float alpha = 1.0f;
+            if constexpr (kOnline) {
+                if (!uwait(bar_pair, j & 1)) {
+                    ok = false;
+                    break;
+                }
+                mx = fmaxf(mx, x_mine[64 * (j & 1) + x_other]);
+                if (mx > m_ref + kRescaleLog2) {  // always at j == 0 (m_ref = -inf)
+                    if (j > 0) alpha = ex2_approx(m_ref - mx);
+                    m_ref = mx;
+                }
+                const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
-                for (int t = 0; t < kTerms; ++t) pt[t][c] = w[t];
+                for (int c = 0; c < kCols / 2; ++c)
+                    f2_unpack(f2_add(f2_pack(s[2 * c], s[2 * c + 1]), nm2), s[2 * c], s[2 * c + 1]);
+            }
+            uint32_t pt[kTP][kCols / 2];
+            auto put = [&](int c, float pa, float pb) {
+                uint32_t w[kTP];
+                split_terms<kTP>(pa, pb, w);
+#pragma unroll
+                for (int t = 0; t < kTP; ++t) pt[t][c] = w[t];
             };
 #pragma unroll
             for (int c = 0; c < kCols / 2; ++c) put(c, ex2_approx(s[2 * c]), ex2_approx(s[2 * c + 1]));  // 2^-inf = 0
@@ -426,7 +503,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
                 break;
             }
             tc_fence_after();
-            if (j > 0 && j % kFold == 0) {
+            if (C::kFoldOn && j > 0 && j % kFold == 0) {
                 // PV_{j-1} closed a run of kFold blocks: fold [O | l] into the
                 // sum (the first fold copies); PV_j then starts afresh. The l
                 // column (64) is the same for both halves: half 0 folds it.
@@ -445,7 +522,27 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
                 }
             }
 #pragma unroll
-            for (int t = 0; t < kTerms; ++t) tmem_st24(lane_base + C::kColP + 48 * t + (kCols / 2) * half, pt[t]);
+            for (int t = 0; t < kTP; ++t) tmem_st24(lane_base + C::kColP + 48 * t + (kCols / 2) * half, pt[t]);
+            if constexpr (kOnline) {
+                // Blocks 0..j-1 are in the current run of [O | l] (unless a
+                // fold just closed it: PV_j then starts afresh) and, from the
+                // first fold on, in the folded sum: bring both to the new
+                // reference before PV_j (released by the next bar_c arrival).
+                // This thread's part: dims [32*half, +32) and column 64 + half
+                // (l, or a zero column).
+                if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+                    for (int which = 0; which < (C::kFoldOn ? 2 : 1); ++which) {
+                        if (C::kFoldOn && which == 0 && j % kFold == 0) continue;  // the run was folded away
+                        if (which == 1 && j < kFold) continue;                     // nothing folded yet
+                        const uint32_t base = lane_base + (which == 0 ? C::kColO : C::kColA);
+                        uint32_t o[33];
+                        tmem_ld32_1(base + 32u * half, base + kHeadDim + half, o);
+#pragma unroll
+                        for (int i = 0; i < 33; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32_1(base + 32u * half, base + kHeadDim + half, o);
+                    }
+                }
+            }
         }
         if (ok) {
             tc_fence_before();
@@ -456,7 +553,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             tc_fence_after();
             uint32_t o[33];  // this thread's 32 output dims and l (column 64)
             tmem_ld32_1(lane_base + C::kColO + 32 * half, lane_base + C::kColO + kHeadDim, o);
-            if (nkb > kFold) {  // plus the folded sum
+            if (C::kFoldOn && nkb > kFold) {  // plus the folded sum
                 uint32_t a[33];
                 tmem_ld32_1(lane_base + C::kColA + 32 * half, lane_base + C::kColA + kHeadDim, a);
 #pragma unroll
@@ -465,11 +562,26 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             const float l = __uint_as_float(o[32]);
             if (row_live) {
                 if (!(l > 0.0f && l <= 3.0e38f)) atomicOr(prm.status, kStatusRange);
-                float4* dst = reinterpret_cast<float4*>(prm.out + (grow * prm.H + h) * kHeadDim + 32 * half);
+                const long long orow = map_row(prm.out_map, grow);
+                if constexpr (C::kBf16Out) {
+                    // bf16 output (round to nearest even) of o / l
+                    const float inv = 1.0f / l;
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(prm.out) + (orow * prm.H + h) * kHeadDim +
+                                                          32 * half);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(__fdiv_rn(__uint_as_float(o[4 * i]), l), __fdiv_rn(__uint_as_float(o[4 * i + 1]), l),
-                                         __fdiv_rn(__uint_as_float(o[4 * i + 2]), l), __fdiv_rn(__uint_as_float(o[4 * i + 3]), l));
+                    for (int i = 0; i < 4; ++i) {
+                        const float* f = reinterpret_cast<const float*>(&o[8 * i]);
+                        dst[i] = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                                            pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+                    }
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(prm.out) + (orow * prm.H + h) * kHeadDim +
+                                                            32 * half);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__fdiv_rn(__uint_as_float(o[4 * i]), l), __fdiv_rn(__uint_as_float(o[4 * i + 1]), l),
+                                             __fdiv_rn(__uint_as_float(o[4 * i + 2]), l), __fdiv_rn(__uint_as_float(o[4 * i + 3]), l));
+                }
             }
         }
     }
@@ -484,38 +596,40 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
 
 // ---------------------------------------------------------------- host
 
-template <int kTerms>
+template <int kTQ, int kTP, bool kOnline>
 cudaError_t launch_terms(const AttnProblemF32& p, const Params& prm, cudaStream_t stream) {
     const uint64_t nk = static_cast<uint64_t>(p.n_seg) * p.k_len;
     const uint64_t row_bytes = kHeadDim * 2;
     const uint64_t ks = static_cast<uint64_t>(p.k_stride);
     Maps maps{};
-    for (int t = 0; t < kTerms; ++t)
-        if (!make_map(&maps.k[t], p.k[t], ks, p.H, row_bytes, ks * row_bytes, kBN, 1) ||
-            !make_map(&maps.v[t], p.v[t], p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
-            return cudaErrorInvalidValue;
-    // Set once per device; host threads that race here both set the same
-    // attribute, and the flag is published atomically.
+    for (int t = 0; t < kTQ; ++t)
+        if (!make_map(&maps.k[t], p.k[t], ks, p.H, row_bytes, ks * row_bytes, kBN, 1)) return cudaErrorInvalidValue;
+    for (int t = 0; t < kTP; ++t)
+        if (!make_map(&maps.v[t], p.v[t], p.H, nk, row_bytes, p.H * row_bytes, 1, kBN)) return cudaErrorInvalidValue;
+    // Set once per device (per instance); host threads that race here both set
+    // the same attribute, and the flag is published atomically.
     static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_set[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(attn_fwd_f32_kernel<kTerms>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem_bytes<kTerms>()));
+        e = cudaFuncSetAttribute(attn_fwd_f32_kernel<kTQ, kTP, kOnline>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_bytes<kTQ, kTP, kOnline>()));
         if (e != cudaSuccess) return e;
         attr_set[dev].store(true, std::memory_order_release);
     }
     dim3 grid(p.n_seg * prm.tiles_per_seg, p.H);
-    attn_fwd_f32_kernel<kTerms><<<grid, kThreads, smem_bytes<kTerms>(), stream>>>(maps, prm);
+    attn_fwd_f32_kernel<kTQ, kTP, kOnline><<<grid, kThreads, smem_bytes<kTQ, kTP, kOnline>(), stream>>>(maps, prm);
     return cudaPeekAtLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention_f32(const AttnProblemF32& p, int* status, long long wait_limit, cudaStream_t stream) {
+    const int tp = p.terms_pv == 0 ? p.terms : p.terms_pv;
     if (p.terms != 2 && p.terms != 3) return cudaErrorInvalidValue;
+    if (tp != p.terms && !(p.terms == 2 && tp == 1 && p.online)) return cudaErrorInvalidValue;
     if (p.n_seg <= 0 || p.H <= 0 || p.q_len <= 0 || p.k_len <= 0) return cudaSuccess;
     Params prm;
     prm.q_hat = p.q_hat;
@@ -527,7 +641,10 @@ cudaError_t launch_attention_f32(const AttnProblemF32& p, int* status, long long
     prm.k_len = p.k_len;
     prm.H = p.H;
     prm.tiles_per_seg = (p.q_len + kBM - 1) / kBM;
-    return p.terms == 3 ? launch_terms<3>(p, prm, stream) : launch_terms<2>(p, prm, stream);
+    prm.out_map = p.out_map;
+    if (tp == 1) return launch_terms<2, 1, true>(p, prm, stream);
+    if (p.online) return p.terms == 3 ? launch_terms<3, 3, true>(p, prm, stream) : launch_terms<2, 2, true>(p, prm, stream);
+    return p.terms == 3 ? launch_terms<3, 3, false>(p, prm, stream) : launch_terms<2, 2, false>(p, prm, stream);
 }
 
 }  // namespace vggt

@@ -22,7 +22,9 @@
 // position with the prologue's own arithmetic (prologue.cuh), writing the
 // head-major k_hat the attention kernel reads. The pooled keys never reach
 // memory, and the result is bit-identical to pooling then running the
-// prologue.
+// prologue. Precise fused mode (calls whose QK LayerNorm affine needs more
+// score precision than bf16 keys give) skips the bf16 rounding of the pooled
+// keys, normalises the fp32 means and writes k_hat as two bf16 terms.
 //
 // Memory-bound: every input byte of K and V is read once, the pooled tokens
 // are written once. One 256-thread block per pooled token: 128 threads pool
@@ -108,7 +110,8 @@ __device__ __forceinline__ void add8x2(uint64_t (&acc)[4], uint2 lo, uint2 hi) {
 }
 
 // kFused: keys normalised and rotated into k_hat (else pooled into k_out);
-// kAffine: the key LayerNorm has an affine. Separate instantiations keep the
+// kAffine: the key LayerNorm has an affine; kPrecise (fused only): fp32 means
+// into the prologue, two-term k_hat. Separate instantiations keep the
 // plain pooling at its register count. Four resident blocks per SM (<= 64
 // registers a thread) measured fastest: occupancy decides this memory-bound
 // kernel more than the few registers it then spills.
@@ -119,7 +122,7 @@ __device__ __forceinline__ void add8x2(uint64_t (&acc)[4], uint2 lo, uint2 hi) {
 // keep the member order). Warp 0 first gathers the pooled position; in fused
 // mode it hands it to the key warps through named barrier 1 (the value warps
 // never wait).
-template <bool kFused, bool kAffine>
+template <bool kFused, bool kAffine, bool kPrecise>
 __global__ void __launch_bounds__(kThreads, 4)
 kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
     __shared__ float2 pooled_pos;
@@ -235,7 +238,8 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
             named_bar_sync(kKeyBar, kKeyBarThreads);  // pooled_pos and the staged affine
             prologue::token_angles(pooled_pos, lane, prologue::lane_freq(freq, lane), sv, cv);
         }
-        // the pooled keys as stored (bf16), then the prologue
+        // the pooled keys as stored (bf16; precise mode: the fp32 means), then
+        // the prologue
         float x1[4], x2[4];
         if (src.copy) {
             x1[0] = prologue::bf16_lo(c_lo.x); x1[1] = prologue::bf16_hi(c_lo.x);
@@ -248,18 +252,24 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
             for (int e = 0; e < 4; ++e) f2_unpack(acc[e], m[2 * e], m[2 * e + 1]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                x1[e] = __bfloat162float(__float2bfloat16_rn(m[e]));
-                x2[e] = __bfloat162float(__float2bfloat16_rn(m[4 + e]));
+                x1[e] = kPrecise ? m[e] : __bfloat162float(__float2bfloat16_rn(m[e]));
+                x2[e] = kPrecise ? m[4 + e] : __bfloat162float(__float2bfloat16_rn(m[4 + e]));
             }
         }
-        uint16_t* out = job.k_hat + (static_cast<size_t>(h) * job.k_hat_stride + dst) * kHeadDim;
-        prologue::norm_rotate_store<kAffine>(x1, x2, aff, sv, cv, live, out, d1);
+        const size_t orow = (static_cast<size_t>(h) * job.k_hat_stride + dst) * kHeadDim;
+        if constexpr (kPrecise) {
+            float r1[4], r2[4];
+            prologue::norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, r1, r2);
+            if (live) prologue::store_two_terms(job.k_hat + orow, job.k_hat_lo + orow, d1, r1, r2);
+        } else {
+            prologue::norm_rotate_store<kAffine>(x1, x2, aff, sv, cv, live, job.k_hat + orow, d1);
+        }
     }
 }
 
-template <bool kFused, bool kAffine>
+template <bool kFused, bool kAffine, bool kPrecise = false>
 cudaError_t launch_pool_kernel(const PoolJob& job, unsigned blocks, cudaStream_t stream) {
-    kv_pool_kernel<kFused, kAffine><<<blocks, kThreads, 0, stream>>>(job, rope_freq_table());
+    kv_pool_kernel<kFused, kAffine, kPrecise><<<blocks, kThreads, 0, stream>>>(job, rope_freq_table());
     return cudaPeekAtLastError();
 }
 
@@ -272,6 +282,9 @@ cudaError_t launch_kv_pool(const PoolJob& job, cudaStream_t stream) {
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
     const unsigned b = static_cast<unsigned>(blocks);
     if (job.k_hat == nullptr) return launch_pool_kernel<false, false>(job, b, stream);
+    if (job.k_hat_lo != nullptr)
+        return job.k_ln.on ? launch_pool_kernel<true, true, true>(job, b, stream)
+                           : launch_pool_kernel<true, false, true>(job, b, stream);
     return job.k_ln.on ? launch_pool_kernel<true, true>(job, b, stream)
                        : launch_pool_kernel<true, false>(job, b, stream);
 }

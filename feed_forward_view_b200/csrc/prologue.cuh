@@ -135,6 +135,21 @@ __device__ __forceinline__ void norm_rotate_store(float (&x1)[4], float (&x2)[4]
     }
 }
 
+// The prologue results o1 (dims d1..d1+3) and o2 (d1+16..d1+19) as two bf16
+// terms: y_0 = bf16(y) at hi + d1 (+16), y_1 = bf16(y - y_0) at lo + d1
+// (+16); y - y_0 is exact in fp32.
+__device__ __forceinline__ void store_two_terms(uint16_t* hi, uint16_t* lo, int d1, const float (&o1)[4],
+                                                const float (&o2)[4]) {
+    const uint32_t a0 = pack2(o1[0], o1[1]), a1 = pack2(o1[2], o1[3]);
+    const uint32_t b0 = pack2(o2[0], o2[1]), b1 = pack2(o2[2], o2[3]);
+    *reinterpret_cast<uint2*>(hi + d1) = make_uint2(a0, a1);
+    *reinterpret_cast<uint2*>(hi + d1 + 16) = make_uint2(b0, b1);
+    *reinterpret_cast<uint2*>(lo + d1) =
+        make_uint2(pack2(o1[0] - bf16_lo(a0), o1[1] - bf16_hi(a0)), pack2(o1[2] - bf16_lo(a1), o1[3] - bf16_hi(a1)));
+    *reinterpret_cast<uint2*>(lo + d1 + 16) =
+        make_uint2(pack2(o2[0] - bf16_lo(b0), o2[1] - bf16_hi(b0)), pack2(o2[2] - bf16_lo(b1), o2[3] - bf16_hi(b1)));
+}
+
 // This lane's RoPE frequency 100^(-(lane%16)/16), chosen from the table with
 // constant indices (no local memory).
 __device__ __forceinline__ float lane_freq(const FreqTable& freq, int lane) {

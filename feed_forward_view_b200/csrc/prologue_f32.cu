@@ -15,7 +15,9 @@
 // The prologue arithmetic (prologue.cuh) is the bf16 path's, fed with fp32
 // inputs. (LayerNorm: "Norm: Layer Normalization" slide; RoPE base 100 and
 // eps 1e-5: the VGGT-Omega config.json table; frequency schedule:
-// "Positional Encoding (4/6)" slide.)
+// "Positional Encoding (4/6)" slide.) The same kernel also takes bf16 inputs:
+// bf16 calls whose QK LayerNorm affine enlarges the scores beyond what a bf16
+// q_hat / k_hat resolves carry q_hat in fp32 and k_hat as two bf16 terms.
 //
 // Memory-bound; one warp per token as in the bf16 prologue, each lane loading
 // its 8 dims of a head as two 16-byte pieces.
@@ -56,22 +58,34 @@ __device__ __forceinline__ void store_terms(const PrologueJobF32& job, size_t ro
     }
 }
 
-template <bool kAffine>
+template <bool kAffine, bool kBf16In>
 __device__ __forceinline__ void process_token_f32(const PrologueJobF32& job, const float* aff, int t, int H,
                                                   int lane, float my_freq) {
     const int d1 = prologue::lane_dim(lane);
-    const float* xt = job.x + static_cast<size_t>(t) * H * kHeadDim;
+    const long long src = map_row(job.in_map, t);
     float sv[4], cv[4];
-    prologue::token_angles(reinterpret_cast<const float2*>(job.pos)[t], lane, my_freq, sv, cv);
+    prologue::token_angles(reinterpret_cast<const float2*>(job.pos)[src], lane, my_freq, sv, cv);
     for (int h0 = 0; h0 < H; h0 += 4) {  // a warp covers 4 heads
         const int h = h0 + (lane >> 3);
         const bool live = h < H;
         float x1[4] = {0.f, 0.f, 0.f, 0.f}, x2[4] = {0.f, 0.f, 0.f, 0.f};
         if (live) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(xt + h * kHeadDim + d1));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(xt + h * kHeadDim + d1 + 16));
-            x1[0] = a.x; x1[1] = a.y; x1[2] = a.z; x1[3] = a.w;
-            x2[0] = b.x; x2[1] = b.y; x2[2] = b.z; x2[3] = b.w;
+            const size_t off = (static_cast<size_t>(src) * H + h) * kHeadDim + d1;
+            if constexpr (kBf16In) {
+                const uint16_t* xt = static_cast<const uint16_t*>(job.x) + off;
+                const uint2 a = __ldg(reinterpret_cast<const uint2*>(xt));
+                const uint2 b = __ldg(reinterpret_cast<const uint2*>(xt + 16));
+                x1[0] = prologue::bf16_lo(a.x); x1[1] = prologue::bf16_hi(a.x);
+                x1[2] = prologue::bf16_lo(a.y); x1[3] = prologue::bf16_hi(a.y);
+                x2[0] = prologue::bf16_lo(b.x); x2[1] = prologue::bf16_hi(b.x);
+                x2[2] = prologue::bf16_lo(b.y); x2[3] = prologue::bf16_hi(b.y);
+            } else {
+                const float* xt = static_cast<const float*>(job.x) + off;
+                const float4 a = __ldg(reinterpret_cast<const float4*>(xt));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(xt + 16));
+                x1[0] = a.x; x1[1] = a.y; x1[2] = a.z; x1[3] = a.w;
+                x2[0] = b.x; x2[1] = b.y; x2[2] = b.z; x2[3] = b.w;
+            }
         }
         float o1[4], o2[4];
         prologue::norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, o1, o2);
@@ -89,7 +103,7 @@ __device__ __forceinline__ void process_token_f32(const PrologueJobF32& job, con
     }
 }
 
-template <bool kAffA, bool kAffB>
+template <bool kAffA, bool kAffB, bool kBf16In>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 qk_prologue_f32_kernel(const __grid_constant__ PrologueJobF32 a, const __grid_constant__ PrologueJobF32 b, int H,
                        FreqTable freq) {
@@ -104,9 +118,9 @@ qk_prologue_f32_kernel(const __grid_constant__ PrologueJobF32 a, const __grid_co
     if (kAffA || kAffB) __syncthreads();
     for (int i = warp; i < total; i += nwarps) {
         if (i < a.n)
-            process_token_f32<kAffA>(a, aff_a, i, H, lane, my_freq);
+            process_token_f32<kAffA, kBf16In>(a, aff_a, i, H, lane, my_freq);
         else
-            process_token_f32<kAffB>(b, aff_b, i - a.n, H, lane, my_freq);
+            process_token_f32<kAffB, kBf16In>(b, aff_b, i - a.n, H, lane, my_freq);
     }
 }
 
@@ -140,8 +154,12 @@ cudaError_t launch_qk_prologue_f32(const PrologueJobF32& a, const PrologueJobF32
     const int sms = sm_count();
     int blocks = (total + kWarpsPerBlock - 1) / kWarpsPerBlock;
     blocks = blocks < sms * 8 ? blocks : sms * 8;
-    auto kernel = a.ln.on ? (b.ln.on ? qk_prologue_f32_kernel<true, true> : qk_prologue_f32_kernel<true, false>)
-                          : (b.ln.on ? qk_prologue_f32_kernel<false, true> : qk_prologue_f32_kernel<false, false>);
+    if (b.n > 0 && b.x_bf16 != a.x_bf16) return cudaErrorInvalidValue;
+    auto kernel = a.x_bf16
+        ? (a.ln.on ? (b.ln.on ? qk_prologue_f32_kernel<true, true, true> : qk_prologue_f32_kernel<true, false, true>)
+                   : (b.ln.on ? qk_prologue_f32_kernel<false, true, true> : qk_prologue_f32_kernel<false, false, true>))
+        : (a.ln.on ? (b.ln.on ? qk_prologue_f32_kernel<true, true, false> : qk_prologue_f32_kernel<true, false, false>)
+                   : (b.ln.on ? qk_prologue_f32_kernel<false, true, false> : qk_prologue_f32_kernel<false, false, false>));
     kernel<<<blocks, kWarpsPerBlock * 32, 0, stream>>>(a, b, H, rope_freq_table());
     return cudaPeekAtLastError();
 }

@@ -392,6 +392,22 @@ __device__ __forceinline__ void tmem_ld32_1(uint32_t taddr, uint32_t taddr1, uin
         : "r"(taddr), "r"(taddr1)
         : "memory");
 }
+// Stores 32 consecutive columns at taddr and one more column at taddr1, and
+// waits for completion.
+__device__ __forceinline__ void tmem_st32_1(uint32_t taddr, uint32_t taddr1, const uint32_t (&r)[33]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33};\n\t"
+        "tcgen05.st.sync.aligned.32x32b.x1.b32 [%1], {%34};\n\t"
+        "tcgen05.wait::st.sync.aligned;"
+        :
+        : "r"(taddr), "r"(taddr1),
+          "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]),
+          "r"(r[32])
+        : "memory");
+}
 // 24 consecutive columns (x16 + x8), waited for.
 __device__ __forceinline__ void tmem_st24(uint32_t taddr, const uint32_t (&r)[24]) {
     asm volatile(

@@ -83,18 +83,24 @@ struct FrameLayout {
     }
 };
 
-// fp32 mode. One fp32 tensor x [n, H, 64] (positions pos [n, 2]) through the
-// prologue; out head-major at row t of head h: (h * out_stride + t) * 64.
-// terms == 0: fp32 results to out[0]; terms == 2 or 3: that many bf16 terms
-// (y_0 = bf16(y), y_1 = bf16(y - y_0), y_2 = bf16(y - y_0 - y_1)) to out[0..].
+// The prologue with fp32 or term-split results (the fp32 mode, and bf16 calls
+// whose affine needs more score precision). One tensor x [., H, 64] (fp32, or
+// bf16 when x_bf16; positions pos [., 2]) through the prologue; n rows out,
+// head-major: row t of head h at (h * out_stride + t) * 64, read from token
+// map_row(in_map, t) of x and pos. terms == 0: fp32 results to out[0];
+// terms == 2 or 3: that many bf16 terms (y_0 = bf16(y), y_1 = bf16(y - y_0),
+// y_2 = bf16(y - y_0 - y_1)) to out[0..]. Both jobs of a launch take the same
+// input type.
 struct PrologueJobF32 {
-    const float* x;
+    const void* x;
     const float* pos;
     void* out[3];
     int n;
     long long out_stride;
     LnAffine ln;
     int terms;
+    bool x_bf16 = false;
+    RowMap in_map;
 };
 cudaError_t launch_qk_prologue_f32(const PrologueJobF32& a, const PrologueJobF32& b, int H,
                                    cudaStream_t stream);
@@ -102,22 +108,29 @@ cudaError_t launch_qk_prologue_f32(const PrologueJobF32& a, const PrologueJobF32
 cudaError_t launch_split_bf16(const float* x, uint16_t* const (&out)[3], int terms, long long n,
                               cudaStream_t stream);
 
-// fp32-mode attention: segments as in AttnProblem; q_hat fp32 head-major
-// (plane stride q_stride), the bf16 terms of k_hat head-major (plane stride
-// k_stride) and of v [n_seg*k_len, H, 64], out fp32 [n_seg*q_len, H, 64];
-// terms 2 or 3.
+// Attention on term-split operands: segments as in AttnProblem; q_hat fp32
+// head-major (plane stride q_stride), the bf16 terms of k_hat head-major
+// (plane stride k_stride) and of v [n_seg*k_len, H, 64].
+//   terms == terms_pv (2 or 3): the fp32 mode; out fp32 [n_seg*q_len, H, 64].
+//   terms == 2, terms_pv == 1: bf16 calls that need precise scores; q_hat and
+//   k_hat in two terms, P and v in one (v[0] = the bf16 v), out bf16, online
+//   softmax required.
+// Query row r is stored at output row map_row(out_map, r).
 struct AttnProblemF32 {
     const float* q_hat;
     const uint16_t* k[3];
     const uint16_t* v[3];
     int terms;
-    float* out;
+    void* out;
     int n_seg;
     int q_len;
     int k_len;
     int H;
     long long q_stride;
     long long k_stride;
+    bool online = false;  // running row maximum, as in AttnProblem
+    int terms_pv = 0;     // 0: the same as terms
+    RowMap out_map;
 };
 cudaError_t launch_attention_f32(const AttnProblemF32& p, int* status, long long wait_limit,
                                  cudaStream_t stream);
@@ -133,7 +146,9 @@ cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, long long n, 
 // [S*Tk,2]. Keys either pooled the same way into k_out (k_hat == nullptr), or
 // (k_out == nullptr) pooled, normalised (k_ln) and rotated at their pooled
 // position, and written head-major: pooled row r of head h at
-// k_hat + (h * k_hat_stride + r) * 64.
+// k_hat + (h * k_hat_stride + r) * 64. With k_hat_lo set as well (precise
+// mode), the pooled keys stay fp32 means (no bf16 rounding) before the
+// prologue, whose results go out as two bf16 terms: k_hat and k_hat_lo.
 struct PoolJob {
     const uint16_t* k;
     const uint16_t* v;
@@ -141,6 +156,7 @@ struct PoolJob {
     uint16_t* k_out;
     uint16_t* k_hat;
     long long k_hat_stride;
+    uint16_t* k_hat_lo = nullptr;
     uint16_t* v_out;
     float* pos_out;
     int S, T;
@@ -168,6 +184,9 @@ struct AttnProblem {
     long long q_stride;
     long long k_stride;
     RowMap out_map;  // output row of query row r: map_row(out_map, r)
+    // Softmax with a running row maximum (any finite inputs) instead of the
+    // maximum-free form, which needs |score| * log2(e) within about 2^6.
+    bool online = false;
 };
 
 // Returns cudaSuccess, or an error from tensor-map encoding or the launch.

@@ -88,8 +88,7 @@ typedef enum vggt_status {
     VGGT_ERR_NULL = -1,        /* a required pointer is NULL                      */
     VGGT_ERR_UNSUPPORTED = -2, /* D != 64, a misaligned pointer, a cache used on
                                   another device than its own, or a QK LayerNorm
-                                  affine that is not finite or exceeds the score
-                                  bound (see vggt_qk_norm)                         */
+                                  affine that is not finite (see vggt_qk_norm)    */
     VGGT_ERR_SHAPE = -3,       /* negative sizes, T != 5 + g*g (plain calls) or a
                                   layout that does not add up to T, bad kv_down, or
                                   a size beyond the library's limits              */
@@ -101,8 +100,8 @@ typedef enum vggt_status {
                                   vggt_get_device_status)                          */
     VGGT_ERR_RANGE = -7        /* an attention row's softmax sum was not a positive
                                   finite number: vggt_attn_core was given vectors
-                                  outside its norm bound (reported by
-                                  vggt_get_device_status)                          */
+                                  outside its norm bound (use vggt_attn_core_online
+                                  for those; reported by vggt_get_device_status)  */
 } vggt_status;
 
 /* Number of special (camera + register) tokens at the head of every frame. */
@@ -178,6 +177,21 @@ VGGT_API int vggt_qk_prologue(const vggt_bf16* x, const float* pos, vggt_bf16* x
 VGGT_API int vggt_attn_core(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
                             vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
                             cudaStream_t stream);
+
+/*
+ * vggt_attn_core for any finite q_hat and k_hat: the softmax keeps a running
+ * row maximum (FlashAttention's online softmax, "Attention" slides of the
+ * VGGT paper-report deck, Section V) and rescales the row's sums only when
+ * that maximum grows by more than 2^8 in exp2 terms. Same arguments, layouts
+ * and rules as vggt_attn_core; no norm bound. Unlike vggt_attn_core it keeps
+ * q_hat exactly as given (the core scales q_hat by log2(e)/8 and rounds it to
+ * bf16 once more), so scores are exact fp32 dot products of the bf16 inputs.
+ * Slower than vggt_attn_core (a shared-memory exchange of block maxima per
+ * key block). Takes no scratch.
+ */
+VGGT_API int vggt_attn_core_online(const vggt_bf16* q_hat, const vggt_bf16* k_hat, const vggt_bf16* v,
+                                   vggt_bf16* out, int n_seg, int q_len, int k_len, int H, int D,
+                                   cudaStream_t stream);
 
 /*
  * Per-frame K/V descriptors (FlashVGGT README: "spatially resampling keys and
@@ -279,13 +293,19 @@ typedef struct vggt_frame_layout {
  * LayerNorm carries; the pages give none, so without it there is no affine).
  * Separate arrays for queries and keys; each is a HOST array of D fp32
  * values or NULL (weight 1, bias 0), read during the call (no reference is
- * kept). Values must be finite.
- * Score bound: the attention kernel evaluates exp(score) without a row
- * maximum (exact up to rounding: softmax ignores a common factor), which
- * needs every score bounded. With Bq = 8 * max|q_weight| + ||q_bias||_2 (a
- * bound on the norm of a normalised query, the plain LayerNorm's being below
- * 8) and Bk likewise, a call needs Bq * Bk / 8 * log2(e) * 1.01 <= 64 (e.g.
- * weights up to 2.3 with zero bias); beyond it returns VGGT_ERR_UNSUPPORTED.
+ * kept). Values must be finite; any finite values are accepted.
+ * Which softmax runs: with Bq = 8 * max|q_weight| + ||q_bias||_2 (a bound on
+ * the norm of a normalised query, the plain LayerNorm's being below 8) and Bk
+ * likewise, every score is at most Bq * Bk / 8 in magnitude. While
+ * Bq * Bk / 8 * log2(e) * 1.01 <= 64 (e.g. weights up to 2.3 with zero bias)
+ * the attention kernel evaluates exp(score) without a row maximum (exact up
+ * to rounding: softmax ignores a common factor); beyond it the kernel keeps a
+ * running row maximum and rescales its sums when it grows (online softmax).
+ * Both give the same result up to rounding. Large affines make the scores
+ * large, and the normalised q and k are stored in bf16 (relative rounding
+ * 2^-9 per element), so a score's error grows with Bq * Bk: results stay
+ * close to exact only while that error (about 2^-9 * |q_hat| * |k_hat| / 8)
+ * is small beside the gaps between a row's largest scores.
  */
 typedef struct vggt_qk_norm {
     const float* q_weight;

@@ -235,6 +235,28 @@ def ln_affine(seed: int, scale: float = 0.5, shift: float = 0.2, D: int = HEAD_D
     return (w(), b(), w(), b())
 
 
+def ln_affine_large(seed: int, max_weight: float = 8.0, bias_norm: float = 4.0, D: int = HEAD_DIM):
+    """A seeded QK LayerNorm affine with large entries ``(q_weight, q_bias,
+    k_weight, k_bias)``: weights of random sign and log-uniform magnitude in
+    [0.5, max_weight], one of them exactly max_weight; biases N(0, 1) scaled
+    to Euclidean norm ``bias_norm``. fp32 CPU tensors."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(30_000 + int(seed))
+
+    def weight():
+        mag = torch.exp(math.log(0.5) + (math.log(max_weight) - math.log(0.5)) * torch.rand(D, generator=gen))
+        sign = torch.where(torch.rand(D, generator=gen) < 0.5, -1.0, 1.0)
+        w = mag * sign
+        w[int(torch.randint(D, (1,), generator=gen))] = max_weight
+        return w
+
+    def bias():
+        b = torch.randn(D, generator=gen)
+        return b * (bias_norm / float(b.norm()))
+
+    return (weight(), bias(), weight(), bias())
+
+
 def make_sequence_qkv(S: int, layout, n_extra: int, seed: int, H: int = HEADS, D: int = HEAD_DIM):
     """``make_layout_qkv`` plus ``n_extra`` sequence tokens after the frames
     (positions (0,0)), drawn from their own generators."""

@@ -101,13 +101,18 @@ def test_pool_and_prologue_argument_checks():
 
 
 def test_core_argument_checks():
+    for name in ("vggt_attn_core", "vggt_attn_core_online"):
+        _core_checks(getattr(F.lib, name))
+
+
+def _core_checks(fn):
     p = [FAKE] * 4
-    assert F.lib.vggt_attn_core(*p, 1, 100, 100, 16, 32, None) == E_UNSUP
-    assert F.lib.vggt_attn_core(*p, -1, 100, 100, 16, 64, None) == E_SHAPE
-    assert F.lib.vggt_attn_core(*p, 1, 1 << 22, 100, 16, 64, None) == E_SHAPE
-    assert F.lib.vggt_attn_core(None, *p[1:], 1, 100, 100, 16, 64, None) == E_NULL
-    assert F.lib.vggt_attn_core(FAKE + 4, *p[1:], 1, 100, 100, 16, 64, None) == E_UNSUP
-    assert F.lib.vggt_attn_core(None, None, None, None, 1, 0, 100, 16, 64, None) == OK
+    assert fn(*p, 1, 100, 100, 16, 32, None) == E_UNSUP
+    assert fn(*p, -1, 100, 100, 16, 64, None) == E_SHAPE
+    assert fn(*p, 1, 1 << 22, 100, 16, 64, None) == E_SHAPE
+    assert fn(None, *p[1:], 1, 100, 100, 16, 64, None) == E_NULL
+    assert fn(FAKE + 4, *p[1:], 1, 100, 100, 16, 64, None) == E_UNSUP
+    assert fn(None, None, None, None, 1, 0, 100, 16, 64, None) == OK
 
 
 def test_binding_rejects_host_tensors():
@@ -176,20 +181,21 @@ def test_ex_descriptor_layout_checks():
     assert _ex_call(d, 1374, kd=0) == E_SHAPE
 
 
-def test_ln_affine_bound_and_finiteness():
+def test_ln_affine_any_finite_values():
+    # Any finite affine is accepted (large ones run the online softmax); only
+    # non-finite weights or biases are refused.
     g = F.lib.vggt_attn_global_ex
     w = lambda c: [c] * 64  # noqa: E731
     assert _ex_call(g, 100, ln=(w(2.0), None, w(2.0), None)) == OK
-    assert _ex_call(g, 100, ln=(w(2.3), None, w(2.3), None)) == OK
-    assert _ex_call(g, 100, ln=(w(2.4), None, w(2.4), None)) == E_UNSUP
-    assert _ex_call(g, 100, ln=(w(-2.4), None, None, None)) == OK        # only the product is bounded
-    # one side alone: Bq * 8 / 8 * log2(e) * 1.01 <= 64 up to Bq = 43.9
-    assert _ex_call(g, 100, ln=(w(5.0), None, None, None)) == OK          # Bq = 40
-    assert _ex_call(g, 100, ln=(w(6.0), None, None, None)) == E_UNSUP     # Bq = 48
-    assert _ex_call(g, 100, ln=(None, w(4.0), None, None)) == OK          # Bq = 8 + ||bias|| = 40
-    assert _ex_call(g, 100, ln=(None, w(5.0), None, None)) == E_UNSUP     # Bq = 48
+    assert _ex_call(g, 100, ln=(w(2.4), None, w(2.4), None)) == OK
+    assert _ex_call(g, 100, ln=(w(-60.0), w(8.0), w(40.0), w(-3.0))) == OK
+    assert _ex_call(g, 100, ln=(w(1e30), None, None, None)) == OK
     assert _ex_call(g, 100, ln=(w(float("nan")), None, None, None)) == E_UNSUP
     assert _ex_call(g, 100, ln=(None, None, None, w(float("inf")))) == E_UNSUP
+    assert _ex_call(g, 100, ln=(None, w(float("-inf")), None, None)) == E_UNSUP
+    one_nan = w(1.0)
+    one_nan[37] = float("nan")
+    assert _ex_call(g, 100, ln=(None, None, one_nan, None)) == E_UNSUP
     # the prologue alone has no score bound, only finiteness
     wp, keep = F._host_f32(w(50.0), "w")
     assert F.lib.vggt_qk_prologue_ex(FAKE, FAKE, FAKE, 0, 16, 64, wp, None, None) == OK
@@ -217,7 +223,7 @@ def test_descriptor_cache_ex_checks_before_allocating():
     c = F.lib.vggt_desc_cache_create_ex
     assert c(ctypes.byref(h), 10, 5 + 25 * 37, 16, 64, 4, None, None) == E_SHAPE
     assert not h.value
-    norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
+    norm, keep = F._norm(([3.0] * 64, None, [float("nan")] * 64, None))
     assert c(ctypes.byref(h), 10, 5 + 25 * 37, 16, 64, 4, F._layout((5, 25, 37, 0)), norm) == E_UNSUP
     assert not h.value
 
@@ -237,7 +243,7 @@ def test_subset_argument_checks():
     assert s(*args(2, 10, 0, 0, H=0)) == OK
     assert s(FAKE, None, FAKE, FAKE, FAKE, 2, 10, 0, 0, 16, 64, 1, None, None) == E_NULL
     assert s(FAKE, FAKE, FAKE + 8, FAKE, FAKE, 2, 10, 0, 0, 16, 64, 1, None, None) == E_UNSUP
-    norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
+    norm, keep = F._norm(([3.0] * 64, None, [float("inf")] * 64, None))
     assert s(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 0, 0, 16, 64, 1, norm, None) == E_UNSUP
 
 
@@ -250,7 +256,7 @@ def test_f32_mode_argument_checks():
             assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 32, None, terms, None) == E_UNSUP
             assert fn(FAKE, None, FAKE, FAKE, FAKE, 2, 10, 16, 64, None, terms, None) == E_NULL
             assert fn(FAKE, FAKE, FAKE + 8, FAKE, FAKE, 2, 10, 16, 64, None, terms, None) == E_UNSUP
-            norm, keep = F._norm(([3.0] * 64, None, [3.0] * 64, None))
+            norm, keep = F._norm(([3.0] * 64, [float("nan")] * 64, None, None))
             assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 64, norm, terms, None) == E_UNSUP
         for terms in (0, 1, 4, -1):  # only two or three bf16 terms
             assert fn(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 16, 64, None, terms, None) == E_UNSUP

@@ -178,10 +178,11 @@ def test_stream_with_layout_and_affine(F):
     check(out, ref, "stream ex")
 
 
-def test_affine_at_the_score_bound(F):
-    # weights 2.3 on queries and keys (the largest the bound admits with no
-    # bias) and k = q: every query's own key scores |q_hat|^2 / 8 ~ 42, about
-    # 61 in log2 units -- exponentials near 2^61 without a row maximum
+def test_affine_with_dominant_self_scores(F):
+    # weights 2.3 on queries and keys and k = q: every query's own key scores
+    # |q_hat|^2 / 8 ~ 42 (about 61 in log2 units) against ~N(0, 5) for the
+    # others; the call runs in precise mode (online softmax, two-term
+    # scores)
     S, g = 2, 9
     q, _, v, pos = synth.make_qkv(S, g, seed=48)
     T = 5 + g * g
