@@ -202,7 +202,10 @@ class OracleLeg:
             kp, vp, pp = O.kv_pool(self.k, self.v, self.pos, w.S, w.T, w.kv_down)
             self.k_hat, self.vv = O.qk_prologue(kp, pp), vp
         elif w.kind in ("global", "global_f32"):
-            self.k_hat, self.vv = O.qk_prologue(self.k, self.pos), self.v
+            ln = synth.workload_affine(w)
+            self.ln = None if ln is None else tuple(x.double().numpy() for x in ln)
+            kw, kb = (None, None) if self.ln is None else self.ln[2:]
+            self.k_hat, self.vv = O.qk_prologue(self.k, self.pos, kw, kb), self.v
 
     def run(self, n_rows: int, seed: int = 0):
         """Returns (TFLOP/s, seconds, rows)."""
@@ -227,7 +230,8 @@ class OracleLeg:
             O.attn_subset(self.q, self.k, self.v, self.pos, w.S, w.T, w.skip, w.n_extra, kind, rows=kept[rows])
             keys = w.n_k if kind == "global" else w.T_k
         else:
-            O.cross_attention(O.qk_prologue(self.q[rows], self.pos[rows]), self.k_hat, self.vv)
+            qw, qb = (None, None) if getattr(self, "ln", None) is None else self.ln[:2]
+            O.cross_attention(O.qk_prologue(self.q[rows], self.pos[rows], qw, qb), self.k_hat, self.vv)
             keys = w.n_k
         dt = time.perf_counter() - t0
         return 4.0 * w.H * w.D * rows.size * keys / dt / 1e12, dt, int(rows.size)
@@ -292,23 +296,37 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- GPU arm
 
 
-def run_gpu(args):
-    import torch
+# Every other workload of the pages' shapes, measured after the headline one
+# on the same GPU (N = 1 only) and reported under "secondary": configurations
+# 1, 2, 3 and 5, the streamed descriptors, the VGGT-Omega token layout, the
+# fp32 mode and a large QK LayerNorm affine (precise mode).
+SECONDARY = ("global_s2_g16", "frame_s8_g37", "global_s8_g37", "descriptor_s200_g37_kd4",
+             "stream_s200_g37_kd4_c10", "omega_global_s32_g32", "omega_frame_s32_g32",
+             "global_s9_g64_f32", "global_s9_g64_affine8")
 
-    import feed_forward_view_b200 as F
-    import synth
 
-    rank, local, world = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    w = synth.ALL_WORKLOADS[args.workload]
+def _event_ms(torch, stream, fn, reps: int, warm: int = 3) -> float:
+    """Average device time of fn() over reps launches, CUDA events on stream."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize(stream.device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize(stream.device)
+    return a.elapsed_time(b) / reps
 
-    q_h, k_h, v_h, pos_h = synth.make_workload(w, seed=rank)
-    q, k, v, pos = (t.to(dev) for t in (q_h, k_h, v_h, pos_h))
-    out = torch.empty_like(q)
-    stream = torch.cuda.current_stream(dev)
-    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, pos))
 
+def make_call(F, w, q):
+    """The public call that one step of workload w makes, as call(q, k, v,
+    pos, out); and the kernel launches per step."""
+    ln = None
+    if w.affine >= 0:
+        import synth
+
+        ln = synth.workload_affine(w)
     if w.kind == "stream":
         # the whole sequence through one descriptor cache, chunk by chunk
         cache = F.DescCache(w.S, w.T, H=w.H, kv_down=w.kv_down)
@@ -319,24 +337,46 @@ def run_gpu(args):
             cache.reset()
             for r0, r1, c in chunks:
                 cache.attend(qq[r0:r1], kk[r0:r1], vv[r0:r1], pp[r0:r1], oo[r0:r1], C=c)
-    elif w.kind.endswith("_f32"):
+        return call, 3 * len(chunks)
+    if w.kind.endswith("_f32"):
         fn32 = F.vggt_attn_global_f32 if w.kind == "global_f32" else F.vggt_attn_frame_f32
 
         def call(qq, kk, vv, pp, oo):
             fn32(qq, kk, vv, pp, oo, S=w.S, T=w.T, terms=w.terms)
-    elif w.kind == "global_batch":
+        return call, 3
+    if w.kind == "global_batch":
         def call(qq, kk, vv, pp, oo):
             F.vggt_attn_global_batch(qq, kk, vv, pp, oo, B=w.B, S=w.S, T=w.T)
-    elif w.kind.startswith("subset"):
+        return call, 2
+    if w.kind.startswith("subset"):
         def call(qq, kk, vv, pp, oo):
             F.vggt_attn_subset(qq, kk, vv, pp, oo, S=w.S, T=w.T, n_skip_back=w.skip, n_extra=w.n_extra,
                                kind=w.kind[len("subset_"):])
-    else:
-        fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
-              "descriptor": F.vggt_attn_descriptor}[w.kind]
-
+        return call, 2 + (1 if w.skip else 0)
+    if ln is not None:  # precise mode: query prologue + key prologue in one launch, attention
         def call(qq, kk, vv, pp, oo):
-            fn(qq, kk, vv, pp, oo, S=w.S, T=w.T, kv_down=w.kv_down)
+            F.vggt_attn_global_ex(qq, kk, vv, pp, oo, S=w.S, T=w.T, ln=ln)
+        return call, 2
+    fn = {"global": F.vggt_attn_global, "frame": F.vggt_attn_frame,
+          "descriptor": F.vggt_attn_descriptor}[w.kind]
+
+    def call(qq, kk, vv, pp, oo):
+        fn(qq, kk, vv, pp, oo, S=w.S, T=w.T, kv_down=w.kv_down)
+    return call, 2 + (1 if w.kind == "descriptor" else 0)
+
+
+def measure(F, torch, w, args, dev, stream, world, local, steps, e2e_steps, seed):
+    """One workload: warm-up, `steps` timed steps between barriers (device
+    time, max over ranks), the kernels timed alone, and the host-buffer leg.
+    Returns a dict of the measurements."""
+    import synth
+
+    peaks, _ = load_peaks()
+    q_h, k_h, v_h, pos_h = synth.make_workload(w, seed=seed)
+    q, k, v, pos = (t.to(dev) for t in (q_h, k_h, v_h, pos_h))
+    out = torch.empty_like(q)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, pos))
+    call, launches = make_call(F, w, q)
 
     def step():
         call(q, k, v, pos, out)
@@ -362,7 +402,7 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -371,24 +411,21 @@ def run_gpu(args):
     ms_local = e0.elapsed_time(e1)
     status = F.vggt_get_device_status()
     ms_total = max_over_ranks(ms_local, world, dev)
-    # per call or chunk: the prologue, the pooling fused with the key
-    # prologue (descriptors) or the value gather (subsets that leave tokens
-    # out), the attention
-    if w.kind == "stream":
-        launches = 3 * len(chunks)
-    else:
-        launches = 2 + (1 if w.kind == "descriptor" or (w.kind.startswith("subset") and w.skip) else 0)
-    ms_step = ms_total / args.steps
+    ms_step = ms_total / steps
     flops = w.flops()
-    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
-    tokens_s = world * w.n_q * args.steps / (ms_total * 1e-3)
+    res = {"w": w, "ms_step": ms_step, "warmed": warmed, "launches": launches, "in_bytes": in_bytes,
+           "out_bytes": out.numel() * out.element_size(), "flops": flops,
+           "value": world * flops * steps / (ms_total * 1e-3) / 1e12,
+           "tokens_s": world * w.n_q * steps / (ms_total * 1e-3), "clocks": clocks.summary()}
 
-    # ---- kernel-only timings (same kernels, launched one by one with events);
-    # a streamed sequence is many calls of growing size: there the step itself
-    # stands for the attention kernel
+    # ---- kernel-only timings (same kernels, launched one by one with events).
+    # A streamed sequence is many calls of growing size, and the fp32 and
+    # precise modes' attention kernel has no entry point of its own: there the
+    # step itself stands for the attention kernel.
     H = w.H
     kind_core = "descriptor" if w.kind == "stream" else w.kind
     f32 = w.kind.endswith("_f32")
+    whole_step = w.kind == "stream" or f32 or w.affine >= 0
     q_hat = torch.empty((H, w.n_q, 64), dtype=torch.bfloat16, device=dev)
     nk_rows = w.n_q if w.kind == "global_batch" else w.n_k  # key rows of all segments
     k_hat = torch.empty((H, nk_rows, 64), dtype=torch.bfloat16, device=dev)
@@ -414,69 +451,45 @@ def run_gpu(args):
         n_seg, q_len, k_len = w.B, w.S * w.T, w.S * w.T
     else:
         n_seg, q_len, k_len = 1, w.n_q, w.n_k
-    reps = max(5, min(args.steps, 50))
-    if w.kind == "stream" or f32:
+    reps = max(5, min(steps, 50))
+    if whole_step:
         attn_ms = ms_step
     else:
-        for _ in range(3):
-            F.vggt_attn_core(q_hat, k_hat, v_use, out_b, n_seg, q_len, k_len)
-        torch.cuda.synchronize(dev)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            F.vggt_attn_core(q_hat, k_hat, v_use, out_b, n_seg, q_len, k_len)
-        a1.record(stream)
-        torch.cuda.synchronize(dev)
-        attn_ms = a0.elapsed_time(a1) / reps
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
-    for _ in range(reps):
-        F.vggt_qk_prologue(qb[:w.n_q], pos[:w.n_q], q_hat)
-    p1.record(stream)
-    torch.cuda.synchronize(dev)
-    pro_ms = p0.elapsed_time(p1) / reps
+        attn_ms = _event_ms(torch, stream, lambda: F.vggt_attn_core(q_hat, k_hat, v_use, out_b, n_seg, q_len, k_len),
+                            reps)
+    res["attn_ms"] = attn_ms
+    res["whole_step"] = whole_step
+    hbm = float(peaks["hbm_gbs"])
+
+    def mem(ms, nbytes):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm, "frac_of_datasheet": gbs / DATASHEET_HBM_GBS}
+
+    pro_ms = _event_ms(torch, stream, lambda: F.vggt_qk_prologue(qb[:w.n_q], pos[:w.n_q], q_hat), reps, warm=0)
     pro_bytes = 2 * w.n_q * H * 64 * 2 + w.n_q * 8  # read x + pos, write x_hat
-    pool = fused_keys = None
+    res["kernels"] = {("qk_prologue_bf16_same_shape" if f32 else "qk_prologue"): mem(pro_ms, pro_bytes)}
     if kind_core == "descriptor":
         # K/V pooling alone: reads k, v and pos of every token, writes the
-        # pooled k, v and positions.
+        # pooled k, v and positions; then the pooling fused with the key
+        # prologue (what the call runs): the same bytes, with normalised keys
+        # written instead of pooled ones.
         kp_o, vp_o, pp_o = (torch.empty_like(t) for t in (kp, vp, pp))
-        for _ in range(3):
-            F.vggt_kv_pool(kb, vb, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
-        torch.cuda.synchronize(dev)
-        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        k0.record(stream)
-        for _ in range(reps):
-            F.vggt_kv_pool(kb, vb, pos, S=w.S, T=w.T, kv_down=w.kv_down, k_out=kp_o, v_out=vp_o, pos_out=pp_o)
-        k1.record(stream)
-        torch.cuda.synchronize(dev)
-        pool_ms = k0.elapsed_time(k1) / reps
         pool_bytes = 2 * (w.n_q + w.n_k) * H * 64 * 2 + (w.n_q + w.n_k) * 8
-        pool = {"ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
-                "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]),
-                "frac_of_datasheet": pool_bytes / (pool_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS}
-        # the pooling fused with the key prologue (what the call runs): the
-        # same bytes, with normalised keys written instead of pooled ones
-        for _ in range(3):
-            F.vggt_descriptor_keys(kb, vb, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
-        torch.cuda.synchronize(dev)
-        k0.record(stream)
-        for _ in range(reps):
-            F.vggt_descriptor_keys(kb, vb, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T, kv_down=w.kv_down)
-        k1.record(stream)
-        torch.cuda.synchronize(dev)
-        fk_ms = k0.elapsed_time(k1) / reps
-        fused_keys = {"ms": fk_ms, "gbs": pool_bytes / (fk_ms * 1e-3) / 1e9,
-                      "frac_hbm": pool_bytes / (fk_ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]),
-                      "frac_of_datasheet": pool_bytes / (fk_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS}
+        pool_ms = _event_ms(torch, stream, lambda: F.vggt_kv_pool(kb, vb, pos, S=w.S, T=w.T, kv_down=w.kv_down,
+                                                                  k_out=kp_o, v_out=vp_o, pos_out=pp_o), reps)
+        fk_ms = _event_ms(torch, stream, lambda: F.vggt_descriptor_keys(kb, vb, pos, k_hat, vp_o, pp_o, S=w.S, T=w.T,
+                                                                        kv_down=w.kv_down), reps)
+        res["kernels"]["kv_pool"] = mem(pool_ms, pool_bytes)
+        res["kernels"]["descriptor_keys"] = mem(fk_ms, pool_bytes)
+    del q_hat, k_hat
 
     # ---- end to end through the public call with host buffers: every step
     # uploads its inputs from pinned host memory and reads its output back.
     # Two device buffer sets and two copy streams (one per PCIe direction) let
     # step i+1's upload and step i-1's download run while step i computes, as a
     # caller streaming scenes through the library would.
-    e2e = None
-    if not args.skip_e2e:
+    res["e2e"] = None
+    if e2e_steps > 0:
         hq, hk, hv, hp = (t.pin_memory() for t in (q_h, k_h, v_h, pos_h))
         hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
         dev_in = [[torch.empty_like(t) for t in (q, k, v, pos)] for _ in range(2)]
@@ -525,22 +538,66 @@ def run_gpu(args):
             downloaded[b].record(stream)
         run_e2e(3)
         torch.cuda.synchronize(dev)
-        n_e2e = max(3, min(args.steps, 30))
         barrier(world, dev)
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record(stream)
-        run_e2e(n_e2e)
+        run_e2e(e2e_steps)
         stream.wait_stream(copy_out)  # the last result is on the host
         stream.wait_stream(copy_in)
         x1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, dev) / n_e2e
-        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size(),
-               "ms_per_step": e2e_ms,
-               "overlap": "uploads and downloads double-buffered on one copy stream per direction"}
+        e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, dev) / e2e_steps
+        res["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": res["out_bytes"],
+                      "ms_per_step": e2e_ms,
+                      "overlap": "uploads and downloads double-buffered on one copy stream per direction"}
+    res["status"] = status or F.vggt_get_device_status()
+    return res
 
-    status2 = F.vggt_get_device_status()
+
+def attention_kernel_name(w) -> str:
+    if w.kind == "stream":
+        return "stream step: per chunk pool + prologue + attn_fwd_kernel"
+    if w.kind.endswith("_f32"):
+        return ("fp32-mode step: prologue, operand split, attn_fwd_f32_kernel (flops counted once per pair; the "
+                f"tensor cores run {w.terms * (w.terms + 1) // 2} products)")
+    if w.affine >= 0:
+        return ("precise-mode step: prologue, attn_fwd_f32_kernel with two-term scores and the online softmax "
+                "(flops counted once per pair; the tensor cores run 3 score products)")
+    return "attn_fwd_kernel"
+
+
+def secondary_entry(res, peaks) -> dict:
+    """The compact record of one secondary workload."""
+    w = res["w"]
+    peak = float(peaks["bf16_tflops"])
+    attn_tf = res["flops"] / (res["attn_ms"] * 1e-3) / 1e12
+    return {
+        "kind": w.kind, "tokens": w.n_q,
+        "keys": w.T if w.kind in ("frame", "frame_f32") else (w.T_k if w.kind == "subset_frame" else w.n_k),
+        "flops": res["flops"], "steps": res["steps"],
+        "ms_per_step": res["ms_step"], "tflops": res["value"], "tokens_per_s": res["tokens_s"],
+        "attention": {"kernel": attention_kernel_name(w), "ms": res["attn_ms"], "tflops": attn_tf,
+                      "frac": attn_tf / peak, "frac_of_sustained": attn_tf / float(peaks.get("bf16_tflops_sustained", peak))},
+        "kernels": res["kernels"],
+        "e2e_tflops": res["e2e"]["value"] if res["e2e"] else None,
+        "clocks": res["clocks"], "device_status": res["status"],
+    }
+
+
+def run_gpu(args):
+    import torch
+
+    import feed_forward_view_b200 as F
+    import synth
+
+    rank, local, world = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    w = synth.ALL_WORKLOADS[args.workload]
+    res = measure(F, torch, w, args, dev, stream, world, local, args.steps,
+                  0 if args.skip_e2e else max(3, min(args.steps, 30)), seed=rank)
 
     # ---- CPU oracle baseline (rank 0 at N = 1 only)
     cpu = None
@@ -553,33 +610,46 @@ def run_gpu(args):
                          + ("; pooling and key prologue redone" if w.kind == "stream"
                             else "; key prologue precomputed")}
 
+    # ---- the other workloads, N = 1 only (the headline line's numbers are
+    # already taken; these follow it on the same GPU)
+    secondary = None
+    if world == 1 and not args.no_secondary:
+        peaks, _ = load_peaks()
+        secondary = {}
+        for name in SECONDARY:
+            if name == w.name:
+                continue
+            r = measure(F, torch, synth.ALL_WORKLOADS[name], args, dev, stream, world, local,
+                        args.secondary_steps, 0 if args.skip_e2e else 10, seed=0)
+            r["steps"] = args.secondary_steps
+            secondary[name] = secondary_entry(r, peaks)
+            del r
+            torch.cuda.empty_cache()
+
     if rank == 0:
         peaks, peak_src = load_peaks()
+        flops, attn_ms, ms_step = res["flops"], res["attn_ms"], res["ms_step"]
         attn_tf = flops / (attn_ms * 1e-3) / 1e12
         scores = flops / (4.0 * w.D)  # query-key pairs x heads
         sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
         peak = float(peaks["bf16_tflops"])
         traffic = profiled_traffic(w)
-        clk = clocks.summary()
+        clk = res["clocks"]
+        f32 = w.kind.endswith("_f32")
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": warmed, "ms_per_step": ms_step,
+            "metric": METRIC, "value": res["value"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": res["warmed"], "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": (f"f32 ({w.terms} bf16 terms, {w.terms * (w.terms + 1) // 2} tensor-core products)"
                       if f32 else "bf16"),
             "data": "synthetic",
             "config": {"workload": w.name, "kind": w.kind, "S": w.S, "T": w.T, "tokens": w.n_q,
-                       "keys": w.T if w.kind == "frame" else (w.T_k if w.kind == "subset_frame" else w.n_k), "H": w.H, "D": w.D,
-                       "kv_down": w.kv_down, "parallelism": f"replicas x{world}",
-                       "l2": f"inputs {in_bytes / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
-            "tokens_per_s": tokens_s,
-            "pct_of_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "tensor",
-                         "kernel": ("stream step: per chunk pool + prologue + attn_fwd_kernel"
-                                    if w.kind == "stream" else
-                                    "fp32-mode step: prologue, operand split, attn_fwd_f32_kernel (flops counted "
-                                    f"once per pair; the tensor cores run {w.terms * (w.terms + 1) // 2} products)"
-                                    if f32 else "attn_fwd_kernel"),
+                       "keys": w.T if w.kind == "frame" else (w.T_k if w.kind == "subset_frame" else w.n_k),
+                       "H": w.H, "D": w.D, "kv_down": w.kv_down, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs {res['in_bytes'] / 2**20:.0f} MiB > L2 {L2_BYTES / 2**20:.0f} MiB; no flush"},
+            "tokens_per_s": res["tokens_s"],
+            "pct_of_peak": 100.0 * res["value"] / world / peak,
+            "roofline": {"bound": "tensor", "kernel": attention_kernel_name(w),
                          "achieved": attn_tf,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
                          "peak_source": f"{peak_src} bf16 burst",
@@ -589,22 +659,18 @@ def run_gpu(args):
                          "share_of_step": attn_ms / ms_step},
             # (the fp32 mode's own prologue runs inside its step; the bf16
             # prologue on the same shape is reported for comparison)
-            "kernels": {("qk_prologue_bf16_same_shape" if f32 else "qk_prologue"): {
-                                        "ms": pro_ms, "gbs": pro_bytes / (pro_ms * 1e-3) / 1e9,
-                                        "frac_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
-                                        "frac_of_datasheet": pro_bytes / (pro_ms * 1e-3) / 1e9 / DATASHEET_HBM_GBS},
-                        **({"kv_pool": pool} if pool else {}),
-                        **({"descriptor_keys": fused_keys} if fused_keys else {})},
+            "kernels": res["kernels"],
             # every score costs one exponential: exponentials per second in
             # the attention kernel, and per SM per clock at the sampled clock
             "exp_per_s": scores / (attn_ms * 1e-3),
             "exp_per_sm_clk": (scores / (attn_ms * 1e-3) / (sm_count * clk["sm_mhz"] * 1e6)
                                if clk.get("sm_mhz") else None),
             "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": launches * args.steps,
+            "e2e": res["e2e"],
+            "gpu_launches": res["launches"] * args.steps,
             "clocks": clk,
-            "device_status": status or status2,
+            "device_status": res["status"],
+            "secondary": secondary,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -625,6 +691,9 @@ def main(argv=None):
     ap.add_argument("--reference-budget-s", type=float, default=150.0)
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle leg")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
+    ap.add_argument("--no-secondary", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--secondary-steps", type=int, default=20,
+                    help="timed steps of each secondary workload (N = 1)")
     args = ap.parse_args(argv)
     if args.impl == "native":
         args.warmup = max(args.warmup, 3)  # at least three untimed steps

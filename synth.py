@@ -52,6 +52,7 @@ class Workload:
     n_extra: int = 0          # sequence tokens after the frames ("subset_*")
     B: int = 1                # scenes per call ("global_batch")
     terms: int = 2            # bf16 terms per fp32 operand ("*_f32")
+    affine: int = -1          # seed of a large QK LayerNorm affine (ln_affine_large), -1: none
 
     @property
     def T(self) -> int:
@@ -157,8 +158,19 @@ F32_WORKLOADS = {w.name: w for w in (
 BATCH_WORKLOADS = {w.name: w for w in (
     Workload("global_b32_s2_g16", "global_batch", S=2, g=16, B=32),
 )}
+# The dense global workload with a large QK LayerNorm affine (weights up to 8,
+# bias norm 4): precise mode (two-term scores, online softmax).
+AFFINE_WORKLOADS = {w.name: w for w in (
+    Workload("global_s9_g64_affine8", "global", S=9, g=64, affine=0),
+)}
 ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS, **STREAM_WORKLOADS, **SUBSET_WORKLOADS, **F32_WORKLOADS,
-                 **BATCH_WORKLOADS}
+                 **BATCH_WORKLOADS, **AFFINE_WORKLOADS}
+
+
+def workload_affine(w: Workload):
+    """The workload's QK LayerNorm affine ``(q_weight, q_bias, k_weight,
+    k_bias)`` as fp32 CPU tensors, or None."""
+    return None if w.affine < 0 else ln_affine_large(w.affine)
 
 
 def grid_side(T: int) -> int:

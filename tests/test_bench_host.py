@@ -79,7 +79,8 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
 
 
 @pytest.mark.parametrize("name", ["global_s2_g16", "frame_s8_g37", "descriptor_s200_g37_kd4",
-                                  "omega_frame_s32_g32", "omega_global_s32_g32", "frame_s8_g37_f32"])
+                                  "omega_frame_s32_g32", "omega_global_s32_g32", "frame_s8_g37_f32",
+                                  "global_s9_g64_affine8"])
 def test_oracle_leg_runs_on_a_small_sample(name):
     import synth
 
@@ -88,3 +89,19 @@ def test_oracle_leg_runs_on_a_small_sample(name):
         pytest.skip("large setup; covered by the reference arm")
     tf, dt, rows = bench.OracleLeg(w).run(8)
     assert tf > 0 and dt > 0 and rows >= 8
+
+
+def test_secondary_workloads_are_known_and_exclude_nothing_of_the_pages_shapes():
+    import synth
+
+    assert all(n in synth.ALL_WORKLOADS for n in bench.SECONDARY)
+    # every configuration of the pages' shapes is either the headline or secondary
+    assert set(synth.WORKLOADS) <= set(bench.SECONDARY) | {bench.DEFAULT_WORKLOAD}
+
+
+def test_attention_kernel_names():
+    import synth
+
+    assert bench.attention_kernel_name(synth.ALL_WORKLOADS["global_s9_g64"]) == "attn_fwd_kernel"
+    assert "precise" in bench.attention_kernel_name(synth.ALL_WORKLOADS["global_s9_g64_affine8"])
+    assert "fp32" in bench.attention_kernel_name(synth.ALL_WORKLOADS["global_s9_g64_f32"])
