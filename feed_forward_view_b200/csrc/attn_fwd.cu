@@ -124,7 +124,6 @@ using attn::Waiter;
 
 constexpr int kBM = 128;                          // query rows per tile
 constexpr int kBN = 96;                           // keys per block
-constexpr int kStages = 8;                        // K/V ring depth
 constexpr int kKVTileBytes = kBN * kHeadDim * 2;  // 12 KB
 constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum block (16)
 // Softmax warps per lane quarter of a tile: 2 = each takes half the score
@@ -134,19 +133,36 @@ constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum bloc
 #endif
 constexpr int kColSplit = VGGT_COL_SPLIT;
 static_assert(kColSplit == 1 || kColSplit == 2, "one or two softmax warps per lane quarter");
-constexpr int kSoftmaxWarps = 8 * kColSplit;         // per CTA: 2 tiles x 4 lane quarters x kColSplit
-constexpr int kThreads = 128 + 32 * kSoftmaxWarps;   // 640 or 384
-constexpr int kCols = kBN / kColSplit;               // score columns per softmax thread
+constexpr int kWarpsPerTile = 4 * kColSplit;  // softmax warps of one query tile
+constexpr int kCols = kBN / kColSplit;        // score columns per softmax thread
+
+// The two CTA shapes. kTiles = 2: two query tiles share every K/V block and
+// the tensor core alternates between them; all 512 TMEM columns, an 8-slot
+// ring, one CTA per SM. kTiles = 1: one query tile, 256 TMEM columns, a
+// 4-slot ring and 384 threads, so that two CTAs share an SM and one's set-up,
+// pipeline fill and drain overlap the other's main loop (short key ranges:
+// frame attention, small problems).
 // Register split: the cap for the CTA's warps at launch; the TMA/MMA
 // warpgroup gives registers up, the softmax warpgroups take them:
-// 2 halves: 128 * 56 + 512 * 104 = 60416 <= 640 * 96;
-// 1 half:   128 * 80 + 256 * 208 = 63488 <= 384 * 168.
-constexpr uint32_t kLaunchRegs = kColSplit == 2 ? 96 : 168;
-constexpr uint32_t kRegsControl = kColSplit == 2 ? 56 : 80;
-constexpr uint32_t kRegsSoftmax = kColSplit == 2 ? 104 : 208;
-static_assert(128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
-constexpr uint32_t kTmemCols = 512;
+//   2 tiles, 2 halves: 128 * 56 + 512 * 104 = 60416 <= 640 * 96;
+//   2 tiles, 1 half:   128 * 80 + 256 * 208 = 63488 <= 384 * 168;
+//   1 tile, 2 halves:  128 * 48 + 256 * 96 = 30720 <= 384 * 80 (two CTAs per SM);
+//   1 tile, 1 half:    128 * 48 + 128 * 208 = 32768 <= 256 * 128.
+template <int kTiles>
+struct Shape {
+    static_assert(kTiles == 1 || kTiles == 2, "one or two query tiles per CTA");
+    static constexpr int kStages = kTiles == 2 ? 8 : 4;  // K/V ring depth
+    static constexpr int kSoftmaxWarps = kWarpsPerTile * kTiles;
+    static constexpr int kThreads = 128 + 32 * kSoftmaxWarps;
+    static constexpr int kMinBlocks = kTiles == 2 ? 1 : 2;  // resident CTAs per SM
+    static constexpr uint32_t kLaunchRegs = kTiles == 2 ? (kColSplit == 2 ? 96 : 168) : (kColSplit == 2 ? 80 : 128);
+    static constexpr uint32_t kRegsControl = kTiles == 2 ? (kColSplit == 2 ? 56 : 80) : 48;
+    static constexpr uint32_t kRegsSoftmax = kTiles == 2 ? (kColSplit == 2 ? 104 : 208) : (kColSplit == 2 ? 96 : 208);
+    static constexpr uint32_t kTmemCols = 256 * kTiles;
+    static_assert(128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+    static_assert(kThreads * kLaunchRegs * kMinBlocks <= 65536, "registers for the resident CTAs");
+};
 
 // TMEM columns of Q_t, S_t, P_t and [O_t | l_t].
 __device__ __forceinline__ constexpr uint32_t col_q(int t) { return 256u * t; }
@@ -177,15 +193,26 @@ constexpr float kFmaFloor = -120.0f;
 #endif
 constexpr int kExp2OnFma = VGGT_EXP2_ON_FMA_PER8;
 
-// 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [-1/2, 1/2]: minimax in relative error
-// (Remez exchange, fit by fit_exp2_poly.py in this directory); worst relative
-// error of the whole float32 evaluation over [-24, 8] is 7.5e-5.
-constexpr float kExp2C0 = 9.999280572e-01f;
-constexpr float kExp2C1 = 6.932609677e-01f;
-constexpr float kExp2C2 = 2.426111251e-01f;
-constexpr float kExp2C3 = 5.517166853e-02f;
+// 2^f ~ c0 + c1 f + ... + cn f^n on [-1/2, 1/2]: minimax in relative error
+// (Remez exchange, fit by fit_exp2_poly.py in this directory). Degree 2
+// (used): worst relative error of the whole float32 evaluation over [-24, 8]
+// 1.7e-3, about the 2^-9 rounding P takes to bf16 anyway, and one packed FMA
+// per pair fewer than degree 3 (7.5e-5): measured +2-3% on the attention
+// kernel, relative Frobenius error against the oracle 3.86e-3 instead of
+// 3.78e-3 at 36 909 tokens.
+#ifndef VGGT_EXP2_DEGREE
+#define VGGT_EXP2_DEGREE 2
+#endif
+constexpr int kExp2Degree = VGGT_EXP2_DEGREE;
+static_assert(kExp2Degree == 2 || kExp2Degree == 3, "polynomial degree 2 or 3");
+__device__ __forceinline__ constexpr float exp2_coef(int i) {
+    return kExp2Degree == 3 ? (i == 0 ? 9.999280572e-01f : i == 1 ? 6.932609677e-01f
+                                         : i == 2 ? 2.426111251e-01f : 5.517166853e-02f)
+                            : (i == 0 ? 1.000443101e+00f : i == 1 ? 7.034479976e-01f : 2.384289354e-01f);
+}
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
+template <int kStages>
 struct SharedStorage {
     uint8_t kv[kStages][2][kKVTileBytes];  // [slot][K, V], 128B-swizzled
     uint8_t ones[kKVTileBytes];            // [1, 0, ..., 0] per key row, 128B-swizzled
@@ -204,16 +231,20 @@ struct SharedStorage {
 // Online instance only, placed after SharedStorage: per (tile, lane quarter)
 // the pair barrier of its two softmax warps and their block maxima, double
 // buffered by block parity ([tile][quarter][parity][half][lane]).
+template <int kTiles>
 struct OnlineShared {
-    uint64_t bar_pair[2][4];
-    float xchg[2][4][2][2][32];
+    uint64_t bar_pair[kTiles][4];
+    float xchg[kTiles][4][2][2][32];
 };
 
-template <bool kOnline>
+template <int kTiles, bool kOnline>
 constexpr size_t smem_bytes() {
-    return sizeof(SharedStorage) + (kOnline ? sizeof(OnlineShared) : 0) + 1024;  // + alignment slack
+    return sizeof(SharedStorage<Shape<kTiles>::kStages>) + (kOnline ? sizeof(OnlineShared<kTiles>) : 0) +
+           1024;  // + alignment slack
 }
-static_assert(smem_bytes<true>() <= 227 * 1024, "shared memory beyond the per-CTA limit");
+static_assert(smem_bytes<2, true>() <= 227 * 1024, "shared memory beyond the per-CTA limit");
+// two one-tile CTAs per SM: 228 KB per SM, 1 KB of it reserved per CTA
+static_assert(2 * (smem_bytes<1, true>() + 1024) <= 228 * 1024, "two one-tile CTAs do not fit an SM");
 
 struct Params {
     const uint16_t* q_hat;  // head-major, head planes q_stride rows apart
@@ -223,7 +254,6 @@ struct Params {
     long long q_stride;     // rows per head plane of q_hat
     int q_len, k_len, H;
     int pairs_per_seg;      // CTAs per segment
-    int tiles_per_cta;      // query tiles a CTA owns: 2, or 1 for grids too small to fill the GPU
     RowMap out_map;         // query row r is stored at output row map_row(out_map, r)
 };
 
@@ -282,8 +312,8 @@ __device__ __forceinline__ constexpr int mufu_pair(int k) {
 // 2^x on the FMA pipe, x in [-125, 125]: t = x + 1.5 * 2^23 rounds x to the
 // nearest integer j and leaves j in the low mantissa bits of t; -j =
 // 1.5 * 2^23 - t exactly; f = x - j exactly (|f| <= 1/2); 2^x = p(f) * 2^j,
-// with 2^j applied by adding j << 23 to the bit pattern of p(f). Six packed
-// adds and FMAs per pair.
+// with 2^j applied by adding j << 23 to the bit pattern of p(f). Three packed
+// adds and FMAs per pair plus one per polynomial degree.
 //
 // Instruction order. A warp issues in order; MUFU accepts one warp-wide ex2
 // every 8 cycles and a packed FMA holds the FMA pipe for 2. Emitting all the
@@ -295,7 +325,7 @@ __device__ __forceinline__ constexpr int mufu_pair(int k) {
 // it was produced, which hides the units' latencies.
 __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint32_t (&pk)[kPairs]) {
     const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
-    constexpr int kStagesFma = 7;  // t, -j, f, three Horner steps, combine + pack
+    constexpr int kStagesFma = 4 + kExp2Degree;  // t, -j, f, the Horner steps, combine + pack
     constexpr int kSteps = (kMufuPairs + 2 > kFmaPairs + kStagesFma - 1)
                                ? kMufuPairs + 2
                                : kFmaPairs + kStagesFma - 1;
@@ -314,19 +344,23 @@ __device__ __forceinline__ void exp_pack_row_mixed(const float (&s)[kCols], uint
             const int i = k - d;
             if (i < 0 || i >= kFmaPairs) continue;
             const int c = fma_pair(i);
-            switch (d) {
-                case 0: tt[i] = f2_add(f2_pack(s[2 * c], s[2 * c + 1]), magic2); break;
-                case 1: ff[i] = f2_fma(tt[i], f2_pack(-1.0f, -1.0f), magic2); break;  // -j
-                case 2: ff[i] = f2_add(f2_pack(s[2 * c], s[2 * c + 1]), ff[i]); break;  // f
-                case 3: y[i] = f2_fma(f2_pack(kExp2C3, kExp2C3), ff[i], f2_pack(kExp2C2, kExp2C2)); break;
-                case 4: y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C1, kExp2C1)); break;
-                case 5: y[i] = f2_fma(y[i], ff[i], f2_pack(kExp2C0, kExp2C0)); break;
-                default: {
-                    uint32_t q0, q1, t0, t1;
-                    u2_unpack(y[i], q0, q1);
-                    u2_unpack(tt[i], t0, t1);
-                    pk[c] = pack_bf16x2(__uint_as_float(q0 + (t0 << 23)), __uint_as_float(q1 + (t1 << 23)));
-                }
+            if (d == 0) {
+                tt[i] = f2_add(f2_pack(s[2 * c], s[2 * c + 1]), magic2);
+            } else if (d == 1) {
+                ff[i] = f2_fma(tt[i], f2_pack(-1.0f, -1.0f), magic2);  // -j
+            } else if (d == 2) {
+                ff[i] = f2_add(f2_pack(s[2 * c], s[2 * c + 1]), ff[i]);  // f
+            } else if (d == 3) {  // the first Horner step
+                constexpr float a = exp2_coef(kExp2Degree), b = exp2_coef(kExp2Degree - 1);
+                y[i] = f2_fma(f2_pack(a, a), ff[i], f2_pack(b, b));
+            } else if (d < 3 + kExp2Degree) {
+                const float cf = exp2_coef(kExp2Degree - 1 - (d - 3));
+                y[i] = f2_fma(y[i], ff[i], f2_pack(cf, cf));
+            } else {
+                uint32_t q0, q1, t0, t1;
+                u2_unpack(y[i], q0, q1);
+                u2_unpack(tt[i], t0, t1);
+                pk[c] = pack_bf16x2(__uint_as_float(q0 + (t0 << 23)), __uint_as_float(q1 + (t1 << 23)));
             }
         }
         if (k >= 2 && k - 2 < kMufuPairs) {
@@ -371,14 +405,17 @@ __device__ __forceinline__ void shift_scores(float (&s)[kCols], float m) {
     }
 }
 
-template <bool kOnline>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kTiles, bool kOnline>
+__global__ void __launch_bounds__(Shape<kTiles>::kThreads, Shape<kTiles>::kMinBlocks)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const Params prm) {
+    using Sh = Shape<kTiles>;
+    constexpr int kStages = Sh::kStages;
+    constexpr int kThreads = Sh::kThreads;
     extern __shared__ uint8_t smem_raw[];
-    SharedStorage& sm = *reinterpret_cast<SharedStorage*>(
+    SharedStorage<kStages>& sm = *reinterpret_cast<SharedStorage<kStages>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    OnlineShared& on = *reinterpret_cast<OnlineShared*>(&sm + 1);  // online instance only
+    OnlineShared<kTiles>& on = *reinterpret_cast<OnlineShared<kTiles>*>(&sm + 1);  // online instance only
 
     // The warp index and the TMEM base go through a lane-0 shuffle so that the
     // compiler knows them to be warp-uniform: everything derived from them
@@ -392,8 +429,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int pair = blockIdx.x - seg * prm.pairs_per_seg;
     const int h = blockIdx.y;
     const int n_qtiles = (prm.q_len + kBM - 1) / kBM;
-    const int tile0 = prm.tiles_per_cta * pair;              // first tile in the segment
-    const int ntile = min(prm.tiles_per_cta, n_qtiles - tile0);  // 1 or 2
+    const int tile0 = kTiles * pair;                  // first tile in the segment
+    const int ntile = min(kTiles, n_qtiles - tile0);  // 1 or 2
     const int k_row0 = seg * prm.k_len;
     const int nkb = (prm.k_len + kBN - 1) / kBN;
     const int last_valid = prm.k_len - (nkb - 1) * kBN;  // keys in the last block
@@ -430,15 +467,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_init(bar_kvempty(s), ntile);  // one commit per tile issuer
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_q(t), kSoftmaxWarps / 2);  // one arrival per softmax warp of the tile
+            mbar_init(bar_q(t), kWarpsPerTile);  // one arrival per softmax warp of the tile
             mbar_init(bar_s(t), 1);
-            mbar_init(bar_c(t), kSoftmaxWarps / 2);
+            mbar_init(bar_c(t), kWarpsPerTile);
             mbar_init(bar_pfree(t), 1);
             mbar_init(bar_o(t), 1);
             mbar_init(bar_tok(t), 1);
         }
         if constexpr (kOnline) {
-            for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < kTiles; ++t)
                 for (int qr = 0; qr < 4; ++qr) mbar_init(smem_u32(&on.bar_pair[t][qr]), kColSplit);
         }
         sm.abort = 0;
@@ -450,7 +487,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tma_prefetch_desc(&tm_v);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
+        tmem_alloc(smem_u32(&sm.tmem_base), Sh::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -459,7 +496,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, sm.tmem_base, 0);
     const Waiter wait{prm.wait_limit, &sm.abort, prm.status};
 
-    if (warp < 4) regs_dec<kRegsControl>();
+    if (warp < 4) regs_dec<Sh::kRegsControl>();
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -569,7 +606,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------ softmax
-        regs_inc<kRegsSoftmax>();
+        regs_inc<Sh::kRegsSoftmax>();
         const int t = (warp - 4) / (4 * kColSplit);
         const int half = ((warp - 4) >> 2) % kColSplit;  // score columns [kCols*half, +kCols)
         const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
@@ -782,7 +819,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, Sh::kTmemCols);
     }
 }
 
@@ -798,6 +835,43 @@ __global__ void wait_probe_kernel(int* status, long long limit) {
         // Nothing ever arrives on `bar`: the wait must run out.
         if (!mbar_wait(smem_u32(&bar), 0, limit, &abort)) atomicOr(status, kStatusTimeout);
     }
+}
+
+// Key blocks up to which one query tile per CTA (two CTAs per SM) is used.
+// Measured (A/B of the two shapes on the same inputs): one tile wins at 6
+// blocks (+21%), 11 (+3.5%) and 15 (+5%: frame attention over 1374-token
+// frames), two tiles from 22 blocks on (+7% at 22, +8% at 43, +14% at 115).
+#ifndef VGGT_SHORT_KEY_BLOCKS
+#define VGGT_SHORT_KEY_BLOCKS 16
+#endif
+constexpr int kShortKeyBlocks = VGGT_SHORT_KEY_BLOCKS;
+
+template <int kTiles, bool kOnline>
+cudaError_t launch_instance(int dev, dim3 grid, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const Params& prm,
+                            cudaStream_t stream) {
+    using Sh = Shape<kTiles>;
+    constexpr size_t smem = smem_bytes<kTiles, kOnline>();
+    // Set once per device and instance; host threads that race here both set
+    // the same attribute, and the flag is published atomically.
+    static std::atomic<bool> attr_set[64];
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        // The register split (setmaxnreg) needs the full launch allocation
+        // (kLaunchRegs per thread); with fewer registers the softmax
+        // warpgroups' increase could never be granted. Refuse to launch such
+        // a build.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<kTiles, kOnline>);
+        if (e != cudaSuccess) return e;
+        if (static_cast<uint32_t>(fa.numRegs) * Sh::kThreads <
+            128 * Sh::kRegsControl + 32 * Sh::kSoftmaxWarps * Sh::kRegsSoftmax)
+            return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(attn_fwd_kernel<kTiles, kOnline>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        attr_set[dev].store(true, std::memory_order_release);
+    }
+    attn_fwd_kernel<kTiles, kOnline><<<grid, Sh::kThreads, smem, stream>>>(tm_k, tm_v, prm);
+    return cudaPeekAtLastError();
 }
 
 }  // namespace
@@ -816,30 +890,24 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
         !make_map(&tm_v, p.v, p.H, nk, row_bytes, p.H * row_bytes, 1, kBN))
         return cudaErrorInvalidValue;
 
-    // Set once per device and instance; host threads that race here both set
-    // the same attribute, and the flag is published atomically.
-    static std::atomic<bool> attr_set[2][64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    const void* kernel = p.online ? reinterpret_cast<const void*>(attn_fwd_kernel<true>)
-                                  : reinterpret_cast<const void*>(attn_fwd_kernel<false>);
-    const size_t smem = p.online ? smem_bytes<true>() : smem_bytes<false>();
-    if (!attr_set[p.online][dev].load(std::memory_order_acquire)) {
-        // The register split (setmaxnreg) needs the full launch allocation
-        // (kLaunchRegs per thread); with fewer registers the softmax
-        // warpgroups' increase could never be granted. Refuse to launch such
-        // a build.
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, kernel);
-        if (e != cudaSuccess) return e;
-        if (static_cast<uint32_t>(fa.numRegs) * kThreads < 128 * kRegsControl + 32 * kSoftmaxWarps * kRegsSoftmax)
-            return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        attr_set[p.online][dev].store(true, std::memory_order_release);
-    }
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_qtiles = (p.q_len + kBM - 1) / kBM;
+    const int nkb = (p.k_len + kBN - 1) / kBN;
+    // Two tiles per CTA share every K/V block and keep the tensor core busy
+    // while one tile's softmax runs; for short key ranges one tile per CTA,
+    // two CTAs per SM, hides each CTA's fixed costs (set-up, the first loads,
+    // the drain) behind the other's work, and it doubles the CTA count of
+    // grids that would not fill the GPU.
+    const long long pair_ctas = static_cast<long long>(p.n_seg) * ((n_qtiles + 1) / 2) * p.H;
+    int tiles = (nkb <= kShortKeyBlocks || pair_ctas < sms) ? 1 : 2;
+#ifdef VGGT_TILES_PER_CTA
+    tiles = VGGT_TILES_PER_CTA;
+#endif
     Params prm;
     prm.q_hat = p.q_hat;
     prm.out = p.out;
@@ -850,25 +918,13 @@ cudaError_t launch_attention(const AttnProblem& p, int* status, long long wait_l
     prm.k_len = p.k_len;
     prm.H = p.H;
     prm.out_map = p.out_map;
-    const int n_qtiles = (p.q_len + kBM - 1) / kBM;
-    // Two tiles per CTA share every K/V block and keep the tensor core busy
-    // while one tile's softmax runs; one tile per CTA doubles the CTA count,
-    // which pays when two-tile CTAs would not even fill the GPU once.
-#ifndef VGGT_TILES_PER_CTA
-    int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long pair_ctas = static_cast<long long>(p.n_seg) * ((n_qtiles + 1) / 2) * p.H;
-    prm.tiles_per_cta = pair_ctas < sms ? 1 : 2;
-#else
-    prm.tiles_per_cta = VGGT_TILES_PER_CTA;
-#endif
-    prm.pairs_per_seg = (n_qtiles + prm.tiles_per_cta - 1) / prm.tiles_per_cta;
+    prm.pairs_per_seg = (n_qtiles + tiles - 1) / tiles;
     dim3 grid(p.n_seg * prm.pairs_per_seg, p.H);
-    if (p.online)
-        attn_fwd_kernel<true><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, prm);
-    else
-        attn_fwd_kernel<false><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, prm);
-    return cudaPeekAtLastError();
+    if (tiles == 1)
+        return p.online ? launch_instance<1, true>(dev, grid, tm_k, tm_v, prm, stream)
+                        : launch_instance<1, false>(dev, grid, tm_k, tm_v, prm, stream);
+    return p.online ? launch_instance<2, true>(dev, grid, tm_k, tm_v, prm, stream)
+                    : launch_instance<2, false>(dev, grid, tm_k, tm_v, prm, stream);
 }
 
 cudaError_t launch_wait_probe(int* status, long long wait_limit, cudaStream_t stream) {

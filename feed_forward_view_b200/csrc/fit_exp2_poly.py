@@ -15,11 +15,11 @@ nearest), so |f| <= 1/2 and f = x - j has no rounding error; then
 2^x = 2^j * p(f), with 2^j applied by adding j to the float32 exponent field.
 
 Running this script prints the float32 coefficients and the worst relative
-error of the float32 Horner evaluation over a dense grid. The degree-3
-values it printed are written into attn_fwd.cu (kExp2C0..kExp2C3: P is
-rounded to bf16 there). The fp32-mode kernel takes every exponential from
-MUFU; a degree-5 fit (`--degree 5`) would match MUFU's ~2^-22 if it needed
-one.
+error of the float32 Horner evaluation over a dense grid. The degree-2 and
+degree-3 values it printed (`--degree 2`, `--degree 3`) are written into
+attn_fwd.cu (exp2_coef; degree 2 is used, since P is rounded to bf16
+there). The fp32-mode kernel takes every exponential from MUFU; a degree-5
+fit (`--degree 5`) would match MUFU's ~2^-22 if it needed one.
 """
 from __future__ import annotations
 

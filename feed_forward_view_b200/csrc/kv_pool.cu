@@ -27,22 +27,20 @@
 // keys, normalises the fp32 means and writes k_hat as two bf16 terms.
 //
 // Memory-bound: every input byte of K and V is read once, the pooled tokens
-// are written once. One 256-thread block per pooled token: 128 threads pool
-// the values, 128 the keys, 16 heads per pass (8 threads per head). Per
-// member token a value thread loads its head's 16 bytes (dims 8*(t%8) ..); a
-// key thread loads the same in plain mode, or the prologue's two 8-byte
-// pieces (dims d1.., d1+16..) in fused mode -- so every member is read with
-// fully coalesced 2 KB rows of K and V, both in flight together. The sums
-// use packed two-lane float32 adds (the kernel is otherwise close to
-// instruction-bound).
+// are written once. One block per pooled token: 128 threads pool the values,
+// 16 heads per pass (8 threads per head, one 16-byte piece per member each);
+// the keys take 128 threads laid out the same way in plain mode, or 64
+// threads in fused mode (4 threads per head, two 16-byte pieces per member
+// each) -- so every member is read with coalesced 128-bit accesses to its
+// 2 KB rows of K and V, both in flight together. The sums use packed two-lane
+// float32 adds (the kernel is otherwise close to instruction-bound).
 #include "prologue.cuh"
 #include "sm100.cuh"
 
 namespace vggt {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kBatch = 8;  // member loads a thread keeps in flight
+constexpr int kBatch = 8;  // member loads a value thread keeps in flight
 
 // Which source tokens pooled token i of a frame averages: a single copied
 // token (src0 + first, copy == true), or the cell rows [r0, r1) x cols
@@ -101,38 +99,118 @@ __device__ __forceinline__ float2 pooled_position(const PoolJob& job, const Sour
     return make_float2(__fdiv_rn(pr, count), __fdiv_rn(pc, count));
 }
 
-// 8 bf16 values (w) added to 4 float32 pairs, two adds per instruction
-__device__ __forceinline__ void add8x2(uint64_t (&acc)[4], uint2 lo, uint2 hi) {
-    acc[0] = f2_add(acc[0], u2_pack(lo.x << 16, lo.x & 0xFFFF0000u));
-    acc[1] = f2_add(acc[1], u2_pack(lo.y << 16, lo.y & 0xFFFF0000u));
-    acc[2] = f2_add(acc[2], u2_pack(hi.x << 16, hi.x & 0xFFFF0000u));
-    acc[3] = f2_add(acc[3], u2_pack(hi.y << 16, hi.y & 0xFFFF0000u));
+// The member sums of one thread: kPieces 16-byte pieces per member (8 dims
+// each) at byte offsets off[0..kPieces) of every member row, summed in member
+// order (row-major over the cell) into packed fp32 pairs acc[4 * piece + e],
+// kB members' loads in flight before their sums; then divided by the member
+// count (IEEE, or the exact product with the reciprocal of a power of two).
+// p: the first member's row (+ the head's offset).
+template <int kPieces, int kB>
+__device__ __forceinline__ void member_means(const uint8_t* p, const int (&off)[kPieces], size_t tok_b,
+                                             size_t row_skip, int cw, int n, bool pow2, float count,
+                                             uint64_t (&acc)[4 * kPieces]) {
+#pragma unroll
+    for (int e = 0; e < 4 * kPieces; ++e) acc[e] = 0;
+    int c = 0;
+    for (int m0 = 0; m0 < n; m0 += kB) {
+        uint4 w[kB][kPieces];
+#pragma unroll
+        for (int j = 0; j < kB; ++j) {
+            if (m0 + j < n) {
+#pragma unroll
+                for (int q = 0; q < kPieces; ++q) w[j][q] = __ldg(reinterpret_cast<const uint4*>(p + off[q]));
+                p += tok_b;
+                if (++c == cw) {
+                    c = 0;
+                    p += row_skip;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kB; ++j) {
+            if (m0 + j < n) {
+#pragma unroll
+                for (int q = 0; q < kPieces; ++q) {
+                    acc[4 * q + 0] = f2_add(acc[4 * q + 0], u2_pack(w[j][q].x << 16, w[j][q].x & 0xFFFF0000u));
+                    acc[4 * q + 1] = f2_add(acc[4 * q + 1], u2_pack(w[j][q].y << 16, w[j][q].y & 0xFFFF0000u));
+                    acc[4 * q + 2] = f2_add(acc[4 * q + 2], u2_pack(w[j][q].z << 16, w[j][q].z & 0xFFFF0000u));
+                    acc[4 * q + 3] = f2_add(acc[4 * q + 3], u2_pack(w[j][q].w << 16, w[j][q].w & 0xFFFF0000u));
+                }
+            }
+        }
+    }
+    if (pow2) {
+        const uint64_t inv2 = f2_pack(1.0f / count, 1.0f / count);
+#pragma unroll
+        for (int e = 0; e < 4 * kPieces; ++e) acc[e] = f2_mul(acc[e], inv2);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4 * kPieces; ++e) {
+            float x, y;
+            f2_unpack(acc[e], x, y);
+            acc[e] = f2_pack(__fdiv_rn(x, count), __fdiv_rn(y, count));
+        }
+    }
+}
+
+// 4 consecutive values of a 16-byte bf16 piece (half 0: the first 4, half 1:
+// the last 4), widened.
+__device__ __forceinline__ void piece_half(uint4 w, int half, float (&x)[4]) {
+    const uint32_t u = half ? w.z : w.x, v = half ? w.w : w.y;
+    x[0] = prologue::bf16_lo(u);
+    x[1] = prologue::bf16_hi(u);
+    x[2] = prologue::bf16_lo(v);
+    x[3] = prologue::bf16_hi(v);
+}
+// 4 consecutive means (pairs acc[first], acc[first + 1]), as stored (bf16)
+// or (kPrecise) as they are.
+template <bool kPrecise>
+__device__ __forceinline__ void means4(const uint64_t (&acc)[8], int first, float (&x)[4]) {
+    f2_unpack(acc[first], x[0], x[1]);
+    f2_unpack(acc[first + 1], x[2], x[3]);
+    if (!kPrecise) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+    }
 }
 
 // kFused: keys normalised and rotated into k_hat (else pooled into k_out);
 // kAffine: the key LayerNorm has an affine; kPrecise (fused only): fp32 means
-// into the prologue, two-term k_hat. Separate instantiations keep the
-// plain pooling at its register count. Four resident blocks per SM (<= 64
-// registers a thread) measured fastest: occupancy decides this memory-bound
-// kernel more than the few registers it then spills.
+// into the prologue, two-term k_hat. Separate instantiations keep the plain
+// pooling at its register count; at most 64 registers a thread (four plain
+// blocks or five fused ones per SM) measured fastest: occupancy decides this
+// memory-bound kernel more than the few registers it then spills.
 //
-// 256 threads: warps 0-3 pool the values, warps 4-7 the keys, 16 heads per
-// pass (8 threads per head). A thread walks its cell's members in row-major
-// order with a pointer, kBatch member loads in flight before the sums (which
-// keep the member order). Warp 0 first gathers the pooled position; in fused
-// mode it hands it to the key warps through named barrier 1 (the value warps
-// never wait).
+// Warps 0-3 pool the values: 16 heads per pass, 8 threads per head, one
+// 16-byte piece (8 dims) per member, kBatch members' loads in flight. The key
+// threads follow: in plain mode warps 4-7, laid out like the value threads;
+// in fused mode warps 4-5, 4 threads per head holding the prologue's two
+// units (dims d1..d1+7 and d1+16..d1+23, two 16-byte pieces per member,
+// kBatch / 2 members in flight), which go on from their means to the
+// prologue arithmetic (norm_rotate2) with no exchange of values. A thread
+// walks its cell's members in row-major order with a pointer; the sums keep
+// the member order. Warp 0 first gathers the pooled position; in fused mode
+// it hands it to the key warps through named barrier 1 (the value warps never
+// wait).
+template <bool kFused>
+constexpr int pool_threads() {
+    return kFused ? 192 : 256;
+}
+
 template <bool kFused, bool kAffine, bool kPrecise>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(pool_threads<kFused>(), kFused ? 5 : 4)
 kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
     __shared__ float2 pooled_pos;
     __shared__ __align__(16) prologue::SmemAffine sk;
-    constexpr uint32_t kKeyBar = 1, kKeyBarThreads = 32 + kThreads / 2;  // warp 0 + the key warps
+    constexpr int kValueThreads = 128;
+    constexpr int kKeyThreads = pool_threads<kFused>() - kValueThreads;
+    constexpr uint32_t kKeyBar = 1, kKeyBarThreads = 32 + kKeyThreads;  // warp 0 + the key warps
+    constexpr int kHeadsPerPass = 16;
 
     const FrameLayout& L = job.layout;
     const int lane = threadIdx.x & 31;
-    const bool keys = threadIdx.x >= kThreads / 2;
-    const int t = threadIdx.x & (kThreads / 2 - 1);  // thread within its half
+    const bool keys = threadIdx.x >= kValueThreads;
+    const int t = keys ? threadIdx.x - kValueThreads : threadIdx.x;  // thread within its group
     const int Tk = L.pooled(job.kd);
     const int s = blockIdx.x / Tk;  // frame
     const int i = blockIdx.x % Tk;  // pooled token within the frame
@@ -145,13 +223,12 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
     const float count = static_cast<float>(n);
     // a power-of-two count divides exactly as a product with its reciprocal
     const bool pow2 = (n & (n - 1)) == 0;
-    const uint64_t inv2 = f2_pack(1.0f / count, 1.0f / count);
     const size_t tok = static_cast<size_t>(job.H) * kHeadDim;  // elements per token
     const size_t tok_b = tok * 2;                              // bytes per token
 
     const float* aff = nullptr;
     if (kAffine && keys) {
-        for (int e = t; e < 2 * kHeadDim; e += kThreads / 2)
+        for (int e = t; e < 2 * kHeadDim; e += kKeyThreads)
             sk.v[e] = e < kHeadDim ? job.k_ln.gamma[e] : job.k_ln.beta[e - kHeadDim];
         aff = sk.v;
     }
@@ -164,112 +241,94 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
         if (kFused) named_bar_arrive(kKeyBar, kKeyBarThreads);
     }
 
-    // 16-byte chunk of a head: dims dv .. dv+7 (values; keys in plain mode);
-    // fused keys take the prologue's dims d1 .. d1+3 and d1+16 .. d1+19
-    const int dv = 8 * (t & 7);
-    const int d1 = prologue::lane_dim(lane);
-    const bool split_keys = kFused && keys;
-    const int o1 = 2 * (split_keys ? d1 : dv), o2 = 2 * (split_keys ? d1 + 16 : dv + 4);
     const uint8_t* in = reinterpret_cast<const uint8_t*>(keys ? job.k : job.v);
-    float sv[4], cv[4];
+    const size_t row_skip = static_cast<size_t>(L.grid_w - cw) * tok_b;
+    const uint8_t* first = in + (grid0 + static_cast<size_t>(src.r0) * L.grid_w + src.c0) * tok_b;
 
-    for (int h0 = 0; h0 < job.H; h0 += kThreads / 16) {
-        const int h = h0 + (t >> 3);
+    if (!kFused || !keys) {
+        // ---- values (and plain keys): dims dv .. dv+7 of head h, token-major out
+        const int dv = 8 * (t & 7);
+        uint16_t* out_base = keys ? job.k_out : job.v_out;
+        for (int h0 = 0; h0 < job.H; h0 += kHeadsPerPass) {
+            const int h = h0 + (t >> 3);
+            if (h >= job.H) continue;
+            const size_t hoff = static_cast<size_t>(h) * kHeadDim * 2;
+            uint4 o;
+            if (src.copy) {
+                o = __ldg(reinterpret_cast<const uint4*>(in + (src0 + src.first) * tok_b + hoff + 2 * dv));
+            } else {
+                uint64_t acc[4];
+                const int off[1] = {2 * dv};
+                member_means<1, kBatch>(first + hoff, off, tok_b, row_skip, cw, n, pow2, count, acc);
+                float m[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f2_unpack(acc[e], m[2 * e], m[2 * e + 1]);
+                o = make_uint4(prologue::pack2(m[0], m[1]), prologue::pack2(m[2], m[3]), prologue::pack2(m[4], m[5]),
+                               prologue::pack2(m[6], m[7]));
+            }
+            *reinterpret_cast<uint4*>(out_base + dst * tok + static_cast<size_t>(h) * kHeadDim + dv) = o;
+        }
+        return;
+    }
+
+    // ---- fused keys: units a (dims d1..d1+3, d1+16..d1+19) and b (d1+4..,
+    // d1+20..) of head h, pooled, then normalised and rotated at the pooled
+    // position
+    const int sub = lane & 3;
+    const int d1 = (sub >> 1) * 32 + 8 * (sub & 1);
+    float sa[4], ca[4], sb[4], cb[4];
+    for (int h0 = 0; h0 < job.H; h0 += kHeadsPerPass) {
+        const int h = h0 + (t >> 2);
         const bool live = h < job.H;
-        uint64_t acc[4] = {0, 0, 0, 0};
-        uint2 c_lo = make_uint2(0, 0), c_hi = make_uint2(0, 0);  // a copied token's values
+        float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+        float b1[4] = {0.f, 0.f, 0.f, 0.f}, b2[4] = {0.f, 0.f, 0.f, 0.f};
         if (live) {
             const size_t hoff = static_cast<size_t>(h) * kHeadDim * 2;
             if (src.copy) {
                 const uint8_t* p = in + (src0 + src.first) * tok_b + hoff;
-                c_lo = __ldg(reinterpret_cast<const uint2*>(p + o1));
-                c_hi = __ldg(reinterpret_cast<const uint2*>(p + o2));
+                const uint4 lo = __ldg(reinterpret_cast<const uint4*>(p + 2 * d1));
+                const uint4 hi = __ldg(reinterpret_cast<const uint4*>(p + 2 * (d1 + 16)));
+                piece_half(lo, 0, a1);
+                piece_half(lo, 1, b1);
+                piece_half(hi, 0, a2);
+                piece_half(hi, 1, b2);
             } else {
-                const uint8_t* p = in + (grid0 + static_cast<size_t>(src.r0) * L.grid_w + src.c0) * tok_b + hoff;
-                const size_t row_skip = static_cast<size_t>(L.grid_w - cw) * tok_b;
-                int c = 0;
-                for (int m0 = 0; m0 < n; m0 += kBatch) {
-                    uint2 lo[kBatch], hi[kBatch];
-#pragma unroll
-                    for (int j = 0; j < kBatch; ++j) {
-                        if (m0 + j < n) {
-                            lo[j] = __ldg(reinterpret_cast<const uint2*>(p + o1));
-                            hi[j] = __ldg(reinterpret_cast<const uint2*>(p + o2));
-                            p += tok_b;
-                            if (++c == cw) {
-                                c = 0;
-                                p += row_skip;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < kBatch; ++j)
-                        if (m0 + j < n) add8x2(acc, lo[j], hi[j]);
-                }
-                if (pow2) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[e] = f2_mul(acc[e], inv2);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float x, y;
-                        f2_unpack(acc[e], x, y);
-                        acc[e] = f2_pack(__fdiv_rn(x, count), __fdiv_rn(y, count));
-                    }
-                }
-            }
-            if (!split_keys) {  // the means (or the copied token), bf16, token-major
-                uint4 o;
-                if (src.copy) {
-                    o = make_uint4(c_lo.x, c_lo.y, c_hi.x, c_hi.y);
-                } else {
-                    float m[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) f2_unpack(acc[e], m[2 * e], m[2 * e + 1]);
-                    o = make_uint4(prologue::pack2(m[0], m[1]), prologue::pack2(m[2], m[3]),
-                                   prologue::pack2(m[4], m[5]), prologue::pack2(m[6], m[7]));
-                }
-                uint16_t* out = (keys ? job.k_out : job.v_out) + dst * tok + static_cast<size_t>(h) * kHeadDim + dv;
-                *reinterpret_cast<uint4*>(out) = o;
+                uint64_t acc[8];
+                const int off[2] = {2 * d1, 2 * (d1 + 16)};
+                member_means<2, kBatch / 2>(first + hoff, off, tok_b, row_skip, cw, n, pow2, count, acc);
+                // the pooled keys as stored (bf16; precise mode: the fp32 means)
+                means4<kPrecise>(acc, 0, a1);
+                means4<kPrecise>(acc, 2, b1);
+                means4<kPrecise>(acc, 4, a2);
+                means4<kPrecise>(acc, 6, b2);
             }
         }
-        if (!split_keys) continue;  // warp-uniform
         if (h0 == 0) {
             named_bar_sync(kKeyBar, kKeyBarThreads);  // pooled_pos and the staged affine
-            prologue::token_angles(pooled_pos, lane, prologue::lane_freq(freq, lane), sv, cv);
+            prologue::token_angles2(pooled_pos, lane, prologue::lane_freq(freq, lane), sa, ca, sb, cb);
         }
-        // the pooled keys as stored (bf16; precise mode: the fp32 means), then
-        // the prologue
-        float x1[4], x2[4];
-        if (src.copy) {
-            x1[0] = prologue::bf16_lo(c_lo.x); x1[1] = prologue::bf16_hi(c_lo.x);
-            x1[2] = prologue::bf16_lo(c_lo.y); x1[3] = prologue::bf16_hi(c_lo.y);
-            x2[0] = prologue::bf16_lo(c_hi.x); x2[1] = prologue::bf16_hi(c_hi.x);
-            x2[2] = prologue::bf16_lo(c_hi.y); x2[3] = prologue::bf16_hi(c_hi.y);
-        } else {
-            float m[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) f2_unpack(acc[e], m[2 * e], m[2 * e + 1]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x1[e] = kPrecise ? m[e] : __bfloat162float(__float2bfloat16_rn(m[e]));
-                x2[e] = kPrecise ? m[4 + e] : __bfloat162float(__float2bfloat16_rn(m[4 + e]));
-            }
-        }
-        const size_t orow = (static_cast<size_t>(h) * job.k_hat_stride + dst) * kHeadDim;
+        float oa1[4], oa2[4], ob1[4], ob2[4];
+        prologue::norm_rotate2<kAffine>(a1, a2, b1, b2, aff, sa, ca, sb, cb, d1, oa1, oa2, ob1, ob2);
+        if (!live) continue;
+        uint16_t* out = job.k_hat + (static_cast<size_t>(h) * job.k_hat_stride + dst) * kHeadDim;
         if constexpr (kPrecise) {
-            float r1[4], r2[4];
-            prologue::norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, r1, r2);
-            if (live) prologue::store_two_terms(job.k_hat + orow, job.k_hat_lo + orow, d1, r1, r2);
+            uint16_t* lo = job.k_hat_lo + (static_cast<size_t>(h) * job.k_hat_stride + dst) * kHeadDim;
+            prologue::store_two_terms(out, lo, d1, oa1, oa2);
+            prologue::store_two_terms(out, lo, d1 + 4, ob1, ob2);
         } else {
-            prologue::norm_rotate_store<kAffine>(x1, x2, aff, sv, cv, live, job.k_hat + orow, d1);
+            *reinterpret_cast<uint4*>(out + d1) =
+                make_uint4(prologue::pack2(oa1[0], oa1[1]), prologue::pack2(oa1[2], oa1[3]),
+                           prologue::pack2(ob1[0], ob1[1]), prologue::pack2(ob1[2], ob1[3]));
+            *reinterpret_cast<uint4*>(out + d1 + 16) =
+                make_uint4(prologue::pack2(oa2[0], oa2[1]), prologue::pack2(oa2[2], oa2[3]),
+                           prologue::pack2(ob2[0], ob2[1]), prologue::pack2(ob2[2], ob2[3]));
         }
     }
 }
 
 template <bool kFused, bool kAffine, bool kPrecise = false>
 cudaError_t launch_pool_kernel(const PoolJob& job, unsigned blocks, cudaStream_t stream) {
-    kv_pool_kernel<kFused, kAffine, kPrecise><<<blocks, kThreads, 0, stream>>>(job, rope_freq_table());
+    kv_pool_kernel<kFused, kAffine, kPrecise><<<blocks, pool_threads<kFused>(), 0, stream>>>(job, rope_freq_table());
     return cudaPeekAtLastError();
 }
 

@@ -72,6 +72,64 @@ __device__ __forceinline__ void token_angles(float2 p, int lane, float my_freq, 
     }
 }
 
+// The arithmetic below is written with explicitly rounded operations
+// (__fadd_rn, __fmul_rn, __fmaf_rn: no contraction left to the compiler) and
+// split into the steps of one "unit" -- the 8 dims d1..d1+3, d1+16..d1+19 an
+// 8-lane thread owns -- so that a thread holding two units (norm_rotate2,
+// the 4-lane layout of the fused pooling pass) performs exactly the same
+// operations in the same order and produces the same bits.
+
+// A unit's partial sum, in a fixed order.
+__device__ __forceinline__ float unit_sum(const float (&x1)[4], const float (&x2)[4]) {
+    return __fadd_rn(__fadd_rn(__fadd_rn(x1[0], x1[1]), __fadd_rn(x1[2], x1[3])),
+                     __fadd_rn(__fadd_rn(x2[0], x2[1]), __fadd_rn(x2[2], x2[3])));
+}
+
+// Centres a unit on the mean and returns its partial sum of squares.
+__device__ __forceinline__ float unit_center_sq(float (&x1)[4], float (&x2)[4], float mean) {
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x1[i] = __fsub_rn(x1[i], mean);
+        x2[i] = __fsub_rn(x2[i], mean);
+        sq = __fmaf_rn(x1[i], x1[i], sq);
+        sq = __fmaf_rn(x2[i], x2[i], sq);
+    }
+    return sq;
+}
+
+// Scale (+ affine) and rotation of a unit at first dim d1.
+template <bool kAffine>
+__device__ __forceinline__ void unit_finish(const float (&x1)[4], const float (&x2)[4], float rstd, const float* aff,
+                                            const float (&sv)[4], const float (&cv)[4], int d1, float (&o1)[4],
+                                            float (&o2)[4]) {
+    float y1[4], y2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        y1[i] = __fmul_rn(x1[i], rstd);
+        y2[i] = __fmul_rn(x2[i], rstd);
+    }
+    if (kAffine) {
+        // volatile: read from shared memory at each use, so the compiler
+        // does not hoist the affine values into registers for the whole token
+        // loop
+        const volatile float* va = aff;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            y1[i] = __fmaf_rn(y1[i], va[d1 + i], va[kHeadDim + d1 + i]);
+            y2[i] = __fmaf_rn(y2[i], va[d1 + 16 + i], va[kHeadDim + d1 + 16 + i]);
+        }
+    }
+    // (y_j, y_{j+16}) -> (y_j cos - y_{j+16} sin, y_{j+16} cos + y_j sin)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o1[i] = __fmaf_rn(y1[i], cv[i], -__fmul_rn(y2[i], sv[i]));
+        o2[i] = __fmaf_rn(y2[i], cv[i], __fmul_rn(y1[i], sv[i]));
+    }
+}
+
+__device__ __forceinline__ float inv_std(float sq) { return rsqrtf(__fmaf_rn(sq, 1.0f / kHeadDim, kEps)); }
+
 // LayerNorm (+ affine) and rotation of one head (8 lanes) whose 8 dims per
 // lane are x1 (dims d1..d1+3) and x2 (d1+16..d1+19); the results, in fp32,
 // go to o1 and o2. Every lane of the warp runs it (the shuffles need the
@@ -80,44 +138,57 @@ __device__ __forceinline__ void token_angles(float2 p, int lane, float my_freq, 
 template <bool kAffine>
 __device__ __forceinline__ void norm_rotate(float (&x1)[4], float (&x2)[4], const float* aff, const float (&sv)[4],
                                             const float (&cv)[4], int d1, float (&o1)[4], float (&o2)[4]) {
-    float sum = (x1[0] + x1[1]) + (x1[2] + x1[3]) + ((x2[0] + x2[1]) + (x2[2] + x2[3]));
-    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-    const float mean = sum * (1.0f / kHeadDim);
-    float sq = 0.f;
+    float sum = unit_sum(x1, x2);
+    sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 1));
+    sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 2));
+    sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 4));
+    const float mean = __fmul_rn(sum, 1.0f / kHeadDim);
+    float sq = unit_center_sq(x1, x2, mean);
+    sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 1));
+    sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 2));
+    sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 4));
+    unit_finish<kAffine>(x1, x2, inv_std(sq), aff, sv, cv, d1, o1, o2);
+}
+
+// The same for a thread that holds two adjacent units of a head (4 lanes per
+// head): unit a at d1 and unit b at d1 + 4, i.e. dims d1..d1+7 and
+// d1+16..d1+23 with d1 = 32*(l/2) + 8*(l%2) for lane l % 4. Its sums are the
+// 8-lane sums after their first exchange (units 2k and 2k+1), and its two
+// exchanges are their second and third: the same operations, the same bits.
+template <bool kAffine>
+__device__ __forceinline__ void norm_rotate2(float (&a1)[4], float (&a2)[4], float (&b1)[4], float (&b2)[4],
+                                             const float* aff, const float (&sa)[4], const float (&ca)[4],
+                                             const float (&sb)[4], const float (&cb)[4], int d1, float (&oa1)[4],
+                                             float (&oa2)[4], float (&ob1)[4], float (&ob2)[4]) {
+    float sum = __fadd_rn(unit_sum(a1, a2), unit_sum(b1, b2));
+    sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 1));
+    sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 2));
+    const float mean = __fmul_rn(sum, 1.0f / kHeadDim);
+    float sq = __fadd_rn(unit_center_sq(a1, a2, mean), unit_center_sq(b1, b2, mean));
+    sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 1));
+    sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 2));
+    const float rstd = inv_std(sq);
+    unit_finish<kAffine>(a1, a2, rstd, aff, sa, ca, d1, oa1, oa2);
+    unit_finish<kAffine>(b1, b2, rstd, aff, sb, cb, d1 + 4, ob1, ob2);
+}
+
+// (sin, cos) of the angles of the two units of a 4-lane thread (see
+// norm_rotate2) at position p, computed like token_angles: lane l computes
+// the pair of (half l/16, frequency l%16), and the values are shuffled to
+// the lanes that own those dims. Every lane of the warp calls it.
+__device__ __forceinline__ void token_angles2(float2 p, int lane, float my_freq, float (&sa)[4], float (&ca)[4],
+                                              float (&sb)[4], float (&cb)[4]) {
+    const float my_pos = (lane < 16) ? p.x : p.y;
+    float sn, cs;
+    sincosf(my_pos * my_freq, &sn, &cs);
+    const int sub = lane & 3;
+    const int src = (sub >> 1) * 16 + 8 * (sub & 1);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        x1[i] -= mean;
-        x2[i] -= mean;
-        sq = fmaf(x1[i], x1[i], sq);
-        sq = fmaf(x2[i], x2[i], sq);
-    }
-    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
-    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
-    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 4);
-    const float rstd = rsqrtf(sq * (1.0f / kHeadDim) + kEps);
-    float y1[4], y2[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        y1[i] = x1[i] * rstd;
-        y2[i] = x2[i] * rstd;
-    }
-    if (kAffine) {
-        // volatile: read from shared memory at each use, so the compiler
-        // does not hoist 16 affine values per lane into registers for the
-        // whole token loop
-        const volatile float* va = aff;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            y1[i] = fmaf(y1[i], va[d1 + i], va[kHeadDim + d1 + i]);
-            y2[i] = fmaf(y2[i], va[d1 + 16 + i], va[kHeadDim + d1 + 16 + i]);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        o1[i] = y1[i] * cv[i] - y2[i] * sv[i];
-        o2[i] = y2[i] * cv[i] + y1[i] * sv[i];
+        sa[i] = __shfl_sync(0xFFFFFFFFu, sn, src + i);
+        ca[i] = __shfl_sync(0xFFFFFFFFu, cs, src + i);
+        sb[i] = __shfl_sync(0xFFFFFFFFu, sn, src + 4 + i);
+        cb[i] = __shfl_sync(0xFFFFFFFFu, cs, src + 4 + i);
     }
 }
 
