@@ -458,6 +458,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     auto k_smem = [&](int s) { return kv_smem0 + static_cast<uint32_t>(2 * kKVTileBytes) * s; };
     auto v_smem = [&](int s) { return k_smem(s) + static_cast<uint32_t>(kKVTileBytes); };
 
+    // One-tile CTAs (short key ranges, where a CTA's start is a large share of
+    // its life) request their first data before the set-up below, so that the
+    // loads' latency runs under it: the softmax warps their rows of q_hat
+    // (this thread's half of its row: 32 bf16 = 16 words, two head dims per
+    // word, low half first), the producer the first K/V block. Measured: the
+    // first scores ready ~1 us sooner, +2% on frame attention. Two-tile CTAs
+    // load after the set-up (the early producer code made ptxas spill there).
+    constexpr bool kEarly = kTiles == 1;
+    constexpr int kQWords = 32 / kColSplit;  // this thread's 2-dim words of the row
+    uint4 q_raw[kQWords / 4];
+    if (kEarly && warp >= 4) {
+        const int t = (warp - 4) / (4 * kColSplit);
+        const int half = ((warp - 4) >> 2) % kColSplit;
+        const int row_in_seg = (tile0 + t) * kBM + (warp & 3) * 32 + lane;
+        if (t < ntile && row_in_seg < prm.q_len) {
+            const long long grow = static_cast<long long>(seg) * prm.q_len + row_in_seg;
+            const uint4* src = reinterpret_cast<const uint4*>(
+                prm.q_hat + (static_cast<long long>(h) * prm.q_stride + grow) * kHeadDim + 2 * kQWords * half);
+#pragma unroll
+            for (int i = 0; i < kQWords / 4; ++i) q_raw[i] = __ldg(src + i);
+        }
+    }
     attn::fill_ones_tile(sm.ones, kKVTileBytes, kThreads);
     fence_proxy_async_smem();  // make the generic-proxy writes visible to the MMA
 
@@ -481,8 +503,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         sm.abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
+        if constexpr (kEarly) {
+            // The first block (its slot is empty; this thread is the TMA
+            // producer below, which continues with block 1).
+            mbar_arrive_expect_tx(bar_kvfull(0), 2 * kKVTileBytes);
+            tma_load_3d(k_smem(0), &tm_k, bar_kvfull(0), 0, k_row0, h);
+            tma_load_3d(v_smem(0), &tm_v, bar_kvfull(0), 0, h, k_row0);
+        }
     }
-    if (warp == 0 && lane == 0) {
+    if (!kEarly && warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -500,8 +529,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int n_issued = 0;  // blocks whose loads were started
-            for (int j = 0; j < nkb; ++j) {
+            int n_issued = kEarly ? 1 : 0;  // blocks whose loads were started (one-tile: the first at set-up)
+            for (int j = n_issued; j < nkb; ++j) {
                 const int s = j % kStages;
                 const uint32_t use = j / kStages;
                 if (use > 0 && !wait(bar_kvempty(s), (use - 1) & 1)) break;
@@ -621,21 +650,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int row_in_seg = (tile0 + t) * kBM + row;
             const bool row_live = row_in_seg < prm.q_len;
             const long long grow = static_cast<long long>(seg) * prm.q_len + row_in_seg;
-            // Q_t into TMEM: this thread's half of its row of q_hat (32 bf16
-            // = 16 words, two head dims per word, low half first) into its
-            // lane, the layout the MMA reads an M x K operand in, each value
-            // multiplied by log2(e)/8 on the way (so that S comes out of the
-            // MMA in log2 units and the exponentials need no multiply). Rows
-            // past the segment are zeros and never stored.
+            // Q_t into TMEM: this thread's half of its row of q_hat (loaded
+            // now, or at the start in one-tile CTAs) into its lane, the layout
+            // the MMA reads an M x K operand in, each value multiplied by
+            // log2(e)/8 on the way (so that S comes out of the MMA in log2
+            // units and the exponentials need no multiply). Rows past the
+            // segment are zeros and never stored.
             {
-                constexpr int kQWords = 32 / kColSplit;  // this thread's 2-dim words of the row
                 uint32_t qr[kQWords];
                 if (row_live) {
                     const uint4* src = reinterpret_cast<const uint4*>(
                         prm.q_hat + (static_cast<long long>(h) * prm.q_stride + grow) * kHeadDim + 2 * kQWords * half);
 #pragma unroll
                     for (int i = 0; i < kQWords / 4; ++i) {
-                        const uint4 w = __ldg(src + i);
+                        const uint4 w = kEarly ? q_raw[i] : __ldg(src + i);
                         if constexpr (kOnline) {  // unscaled: the shift applies log2(e)/8 in fp32
                             qr[4 * i] = w.x;
                             qr[4 * i + 1] = w.y;
