@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "pdl.cuh"
 #include "sm100.cuh"
 #include "vggt_internal.h"
 

@@ -409,6 +409,8 @@ template <int kTiles, bool kOnline>
 __global__ void __launch_bounds__(Shape<kTiles>::kThreads, Shape<kTiles>::kMinBlocks)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const Params prm) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     using Sh = Shape<kTiles>;
     constexpr int kStages = Sh::kStages;
     constexpr int kThreads = Sh::kThreads;
@@ -898,8 +900,7 @@ cudaError_t launch_instance(int dev, dim3 grid, const CUtensorMap& tm_k, const C
         if (e != cudaSuccess) return e;
         attr_set[dev].store(true, std::memory_order_release);
     }
-    attn_fwd_kernel<kTiles, kOnline><<<grid, Sh::kThreads, smem, stream>>>(tm_k, tm_v, prm);
-    return cudaPeekAtLastError();
+    return launch_pdl(attn_fwd_kernel<kTiles, kOnline>, grid, dim3(Sh::kThreads), smem, stream, tm_k, tm_v, prm);
 }
 
 }  // namespace

@@ -213,6 +213,8 @@ __device__ __forceinline__ void split_terms(float a, float b, uint32_t (&w)[kTer
 template <int kTQ, int kTP, bool kOnline>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     using C = Cfg<kTQ, kTP>;
     constexpr int kSK = C::kStagesK, kSV = C::kStagesV;
     extern __shared__ uint8_t smem_raw[];
@@ -620,8 +622,8 @@ cudaError_t launch_terms(const AttnProblemF32& p, const Params& prm, cudaStream_
         attr_set[dev].store(true, std::memory_order_release);
     }
     dim3 grid(p.n_seg * prm.tiles_per_seg, p.H);
-    attn_fwd_f32_kernel<kTQ, kTP, kOnline><<<grid, kThreads, smem_bytes<kTQ, kTP, kOnline>(), stream>>>(maps, prm);
-    return cudaPeekAtLastError();
+    return launch_pdl(attn_fwd_f32_kernel<kTQ, kTP, kOnline>, grid, dim3(kThreads), smem_bytes<kTQ, kTP, kOnline>(), stream,
+                      maps, prm);
 }
 
 }  // namespace

@@ -34,6 +34,7 @@
 // each) -- so every member is read with coalesced 128-bit accesses to its
 // 2 KB rows of K and V, both in flight together. The sums use packed two-lane
 // float32 adds (the kernel is otherwise close to instruction-bound).
+#include "pdl.cuh"
 #include "prologue.cuh"
 #include "sm100.cuh"
 
@@ -200,6 +201,8 @@ constexpr int pool_threads() {
 template <bool kFused, bool kAffine, bool kPrecise>
 __global__ void __launch_bounds__(pool_threads<kFused>(), kFused ? 5 : 4)
 kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     __shared__ float2 pooled_pos;
     __shared__ __align__(16) prologue::SmemAffine sk;
     constexpr int kValueThreads = 128;
@@ -328,8 +331,8 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
 
 template <bool kFused, bool kAffine, bool kPrecise = false>
 cudaError_t launch_pool_kernel(const PoolJob& job, unsigned blocks, cudaStream_t stream) {
-    kv_pool_kernel<kFused, kAffine, kPrecise><<<blocks, pool_threads<kFused>(), 0, stream>>>(job, rope_freq_table());
-    return cudaPeekAtLastError();
+    return launch_pdl(kv_pool_kernel<kFused, kAffine, kPrecise>, dim3(blocks), dim3(pool_threads<kFused>()), 0, stream,
+                      job, rope_freq_table());
 }
 
 }  // namespace

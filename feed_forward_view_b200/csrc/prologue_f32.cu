@@ -21,6 +21,7 @@
 //
 // Memory-bound; one warp per token as in the bf16 prologue, each lane loading
 // its 8 dims of a head as two 16-byte pieces.
+#include "pdl.cuh"
 #include "prologue.cuh"
 
 namespace vggt {
@@ -107,6 +108,8 @@ template <bool kAffA, bool kAffB, bool kBf16In>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 qk_prologue_f32_kernel(const __grid_constant__ PrologueJobF32 a, const __grid_constant__ PrologueJobF32 b, int H,
                        FreqTable freq) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     const int lane = threadIdx.x & 31;
     const int warp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -129,6 +132,8 @@ template <int kTerms>
 __global__ void __launch_bounds__(256)
 split_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__ t0, uint2* __restrict__ t1,
                   uint2* __restrict__ t2, long long n4) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n4; i += static_cast<long long>(gridDim.x) * 256) {
         const float4 v = __ldg(x + i);
         uint32_t a[kTerms], b[kTerms];
@@ -160,8 +165,7 @@ cudaError_t launch_qk_prologue_f32(const PrologueJobF32& a, const PrologueJobF32
                    : (b.ln.on ? qk_prologue_f32_kernel<false, true, true> : qk_prologue_f32_kernel<false, false, true>))
         : (a.ln.on ? (b.ln.on ? qk_prologue_f32_kernel<true, true, false> : qk_prologue_f32_kernel<true, false, false>)
                    : (b.ln.on ? qk_prologue_f32_kernel<false, true, false> : qk_prologue_f32_kernel<false, false, false>));
-    kernel<<<blocks, kWarpsPerBlock * 32, 0, stream>>>(a, b, H, rope_freq_table());
-    return cudaPeekAtLastError();
+    return launch_pdl(kernel, dim3(blocks), dim3(kWarpsPerBlock * 32), 0, stream, a, b, H, rope_freq_table());
 }
 
 cudaError_t launch_split_bf16(const float* x, uint16_t* const (&out)[3], int terms, long long n,
@@ -172,10 +176,9 @@ cudaError_t launch_split_bf16(const float* x, uint16_t* const (&out)[3], int ter
     const long long cap = static_cast<long long>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
     auto kernel = terms == 3 ? split_bf16_kernel<3> : split_bf16_kernel<2>;
-    kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<const float4*>(x), reinterpret_cast<uint2*>(out[0]), reinterpret_cast<uint2*>(out[1]),
-        reinterpret_cast<uint2*>(out[2]), n4);
-    return cudaPeekAtLastError();
+    return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                      reinterpret_cast<const float4*>(x), reinterpret_cast<uint2*>(out[0]),
+                      reinterpret_cast<uint2*>(out[1]), reinterpret_cast<uint2*>(out[2]), n4);
 }
 
 }  // namespace vggt

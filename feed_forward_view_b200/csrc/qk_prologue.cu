@@ -10,6 +10,7 @@
 // of both jobs.
 #include <cmath>
 
+#include "pdl.cuh"
 #include "prologue.cuh"
 
 namespace vggt {
@@ -23,6 +24,8 @@ template <bool kAffA, bool kAffB>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 qk_prologue_kernel(const __grid_constant__ PrologueJob a, const __grid_constant__ PrologueJob b, int H,
                    FreqTable freq) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     const int lane = threadIdx.x & 31;
     const int warp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -43,6 +46,8 @@ qk_prologue_kernel(const __grid_constant__ PrologueJob a, const __grid_constant_
 // One warp per destination row, 16 bytes per lane per step.
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n, int chunks, RowMap m) {
+    griddep_launch_dependents();
+    griddep_wait();  // before any global memory access (pdl.cuh)
     const int lane = threadIdx.x & 31;
     const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
     for (long long c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); c < n; c += warps) {
@@ -64,9 +69,8 @@ cudaError_t launch_gather_rows(const uint16_t* src, uint16_t* dst, long long n, 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     long long blocks = (n + 7) / 8;
     if (blocks > static_cast<long long>(sms) * 8) blocks = static_cast<long long>(sms) * 8;
-    gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n, row_elems / 8, m);
-    return cudaPeekAtLastError();
+    return launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                      reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n, row_elems / 8, m);
 }
 
 FreqTable rope_freq_table() {
@@ -88,8 +92,7 @@ cudaError_t launch_qk_prologue(const PrologueJob& a, const PrologueJob& b, int H
     blocks = blocks < sms * 8 ? blocks : sms * 8;
     auto kernel = a.ln.on ? (b.ln.on ? qk_prologue_kernel<true, true> : qk_prologue_kernel<true, false>)
                           : (b.ln.on ? qk_prologue_kernel<false, true> : qk_prologue_kernel<false, false>);
-    kernel<<<blocks, kWarpsPerBlock * 32, 0, stream>>>(a, b, H, rope_freq_table());
-    return cudaPeekAtLastError();
+    return launch_pdl(kernel, dim3(blocks), dim3(kWarpsPerBlock * 32), 0, stream, a, b, H, rope_freq_table());
 }
 
 }  // namespace vggt
