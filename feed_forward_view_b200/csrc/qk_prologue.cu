@@ -8,6 +8,7 @@
 // Memory-bound: one read and one write of 2 KB per token (H = 16).
 // Mapping: one warp per token, 8 lanes per head, grid-stride over the tokens
 // of both jobs.
+#include <atomic>
 #include <cmath>
 
 #include "pdl.cuh"
@@ -88,10 +89,23 @@ cudaError_t launch_qk_prologue(const PrologueJob& a, const PrologueJob& b, int H
     if (e != cudaSuccess) return e;
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int blocks = (total + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    blocks = blocks < sms * 8 ? blocks : sms * 8;
     auto kernel = a.ln.on ? (b.ln.on ? qk_prologue_kernel<true, true> : qk_prologue_kernel<true, false>)
                           : (b.ln.on ? qk_prologue_kernel<false, true> : qk_prologue_kernel<false, false>);
+    // As many blocks as are resident at once (the warps stride over the
+    // tokens): a grid beyond that leaves a second, partial wave that starts
+    // only as the first one ends, and that the next launch then waits for.
+    static std::atomic<int> per_sm_cache[64][4];
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const int inst = (a.ln.on ? 2 : 0) + (b.ln.on ? 1 : 0);
+    int per_sm = per_sm_cache[dev][inst].load(std::memory_order_acquire);
+    if (per_sm == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWarpsPerBlock * 32, 0);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        per_sm_cache[dev][inst].store(per_sm, std::memory_order_release);
+    }
+    int blocks = (total + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    blocks = blocks < sms * per_sm ? blocks : sms * per_sm;
     return launch_pdl(kernel, dim3(blocks), dim3(kWarpsPerBlock * 32), 0, stream, a, b, H, rope_freq_table());
 }
 
