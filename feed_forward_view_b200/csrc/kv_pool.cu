@@ -201,7 +201,6 @@ constexpr int pool_threads() {
 template <bool kFused, bool kAffine, bool kPrecise>
 __global__ void __launch_bounds__(pool_threads<kFused>(), kFused ? 5 : 4)
 kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
-    griddep_launch_dependents();
     griddep_wait();  // before any global memory access (pdl.cuh)
     __shared__ float2 pooled_pos;
     __shared__ __align__(16) prologue::SmemAffine sk;
@@ -271,6 +270,7 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
             }
             *reinterpret_cast<uint4*>(out_base + dst * tok + static_cast<size_t>(h) * kHeadDim + dv) = o;
         }
+        griddep_launch_dependents();
         return;
     }
 
@@ -327,6 +327,7 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
                            prologue::pack2(ob2[0], ob2[1]), prologue::pack2(ob2[2], ob2[3]));
         }
     }
+    griddep_launch_dependents();
 }
 
 template <bool kFused, bool kAffine, bool kPrecise = false>

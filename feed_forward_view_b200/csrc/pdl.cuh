@@ -4,12 +4,16 @@
 // in the stream is still finishing, so that its CTAs are dispatched during the
 // previous kernel's last wave instead of after it. Such a kernel must run
 // griddep_wait() before it reads or writes global memory that earlier work may
-// touch. Every kernel of the library starts with
-//   griddep_launch_dependents();  // the next kernel may be scheduled
-//   griddep_wait();               // the previous work has completed
-// so that only the launch itself overlaps: everything the kernel does happens
-// after the preceding work has finished and its writes are visible, exactly
-// as with an ordinary launch. Both instructions do nothing when there is no
+// touch. Every kernel of the library starts with griddep_wait(), so that only
+// the launch itself overlaps: everything the kernel does happens after the
+// preceding work has finished and its writes are visible, exactly as with an
+// ordinary launch. griddep_launch_dependents() lets the next kernel be
+// scheduled once every CTA of this one has issued it: the attention kernels
+// issue it first thing (their grids are often a single wave, whose free SMs
+// the next kernel can then take at once), the memory-bound kernels at the end
+// of each CTA's work (their grids are many waves, and an early signal only
+// parks the next kernel's CTAs, waiting, through most of this one: measured
+// slower at 274 800 tokens). Both instructions do nothing when there is no
 // programmatic dependency (an ordinary launch, or nothing before it).
 #pragma once
 

@@ -108,7 +108,6 @@ template <bool kAffA, bool kAffB, bool kBf16In>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 qk_prologue_f32_kernel(const __grid_constant__ PrologueJobF32 a, const __grid_constant__ PrologueJobF32 b, int H,
                        FreqTable freq) {
-    griddep_launch_dependents();
     griddep_wait();  // before any global memory access (pdl.cuh)
     const int lane = threadIdx.x & 31;
     const int warp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -125,6 +124,7 @@ qk_prologue_f32_kernel(const __grid_constant__ PrologueJobF32 a, const __grid_co
         else
             process_token_f32<kAffB, kBf16In>(b, aff_b, i - a.n, H, lane, my_freq);
     }
+    griddep_launch_dependents();
 }
 
 // The kTerms bf16 terms of x, 4 values per thread per step.
@@ -132,7 +132,6 @@ template <int kTerms>
 __global__ void __launch_bounds__(256)
 split_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__ t0, uint2* __restrict__ t1,
                   uint2* __restrict__ t2, long long n4) {
-    griddep_launch_dependents();
     griddep_wait();  // before any global memory access (pdl.cuh)
     for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n4; i += static_cast<long long>(gridDim.x) * 256) {
         const float4 v = __ldg(x + i);
@@ -143,6 +142,7 @@ split_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__ t0, uint2* _
         t1[i] = make_uint2(a[1], b[1]);
         if (kTerms == 3) t2[i] = make_uint2(a[kTerms - 1], b[kTerms - 1]);
     }
+    griddep_launch_dependents();
 }
 
 int sm_count() {

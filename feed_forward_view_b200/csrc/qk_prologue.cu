@@ -25,7 +25,6 @@ template <bool kAffA, bool kAffB>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 qk_prologue_kernel(const __grid_constant__ PrologueJob a, const __grid_constant__ PrologueJob b, int H,
                    FreqTable freq) {
-    griddep_launch_dependents();
     griddep_wait();  // before any global memory access (pdl.cuh)
     const int lane = threadIdx.x & 31;
     const int warp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -42,12 +41,12 @@ qk_prologue_kernel(const __grid_constant__ PrologueJob a, const __grid_constant_
         else
             prologue::process_token<kAffB>(b, aff_b, i - a.n, H, lane, my_freq);
     }
+    griddep_launch_dependents();
 }
 
 // One warp per destination row, 16 bytes per lane per step.
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n, int chunks, RowMap m) {
-    griddep_launch_dependents();
     griddep_wait();  // before any global memory access (pdl.cuh)
     const int lane = threadIdx.x & 31;
     const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
@@ -56,6 +55,7 @@ gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long 
         uint4* d = dst + c * chunks;
         for (int i = lane; i < chunks; i += 32) d[i] = __ldg(s + i);
     }
+    griddep_launch_dependents();
 }
 
 }  // namespace
