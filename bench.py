@@ -38,7 +38,7 @@ DATASHEET_BF16_TFLOPS = 2250.0
 DATASHEET_HBM_GBS = 8000.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_kernel_global_s6_g64.txt")
 KERNEL_SOURCES = ("feed_forward_view_b200/csrc/attn_fwd.cu", "feed_forward_view_b200/csrc/attn_common.cuh",
-                  "feed_forward_view_b200/csrc/sm100.cuh")
+                  "feed_forward_view_b200/csrc/sm100.cuh", "feed_forward_view_b200/csrc/pdl.cuh")
 
 
 # ----------------------------------------------------------------------------- helpers
