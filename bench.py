@@ -306,16 +306,27 @@ SECONDARY = ("global_s2_g16", "frame_s8_g37", "global_s8_g37", "descriptor_s200_
 
 
 def _event_ms(torch, stream, fn, reps: int, warm: int = 3) -> float:
-    """Average device time of fn() over reps launches, CUDA events on stream."""
+    """Average device time of fn() over reps back-to-back launches. The reps
+    calls are captured once into a CUDA graph and one replay is timed with
+    CUDA events on the stream: called one by one from Python, a launch of a
+    few microseconds waits for the host's per-call work (the binding's checks
+    and marshalling take longer than the smallest kernels), and the timing
+    would then measure the host instead of the kernel."""
     for _ in range(warm):
         fn()
     torch.cuda.synchronize(stream.device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()  # the first replay uploads the graph
+    torch.cuda.synchronize(stream.device)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(reps):
-        fn()
+    g.replay()
     b.record(stream)
     torch.cuda.synchronize(stream.device)
+    del g
     return a.elapsed_time(b) / reps
 
 
@@ -665,6 +676,7 @@ def run_gpu(args):
                          "frac_of_sustained": attn_tf / float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_of_datasheet": attn_tf / DATASHEET_BF16_TFLOPS,
                          "traffic": traffic, "kernel_ms": attn_ms,
+                         "kernel_timing": "CUDA events around one replay of a CUDA graph of back-to-back launches",
                          "share_of_step": attn_ms / ms_step},
             # (the fp32 mode's own prologue runs inside its step; the bf16
             # prologue on the same shape is reported for comparison)
