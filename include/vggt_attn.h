@@ -60,6 +60,13 @@
  *     attributes, which cannot happen during a capture: make one ordinary
  *     call per device (and per variant: frame/global/descriptor, fp32 mode)
  *     before capturing.
+ *   - Every kernel is launched with programmatic dependent launch and waits
+ *     (griddepcontrol.wait) for the previous work in its stream to complete
+ *     before it touches memory, so calls are ordered in their stream exactly
+ *     as ordinary launches are. A caller's own kernel that it launches right
+ *     after a call with the programmatic-stream-serialization attribute may
+ *     start early, like the library's, and must wait the same way before it
+ *     reads the call's outputs.
  *   - Host threads may call the library concurrently (each on its own
  *     stream); a device's one-time set-up is serialised inside. A descriptor
  *     cache handle is not: one thread (or one stream order) at a time.
