@@ -311,7 +311,7 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
             prologue::token_angles2(pooled_pos, lane, prologue::lane_freq(freq, lane), sa, ca, sb, cb);
         }
         float oa1[4], oa2[4], ob1[4], ob2[4];
-        prologue::norm_rotate2<kAffine>(a1, a2, b1, b2, aff, sa, ca, sb, cb, d1, oa1, oa2, ob1, ob2);
+        prologue::norm_rotate2<kAffine, false>(a1, a2, b1, b2, aff, sa, ca, sb, cb, d1, oa1, oa2, ob1, ob2);
         if (!live) continue;
         uint16_t* out = job.k_hat + (static_cast<size_t>(h) * job.k_hat_stride + dst) * kHeadDim;
         if constexpr (kPrecise) {

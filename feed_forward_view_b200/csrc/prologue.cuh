@@ -19,6 +19,7 @@
 
 #include <cuda_bf16.h>
 
+#include "sm100.cuh"
 #include "vggt_internal.h"
 
 namespace vggt {
@@ -72,59 +73,125 @@ __device__ __forceinline__ void token_angles(float2 p, int lane, float my_freq, 
     }
 }
 
-// The arithmetic below is written with explicitly rounded operations
-// (__fadd_rn, __fmul_rn, __fmaf_rn: no contraction left to the compiler) and
-// split into the steps of one "unit" -- the 8 dims d1..d1+3, d1+16..d1+19 an
-// 8-lane thread owns -- so that a thread holding two units (norm_rotate2,
-// the 4-lane layout of the fused pooling pass) performs exactly the same
-// operations in the same order and produces the same bits.
+// The arithmetic below is written with explicitly rounded operations (no
+// contraction left to the compiler) and split into the steps of one "unit" --
+// the 8 dims d1..d1+3, d1+16..d1+19 an 8-lane thread owns -- so that a thread
+// holding two units (norm_rotate2, the 4-lane layout of the fused pooling
+// pass) performs exactly the same operations in the same order and produces
+// the same bits. A unit is handled as four pairs of adjacent dims, (d1, d1+1),
+// (d1+2, d1+3), (d1+16, d1+17), (d1+18, d1+19): the even dims of the pairs in
+// one lane, the odd dims in another. kPacked selects packed two-lane fp32
+// instructions (add / mul / fma .rn.f32x2: each lane an ordinary round-to-
+// nearest operation, two results per instruction) or the same operations one
+// by one: identical results. The prologue kernels take the packed form (they
+// are partly issue-bound at the power-capped clock, and it halves their
+// arithmetic instructions); the fused pooling pass the scalar one (at its
+// 64-register cap the register pairs cost it spills and 1.5%).
 
-// A unit's partial sum, in a fixed order.
+// A unit's partial sum: ((x0 + x2) + (x16 + x18)) + ((x1 + x3) + (x17 + x19)).
+template <bool kPacked>
 __device__ __forceinline__ float unit_sum(const float (&x1)[4], const float (&x2)[4]) {
-    return __fadd_rn(__fadd_rn(__fadd_rn(x1[0], x1[1]), __fadd_rn(x1[2], x1[3])),
-                     __fadd_rn(__fadd_rn(x2[0], x2[1]), __fadd_rn(x2[2], x2[3])));
+    if constexpr (kPacked) {
+        const uint64_t e = f2_add(f2_add(f2_pack(x1[0], x1[1]), f2_pack(x1[2], x1[3])),
+                                  f2_add(f2_pack(x2[0], x2[1]), f2_pack(x2[2], x2[3])));
+        float lo, hi;
+        f2_unpack(e, lo, hi);
+        return __fadd_rn(lo, hi);
+    } else {
+        return __fadd_rn(__fadd_rn(__fadd_rn(x1[0], x1[2]), __fadd_rn(x2[0], x2[2])),
+                         __fadd_rn(__fadd_rn(x1[1], x1[3]), __fadd_rn(x2[1], x2[3])));
+    }
 }
 
-// Centres a unit on the mean and returns its partial sum of squares.
+// Centres a unit on the mean (x + (-mean): the same rounding as x - mean) and
+// returns its partial sum of squares: (((x0^2 + x2^2) + x16^2) + x18^2) +
+// (((x1^2 + x3^2) + x17^2) + x19^2), each step a fused multiply-add.
+template <bool kPacked>
 __device__ __forceinline__ float unit_center_sq(float (&x1)[4], float (&x2)[4], float mean) {
-    float sq = 0.f;
+    if constexpr (!kPacked) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        x1[i] = __fsub_rn(x1[i], mean);
-        x2[i] = __fsub_rn(x2[i], mean);
-        sq = __fmaf_rn(x1[i], x1[i], sq);
-        sq = __fmaf_rn(x2[i], x2[i], sq);
+        for (int i = 0; i < 4; ++i) {
+            x1[i] = __fadd_rn(x1[i], -mean);
+            x2[i] = __fadd_rn(x2[i], -mean);
+        }
+        float lo = __fmul_rn(x1[0], x1[0]), hi = __fmul_rn(x1[1], x1[1]);
+        lo = __fmaf_rn(x1[2], x1[2], lo);
+        hi = __fmaf_rn(x1[3], x1[3], hi);
+        lo = __fmaf_rn(x2[0], x2[0], lo);
+        hi = __fmaf_rn(x2[1], x2[1], hi);
+        lo = __fmaf_rn(x2[2], x2[2], lo);
+        hi = __fmaf_rn(x2[3], x2[3], hi);
+        return __fadd_rn(lo, hi);
     }
-    return sq;
+    const uint64_t nm = f2_pack(-mean, -mean);
+    const uint64_t a = f2_add(f2_pack(x1[0], x1[1]), nm), b = f2_add(f2_pack(x1[2], x1[3]), nm);
+    const uint64_t c = f2_add(f2_pack(x2[0], x2[1]), nm), d = f2_add(f2_pack(x2[2], x2[3]), nm);
+    f2_unpack(a, x1[0], x1[1]);
+    f2_unpack(b, x1[2], x1[3]);
+    f2_unpack(c, x2[0], x2[1]);
+    f2_unpack(d, x2[2], x2[3]);
+    uint64_t q = f2_mul(a, a);
+    q = f2_fma(b, b, q);
+    q = f2_fma(c, c, q);
+    q = f2_fma(d, d, q);
+    float lo, hi;
+    f2_unpack(q, lo, hi);
+    return __fadd_rn(lo, hi);
 }
 
 // Scale (+ affine) and rotation of a unit at first dim d1.
-template <bool kAffine>
+template <bool kAffine, bool kPacked>
 __device__ __forceinline__ void unit_finish(const float (&x1)[4], const float (&x2)[4], float rstd, const float* aff,
                                             const float (&sv)[4], const float (&cv)[4], int d1, float (&o1)[4],
                                             float (&o2)[4]) {
-    float y1[4], y2[4];
+    if constexpr (!kPacked) {
+        float y1[4], y2[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        y1[i] = __fmul_rn(x1[i], rstd);
-        y2[i] = __fmul_rn(x2[i], rstd);
+        for (int i = 0; i < 4; ++i) {
+            y1[i] = __fmul_rn(x1[i], rstd);
+            y2[i] = __fmul_rn(x2[i], rstd);
+        }
+        if (kAffine) {
+            const volatile float* va = aff;  // (see below)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                y1[i] = __fmaf_rn(y1[i], va[d1 + i], va[kHeadDim + d1 + i]);
+                y2[i] = __fmaf_rn(y2[i], va[d1 + 16 + i], va[kHeadDim + d1 + 16 + i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o1[i] = __fmaf_rn(y1[i], cv[i], __fmul_rn(y2[i], -sv[i]));
+            o2[i] = __fmaf_rn(y2[i], cv[i], __fmul_rn(y1[i], sv[i]));
+        }
+        return;
     }
+    const uint64_t r2 = f2_pack(rstd, rstd);
+    // y1 pairs (j, j+1) for j = d1, d1 + 2; y2 pairs at j + 16
+    uint64_t y1[2] = {f2_mul(f2_pack(x1[0], x1[1]), r2), f2_mul(f2_pack(x1[2], x1[3]), r2)};
+    uint64_t y2[2] = {f2_mul(f2_pack(x2[0], x2[1]), r2), f2_mul(f2_pack(x2[2], x2[3]), r2)};
     if (kAffine) {
         // volatile: read from shared memory at each use, so the compiler
         // does not hoist the affine values into registers for the whole token
         // loop
         const volatile float* va = aff;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            y1[i] = __fmaf_rn(y1[i], va[d1 + i], va[kHeadDim + d1 + i]);
-            y2[i] = __fmaf_rn(y2[i], va[d1 + 16 + i], va[kHeadDim + d1 + 16 + i]);
+        for (int k = 0; k < 2; ++k) {
+            const int j = d1 + 2 * k;
+            y1[k] = f2_fma(y1[k], f2_pack(va[j], va[j + 1]), f2_pack(va[kHeadDim + j], va[kHeadDim + j + 1]));
+            y2[k] = f2_fma(y2[k], f2_pack(va[j + 16], va[j + 17]),
+                           f2_pack(va[kHeadDim + j + 16], va[kHeadDim + j + 17]));
         }
     }
-    // (y_j, y_{j+16}) -> (y_j cos - y_{j+16} sin, y_{j+16} cos + y_j sin)
+    // (y_j, y_{j+16}) -> (y_j cos - y_{j+16} sin, y_{j+16} cos + y_j sin);
+    // -(y_{j+16} sin) is formed as y_{j+16} (-sin), the same value
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        o1[i] = __fmaf_rn(y1[i], cv[i], -__fmul_rn(y2[i], sv[i]));
-        o2[i] = __fmaf_rn(y2[i], cv[i], __fmul_rn(y1[i], sv[i]));
+    for (int k = 0; k < 2; ++k) {
+        const uint64_t c2 = f2_pack(cv[2 * k], cv[2 * k + 1]);
+        const uint64_t s2 = f2_pack(sv[2 * k], sv[2 * k + 1]);
+        const uint64_t ns2 = f2_pack(-sv[2 * k], -sv[2 * k + 1]);
+        f2_unpack(f2_fma(y1[k], c2, f2_mul(y2[k], ns2)), o1[2 * k], o1[2 * k + 1]);
+        f2_unpack(f2_fma(y2[k], c2, f2_mul(y1[k], s2)), o2[2 * k], o2[2 * k + 1]);
     }
 }
 
@@ -135,19 +202,19 @@ __device__ __forceinline__ float inv_std(float sq) { return rsqrtf(__fmaf_rn(sq,
 // go to o1 and o2. Every lane of the warp runs it (the shuffles need the
 // whole warp); lanes that hold no head hold zeros. kAffine: apply the affine
 // staged at aff (gamma[64] then beta[64] in shared memory).
-template <bool kAffine>
+template <bool kAffine, bool kPacked>
 __device__ __forceinline__ void norm_rotate(float (&x1)[4], float (&x2)[4], const float* aff, const float (&sv)[4],
                                             const float (&cv)[4], int d1, float (&o1)[4], float (&o2)[4]) {
-    float sum = unit_sum(x1, x2);
+    float sum = unit_sum<kPacked>(x1, x2);
     sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 1));
     sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 2));
     sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 4));
     const float mean = __fmul_rn(sum, 1.0f / kHeadDim);
-    float sq = unit_center_sq(x1, x2, mean);
+    float sq = unit_center_sq<kPacked>(x1, x2, mean);
     sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 1));
     sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 2));
     sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 4));
-    unit_finish<kAffine>(x1, x2, inv_std(sq), aff, sv, cv, d1, o1, o2);
+    unit_finish<kAffine, kPacked>(x1, x2, inv_std(sq), aff, sv, cv, d1, o1, o2);
 }
 
 // The same for a thread that holds two adjacent units of a head (4 lanes per
@@ -155,21 +222,21 @@ __device__ __forceinline__ void norm_rotate(float (&x1)[4], float (&x2)[4], cons
 // d1+16..d1+23 with d1 = 32*(l/2) + 8*(l%2) for lane l % 4. Its sums are the
 // 8-lane sums after their first exchange (units 2k and 2k+1), and its two
 // exchanges are their second and third: the same operations, the same bits.
-template <bool kAffine>
+template <bool kAffine, bool kPacked>
 __device__ __forceinline__ void norm_rotate2(float (&a1)[4], float (&a2)[4], float (&b1)[4], float (&b2)[4],
                                              const float* aff, const float (&sa)[4], const float (&ca)[4],
                                              const float (&sb)[4], const float (&cb)[4], int d1, float (&oa1)[4],
                                              float (&oa2)[4], float (&ob1)[4], float (&ob2)[4]) {
-    float sum = __fadd_rn(unit_sum(a1, a2), unit_sum(b1, b2));
+    float sum = __fadd_rn(unit_sum<kPacked>(a1, a2), unit_sum<kPacked>(b1, b2));
     sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 1));
     sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, 2));
     const float mean = __fmul_rn(sum, 1.0f / kHeadDim);
-    float sq = __fadd_rn(unit_center_sq(a1, a2, mean), unit_center_sq(b1, b2, mean));
+    float sq = __fadd_rn(unit_center_sq<kPacked>(a1, a2, mean), unit_center_sq<kPacked>(b1, b2, mean));
     sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 1));
     sq = __fadd_rn(sq, __shfl_xor_sync(0xFFFFFFFFu, sq, 2));
     const float rstd = inv_std(sq);
-    unit_finish<kAffine>(a1, a2, rstd, aff, sa, ca, d1, oa1, oa2);
-    unit_finish<kAffine>(b1, b2, rstd, aff, sb, cb, d1 + 4, ob1, ob2);
+    unit_finish<kAffine, kPacked>(a1, a2, rstd, aff, sa, ca, d1, oa1, oa2);
+    unit_finish<kAffine, kPacked>(b1, b2, rstd, aff, sb, cb, d1 + 4, ob1, ob2);
 }
 
 // (sin, cos) of the angles of the two units of a 4-lane thread (see
@@ -199,7 +266,7 @@ __device__ __forceinline__ void norm_rotate_store(float (&x1)[4], float (&x2)[4]
                                                   const float (&sv)[4], const float (&cv)[4], bool live,
                                                   uint16_t* dst, int d1) {
     float o1[4], o2[4];
-    norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, o1, o2);
+    norm_rotate<kAffine, true>(x1, x2, aff, sv, cv, d1, o1, o2);
     if (live) {
         *reinterpret_cast<uint2*>(dst + d1) = make_uint2(pack2(o1[0], o1[1]), pack2(o1[2], o1[3]));
         *reinterpret_cast<uint2*>(dst + d1 + 16) = make_uint2(pack2(o2[0], o2[1]), pack2(o2[2], o2[3]));

@@ -89,7 +89,7 @@ __device__ __forceinline__ void process_token_f32(const PrologueJobF32& job, con
             }
         }
         float o1[4], o2[4];
-        prologue::norm_rotate<kAffine>(x1, x2, aff, sv, cv, d1, o1, o2);
+        prologue::norm_rotate<kAffine, true>(x1, x2, aff, sv, cv, d1, o1, o2);
         if (!live) continue;
         const size_t row = (static_cast<size_t>(h) * job.out_stride + t) * kHeadDim;
         if (job.terms == 2) {
