@@ -31,11 +31,12 @@
 // softmax (kTQ = 2, kTP = 1).
 //
 // One CTA per 128-row query tile of one head. Warps: 0 TMA producer for the
-// K terms of 96 keys, 2 for the V terms (separate rings: 4 + 4 slots for two
-// terms, 3 + 2 for three), 1 MMA issuer, 3 idle, 4-11 softmax (2 per TMEM
-// lane quarter, 48 score columns each). Tensor memory: the Q terms (32
-// columns each), S (96), the P terms (48 each), [O | l] (80) and its folded
-// sum (80, see kFold). The softmax warps and the issuer meet once
+// K terms of a key block (96 keys; 64 in the precise instance, see Cfg), 2
+// for the V terms (separate rings: 4 + 4 slots for two terms, 3 + 2 for
+// three, 3 + 4 in the precise instance), 1 MMA issuer, 3 idle, 4-11 softmax
+// (2 per TMEM lane quarter, half the block's score columns each). Tensor
+// memory: the Q terms (32 columns each), S (one column per key), the P terms
+// (half that each), [O | l] (80) and its folded sum (80, see kFold). The softmax warps and the issuer meet once
 // per key block exactly as in the bf16 kernel (attn_fwd.cu): right after
 // loading S_j the softmax warps arrive on bar_c (P_{j-1} written, S free; the
 // first warp has checked that K_{j+1} landed), and on that signal the issuer
@@ -64,13 +65,9 @@ using attn::make_map;
 using attn::Waiter;
 
 constexpr int kBM = 128;                          // query rows per CTA
-constexpr int kBN = 96;                           // keys per block
-constexpr int kTileBytes = kBN * kHeadDim * 2;    // one 96 x 64 bf16 tile, 12 KB
 constexpr int kOCols = kHeadDim + 16;             // O (64) and the row-sum block
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 128 + 32 * kSoftmaxWarps;  // 384
-constexpr int kCols = 48;                           // score columns per softmax thread
-constexpr uint32_t kTmemCols = 512;
 
 // Per term counts -- kTQ for Q and K (the score product), kTP for P and V
 // (the value product): the K and V ring depths (separate rings, each with its
@@ -79,25 +76,48 @@ constexpr uint32_t kTmemCols = 512;
 //   fp32 mode, two terms (kTQ = kTP = 2): 4 + 4 slots of 2 tiles;
 //   three terms (3, 3): 3 + 2 slots of 3 tiles (a third V slot does not fit
 //   beside them in 227 KB);
-//   precise scores for bf16 calls (2, 1): 4 K slots of 2 tiles, 6 V slots of
-//   one tile (the bf16 v itself); P in one bf16 term and a bf16 output, so the
-//   value product needs no fold.
+//   precise scores for bf16 calls (2, 1): 64-key blocks, 3 K slots of 2
+//   tiles, 4 V slots of one tile (the bf16 v itself); P in one bf16 term and
+//   a bf16 output, so the value product needs no fold. With 64 keys a block,
+//   a CTA needs 240 of 256 TMEM columns and ~90 KB of shared memory, so two
+//   CTAs share an SM (one alone left the SM latency-bound: tensor pipe 48 %,
+//   MUFU 47 %, 8 softmax warps).
 template <int kTQ, int kTP>
 struct Cfg {
     static_assert((kTQ == 2 || kTQ == 3) && (kTP == kTQ || (kTQ == 2 && kTP == 1)), "term counts");
-    static constexpr int kStagesK = kTQ == 2 ? 4 : 3;
-    static constexpr int kStagesV = kTP == 1 ? 6 : (kTP == 2 ? 4 : 2);
+    static constexpr int kBN = kTP == 1 ? 64 : 96;             // keys per block
+    static constexpr int kTileBytes = kBN * kHeadDim * 2;      // one kBN x 64 bf16 tile
+    static constexpr int kCols = kBN / 2;                      // score columns per softmax thread
+    static constexpr int kMinBlocks = kTP == 1 ? 2 : 1;        // resident CTAs per SM
+    static constexpr uint32_t kTmemCols = kTP == 1 ? 256 : 512;
+    static constexpr int kStagesK = kTP == 1 ? 3 : (kTQ == 2 ? 4 : 3);
+    static constexpr int kStagesV = kTP == 1 ? 4 : (kTP == 2 ? 4 : 2);
     static constexpr int kPairsS = kTQ * (kTQ + 1) / 2;   // term products kept in S
     static constexpr int kPairsPV = kTP * (kTP + 1) / 2;  // and in [O | l]
     static constexpr bool kFoldOn = kTP > 1;              // fp32 outputs: fold every kFold blocks
     static constexpr bool kBf16Out = kTP == 1;
     static constexpr uint32_t kColQ = 0;                  // 32 per term
     static constexpr uint32_t kColS = 32 * kTQ;
-    static constexpr uint32_t kColP = kColS + kBN;        // 48 per term
+    static constexpr uint32_t kColP = kColS + kBN;        // kBN / 2 per term
     static constexpr uint32_t kColO = kColP + (kBN / 2) * kTP;
     static constexpr uint32_t kColA = kColO + kOCols;     // the folded partial sums
-    static_assert(kColA + kOCols <= kTmemCols, "tensor memory columns");
+    static_assert((kFoldOn ? kColA : kColO) + kOCols <= kTmemCols, "tensor memory columns");
+    static_assert(kCols == 32 || kCols == 48, "score columns per thread");
 };
+
+// TMEM loads and stores of the widths the two block sizes use.
+template <int N>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 32 || N == 48, "unsupported width");
+    if constexpr (N == 32) tmem_ld32(taddr, r);
+    if constexpr (N == 48) tmem_ld48(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 24, "unsupported width");
+    if constexpr (N == 16) tmem_st16(taddr, r);
+    if constexpr (N == 24) tmem_st24(taddr, r);
+}
 
 // The kept term products in order of size: (0,0), then (0,1) (1,0), then
 // (0,2) (1,1) (2,0). Product i multiplies term pair_a(i) of the left operand
@@ -145,9 +165,9 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 template <int kTQ, int kTP>
 struct SharedStorage {
     using C = Cfg<kTQ, kTP>;
-    uint8_t k[C::kStagesK][kTQ][kTileBytes];  // K terms, 128B-swizzled
-    uint8_t v[C::kStagesV][kTP][kTileBytes];  // V terms, 128B-swizzled
-    uint8_t ones[kTileBytes];                    // [1, 0, ..., 0] per key row, 128B-swizzled
+    uint8_t k[C::kStagesK][kTQ][C::kTileBytes];  // K terms, 128B-swizzled
+    uint8_t v[C::kStagesV][kTP][C::kTileBytes];  // V terms, 128B-swizzled
+    uint8_t ones[C::kTileBytes];                 // [1, 0, ..., 0] per key row, 128B-swizzled
     uint64_t bar_kfull[C::kStagesK];
     uint64_t bar_kempty[C::kStagesK];
     uint64_t bar_vfull[C::kStagesV];
@@ -176,6 +196,8 @@ constexpr size_t smem_bytes() {
 static_assert(smem_bytes<2, 2, true>() <= 227 * 1024 && smem_bytes<3, 3, true>() <= 227 * 1024 &&
                   smem_bytes<2, 1, true>() <= 227 * 1024,
               "shared memory beyond the per-CTA limit");
+// two (2, 1) CTAs per SM: 228 KB per SM, 1 KB of it reserved per CTA
+static_assert(2 * (smem_bytes<2, 1, true>() + 1024) <= 228 * 1024, "two precise-mode CTAs do not fit an SM");
 
 // The TMA maps of the K terms (head-major planes) and the V terms
 // (token-major), unused entries zero.
@@ -211,11 +233,14 @@ __device__ __forceinline__ void split_terms(float a, float b, uint32_t (&w)[kTer
 }
 
 template <int kTQ, int kTP, bool kOnline>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, Cfg<kTQ, kTP>::kMinBlocks)
 attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
     griddep_launch_dependents();
     griddep_wait();  // before any global memory access (pdl.cuh)
     using C = Cfg<kTQ, kTP>;
+    constexpr int kBN = C::kBN;
+    constexpr int kTileBytes = C::kTileBytes;
+    constexpr int kCols = C::kCols;
     constexpr int kSK = C::kStagesK, kSV = C::kStagesV;
     extern __shared__ uint8_t smem_raw[];
     SharedStorage<kTQ, kTP>& sm = *reinterpret_cast<SharedStorage<kTQ, kTP>*>(
@@ -278,7 +303,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
         for (int t = 0; t < (warp == 0 ? kTQ : kTP); ++t) tma_prefetch_desc(warp == 0 ? &maps.k[t] : &maps.v[t]);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
+        tmem_alloc(smem_u32(&sm.tmem_base), C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -341,7 +366,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             }
             __syncwarp();
         };
-        // PV_j: the kept products P_a [V_b | 1], 6 steps of 16 keys each; the
+        // PV_j: the kept products P_a [V_b | 1], kBN / 16 steps of 16 keys each; the
         // products with V_0 carry the ones column (the B operand's second
         // 64-column block, a leading byte offset away from the V_0 tile), so
         // the row sum collects every term of P
@@ -356,8 +381,8 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
                     const uint64_t vd = b == 0 ? smem_desc_sw128(v0_addr, ones_smem - v0_addr, 1024)
                                                : smem_desc_sw128(v_tile(s, b), 16, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < 6; ++kk)
-                        mma_ts(o_tm, p_tm + 48 * pair_a(i) + 8 * kk, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4),
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_ts(o_tm, p_tm + (kBN / 2) * pair_a(i) + 8 * kk, vd + static_cast<uint64_t>((kk * 16 * 128) >> 4),
                                b == 0 ? idesc_o : idesc_o64,
                                ((C::kFoldOn ? j % kFold != 0 : j > 0) || i > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -381,7 +406,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
         drain_wait(bar_o, 0, prm.wait_limit);
     } else if (warp >= 4) {
         // ------------------------------------------------------ softmax
-        const int half = (warp - 4) >> 2;  // score columns [48*half, +48)
+        const int half = (warp - 4) >> 2;  // score columns [kCols*half, +kCols)
         const int quarter = warp & 3;      // TMEM lanes [32*quarter, +32)
         const int row = quarter * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -438,7 +463,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
             float s[kCols];
             {
                 uint32_t r[kCols];
-                tmem_ld48(lane_base + C::kColS + kCols * half, r);
+                tmem_load_cols(lane_base + C::kColS + kCols * half, r);
 #pragma unroll
                 for (int i = 0; i < kCols; ++i) s[i] = __uint_as_float(r[i]);
             }
@@ -524,7 +549,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
                 }
             }
 #pragma unroll
-            for (int t = 0; t < kTP; ++t) tmem_st24(lane_base + C::kColP + 48 * t + (kCols / 2) * half, pt[t]);
+            for (int t = 0; t < kTP; ++t) tmem_store_cols(lane_base + C::kColP + (kBN / 2) * t + (kCols / 2) * half, pt[t]);
             if constexpr (kOnline) {
                 // Blocks 0..j-1 are in the current run of [O | l] (unless a
                 // fold just closed it: PV_j then starts afresh) and, from the
@@ -592,7 +617,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
@@ -600,6 +625,7 @@ attn_fwd_f32_kernel(const __grid_constant__ Maps maps, const Params prm) {
 
 template <int kTQ, int kTP, bool kOnline>
 cudaError_t launch_terms(const AttnProblemF32& p, const Params& prm, cudaStream_t stream) {
+    constexpr int kBN = Cfg<kTQ, kTP>::kBN;
     const uint64_t nk = static_cast<uint64_t>(p.n_seg) * p.k_len;
     const uint64_t row_bytes = kHeadDim * 2;
     const uint64_t ks = static_cast<uint64_t>(p.k_stride);
