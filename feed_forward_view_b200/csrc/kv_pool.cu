@@ -182,29 +182,34 @@ __device__ __forceinline__ void means4(const uint64_t (&acc)[8], int first, floa
 // blocks or five fused ones per SM) measured fastest: occupancy decides this
 // memory-bound kernel more than the few registers it then spills.
 //
-// Warps 0-3 pool the values: 16 heads per pass, 8 threads per head, one
-// 16-byte piece (8 dims) per member, kBatch members' loads in flight. The key
-// threads follow: in plain mode warps 4-7, laid out like the value threads;
-// in fused mode warps 4-5, 4 threads per head holding the prologue's two
-// units (dims d1..d1+7 and d1+16..d1+23, two 16-byte pieces per member,
-// kBatch / 2 members in flight), which go on from their means to the
-// prologue arithmetic (norm_rotate2) with no exchange of values. A thread
+// Plain mode (256 threads): warps 0-3 pool the values, warps 4-7 the keys,
+// 16 heads per pass, 8 threads per head, one 16-byte piece (8 dims) per
+// member, kBatch members' loads in flight. Fused mode (128 threads): warps
+// 0-1 pool the values, 4 threads per head with two 16-byte pieces (16 dims)
+// per member and kBatch / 2 members in flight; warps 2-3 the keys, 4 threads
+// per head holding the prologue's two units (dims d1..d1+7 and d1+16..d1+23,
+// two 16-byte pieces per member, kBatch / 2 members in flight), which go on
+// from their means to the prologue arithmetic (norm_rotate2) with no
+// exchange of values. (The key threads carry the longer path -- their means
+// and then the prologue -- so the two groups are given the same number of
+// warps; with four value warps beside two key warps, the value warps idled
+// half the block and five blocks fitted an SM, against eight now.) A thread
 // walks its cell's members in row-major order with a pointer; the sums keep
 // the member order. Warp 0 first gathers the pooled position; in fused mode
 // it hands it to the key warps through named barrier 1 (the value warps never
 // wait).
 template <bool kFused>
 constexpr int pool_threads() {
-    return kFused ? 192 : 256;
+    return kFused ? 128 : 256;
 }
 
 template <bool kFused, bool kAffine, bool kPrecise>
-__global__ void __launch_bounds__(pool_threads<kFused>(), kFused ? 5 : 4)
+__global__ void __launch_bounds__(pool_threads<kFused>(), kFused ? 8 : 4)
 kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
     griddep_wait();  // before any global memory access (pdl.cuh)
     __shared__ float2 pooled_pos;
     __shared__ __align__(16) prologue::SmemAffine sk;
-    constexpr int kValueThreads = 128;
+    constexpr int kValueThreads = kFused ? 64 : 128;
     constexpr int kKeyThreads = pool_threads<kFused>() - kValueThreads;
     constexpr uint32_t kKeyBar = 1, kKeyBarThreads = 32 + kKeyThreads;  // warp 0 + the key warps
     constexpr int kHeadsPerPass = 16;
@@ -248,27 +253,39 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
     const uint8_t* first = in + (grid0 + static_cast<size_t>(src.r0) * L.grid_w + src.c0) * tok_b;
 
     if (!kFused || !keys) {
-        // ---- values (and plain keys): dims dv .. dv+7 of head h, token-major out
-        const int dv = 8 * (t & 7);
+        // ---- values (and plain keys): dims dv .. dv + 8 * kPieces - 1 of head h,
+        // token-major out
+        constexpr int kShift = kFused ? 2 : 3;    // log2 of the threads per head
+        constexpr int kPieces = 8 >> kShift;      // 16-byte pieces (8 dims) per member
+        const int dv = 8 * kPieces * (t & ((1 << kShift) - 1));
         uint16_t* out_base = keys ? job.k_out : job.v_out;
         for (int h0 = 0; h0 < job.H; h0 += kHeadsPerPass) {
-            const int h = h0 + (t >> 3);
+            const int h = h0 + (t >> kShift);
             if (h >= job.H) continue;
             const size_t hoff = static_cast<size_t>(h) * kHeadDim * 2;
-            uint4 o;
+            uint4 o[kPieces];
             if (src.copy) {
-                o = __ldg(reinterpret_cast<const uint4*>(in + (src0 + src.first) * tok_b + hoff + 2 * dv));
-            } else {
-                uint64_t acc[4];
-                const int off[1] = {2 * dv};
-                member_means<1, kBatch>(first + hoff, off, tok_b, row_skip, cw, n, pow2, count, acc);
-                float m[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) f2_unpack(acc[e], m[2 * e], m[2 * e + 1]);
-                o = make_uint4(prologue::pack2(m[0], m[1]), prologue::pack2(m[2], m[3]), prologue::pack2(m[4], m[5]),
-                               prologue::pack2(m[6], m[7]));
+                for (int q = 0; q < kPieces; ++q)
+                    o[q] = __ldg(reinterpret_cast<const uint4*>(in + (src0 + src.first) * tok_b + hoff + 2 * (dv + 8 * q)));
+            } else {
+                uint64_t acc[4 * kPieces];
+                int off[kPieces];
+#pragma unroll
+                for (int q = 0; q < kPieces; ++q) off[q] = 2 * (dv + 8 * q);
+                member_means<kPieces, kBatch / kPieces>(first + hoff, off, tok_b, row_skip, cw, n, pow2, count, acc);
+#pragma unroll
+                for (int q = 0; q < kPieces; ++q) {
+                    float m[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) f2_unpack(acc[4 * q + e], m[2 * e], m[2 * e + 1]);
+                    o[q] = make_uint4(prologue::pack2(m[0], m[1]), prologue::pack2(m[2], m[3]),
+                                      prologue::pack2(m[4], m[5]), prologue::pack2(m[6], m[7]));
+                }
             }
-            *reinterpret_cast<uint4*>(out_base + dst * tok + static_cast<size_t>(h) * kHeadDim + dv) = o;
+#pragma unroll
+            for (int q = 0; q < kPieces; ++q)
+                *reinterpret_cast<uint4*>(out_base + dst * tok + static_cast<size_t>(h) * kHeadDim + dv + 8 * q) = o[q];
         }
         griddep_launch_dependents();
         return;
