@@ -1,8 +1,11 @@
 """Host logic of bench.py without a GPU: max-over-ranks timing across two gloo
 ranks (the path of a multi-GPU run, where every rank is an independent
 replica), clock-sample parsing and the profile/traffic bookkeeping."""
+import json
 import os
+import pathlib
 import socket
+import sys
 
 import pytest
 import torch.multiprocessing as mp
@@ -105,3 +108,30 @@ def test_attention_kernel_names():
     assert bench.attention_kernel_name(synth.ALL_WORKLOADS["global_s9_g64"]) == "attn_fwd_kernel"
     assert "precise" in bench.attention_kernel_name(synth.ALL_WORKLOADS["global_s9_g64_affine8"])
     assert "fp32" in bench.attention_kernel_name(synth.ALL_WORKLOADS["global_s9_g64_f32"])
+
+
+_REFERENCE_ARM_CHILD = r"""
+import json, sys
+sys.path.insert(0, sys.argv[1])
+import bench
+rc = bench.main(["--impl", "reference", "--workload", "global_s2_g16", "--steps", "1", "--warmup", "0",
+                 "--reference-budget-s", "2"])
+maps = open("/proc/self/maps").read()
+print(json.dumps({"rc": rc, "lib_mapped": "libvggt_attn" in maps,
+                  "package_imported": "feed_forward_view_b200" in sys.modules}))
+"""
+
+
+def test_reference_arm_never_loads_the_product_library():
+    # The oracle arm's process must hold neither the package nor its shared
+    # library: it times the oracle alone.
+    import subprocess
+
+    root = str(pathlib.Path(__file__).resolve().parents[1])
+    res = subprocess.run([sys.executable, "-c", _REFERENCE_ARM_CHILD, root], capture_output=True, text=True,
+                         timeout=600, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    arm, probe = json.loads(lines[0]), json.loads(lines[-1])
+    assert arm["impl"] == "reference" and arm["value"] > 0
+    assert probe == {"rc": 0, "lib_mapped": False, "package_imported": False}
