@@ -213,6 +213,8 @@ kv_pool_kernel(const __grid_constant__ PoolJob job, FreqTable freq) {
     constexpr int kKeyThreads = pool_threads<kFused>() - kValueThreads;
     constexpr uint32_t kKeyBar = 1, kKeyBarThreads = 32 + kKeyThreads;  // warp 0 + the key warps
     constexpr int kHeadsPerPass = 16;
+    static_assert(kValueThreads / (kFused ? 4 : 8) == kHeadsPerPass && (!kFused || kKeyThreads / 4 == kHeadsPerPass),
+                  "each group covers kHeadsPerPass heads per pass");
 
     const FrameLayout& L = job.layout;
     const int lane = threadIdx.x & 31;
